@@ -1,0 +1,59 @@
+"""The diagonal enumeration, pinned by brute force and a hand-written table.
+
+Source: skill page "Diagonal Batching for Recurrent Memory Transformers", "Implementation"
+(the diagonal scheduler) and "Architecture Overview" (dependency preservation): the
+(layer, segment) grid is swept along anti-diagonals d = l + s, and cell (l, s) needs
+(l-1, s) and (l, s-1) to have run first.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+from oracle import armt
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def brute_force_diagonals(L, S):
+    """Group all L*S cells by l+s, each group in ascending l -- no diagonal-index loop."""
+    cells = sorted(itertools.product(range(L), range(S)), key=lambda c: (c[0] + c[1], c[0]))
+    groups = {}
+    for l, s in cells:
+        groups.setdefault(l + s, []).append((l, s))
+    return [groups[k] for k in sorted(groups)]
+
+
+@pytest.mark.parametrize("L,S", [(L, S) for L in range(1, 13) for S in range(1, 13)])
+def test_diagonals_brute_force(L, S):
+    diags = armt.diagonals(L, S)
+    assert diags == brute_force_diagonals(L, S)
+    assert len(diags) == L + S - 1
+    flat = [c for d in diags for c in d]
+    assert len(flat) == L * S and len(set(flat)) == L * S
+    where = {c: i for i, d in enumerate(diags) for c in d}
+    for (l, s), i in where.items():
+        assert l + s == i
+        if l > 0:
+            assert where[(l - 1, s)] == i - 1
+        if s > 0:
+            assert where[(l, s - 1)] == i - 1
+        # at most one cell per layer on a diagonal (layer state is updated in place)
+    for d in diags:
+        ls = [l for l, _ in d]
+        assert ls == sorted(ls) and len(set(ls)) == len(ls)
+    # size of diagonal d (a count of lattice points on the line l + s = d inside the grid)
+    sizes = [len(d) for d in diags]
+    for i, n in enumerate(sizes):
+        assert n == sum(1 for l in range(L) if 0 <= i - l < S)
+
+
+def test_diagonals_golden_table():
+    rows = np.loadtxt(os.path.join(GOLDEN, "schedule_L3_S4.txt"), dtype=np.int32, comments="#")
+    np.testing.assert_array_equal(armt.schedule_triples(3, 4, "diagonal"), rows)
+
+
+def test_sequential_steps():
+    t = armt.schedule_triples(3, 2, "sequential")
+    np.testing.assert_array_equal(t, [[0, 0, 0], [1, 1, 0], [2, 2, 0], [3, 0, 1], [4, 1, 1], [5, 2, 1]])
