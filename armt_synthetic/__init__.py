@@ -10,14 +10,18 @@ ARMT on sequences of up to 131,072 tokens. The pages give no checkpoint, so weig
 random: every projection ~ N(0, 0.02), RMSNorm gains = 1, memory tokens ~ N(0, 0.02),
 embeddings ~ N(0, 1).
 
-Draw order (one numpy PCG64 stream per seed, float32 standard normals):
-  weights seed: for l in 0..L-1: wq, wk, wv, wo, w_gate, w_up, w_down, w_mq, w_mk, w_mv, w_mo;
-                then mem_tokens.
-  embedding seed: one [n_segments * seg_len, d_model] draw.
+Streams (numpy PCG64 seeded with an integer tuple; float32 standard normals, row-major):
+  weight matrix k of layer l:  PCG64([seed, l, i_k]), i_k = position of k in LAYER_KEYS
+  memory tokens:               PCG64([seed, L, 0])
+  embeddings of segment s:     PCG64([emb_seed, s])   (so a prefix of segments is the same
+                                                       whatever the total segment count)
+Independent streams let the draws run in parallel threads.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
+import os
 from dataclasses import dataclass
 
 import numpy as np
@@ -86,7 +90,15 @@ CONFIGS = {
 
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); returns float32 holding them."""
-    return bf16_bits_to_f32(bf16_bits(a))
+    out = np.array(a, dtype=np.float32, copy=True)
+    _round_bf16_inplace(out)
+    return out
+
+
+def _round_bf16_inplace(a: np.ndarray) -> None:
+    u = a.reshape(-1).view(np.uint32)
+    u += np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    u &= np.uint32(0xFFFF0000)
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -100,6 +112,19 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
+def _normal(key: tuple, shape: tuple, std: float, bf16: bool) -> np.ndarray:
+    a = np.random.Generator(np.random.PCG64(list(key))).standard_normal(shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    if bf16:
+        _round_bf16_inplace(a)
+    return a
+
+
+def _pool():
+    return cf.ThreadPoolExecutor(max_workers=max(1, min(32, os.cpu_count() or 1)))
+
+
 def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02) -> dict:
     """Random-init weights of an ARMT with cfg's shapes.
 
@@ -107,23 +132,28 @@ def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02) ->
     [n_mem, d_model]. Values are float32; for a bf16 model they are already rounded to
     bf16 (so float32 and bf16 storage hold the same numbers).
     """
-    rng = np.random.Generator(np.random.PCG64(seed))
     shapes = cfg.weight_shapes()
-    w = {k: [] for k in LAYER_KEYS}
-    for _ in range(cfg.n_layers):
-        for k in LAYER_KEYS:
-            w[k].append(rng.standard_normal(shapes[k], dtype=np.float32) * np.float32(std))
-    w["mem_tokens"] = rng.standard_normal((cfg.n_mem, cfg.d_model), dtype=np.float32) * np.float32(std)
+    bf16 = cfg.dtype == "bf16"
+    jobs = [(l, i, k) for l in range(cfg.n_layers) for i, k in enumerate(LAYER_KEYS)]
+    with _pool() as ex:
+        mats = list(ex.map(lambda j: _normal((seed, j[0], j[1]), shapes[j[2]], std, bf16), jobs))
+    w = {k: [None] * cfg.n_layers for k in LAYER_KEYS}
+    for (l, _, k), m in zip(jobs, mats):
+        w[k][l] = m
+    w["mem_tokens"] = _normal((seed, cfg.n_layers, 0), (cfg.n_mem, cfg.d_model), std, bf16)
     w["g_attn"] = [np.ones(cfg.d_model, np.float32) for _ in range(cfg.n_layers)]
     w["g_mlp"] = [np.ones(cfg.d_model, np.float32) for _ in range(cfg.n_layers)]
-    if cfg.dtype == "bf16":
-        for k, v in w.items():
-            w[k] = [round_to_bf16(a) for a in v] if isinstance(v, list) else round_to_bf16(v)
     return w
 
 
 def make_embeddings(cfg: ArmtConfig, n_segments: int, seed: int = EMB_SEED) -> np.ndarray:
     """Input embeddings [n_segments * seg_len, d_model] ~ N(0, 1) (bf16-rounded for a bf16 model)."""
-    rng = np.random.Generator(np.random.PCG64(seed))
-    e = rng.standard_normal((n_segments * cfg.seg_len, cfg.d_model), dtype=np.float32)
-    return round_to_bf16(e) if cfg.dtype == "bf16" else e
+    out = np.empty((n_segments * cfg.seg_len, cfg.d_model), np.float32)
+    seg = cfg.seg_len
+
+    def fill(s):
+        out[s * seg:(s + 1) * seg] = _normal((seed, s), (seg, cfg.d_model), 1.0, cfg.dtype == "bf16")
+
+    with _pool() as ex:
+        list(ex.map(fill, range(n_segments)))
+    return out

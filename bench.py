@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Throughput of diagonal-batched ARMT prefill on B200.
+
+Workload (per GPU): a LLaMA-1B-shaped ARMT -- 16 layers, d_model 2048, 32 query / 8 KV
+heads of 64, SwiGLU 8192, RMSNorm, RoPE theta 500000, associative memory d_k = d_v = 64 --
+prefilling one 131,072-token sequence as 128 segments of 1024 tokens + 16 memory tokens,
+bf16 storage with fp32 accumulation. Seeded N(0, 1) embeddings, random-init N(0, 0.02)
+weights. One step = one rmt_forward over all 128 segments (143 anti-diagonals, 14 kernel
+kinds per diagonal), schedule DIAGONAL. Inputs (1.96 GB of weights, 0.54 GB of embeddings)
+are larger than the 126 MB L2, so no flush is needed between steps.
+
+`python bench.py --gpus N --steps K --warmup W` prints one JSON line (rank 0). For N > 1
+(torchrun) every rank runs an independent replica on its own GPU: the method has no
+cross-GPU exchange, so the value is N x 131,072 tokens over the slowest rank's time.
+`--impl reference` times the oracle (numpy, host cores) on a bounded sample of the same
+workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from armt_synthetic import CONFIGS, make_embeddings, make_weights  # noqa: E402
+
+METRIC = "ARMT prefill tokens/s at 131K (1B-shape, 1 B200); grouped-GEMM % tensor peak"
+UNIT = "tokens/s"
+N_SEGMENTS = 128
+WORKLOAD = "LLaMA-1B-shaped ARMT prefill of one 131,072-token sequence (128 x (1024 + 16 memory) tokens)"
+DATA = "synthetic: seeded N(0,1) embeddings, random-init N(0,0.02) weights"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes per launch of the gate/up GEMM measured by ncu (profiles/gateup_gemm_1b.md); None
+# until a capture of the current kernel exists.
+GATEUP_TRAFFIC_BYTES_PER_LAUNCH = None
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--segments", type=int, default=N_SEGMENTS)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-sequential", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons every 200 ms while running."""
+
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=lambda: self.lines.extend(iter(self.proc.stdout.readline, "")),
+                                       daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": float(max(power))}
+
+
+# ------------------------------------------------------------------------ reference arm
+
+def run_reference(args, world: int, rank: int) -> int:
+    """The oracle (numpy, strictly sequential) on the host cores: each step runs the next
+    block of (layer, segment) cells of the same workload in sequential order, carrying the
+    recurrent state; the block size is calibrated so the whole run stays within minutes."""
+    if rank != 0:
+        return 0
+    from oracle import armt
+
+    cfg = CONFIGS["1b"]
+    L, seg = cfg.n_layers, cfg.seg_len
+    w = make_weights(cfg)
+    lws = [armt.layer_weights(w, l, np.float32) for l in range(L)]
+    mem = w["mem_tokens"]
+    K, W = max(1, args.steps), max(0, args.warmup)
+    # calibrate on one cell (counts as warm-up work)
+    emb0 = make_embeddings(cfg, 1)
+    x = np.concatenate([emb0[:seg], mem])
+    A0, z0 = np.zeros((cfg.d_k, cfg.d_v), np.float32), np.zeros(cfg.d_k, np.float32)
+    t0 = time.perf_counter()
+    armt.armt_cell(x, lws[0], A0, z0, cfg)
+    t_cell = time.perf_counter() - t0
+    budget = min(30.0, max(2.0, 150.0 / (K + W)))
+    cells_per_step = max(1, int(budget / t_cell))
+    n_cells = (K + W) * cells_per_step
+    n_seg = min(N_SEGMENTS, math.ceil(n_cells / L) + 1)
+    emb = make_embeddings(cfg, n_seg)
+    A = [np.zeros((cfg.d_k, cfg.d_v), np.float32) for _ in range(L)]
+    z = [np.zeros(cfg.d_k, np.float32) for _ in range(L)]
+    state = {"c": 0, "x": None}
+
+    def run_cells(n):
+        for _ in range(n):
+            s, l = divmod(state["c"] % (n_seg * L), L)
+            if l == 0:
+                state["x"] = np.concatenate([emb[s * seg:(s + 1) * seg], mem])
+                if s == 0:
+                    for i in range(L):
+                        A[i][:] = 0
+                        z[i][:] = 0
+            state["x"], A[l], z[l] = armt.armt_cell(state["x"], lws[l], A[l], z[l], cfg)
+            state["c"] += 1
+
+    for _ in range(W):
+        run_cells(cells_per_step)
+    times = []
+    for _ in range(K):
+        t0 = time.perf_counter()
+        run_cells(cells_per_step)
+        times.append(time.perf_counter() - t0)
+    step_s = float(np.mean(times))
+    tokens_per_step = cells_per_step * seg / L  # one cell = one layer of one segment
+    value = tokens_per_step / step_s
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": DATA,
+        "config": {"workload": WORKLOAD, "layers": L, "segments": N_SEGMENTS, "seg_len": seg, "n_mem": cfg.n_mem,
+                   "tokens": N_SEGMENTS * seg, "schedule": "sequential (oracle)", "batch": 1},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{cells_per_step} (layer, segment) cells per step in sequential order "
+                                   f"({tokens_per_step:.0f} token-equivalents of the 16-layer model)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def cpu_baseline(cfg, w, emb) -> dict:
+    """The oracle as it stands, on one segment (1024 tokens through all 16 layers)."""
+    from oracle import armt
+    seg = cfg.seg_len
+    t0 = time.perf_counter()
+    armt.forward(cfg, w, emb[:seg], 1, dtype=np.float32)
+    dt = time.perf_counter() - t0
+    return {"value": seg / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"1 of {N_SEGMENTS} segments (1024 tokens through 16 layers, {dt:.1f} s); per-segment cost "
+                      "is the same for every segment"}
+
+
+def main() -> int:
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import torch.distributed as dist
+
+    from recurrent_memory_transformer_anti_b200 import rmt
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    K, W = max(1, args.steps), max(3, args.warmup)
+    S = args.segments
+    cfg = CONFIGS["1b"]
+    w = make_weights(cfg)
+    emb = make_embeddings(cfg, S)
+    h = rmt.rmt_create(rmt.weights_storage(w, "bf16", dev), cfg)
+    e = rmt.storage(emb, "bf16", dev)
+    out = torch.empty_like(e)
+    A = torch.empty(cfg.n_layers, cfg.d_k, cfg.d_v, device=dev)
+    z = torch.empty(cfg.n_layers, cfg.d_k, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def run(schedule, n):
+        for _ in range(n):
+            rmt.rmt_forward(h, e, S, schedule, out, A, z, stream)
+
+    def timed(schedule, n):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(schedule, n)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1) / n
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    run("diagonal", W)
+    rmt.rmt_sync(h, stream)
+
+    # ---- timed region: K diagonal-batched forwards, gate/up GEMM launches probed
+    rmt.rmt_probe(h, ["gateup"])
+    props = torch.cuda.get_device_properties(local)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler.start()
+    ms = timed("diagonal", K)
+    clocks = sampler.stop()
+    probe = rmt.rmt_probe_read(h, "gateup")
+    rmt.rmt_sync(h, stream)
+    rmt.rmt_probe(h, [])
+    tokens = S * cfg.seg_len
+    value = world * tokens / (ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    achieved = probe["flops"] / (probe["ms"] / 1e3) / 1e12 if probe["ms"] > 0 else None
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "kernel": "grouped GEMM gate/up + SwiGLU epilogue (tcgen05)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak if achieved else None,
+                "peak_source": f"bf16_tflops_sustained ({peak_src})",
+                "launches": probe["launches"], "kernel_ms_per_step": probe["ms"] / K,
+                "traffic": GATEUP_TRAFFIC_BYTES_PER_LAUNCH}
+
+    # ---- per-kernel breakdown of one forward (outside the timed region)
+    rmt.rmt_probe(h, list(rmt.KERNELS))
+    run("diagonal", 1)
+    rmt.rmt_sync(h, stream)
+    breakdown = {}
+    for k in rmt.KERNELS:
+        r = rmt.rmt_probe_read(h, k)
+        if r["launches"]:
+            breakdown[k] = {"ms": round(r["ms"], 3), "launches": r["launches"],
+                            "tflops": round(r["flops"] / r["ms"] / 1e9, 1) if r["ms"] > 0 and r["flops"] else None,
+                            "gbs": round(r["bytes"] / r["ms"] / 1e6, 1) if r["ms"] > 0 else None}
+    rmt.rmt_probe(h, [])
+
+    # ---- sequential schedule on the same kernels (the 1.8x comparison of the abstract)
+    seq = None
+    if not args.no_sequential:
+        run("sequential", 1)
+        seq_ms = timed("sequential", max(1, min(K, 3)))
+        seq = {"ms_per_step": seq_ms, "tokens_per_s": world * tokens / (seq_ms / 1e3),
+               "diagonal_speedup": seq_ms / ms}
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    e_host = e.cpu().pin_memory()
+    o_host = torch.empty_like(e_host).pin_memory()
+    A_host = torch.empty(A.shape, dtype=A.dtype).pin_memory()
+    z_host = torch.empty(z.shape, dtype=z.dtype).pin_memory()
+    rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
+    torch.cuda.synchronize()
+    n_e2e = max(1, min(K, 3))
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    rmt.rmt_sync(h, stream)
+    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": e_host.numel() * e_host.element_size(),
+           "d2h_bytes_per_step": o_host.numel() * o_host.element_size() + A_host.numel() * 4 + z_host.numel() * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, w, emb)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": DATA,
+            "config": {"workload": WORKLOAD, "layers": cfg.n_layers, "d_model": cfg.d_model, "segments": S,
+                       "seg_len": cfg.seg_len, "n_mem": cfg.n_mem, "tokens": tokens, "schedule": "diagonal",
+                       "batch": 1, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (weights 1.96 GB, embeddings 0.54 GB): no flush"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": probe["all_launches"],
+            "clocks": clocks,
+            "sequential": seq,
+            "breakdown_one_step": breakdown,
+        }
+        print(json.dumps(line))
+    rmt.rmt_destroy(h)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

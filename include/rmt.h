@@ -1,0 +1,208 @@
+/*
+ * rmt.h -- C ABI of the diagonal-batched ARMT prefill library (librmt.so, sm_100a).
+ *
+ * The method: "Diagonal Batching Unlocks Parallelism in Recurrent Memory Transformers
+ * for Long Contexts" (arXiv 2506.05229; abstract, and the skill page of the same title:
+ * "Core Concept", "Architecture Overview", "Implementation"). An ARMT runs a grid of
+ * (layer l, segment s) cells; cell (l, s) needs the output of (l-1, s) and layer l's
+ * associative memory after (l, s-1). The grid is swept in anti-diagonals d = l + s and
+ * every cell of a diagonal runs in the same grouped launches, each cell with its own
+ * layer's weights. The result is the sequential model's result, reordered only.
+ *
+ * Conventions for every entry point:
+ *  - Status codes only: no exceptions or aborts cross the ABI. A non-OK status leaves
+ *    a message for rmt_last_error() (thread-local) and leaves any handle usable.
+ *  - "device or host" pointers may point to device memory or to host memory (pinned or
+ *    pageable); host buffers are copied inside the call, on the given stream.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *    stream) and the call returns without waiting, unless stated otherwise. Device-side
+ *    faults of a bounded wait show up at rmt_sync() as RMT_ETIMEOUT.
+ *  - Matrices are row-major; projection weights are [out_features, in_features] like
+ *    nn.Linear. bf16 values are passed as their 16-bit patterns.
+ */
+#ifndef RMT_H
+#define RMT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RMT_OK = 0,
+  RMT_EINVAL = 1,    /* bad argument: null pointer, unsupported shape, size out of range */
+  RMT_ENOMEM = 2,    /* device or pinned allocation failed */
+  RMT_ECUDA = 3,     /* a CUDA runtime call or launch failed */
+  RMT_ETIMEOUT = 4,  /* a bounded device-side wait gave up (reported by rmt_sync) */
+  RMT_ESTATE = 5     /* call not valid in this state (e.g. trace before any forward) */
+} rmt_status;
+
+typedef enum { RMT_DIAGONAL = 0, RMT_SEQUENTIAL = 1 } rmt_schedule;
+
+/* Storage type of weights, embeddings, outputs and inter-kernel activations.
+ * RMT_F32: every GEMM is an fp32 FMA kernel (no tensor cores).
+ * RMT_BF16: GEMMs and attention run on tensor cores with fp32 accumulation; the residual
+ * stream, softmax, RMSNorm statistics and the memory state stay fp32. */
+typedef enum { RMT_F32 = 0, RMT_BF16 = 1 } rmt_dtype;
+
+/* Model shape. A cell has M = seg_len + n_mem rows: the segment's tokens followed by the
+ * n_mem memory tokens. Limits (else RMT_EINVAL): all sizes > 0; n_heads % n_kv_heads == 0;
+ * head_dim in {32, 64, 128}; d_k, d_v multiples of 32, at most 128; n_mem <= 64 and
+ * n_mem*(d_k+d_v) <= 4096; d_ff % 64 == 0; d_model % 4 == 0.
+ * RMT_BF16 also needs d_model, n_heads*head_dim and d_v multiples of 64, and projection
+ * widths that tile by 256/128/64/32 columns: (n_heads+2*n_kv_heads)*head_dim in whole
+ * heads, 2*d_ff by at least 128, d_model and d_k. */
+typedef struct {
+  int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, d_ff, seg_len, n_mem, d_k, d_v;
+  float rope_theta; /* RoPE base (500000 for the LLaMA-shaped models) */
+  float rms_eps;    /* RMSNorm epsilon (1e-5) */
+  float mem_eps;    /* associative-memory epsilon in both denominators (1e-6) */
+  rmt_dtype dtype;
+} rmt_cfg;
+
+/* Model weights, in cfg.dtype. Each `const void* const*` member is a host array of
+ * n_layers pointers (one per layer); each pointer may be device or host memory.
+ *   wq [H*dh, d]  wk [Hkv*dh, d]  wv [Hkv*dh, d]  wo [d, H*dh]
+ *   w_gate [F, d]  w_up [F, d]  w_down [d, F]                 (SwiGLU MLP)
+ *   w_mq [d_k, d]  w_mk [d_k, d]  w_mv [d_v, d]  w_mo [d, d_v] (associative memory)
+ *   g_attn [d]  g_mlp [d]                                      (RMSNorm gains)
+ *   mem_tokens [n_mem, d]: one matrix, appended after every segment at layer 0. */
+typedef struct {
+  const void* const* wq;
+  const void* const* wk;
+  const void* const* wv;
+  const void* const* wo;
+  const void* const* w_gate;
+  const void* const* w_up;
+  const void* const* w_down;
+  const void* const* w_mq;
+  const void* const* w_mk;
+  const void* const* w_mv;
+  const void* const* w_mo;
+  const void* const* g_attn;
+  const void* const* g_mlp;
+  const void* mem_tokens;
+} rmt_weights;
+
+typedef struct rmt_handle rmt_handle;
+
+/* Validate cfg, copy and pack the weights into library-owned device memory (on the
+ * current CUDA device), allocate activations and state. Synchronous. The caller may free
+ * its weight buffers when this returns. *out is set only on RMT_OK. */
+rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle** out);
+
+/* ARMT prefill of n_segments segments (batch 1).
+ *   emb        [n_segments*seg_len, d_model] in cfg.dtype, device or host.
+ *   out_hidden [n_segments*seg_len, d_model] in cfg.dtype, device or host: the last
+ *              layer's hidden states at the segment-token rows (memory rows dropped).
+ *   out_A      [n_layers, d_k, d_v] fp32 or NULL; out_z [n_layers, d_k] fp32 or NULL:
+ *              the memory state after the last segment. The state starts at zero.
+ * schedule RMT_DIAGONAL runs one grouped launch per step over all cells of an
+ * anti-diagonal; RMT_SEQUENTIAL runs the same kernels one cell per step, segments
+ * outermost. Both give the same bits. Asynchronous on `stream`; a handle runs one forward
+ * at a time (calls on one handle must be ordered on one stream). */
+rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule,
+                       void* out_hidden, float* out_A, float* out_z, void* stream);
+
+/* The execution order as int32 triples (step, layer, segment), one per cell, n_layers*
+ * n_segments of them: steps ascend; within a diagonal step layers ascend. Host memory,
+ * cap = capacity of out_dls in int32 elements (>= 3*L*S). Needs no GPU. */
+rmt_status rmt_schedule_table(int32_t n_layers, int32_t n_segments, rmt_schedule schedule,
+                              int32_t* out_dls, size_t cap);
+rmt_status rmt_get_schedule(const rmt_handle* h, int32_t n_segments, rmt_schedule schedule,
+                            int32_t* out_dls, size_t cap);
+
+/* The (step, layer, segment) triples the device recorded for each cell during the last
+ * forward, in schedule-table order (written by the memory-update kernel of each cell).
+ * Synchronizes the device. RMT_ESTATE before the first forward. */
+rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap);
+
+/* Wait for `stream`, then report (and clear) the handle's device error word: RMT_ETIMEOUT
+ * if a bounded device wait gave up, RMT_ECUDA on a CUDA error. With h == NULL the error
+ * word of the kernel-level entry points on the current device is checked. */
+rmt_status rmt_sync(rmt_handle* h, void* stream);
+
+/* Kernel kinds of one schedule step, in launch order (see rmt_forward). */
+typedef enum {
+  RMT_K_ASSEMBLE = 0,  /* layer-0 input: segment embeddings + memory tokens */
+  RMT_K_MEMQ = 1,      /* memory-query projection (grouped GEMM) */
+  RMT_K_MEMREAD = 2,   /* associative read */
+  RMT_K_MEMO = 3,      /* read-out projection + residual (grouped GEMM) */
+  RMT_K_RMSNORM1 = 4,
+  RMT_K_QKV = 5,       /* QKV projection + RoPE (grouped GEMM) */
+  RMT_K_ATTENTION = 6,
+  RMT_K_O = 7,         /* output projection + residual (grouped GEMM) */
+  RMT_K_RMSNORM2 = 8,
+  RMT_K_GATEUP = 9,    /* gate/up projection + SwiGLU (grouped GEMM) */
+  RMT_K_DOWN = 10,     /* down projection + residual (grouped GEMM) */
+  RMT_K_MEMKV = 11,    /* memory key/value projection of the memory-token rows */
+  RMT_K_MEMUPDATE = 12,/* delta-rule update */
+  RMT_K_EMIT = 13,     /* segment output */
+  RMT_K_COUNT = 14
+} rmt_kernel;
+
+/* Start (or restart) timing every launch of the kernel kinds in `mask` (bit k = kind k)
+ * in later forwards on this handle, with a CUDA event pair around each launch on the
+ * forward's stream; mask 0 stops timing. Resets all probe counters. */
+rmt_status rmt_probe(rmt_handle* h, uint32_t mask);
+
+/* Probe totals since rmt_probe for one kind: summed event time in ms, launches, and the
+ * algorithmic flops and bytes of those launches (the minimum a launch must compute and
+ * move); plus the number of kernels of all kinds the handle launched. Any output may be
+ * NULL. Synchronizes the device. */
+rmt_status rmt_probe_read(rmt_handle* h, rmt_kernel kind, double* ms, int64_t* launches, double* flops,
+                          double* bytes, int64_t* all_launches);
+
+/* Free everything the handle owns. Synchronizes the device. NULL is accepted. */
+rmt_status rmt_destroy(rmt_handle* h);
+
+/* Message of the last non-OK status on this thread ("" if none). */
+const char* rmt_last_error(void);
+
+/* ------------------------------------------------------------------------------------
+ * Kernel-level entry points: the same kernels the forward launches, on caller buffers
+ * (device pointers only), for testing and measurement. All asynchronous on `stream`.
+ * ------------------------------------------------------------------------------------ */
+
+/* Grouped GEMM on tensor cores (tcgen05, TMEM accumulators, TMA-fed):
+ *   C[g] = A[g] . B[g]^T for g in 0..G-1, bf16 inputs, fp32 accumulation.
+ * A [G, M, K] bf16, B [G, N, K] bf16 (a distinct weight per group, [out, in]),
+ * C [G, M, N] in out_dtype (RMT_F32 or RMT_BF16). Needs K % 64 == 0 and N % 64 == 0;
+ * M is arbitrary (ragged last tile). Pointers 16-byte aligned. "Architecture Overview":
+ * GroupedGEMM operations batched across layers within a diagonal. */
+rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t G, int32_t M,
+                                 int32_t N, int32_t K, rmt_dtype out_dtype, void* stream);
+
+/* Segment-local causal attention with grouped KV heads, per cell:
+ *   out[g, i, h] = softmax_j<=i(q[g,i,h] . k[g,j,h/(H/Hkv)] / sqrt(dh)) v[g,j,h/(H/Hkv)]
+ * qkv [G, M, (H + 2*Hkv)*dh] (q heads, then k heads, then v heads, RoPE already applied),
+ * out [G, M, H*dh]; dtype RMT_F32 or RMT_BF16 (softmax in fp32). dh in {32, 64, 128}. */
+rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32_t H, int32_t Hkv,
+                         int32_t dh, rmt_dtype dtype, void* stream);
+
+/* Associative read, per row r of each group g (phi(x) = elu(x) + 1):
+ *   o[g,r] = phi(q[g,r]) A[g] / (phi(q[g,r]) . z[g] + eps)
+ * q [G, M, dk] fp32 (before phi), A [G, dk, dv] fp32, z [G, dk] fp32, o [G, M, dv] in
+ * dtype. dk, dv multiples of 32, <= 128. */
+rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void* o, int32_t G,
+                           int32_t M, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
+
+/* Delta-rule write of n rows per group, all rows against the pre-update state:
+ *   v_bar = phi(k) A / (phi(k) . z + eps);  A += phi(k)^T (v - v_bar);  z += sum_r phi(k_r)
+ * k [G, n, dk] fp32 (before phi), v [G, n, dv] fp32, A [G, dk, dv] and z [G, dk] fp32,
+ * updated in place. n <= 64; dk, dv multiples of 32, <= 128. */
+rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G,
+                             int32_t n, int32_t dk, int32_t dv, float eps, void* stream);
+
+/* RMSNorm of fp32 rows into dtype: y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g.
+ * x [rows, d] fp32, g [d] and y [rows, d] in dtype. d % 4 == 0. */
+rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int32_t d, float eps,
+                       rmt_dtype dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMT_H */

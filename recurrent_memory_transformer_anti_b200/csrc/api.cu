@@ -1,0 +1,783 @@
+// C ABI of the diagonal-batched ARMT prefill library: handle, weight packing, the host
+// scheduler and the launch sequence of one schedule step.
+//
+// Scheduler ("Implementation" of the diagonal-batching skill page): the (layer, segment)
+// grid is swept in anti-diagonals d = l + s, cells of a diagonal in ascending layer order,
+// d = 0 .. L+S-2; the layers on diagonal d are max(0, d-S+1) .. min(d, L-1). The
+// sequential schedule runs one cell per step, segments outermost. Either way one step is
+// the same fixed launch sequence over the step's cells (a cell table on the device):
+//   [layer-0 input] -> mem-q GEMM -> memory read -> mem-o GEMM (+residual) -> RMSNorm
+//   -> QKV GEMM (+RoPE) -> attention -> O GEMM (+residual) -> RMSNorm
+//   -> gate/up GEMM (+SwiGLU) -> down GEMM (+residual) -> memory k/v -> memory update
+//   -> [segment output]
+// Each kernel does the same arithmetic for a cell whatever else shares its launch, so the
+// two schedules give identical bits ("Dependency Preservation" in "Architecture
+// Overview"; arXiv 2506.05229 abstract: a pure run-time reordering with exact recurrence).
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "launch.h"
+#include "rmt.h"
+
+using namespace rmt;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+rmt_status fail(rmt_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+#define RMT_CUDA(call)                                                                             \
+  do {                                                                                             \
+    cudaError_t e_ = (call);                                                                       \
+    if (e_ != cudaSuccess) return fail(RMT_ECUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+bool is_host_ptr(const void* p) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return true;
+  }
+  return attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged;
+}
+
+struct Table {
+  std::vector<Cell> cells;  // host copy, execution order
+  std::vector<int> off, cnt;
+  Cell* dev = nullptr;
+};
+
+void build_table(int L, int S, rmt_schedule sch, Table& t) {
+  t.cells.clear();
+  t.off.clear();
+  t.cnt.clear();
+  if (sch == RMT_DIAGONAL) {
+    for (int d = 0; d <= L + S - 2; ++d) {
+      const int lo = d - S + 1 > 0 ? d - S + 1 : 0, hi = d < L - 1 ? d : L - 1;
+      if (lo > hi) continue;
+      t.off.push_back(static_cast<int>(t.cells.size()));
+      for (int l = lo; l <= hi; ++l) t.cells.push_back(Cell{l, d - l});
+      t.cnt.push_back(hi - lo + 1);
+    }
+  } else {
+    for (int s = 0; s < S; ++s)
+      for (int l = 0; l < L; ++l) {
+        t.off.push_back(static_cast<int>(t.cells.size()));
+        t.cells.push_back(Cell{l, s});
+        t.cnt.push_back(1);
+      }
+  }
+}
+
+// Identity cell table (g, 0), g = 0..n-1, for the kernel-level entry points.
+struct DeviceScratch {
+  Cell* cells = nullptr;
+  int cap = 0;
+  int* err = nullptr;
+};
+DeviceScratch g_dev_scratch[64];
+
+rmt_status device_scratch(int G, const Cell** cells, int** err) {
+  int dev = 0;
+  RMT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RMT_EINVAL, "device index out of range");
+  DeviceScratch& s = g_dev_scratch[dev];
+  if (!s.err) {
+    RMT_CUDA(cudaMalloc(&s.err, sizeof(int)));
+    RMT_CUDA(cudaMemset(s.err, 0, sizeof(int)));
+  }
+  if (G > s.cap) {
+    const int cap = G > 4096 ? G : 4096;
+    std::vector<Cell> h(cap);
+    for (int g = 0; g < cap; ++g) h[g] = Cell{g, 0};
+    Cell* p = nullptr;
+    if (cudaMalloc(&p, sizeof(Cell) * cap) != cudaSuccess) return fail(RMT_ENOMEM, "cell table allocation failed");
+    RMT_CUDA(cudaMemcpy(p, h.data(), sizeof(Cell) * cap, cudaMemcpyHostToDevice));
+    if (s.cells) cudaFree(s.cells);
+    s.cells = p;
+    s.cap = cap;
+  }
+  *cells = s.cells;
+  if (err) *err = s.err;
+  return RMT_OK;
+}
+
+}  // namespace
+
+struct rmt_handle {
+  rmt_cfg cfg{};
+  int dev = 0;
+  bool bf16 = false;
+  int M = 0, es = 4, Nqkv = 0, nsplit = 0;
+  // packed weights (cfg dtype)
+  void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_d = nullptr, *w_mq = nullptr, *w_mo = nullptr,
+       *w_mkv = nullptr, *g1 = nullptr, *g2 = nullptr, *memtok = nullptr;
+  // activations and state
+  float* x = nullptr;
+  __nv_bfloat16* xb = nullptr;
+  void *hbuf = nullptr, *qkv = nullptr, *att = nullptr, *u = nullptr, *om = nullptr;
+  float *qm = nullptr, *part = nullptr, *A = nullptr, *z = nullptr;
+  float2* rope = nullptr;
+  int* err = nullptr;
+  int* trace = nullptr;
+  size_t trace_cap = 0;
+  int traced_cells = -1;
+  void* emb_stage = nullptr;
+  size_t emb_stage_bytes = 0;
+  void* out_stage = nullptr;
+  size_t out_stage_bytes = 0;
+  std::map<std::pair<int, int>, Table> tables;
+  CUtensorMap tm_xb, tm_om, tm_h, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo;
+  int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
+  std::vector<void*> allocs;
+  // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
+  struct ProbeRec {
+    int kind;
+    double flops, bytes;
+    cudaEvent_t a, b;
+  };
+  uint32_t probe_mask = 0;
+  std::vector<cudaEvent_t> probe_pool;
+  size_t probe_used = 0;
+  std::vector<ProbeRec> probe_recs;
+  int64_t launches = 0;
+
+  cudaEvent_t probe_event() {
+    if (probe_used == probe_pool.size()) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      probe_pool.push_back(e);
+    }
+    return probe_pool[probe_used++];
+  }
+
+  void* alloc(size_t bytes) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    allocs.push_back(p);
+    return p;
+  }
+  void release() {
+    for (void* p : allocs) cudaFree(p);
+    allocs.clear();
+    for (auto& kv : tables)
+      if (kv.second.dev) cudaFree(kv.second.dev);
+    tables.clear();
+    if (trace) cudaFree(trace);
+    if (emb_stage) cudaFree(emb_stage);
+    if (out_stage) cudaFree(out_stage);
+    trace = nullptr;
+    emb_stage = out_stage = nullptr;
+    for (cudaEvent_t e : probe_pool) cudaEventDestroy(e);
+    probe_pool.clear();
+    probe_recs.clear();
+    probe_used = 0;
+  }
+};
+
+namespace {
+
+bool validate_cfg(const rmt_cfg* c, std::string& why) {
+  if (c->n_layers <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+      c->d_ff <= 0 || c->seg_len <= 0 || c->n_mem <= 0 || c->d_k <= 0 || c->d_v <= 0) {
+    why = "all sizes must be positive";
+    return false;
+  }
+  if (c->dtype != RMT_F32 && c->dtype != RMT_BF16) return why = "dtype must be RMT_F32 or RMT_BF16", false;
+  if (c->n_heads % c->n_kv_heads) return why = "n_heads must be a multiple of n_kv_heads", false;
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return why = "head_dim must be 32, 64 or 128", false;
+  if (c->d_k % 32 || c->d_v % 32 || c->d_k > 128 || c->d_v > 128)
+    return why = "d_k and d_v must be multiples of 32, at most 128", false;
+  if (c->n_mem > 64 || c->n_mem * (c->d_k + c->d_v) > 4096) return why = "n_mem <= 64 and n_mem*(d_k+d_v) <= 4096", false;
+  if (c->d_ff % 64) return why = "d_ff must be a multiple of 64", false;
+  if (c->d_model % 4) return why = "d_model must be a multiple of 4", false;
+  if (!(c->rope_theta > 0.f) || !(c->rms_eps >= 0.f) || !(c->mem_eps >= 0.f))
+    return why = "rope_theta > 0, rms_eps >= 0, mem_eps >= 0", false;
+  if (c->dtype == RMT_BF16) {
+    const int hd = c->n_heads * c->head_dim, nqkv = (c->n_heads + 2 * c->n_kv_heads) * c->head_dim;
+    if (c->d_model % 64 || hd % 64 || c->d_v % 64)
+      return why = "bf16: d_model, n_heads*head_dim and d_v must be multiples of 64", false;
+    if (!tc_pick_bn(nqkv, kEpiRope, c->head_dim) || !tc_pick_bn(2 * c->d_ff, kEpiSwiGLU, 0) ||
+        !tc_pick_bn(c->d_model, kEpiResid, 0) || !tc_pick_bn(c->d_k, kEpiStoreF32, 0))
+      return why = "bf16: projection widths do not fit the tensor-core tiles", false;
+  }
+  const double slot_bytes = double(2 * c->n_layers + 2) * (c->seg_len + c->n_mem) * c->d_model * 4.0;
+  if (slot_bytes > 64e9) return why = "model too large for one device", false;
+  return true;
+}
+
+rmt_status copy_in(void* dst, const void* src, size_t bytes, const char* what) {
+  if (!src) return fail(RMT_EINVAL, std::string("null weight pointer: ") + what);
+  RMT_CUDA(cudaMemcpy(dst, src, bytes, cudaMemcpyDefault));
+  return RMT_OK;
+}
+
+#define RMT_TRY(expr)            \
+  do {                           \
+    rmt_status s_ = (expr);      \
+    if (s_ != RMT_OK) return s_; \
+  } while (0)
+
+rmt_status pack_weights(rmt_handle* h, const rmt_weights* w) {
+  const rmt_cfg& c = h->cfg;
+  const size_t es = h->es, L = c.n_layers, d = c.d_model, hd = size_t(c.n_heads) * c.head_dim,
+               kvd = size_t(c.n_kv_heads) * c.head_dim, F = c.d_ff, dk = c.d_k, dv = c.d_v;
+  const void* const* arrays[] = {w->wq, w->wk, w->wv, w->wo, w->w_gate, w->w_up, w->w_down,
+                                 w->w_mq, w->w_mk, w->w_mv, w->w_mo, w->g_attn, w->g_mlp};
+  for (auto a : arrays)
+    if (!a) return fail(RMT_EINVAL, "null per-layer weight array");
+  auto at = [&](void* base, size_t elems_per_layer, size_t l, size_t off = 0) {
+    return static_cast<char*>(base) + (l * elems_per_layer + off) * es;
+  };
+  const size_t nqkv = size_t(h->Nqkv);
+  for (size_t l = 0; l < L; ++l) {
+    RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l), w->wq[l], hd * d * es, "wq"));
+    RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, hd * d), w->wk[l], kvd * d * es, "wk"));
+    RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, (hd + kvd) * d), w->wv[l], kvd * d * es, "wv"));
+    RMT_TRY(copy_in(at(h->w_o, d * hd, l), w->wo[l], d * hd * es, "wo"));
+    // gate/up interleaved in blocks of kSwiGLUBlock rows: [g0 u0 g1 u1 ...]
+    if (!w->w_gate[l] || !w->w_up[l]) return fail(RMT_EINVAL, "null w_gate/w_up");
+    const size_t blk = size_t(kSwiGLUBlock) * d * es;
+    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l), 2 * blk, w->w_gate[l], blk, blk, F / kSwiGLUBlock, cudaMemcpyDefault));
+    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l) + blk, 2 * blk, w->w_up[l], blk, blk, F / kSwiGLUBlock,
+                          cudaMemcpyDefault));
+    RMT_TRY(copy_in(at(h->w_d, d * F, l), w->w_down[l], d * F * es, "w_down"));
+    RMT_TRY(copy_in(at(h->w_mq, dk * d, l), w->w_mq[l], dk * d * es, "w_mq"));
+    RMT_TRY(copy_in(at(h->w_mo, d * dv, l), w->w_mo[l], d * dv * es, "w_mo"));
+    RMT_TRY(copy_in(at(h->w_mkv, (dk + dv) * d, l), w->w_mk[l], dk * d * es, "w_mk"));
+    RMT_TRY(copy_in(at(h->w_mkv, (dk + dv) * d, l, dk * d), w->w_mv[l], dv * d * es, "w_mv"));
+    RMT_TRY(copy_in(at(h->g1, d, l), w->g_attn[l], d * es, "g_attn"));
+    RMT_TRY(copy_in(at(h->g2, d, l), w->g_mlp[l], d * es, "g_mlp"));
+  }
+  RMT_TRY(copy_in(h->memtok, w->mem_tokens, size_t(c.n_mem) * d * es, "mem_tokens"));
+  return RMT_OK;
+}
+
+rmt_status build_maps(rmt_handle* h) {
+  const rmt_cfg& c = h->cfg;
+  const uint64_t L = c.n_layers, d = c.d_model, hd = uint64_t(c.n_heads) * c.head_dim, F = c.d_ff, M = h->M;
+  h->bn_mq = tc_pick_bn(c.d_k, kEpiStoreF32, 0);
+  h->bn_mo = tc_pick_bn(c.d_model, kEpiResid, 0);
+  h->bn_qkv = tc_pick_bn(h->Nqkv, kEpiRope, c.head_dim);
+  h->bn_o = tc_pick_bn(c.d_model, kEpiResid, 0);
+  h->bn_gu = tc_pick_bn(2 * c.d_ff, kEpiSwiGLU, 0);
+  h->bn_d = tc_pick_bn(c.d_model, kEpiResidCast, 0);
+  bool ok = make_tmap_bf16_3d(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) &&
+            make_tmap_bf16_3d(&h->tm_om, h->om, c.d_v, M, L, 128) &&
+            make_tmap_bf16_3d(&h->tm_h, h->hbuf, d, M, L, 128) &&
+            make_tmap_bf16_3d(&h->tm_att, h->att, hd, M, L, 128) &&
+            make_tmap_bf16_3d(&h->tm_u, h->u, F, M, L, 128) &&
+            make_tmap_bf16_3d(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) &&
+            make_tmap_bf16_3d(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->bn_mo) &&
+            make_tmap_bf16_3d(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) &&
+            make_tmap_bf16_3d(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
+            make_tmap_bf16_3d(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) &&
+            make_tmap_bf16_3d(&h->tm_wd, h->w_d, F, d, L, h->bn_d);
+  return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
+}
+
+enum Proj { kProjMemQ, kProjMemO, kProjQkv, kProjO, kProjGateUp, kProjDown };
+
+cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream_t st) {
+  const rmt_cfg& c = h->cfg;
+  const int d = c.d_model, hd = c.n_heads * c.head_dim;
+  EpiParams ep{};
+  ep.x = h->x;
+  ep.ldx = d;
+  ep.rope = h->rope;
+  ep.head_dim = c.head_dim;
+  ep.rope_cols = (c.n_heads + c.n_kv_heads) * c.head_dim;
+  ep.out_mode = ep.src_mode = ep.dst_mode = kByLayer;
+  int N = 0, K = 0;
+  EpiKind epi = kEpiStoreF32;
+  IndexMode amode = kByLayer;
+  const float* a32 = nullptr;
+  const void* w = nullptr;
+  const CUtensorMap *ta = nullptr, *tb = nullptr;
+  int bn = 0;
+  switch (p) {
+    case kProjMemQ:
+      N = c.d_k, K = d, epi = kEpiStoreF32, amode = kInSlot;
+      ep.out = h->qm, ep.ldo = c.d_k;
+      a32 = h->x, w = h->w_mq, ta = &h->tm_xb, tb = &h->tm_wmq, bn = h->bn_mq;
+      break;
+    case kProjMemO:
+      N = d, K = c.d_v, epi = kEpiResid;
+      ep.src_mode = kInSlot, ep.dst_mode = kOutSlot;
+      a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
+      break;
+    case kProjQkv:
+      N = h->Nqkv, K = d, epi = kEpiRope;
+      ep.out = h->qkv, ep.ldo = h->Nqkv;
+      a32 = static_cast<const float*>(h->hbuf), w = h->w_qkv, ta = &h->tm_h, tb = &h->tm_wqkv, bn = h->bn_qkv;
+      break;
+    case kProjO:
+      N = d, K = hd, epi = kEpiResid;
+      ep.src_mode = ep.dst_mode = kOutSlot;
+      a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
+      break;
+    case kProjGateUp:
+      N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU;
+      ep.out = h->u, ep.ldo = c.d_ff;
+      a32 = static_cast<const float*>(h->hbuf), w = h->w_gu, ta = &h->tm_h, tb = &h->tm_wgu, bn = h->bn_gu;
+      break;
+    case kProjDown:
+      N = d, K = c.d_ff, epi = h->bf16 ? kEpiResidCast : kEpiResid;
+      ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb;
+      a32 = static_cast<const float*>(h->u), w = h->w_d, ta = &h->tm_u, tb = &h->tm_wd, bn = h->bn_d;
+      break;
+  }
+  if (h->bf16) {
+    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
+    return launch_tc_gemm(*ta, *tb, a, bn, st);
+  }
+  SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, K, amode, static_cast<const float*>(w), epi, ep};
+  return launch_simt_gemm(a, st);
+}
+
+// Launch one kernel of a step: count it and, if its kind is probed, bracket it with events.
+template <typename F>
+cudaError_t launch_kind(rmt_handle* h, int kind, double flops, double bytes, cudaStream_t st, F&& fn) {
+  const bool on = (h->probe_mask >> kind) & 1u;
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (on && (a = h->probe_event()) != nullptr) cudaEventRecord(a, st);
+  const cudaError_t e = fn();
+  ++h->launches;
+  if (on && a && (b = h->probe_event()) != nullptr) {
+    cudaEventRecord(b, st);
+    h->probe_recs.push_back(rmt_handle::ProbeRec{kind, flops, bytes, a, b});
+  }
+  return e;
+}
+
+cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* emb, void* out, cudaStream_t st) {
+  const rmt_cfg& c = h->cfg;
+  const int L = c.n_layers, d = c.d_model, M = h->M, G = t.cnt[step], off = t.off[step];
+  const Cell* cells = t.dev + off;
+  const Cell first = t.cells[off], last = t.cells[off + G - 1];
+  const size_t slot_elems = size_t(M) * d;
+  // algorithmic work per launch (flops; bytes that must cross HBM at least once)
+  const double g = G, m = M, dd = d, es = h->es, dk = c.d_k, dv = c.d_v, hd = double(c.n_heads) * c.head_dim,
+               nq = h->Nqkv, F = c.d_ff, n = c.n_mem, ea = h->bf16 ? 2.0 : 4.0;
+  cudaError_t e;
+  if (first.l == 0) {
+    const int sl = in_slot(L, 0, first.s);
+    e = launch_kind(h, RMT_K_ASSEMBLE, 0, m * dd * (es + 4 + (h->bf16 ? 2 : 0)), st, [&] {
+      return launch_assemble(emb, h->memtok, h->x + sl * slot_elems, h->bf16 ? h->xb + sl * slot_elems : nullptr,
+                             c.seg_len, c.n_mem, d, first.s, h->bf16, st);
+    });
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_kind(h, RMT_K_MEMQ, 2 * g * m * dk * dd, g * (m * dd * ea + dk * dd * es + m * dk * 4), st,
+                  [&] { return run_proj(h, kProjMemQ, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk), g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es),
+                  st, [&] {
+                    MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
+                    return launch_mem_read(a, h->bf16, st);
+                  });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv, g * (m * dv * es + dd * dv * es + 2 * m * dd * 4), st,
+                  [&] { return run_proj(h, kProjMemO, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_RMSNORM1, 3 * g * m * dd, g * (m * dd * 4 + dd * es + m * dd * es), st, [&] {
+    RmsArgs a{h->x, h->g1, h->hbuf, M, d, c.rms_eps, G, cells, kOutSlot, kByLayer, L};
+    return launch_rmsnorm(a, h->bf16, st);
+  });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_QKV, 2 * g * m * nq * dd, g * (m * dd * es + nq * dd * es + m * nq * es), st,
+                  [&] { return run_proj(h, kProjQkv, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_ATTENTION, g * c.n_heads * 4.0 * c.head_dim * m * (m + 1) / 2,
+                  g * (m * nq * es + m * hd * es), st, [&] {
+                    AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L};
+                    return launch_attention(a, h->bf16, st);
+                  });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd, g * (m * hd * es + dd * hd * es + 2 * m * dd * 4), st,
+                  [&] { return run_proj(h, kProjO, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_RMSNORM2, 3 * g * m * dd, g * (m * dd * 4 + dd * es + m * dd * es), st, [&] {
+    RmsArgs a{h->x, h->g2, h->hbuf, M, d, c.rms_eps, G, cells, kOutSlot, kByLayer, L};
+    return launch_rmsnorm(a, h->bf16, st);
+  });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_GATEUP, 2 * g * m * 2 * F * dd, g * (m * dd * es + 2 * F * dd * es + m * F * es), st,
+                  [&] { return run_proj(h, kProjGateUp, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_DOWN, 2 * g * m * dd * F,
+                  g * (m * F * es + dd * F * es + 2 * m * dd * 4 + (h->bf16 ? m * dd * 2 : 0)), st,
+                  [&] { return run_proj(h, kProjDown, cells, G, st); });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_MEMKV, 2 * g * n * (dk + dv) * dd,
+                  g * (n * dd * 4 + (dk + dv) * dd * es + h->nsplit * n * (dk + dv) * 4), st, [&] {
+                    MemKvArgs a{h->x, M, d, c.seg_len, c.n_mem, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
+                    return launch_mem_kv(a, h->bf16, st);
+                  });
+  if (e != cudaSuccess) return e;
+  e = launch_kind(h, RMT_K_MEMUPDATE, g * 4 * n * dk * dv,
+                  g * (h->nsplit * n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), st, [&] {
+                    MemUpdateArgs a{h->part, h->nsplit, nullptr, nullptr, h->A, h->z, c.n_mem, c.d_k, c.d_v, c.mem_eps,
+                                    G, cells, kByLayer, kByLayer, L, h->trace, off, step};
+                    return launch_mem_update(a, st);
+                  });
+  if (e != cudaSuccess) return e;
+  if (last.l == L - 1) {
+    e = launch_kind(h, RMT_K_EMIT, 0, double(c.seg_len) * dd * (4 + es), st, [&] {
+      return launch_emit(h->x + out_slot(L, L - 1, last.s) * slot_elems, out, c.seg_len, d, last.s, h->bf16, st);
+    });
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (dev >= 0 && cudaGetDevice(&prev) == cudaSuccess && prev != dev)
+      cudaSetDevice(dev);
+    else
+      prev = -1;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* rmt_last_error(void) { return g_last_error.c_str(); }
+
+rmt_status rmt_schedule_table(int32_t n_layers, int32_t n_segments, rmt_schedule schedule, int32_t* out_dls,
+                              size_t cap) {
+  if (n_layers <= 0 || n_segments <= 0) return fail(RMT_EINVAL, "n_layers and n_segments must be positive");
+  if (schedule != RMT_DIAGONAL && schedule != RMT_SEQUENTIAL) return fail(RMT_EINVAL, "unknown schedule");
+  if (!out_dls) return fail(RMT_EINVAL, "out_dls is null");
+  const size_t need = 3 * size_t(n_layers) * size_t(n_segments);
+  if (cap < need) return fail(RMT_EINVAL, "out_dls capacity below 3*n_layers*n_segments");
+  Table t;
+  build_table(n_layers, n_segments, schedule, t);
+  size_t k = 0;
+  for (size_t step = 0; step < t.off.size(); ++step)
+    for (int i = 0; i < t.cnt[step]; ++i) {
+      const Cell c = t.cells[t.off[step] + i];
+      out_dls[k++] = int32_t(step);
+      out_dls[k++] = c.l;
+      out_dls[k++] = c.s;
+    }
+  return RMT_OK;
+}
+
+rmt_status rmt_get_schedule(const rmt_handle* h, int32_t n_segments, rmt_schedule schedule, int32_t* out_dls,
+                            size_t cap) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  return rmt_schedule_table(h->cfg.n_layers, n_segments, schedule, out_dls, cap);
+}
+
+rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle** out) {
+  if (!weights || !cfg || !out) return fail(RMT_EINVAL, "null argument to rmt_create");
+  std::string why;
+  if (!validate_cfg(cfg, why)) return fail(RMT_EINVAL, "invalid cfg: " + why);
+  rmt_handle* h = new rmt_handle();
+  h->cfg = *cfg;
+  auto bail = [&](rmt_status st) {
+    h->release();
+    delete h;
+    return st;
+  };
+  if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(RMT_ECUDA, "no CUDA device"));
+  const rmt_cfg& c = h->cfg;
+  h->bf16 = c.dtype == RMT_BF16;
+  h->es = h->bf16 ? 2 : 4;
+  h->M = c.seg_len + c.n_mem;
+  h->Nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  h->nsplit = (c.d_model + kMemKvSplit - 1) / kMemKvSplit;
+  const size_t L = c.n_layers, d = c.d_model, M = h->M, es = h->es, hd = size_t(c.n_heads) * c.head_dim,
+               F = c.d_ff, dk = c.d_k, dv = c.d_v;
+  struct {
+    void** p;
+    size_t bytes;
+  } plan[] = {
+      {&h->w_qkv, L * h->Nqkv * d * es}, {&h->w_o, L * d * hd * es},        {&h->w_gu, L * 2 * F * d * es},
+      {&h->w_d, L * d * F * es},         {&h->w_mq, L * dk * d * es},       {&h->w_mo, L * d * dv * es},
+      {&h->w_mkv, L * (dk + dv) * d * es}, {&h->g1, L * d * es},            {&h->g2, L * d * es},
+      {&h->memtok, size_t(c.n_mem) * d * es},
+      {reinterpret_cast<void**>(&h->x), n_slots(c.n_layers) * M * d * 4},
+      {&h->hbuf, L * M * d * es},        {&h->qkv, L * M * h->Nqkv * es},   {&h->att, L * M * hd * es},
+      {&h->u, L * M * F * es},           {&h->om, L * M * dv * es},
+      {reinterpret_cast<void**>(&h->qm), L * M * dk * 4},
+      {reinterpret_cast<void**>(&h->part), L * h->nsplit * size_t(c.n_mem) * (dk + dv) * 4},
+      {reinterpret_cast<void**>(&h->A), L * dk * dv * 4},
+      {reinterpret_cast<void**>(&h->z), L * dk * 4},
+      {reinterpret_cast<void**>(&h->rope), M * (c.head_dim / 2) * sizeof(float2)},
+      {reinterpret_cast<void**>(&h->err), sizeof(int)},
+  };
+  for (auto& e : plan) {
+    *e.p = h->alloc(e.bytes);
+    if (!*e.p) return bail(fail(RMT_ENOMEM, "device allocation failed"));
+  }
+  if (h->bf16) {
+    h->xb = static_cast<__nv_bfloat16*>(h->alloc(n_slots(c.n_layers) * M * d * 2));
+    if (!h->xb) return bail(fail(RMT_ENOMEM, "device allocation failed"));
+  }
+  rmt_status st = pack_weights(h, weights);
+  if (st != RMT_OK) return bail(st);
+  // RoPE table: angle p * theta^(-2i/dh) at segment-local position p, in double precision
+  {
+    const int half = c.head_dim / 2;
+    std::vector<float2> tab(M * half);
+    for (size_t p = 0; p < M; ++p)
+      for (int i = 0; i < half; ++i) {
+        const double ang = double(p) * std::pow(double(c.rope_theta), -2.0 * i / c.head_dim);
+        tab[p * half + i] = make_float2(float(std::cos(ang)), float(std::sin(ang)));
+      }
+    if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(fail(RMT_ECUDA, "rope table upload failed"));
+  }
+  if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(h->x, 0, n_slots(c.n_layers) * M * d * 4) != cudaSuccess)
+    return bail(fail(RMT_ECUDA, "cudaMemset failed"));
+  if (h->bf16) {
+    if ((st = build_maps(h)) != RMT_OK) return bail(st);
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return bail(fail(RMT_ECUDA, "weight packing failed"));
+  *out = h;
+  return RMT_OK;
+}
+
+rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, void* out_hidden,
+                       float* out_A, float* out_z, void* stream) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  if (!emb || !out_hidden) return fail(RMT_EINVAL, "emb and out_hidden must not be null");
+  if (n_segments <= 0) return fail(RMT_EINVAL, "n_segments must be positive");
+  if (schedule != RMT_DIAGONAL && schedule != RMT_SEQUENTIAL) return fail(RMT_EINVAL, "unknown schedule");
+  DeviceGuard guard(h->dev);
+  const rmt_cfg& c = h->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t io_bytes = size_t(n_segments) * c.seg_len * c.d_model * h->es;
+  const void* emb_dev = emb;
+  if (is_host_ptr(emb)) {
+    if (h->emb_stage_bytes < io_bytes) {
+      if (h->emb_stage) cudaFree(h->emb_stage);
+      h->emb_stage = nullptr;
+      h->emb_stage_bytes = 0;
+      if (cudaMalloc(&h->emb_stage, io_bytes) != cudaSuccess) return fail(RMT_ENOMEM, "staging allocation failed");
+      h->emb_stage_bytes = io_bytes;
+    }
+    RMT_CUDA(cudaMemcpyAsync(h->emb_stage, emb, io_bytes, cudaMemcpyHostToDevice, st));
+    emb_dev = h->emb_stage;
+  }
+  void* out_dev = out_hidden;
+  const bool out_host = is_host_ptr(out_hidden);
+  if (out_host) {
+    if (h->out_stage_bytes < io_bytes) {
+      if (h->out_stage) cudaFree(h->out_stage);
+      h->out_stage = nullptr;
+      h->out_stage_bytes = 0;
+      if (cudaMalloc(&h->out_stage, io_bytes) != cudaSuccess) return fail(RMT_ENOMEM, "staging allocation failed");
+      h->out_stage_bytes = io_bytes;
+    }
+    out_dev = h->out_stage;
+  }
+  const auto key = std::make_pair(int(n_segments), int(schedule));
+  auto it = h->tables.find(key);
+  if (it == h->tables.end()) {
+    Table t;
+    build_table(c.n_layers, n_segments, schedule, t);
+    if (cudaMalloc(&t.dev, sizeof(Cell) * t.cells.size()) != cudaSuccess)
+      return fail(RMT_ENOMEM, "cell table allocation failed");
+    if (cudaMemcpy(t.dev, t.cells.data(), sizeof(Cell) * t.cells.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(t.dev);
+      return fail(RMT_ECUDA, "cell table upload failed");
+    }
+    it = h->tables.emplace(key, std::move(t)).first;
+  }
+  const Table& t = it->second;
+  const size_t ncell = t.cells.size();
+  if (h->trace_cap < ncell) {
+    if (h->trace) cudaFree(h->trace);
+    h->trace = nullptr;
+    h->trace_cap = 0;
+    if (cudaMalloc(&h->trace, 3 * sizeof(int) * ncell) != cudaSuccess) return fail(RMT_ENOMEM, "trace allocation failed");
+    h->trace_cap = ncell;
+  }
+  const size_t L = c.n_layers;
+  RMT_CUDA(cudaMemsetAsync(h->A, 0, L * c.d_k * c.d_v * sizeof(float), st));
+  RMT_CUDA(cudaMemsetAsync(h->z, 0, L * c.d_k * sizeof(float), st));
+  for (int step = 0; step < int(t.off.size()); ++step) {
+    cudaError_t e = enqueue_step(h, t, step, emb_dev, out_dev, st);
+    if (e != cudaSuccess) return fail(RMT_ECUDA, std::string("launch failed: ") + cudaGetErrorString(e));
+  }
+  if (out_host) RMT_CUDA(cudaMemcpyAsync(out_hidden, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
+  if (out_A) RMT_CUDA(cudaMemcpyAsync(out_A, h->A, L * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
+  if (out_z) RMT_CUDA(cudaMemcpyAsync(out_z, h->z, L * c.d_k * sizeof(float), cudaMemcpyDefault, st));
+  h->traced_cells = int(ncell);
+  RMT_CUDA(cudaGetLastError());
+  return RMT_OK;
+}
+
+rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap) {
+  if (!h || !out_dls) return fail(RMT_EINVAL, "null argument");
+  if (h->traced_cells < 0) return fail(RMT_ESTATE, "no forward has run on this handle");
+  if (cap < 3 * size_t(h->traced_cells)) return fail(RMT_EINVAL, "out_dls capacity too small");
+  DeviceGuard guard(h->dev);
+  RMT_CUDA(cudaDeviceSynchronize());
+  RMT_CUDA(cudaMemcpy(out_dls, h->trace, 3 * sizeof(int) * h->traced_cells, cudaMemcpyDeviceToHost));
+  return RMT_OK;
+}
+
+rmt_status rmt_sync(rmt_handle* h, void* stream) {
+  int* err = nullptr;
+  if (h) {
+    err = h->err;
+  } else {
+    const Cell* cells = nullptr;
+    rmt_status s = device_scratch(1, &cells, &err);
+    if (s != RMT_OK) return s;
+  }
+  DeviceGuard guard(h ? h->dev : -1);
+  RMT_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(cudaGetLastError());
+  int word = 0;
+  RMT_CUDA(cudaMemcpy(&word, err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word) {
+    RMT_CUDA(cudaMemset(err, 0, sizeof(int)));
+    return fail(RMT_ETIMEOUT, "a bounded device wait gave up (error word " + std::to_string(word) + ")");
+  }
+  return RMT_OK;
+}
+
+rmt_status rmt_probe(rmt_handle* h, uint32_t mask) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  DeviceGuard guard(h->dev);
+  RMT_CUDA(cudaDeviceSynchronize());
+  h->probe_mask = mask;
+  h->probe_recs.clear();
+  h->probe_used = 0;
+  h->launches = 0;
+  return RMT_OK;
+}
+
+rmt_status rmt_probe_read(rmt_handle* h, rmt_kernel kind, double* ms, int64_t* launches, double* flops, double* bytes,
+                          int64_t* all_launches) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  if (int(kind) < 0 || int(kind) >= RMT_K_COUNT) return fail(RMT_EINVAL, "unknown kernel kind");
+  DeviceGuard guard(h->dev);
+  RMT_CUDA(cudaDeviceSynchronize());
+  double t = 0, f = 0, b = 0;
+  int64_t nl = 0;
+  for (const auto& r : h->probe_recs) {
+    if (r.kind != int(kind)) continue;
+    float e = 0.f;
+    RMT_CUDA(cudaEventElapsedTime(&e, r.a, r.b));
+    t += e;
+    f += r.flops;
+    b += r.bytes;
+    ++nl;
+  }
+  if (ms) *ms = t;
+  if (launches) *launches = nl;
+  if (flops) *flops = f;
+  if (bytes) *bytes = b;
+  if (all_launches) *all_launches = h->launches;
+  return RMT_OK;
+}
+
+rmt_status rmt_destroy(rmt_handle* h) {
+  if (!h) return RMT_OK;
+  {
+    DeviceGuard guard(h->dev);
+    cudaDeviceSynchronize();
+    h->release();
+  }
+  delete h;
+  return RMT_OK;
+}
+
+// ----------------------------------------------------------------- kernel-level entry points
+
+rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t G, int32_t M, int32_t N, int32_t K,
+                                 rmt_dtype out_dtype, void* stream) {
+  if (!A || !B || !C) return fail(RMT_EINVAL, "null pointer");
+  if (G <= 0 || M <= 0 || N <= 0 || K <= 0) return fail(RMT_EINVAL, "sizes must be positive");
+  if (K % 64 || N % 64) return fail(RMT_EINVAL, "K and N must be multiples of 64");
+  if (out_dtype != RMT_F32 && out_dtype != RMT_BF16) return fail(RMT_EINVAL, "bad out_dtype");
+  const Cell* cells = nullptr;
+  int* err = nullptr;
+  RMT_TRY(device_scratch(G, &cells, &err));
+  CUtensorMap ta, tb;
+  const int epi = out_dtype == RMT_F32 ? kEpiStoreF32 : kEpiStoreAct;
+  const int bn = tc_pick_bn(N, epi, 0);
+  if (!make_tmap_bf16_3d(&ta, A, K, M, G, 128) || !make_tmap_bf16_3d(&tb, B, K, N, G, bn))
+    return fail(RMT_EINVAL, "tensor map encoding failed (pointers must be 16-byte aligned)");
+  EpiParams ep{};
+  ep.out = C;
+  ep.ldo = N;
+  ep.out_mode = kByLayer;
+  TcGemmArgs a{M, N, K, G, cells, G, kByLayer, static_cast<EpiKind>(epi), ep, err};
+  RMT_CUDA(launch_tc_gemm(ta, tb, a, bn, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32_t H, int32_t Hkv, int32_t dh,
+                         rmt_dtype dtype, void* stream) {
+  if (!qkv || !out) return fail(RMT_EINVAL, "null pointer");
+  if (G <= 0 || M <= 0 || H <= 0 || Hkv <= 0 || H % Hkv) return fail(RMT_EINVAL, "bad sizes");
+  if (dh != 32 && dh != 64 && dh != 128) return fail(RMT_EINVAL, "dh must be 32, 64 or 128");
+  if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(G, &cells, nullptr));
+  AttnArgs a{qkv, out, M, H, Hkv, dh, G, cells, kByLayer, G};
+  RMT_CUDA(launch_attention(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void* o, int32_t G, int32_t M, int32_t dk,
+                           int32_t dv, float eps, rmt_dtype dtype, void* stream) {
+  if (!q || !A || !z || !o) return fail(RMT_EINVAL, "null pointer");
+  if (G <= 0 || M <= 0 || dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128)
+    return fail(RMT_EINVAL, "bad sizes");
+  if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(G, &cells, nullptr));
+  MemReadArgs a{q, A, z, o, M, dk, dv, eps, G, cells, kByLayer, kByLayer, G};
+  RMT_CUDA(launch_mem_read(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n, int32_t dk,
+                             int32_t dv, float eps, void* stream) {
+  if (!k || !v || !A || !z) return fail(RMT_EINVAL, "null pointer");
+  if (G <= 0 || n <= 0 || n > 64 || dk % 32 || dv % 32 || dk <= 0 || dv <= 0 || dk > 128 || dv > 128)
+    return fail(RMT_EINVAL, "bad sizes");
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(G, &cells, nullptr));
+  MemUpdateArgs a{nullptr, 0, k, v, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0};
+  RMT_CUDA(launch_mem_update(a, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int32_t d, float eps, rmt_dtype dtype,
+                       void* stream) {
+  if (!x || !g || !y) return fail(RMT_EINVAL, "null pointer");
+  if (rows <= 0 || d <= 0 || d % 4) return fail(RMT_EINVAL, "bad sizes");
+  if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(1, &cells, nullptr));
+  RmsArgs a{x, g, y, rows, d, eps, 1, cells, kByLayer, kByLayer, 1};
+  RMT_CUDA(launch_rmsnorm(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+}  // extern "C"

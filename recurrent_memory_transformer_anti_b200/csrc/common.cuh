@@ -1,0 +1,82 @@
+// Shared device-side definitions: cell tables, activation-slot addressing, epilogue kinds.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rmt {
+
+// Device error word values (OR-ed together; read and cleared by rmt_sync).
+enum : int {
+  kErrTimeoutProducer = 1,
+  kErrTimeoutMma = 2,
+  kErrTimeoutEpilogue = 4,
+  kErrBadArgs = 8,
+};
+
+// One (layer, segment) cell of the grid.
+struct Cell {
+  int l, s;
+};
+
+// Activation slots. The residual stream of cell (l, s) lives in a [M, d] fp32 slot:
+//   output slot  : ((l + s) % 2) * L + l            (written by cell (l, s))
+//   input slot   : output slot of (l-1, s), or 2L + s % 2 for layer 0 (embeddings + memory)
+// Cell (l, s) runs on diagonal l + s; its input was written on diagonal l + s - 1 and is
+// next overwritten on diagonal l + s + 1, so two parities suffice for both schedules.
+__host__ __device__ inline int out_slot(int L, int l, int s) { return ((l + s) & 1) * L + l; }
+__host__ __device__ inline int in_slot(int L, int l, int s) {
+  return l == 0 ? 2 * L + (s & 1) : ((l + s - 1) & 1) * L + (l - 1);
+}
+constexpr int n_slots(int L) { return 2 * L + 2; }
+
+// How a kernel turns a cell into an index of a stacked [*, M, cols] buffer.
+enum IndexMode : int { kByLayer = 0, kInSlot = 1, kOutSlot = 2 };
+
+__device__ __forceinline__ int cell_index(IndexMode mode, int L, Cell c) {
+  return mode == kByLayer ? c.l : (mode == kInSlot ? in_slot(L, c.l, c.s) : out_slot(L, c.l, c.s));
+}
+
+// GEMM epilogues shared by the tensor-core and the fp32 kernels.
+enum EpiKind : int {
+  kEpiStoreF32 = 0,   // out(f32) = acc
+  kEpiStoreAct = 1,   // out(T) = acc
+  kEpiResid = 2,      // x(f32)[dst] = x(f32)[src] + acc
+  kEpiResidCast = 3,  // as kEpiResid, and also xb(bf16)[dst] = bf16(result)
+  kEpiRope = 4,       // out(T) = RoPE(acc) for columns < rope_cols, acc elsewhere
+  kEpiSwiGLU = 5,     // out(T)[:, j] = silu(gate_j) * up_j, gate/up interleaved in blocks of 64
+};
+
+constexpr int kSwiGLUBlock = 64;
+
+struct EpiParams {
+  void* out;             // kEpiStore*, kEpiRope, kEpiSwiGLU output (stacked [*, M, ldo])
+  int ldo;               // output row stride (elements)
+  IndexMode out_mode;
+  float* x;              // residual stream base ([n_slots, M, ldx] fp32)
+  int ldx;
+  IndexMode src_mode, dst_mode;
+  __nv_bfloat16* xb;     // bf16 copy of the residual stream ([n_slots, M, ldx]) or null
+  const float2* rope;    // [M, head_dim/2] (cos, sin)
+  int rope_cols;         // columns (q and k heads) that get RoPE
+  int head_dim;
+};
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// phi(x) = elu(x) + 1
+__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// silu(x) = x * sigmoid(x)
+__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+
+}  // namespace rmt

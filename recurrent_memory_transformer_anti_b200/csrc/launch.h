@@ -1,0 +1,134 @@
+// Internal launcher interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace rmt {
+
+// ------------------------------------------------------------------ grouped GEMMs
+// Group g computes rows 0..M-1 of cell cells[g]: Y = X . W^T with
+//   X = slice cell_index(a_mode, cells[g]) of a [*, M, K] stack,
+//   W = slice cells[g].l of a [L, N, K] stack.
+struct TcGemmArgs {
+  int M, N, K;
+  int G;
+  const Cell* cells;  // device array of G cells
+  int L;
+  IndexMode a_mode;
+  EpiKind epi;
+  EpiParams ep;
+  int* err;  // device error word (may be null)
+};
+
+// tensor-core path (bf16 operands in TMA tensor maps)
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                       uint32_t box_rows);
+int tc_pick_bn(int N, int epi, int head_dim);  // 0 if no tile width fits
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn,
+                           cudaStream_t st);
+
+// fp32 FMA path (fp32 operands by pointer)
+struct SimtGemmArgs {
+  int M, N, K;
+  int G;
+  const Cell* cells;
+  int L;
+  const float* a;  // [*, M, lda]
+  int lda;
+  IndexMode a_mode;
+  const float* w;  // [L, N, K]
+  EpiKind epi;
+  EpiParams ep;
+};
+cudaError_t launch_simt_gemm(const SimtGemmArgs& args, cudaStream_t st);
+
+// ------------------------------------------------------------------ attention
+// qkv: [*, M, (H + 2 Hkv) dh] slice by layer; out: [*, M, H dh] slice by layer.
+struct AttnArgs {
+  const void* qkv;
+  void* out;
+  int M, H, Hkv, dh;
+  int G;
+  const Cell* cells;
+  IndexMode mode;  // slice index of both buffers
+  int L;
+};
+cudaError_t launch_attention(const AttnArgs& a, bool bf16, cudaStream_t st);
+
+// ------------------------------------------------------------------ associative memory
+struct MemReadArgs {
+  const float* q;  // [*, M, dk] raw (before phi)
+  const float* A;  // [*, dk, dv]
+  const float* z;  // [*, dk]
+  void* o;         // [*, M, dv]
+  int M, dk, dv;
+  float eps;
+  int G;
+  const Cell* cells;
+  IndexMode mode;        // slice of q and o
+  IndexMode state_mode;  // slice of A and z
+  int L;
+};
+cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st);
+
+// Partial products of the memory-token rows with [W_mk; W_mv], split along d_model so the
+// reduction order is fixed: part[l][split][r][j] = sum_{k in split} Y[r][k] W_mkv[l][j][k],
+// Y = rows row0 .. row0+n-1 of the cell's output slot.
+constexpr int kMemKvSplit = 64;  // d_model columns per split
+struct MemKvArgs {
+  const float* x;  // residual stream [n_slots, M, d]
+  int M, d, row0, n;
+  const void* w;   // [L, dkv, d] in T
+  float* part;     // [L, nsplit, n, dkv] fp32
+  int dkv;
+  int G;
+  const Cell* cells;
+  int L;
+};
+cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st);
+
+// Delta-rule update of A, z from raw keys/values of n rows. Keys/values come either from
+// the split partials above (part != null: k = columns 0..dk-1, v = columns dk..dk+dv-1 of
+// the reduced rows) or from plain arrays k [*, n, dk], v [*, n, dv].
+struct MemUpdateArgs {
+  const float* part;  // [*, nsplit, n, dk + dv] or null
+  int nsplit;
+  const float* k;     // [*, n, dk] (when part == null)
+  const float* v;     // [*, n, dv]
+  float* A;           // [*, dk, dv]
+  float* z;           // [*, dk]
+  int n, dk, dv;
+  float eps;
+  int G;
+  const Cell* cells;
+  IndexMode kv_mode, state_mode;
+  int L;
+  int* trace;         // optional: trace[3*(trace_base+g) + {0,1,2}] = (step, l, s)
+  int trace_base, step;
+};
+cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------------------ row kernels
+struct RmsArgs {
+  const float* x;  // [*, M, d] fp32
+  const void* g;   // [L, d] in T
+  void* y;         // [*, M, d] in T
+  int M, d;
+  float eps;
+  int G;
+  const Cell* cells;
+  IndexMode x_mode, y_mode;
+  int L;
+};
+cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st);
+
+// Layer-0 input of segment s: rows 0..seg-1 from emb, rows seg..M-1 from the memory tokens.
+cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __nv_bfloat16* xb_slot, int seg, int n_mem,
+                            int d, int s, bool bf16, cudaStream_t st);
+// Segment output: rows 0..seg-1 of an fp32 slot, cast to T, to out + s*seg*d.
+cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, bool bf16, cudaStream_t st);
+
+}  // namespace rmt

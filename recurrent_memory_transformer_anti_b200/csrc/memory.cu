@@ -1,0 +1,258 @@
+// Associative memory of an ARMT layer (the model the diagonal-batching paper accelerates;
+// arXiv 2506.05229 applies it to a LLaMA-1B ARMT). The pages cite ARMT by name only; the
+// kernels implement phi(x) = elu(x) + 1 and
+//   read   : o = phi(q) A / (phi(q) . z + eps)                     per row
+//   update : v_bar = phi(K) A / (phi(K) . z + eps)
+//            A += phi(K)^T (V - v_bar),  z += sum over rows of phi(K)   (pre-update A, z)
+// with A (d_k x d_v) and z (d_k) in fp32. Every reduction runs in a fixed order, so a cell
+// gives the same bits whichever other cells share its launch.
+#include "common.cuh"
+#include "launch.h"
+
+namespace rmt {
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ----------------------------------------------------------------------------- read
+// CTA = 128 rows of one cell, 8 warps x 16 rows, 4 rows in flight per warp. A and z sit in
+// shared memory; lane j owns output columns j, j+32, ...; q_i reaches all lanes by shuffle.
+constexpr int kReadRows = 128, kReadWarps = 8, kReadBatch = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemReadArgs a) {
+  extern __shared__ float sm[];
+  const int dk = a.dk, dv = a.dv, nk = dk >> 5, nv = dv >> 5;
+  float* As = sm;            // [dk][dv]
+  float* zs = sm + dk * dv;  // [dk]
+  const Cell c = a.cells[blockIdx.y];
+  const size_t si = cell_index(a.state_mode, a.L, c), qi = cell_index(a.mode, a.L, c);
+  const float4* A4 = reinterpret_cast<const float4*>(a.A + si * dk * dv);
+  for (int i = threadIdx.x; i < (dk * dv) >> 2; i += blockDim.x) reinterpret_cast<float4*>(As)[i] = A4[i];
+  for (int i = threadIdx.x; i < dk; i += blockDim.x) zs[i] = a.z[si * dk + i];
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* q = a.q + qi * a.M * dk;
+  T* o = static_cast<T*>(a.o) + qi * a.M * dv;
+  const int r_begin = blockIdx.x * kReadRows + warp * (kReadRows / kReadWarps);
+  const int r_end = min(r_begin + kReadRows / kReadWarps, a.M);
+  for (int r0 = r_begin; r0 < r_end; r0 += kReadBatch) {
+    float fq[kReadBatch][4], acc[kReadBatch][4], den[kReadBatch];
+#pragma unroll
+    for (int b = 0; b < kReadBatch; ++b) {
+      const int row = r0 + b;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        fq[b][u] = (u < nk && row < r_end) ? phi_f(q[static_cast<size_t>(row) * dk + 32 * u + lane]) : 0.f;
+        acc[b][u] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kReadBatch; ++b) {
+      float d = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (u < nk) d = fmaf(fq[b][u], zs[32 * u + lane], d);
+      den[b] = warp_sum(d) + a.eps;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u >= nk) break;
+      for (int j = 0; j < 32; ++j) {
+        const float* Ai = As + (32 * u + j) * dv;
+        float qb[kReadBatch];
+#pragma unroll
+        for (int b = 0; b < kReadBatch; ++b) qb[b] = __shfl_sync(0xffffffffu, fq[b][u], j);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          if (v < nv) {
+            const float av = Ai[32 * v + lane];
+#pragma unroll
+            for (int b = 0; b < kReadBatch; ++b) acc[b][v] = fmaf(qb[b], av, acc[b][v]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kReadBatch; ++b) {
+      const int row = r0 + b;
+      if (row >= r_end) break;
+      const float inv = 1.f / den[b];
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        if (v < nv) o[static_cast<size_t>(row) * dv + 32 * v + lane] = from_f32<T>(acc[b][v] * inv);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ key/value projection
+// CTA = one split of kMemKvSplit columns of d_model for one cell: the n memory rows and the
+// dkv weight rows of that split are staged in shared memory, then each thread forms up to
+// 16 of the n x dkv partial dot products.
+constexpr int kKvThreads = 256, kKvMaxOut = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
+  extern __shared__ float sm[];
+  constexpr int KS = kMemKvSplit;
+  float* Ys = sm;                // [n][KS]
+  float* Ws = sm + a.n * KS;     // [KS][dkv + 1]
+  const int ldw = a.dkv + 1;
+  const Cell c = a.cells[blockIdx.y];
+  const int split = blockIdx.x, k0 = split * KS;
+  const int kw = min(KS, a.d - k0);
+  const float* Y = a.x + (static_cast<size_t>(out_slot(a.L, c.l, c.s)) * a.M + a.row0) * a.d + k0;
+  const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
+  for (int e = threadIdx.x; e < a.n * KS; e += kKvThreads) {
+    const int r = e / KS, k = e % KS;
+    Ys[e] = k < kw ? Y[static_cast<size_t>(r) * a.d + k] : 0.f;
+  }
+  for (int e = threadIdx.x; e < a.dkv * KS; e += kKvThreads) {
+    const int j = e / KS, k = e % KS;
+    Ws[k * ldw + j] = k < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k]) : 0.f;
+  }
+  __syncthreads();
+  const int nout = a.n * a.dkv;
+  float acc[kKvMaxOut];
+#pragma unroll
+  for (int i = 0; i < kKvMaxOut; ++i) acc[i] = 0.f;
+  for (int k = 0; k < KS; ++k) {
+#pragma unroll
+    for (int i = 0; i < kKvMaxOut; ++i) {
+      const int e = threadIdx.x + i * kKvThreads;
+      if (e < nout) {
+        const int r = e / a.dkv, j = e % a.dkv;
+        acc[i] = fmaf(Ys[r * KS + k], Ws[k * ldw + j], acc[i]);
+      }
+    }
+  }
+  const int nsplit = (a.d + KS - 1) / KS;
+  float* part = a.part + (static_cast<size_t>(c.l) * nsplit + split) * nout;
+#pragma unroll
+  for (int i = 0; i < kKvMaxOut; ++i) {
+    const int e = threadIdx.x + i * kKvThreads;
+    if (e < nout) part[e] = acc[i];
+  }
+}
+
+// --------------------------------------------------------------------------- update
+// CTA = one cell. Shared memory: raw k|v rows, phi(k), A, z, row denominators, V - v_bar.
+constexpr int kUpdThreads = 256;
+
+__global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdateArgs a) {
+  extern __shared__ float sm[];
+  const int n = a.n, dk = a.dk, dv = a.dv, dkv = dk + dv;
+  float* KV = sm;              // [n][dkv]: phi(k) in columns < dk, v after
+  float* As = KV + n * dkv;    // [dk][dv]
+  float* zs = As + dk * dv;    // [dk]
+  float* den = zs + dk;        // [n]
+  float* D = den + n;          // [n][dv]
+  const Cell c = a.cells[blockIdx.x];
+  const size_t ki = cell_index(a.kv_mode, a.L, c), si = cell_index(a.state_mode, a.L, c);
+  float* A = a.A + si * dk * dv;
+  float* z = a.z + si * dk;
+
+  for (int e = threadIdx.x; e < n * dkv; e += kUpdThreads) {
+    const int r = e / dkv, j = e % dkv;
+    float val;
+    if (a.part) {
+      const float* p = a.part + ki * a.nsplit * n * dkv + e;
+      val = 0.f;
+      for (int sp = 0; sp < a.nsplit; ++sp) val += p[static_cast<size_t>(sp) * n * dkv];
+    } else {
+      val = j < dk ? a.k[(ki * n + r) * dk + j] : a.v[(ki * n + r) * dv + (j - dk)];
+    }
+    KV[e] = j < dk ? phi_f(val) : val;
+  }
+  for (int e = threadIdx.x; e < dk * dv; e += kUpdThreads) As[e] = A[e];
+  for (int e = threadIdx.x; e < dk; e += kUpdThreads) zs[e] = z[e];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < n; r += kUpdThreads / 32) {
+    float d = 0.f;
+    for (int i = lane; i < dk; i += 32) d = fmaf(KV[r * dkv + i], zs[i], d);
+    d = warp_sum(d);
+    if (lane == 0) den[r] = d + a.eps;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * dv; e += kUpdThreads) {
+    const int r = e / dv, j = e % dv;
+    float num = 0.f;
+    for (int i = 0; i < dk; ++i) num = fmaf(KV[r * dkv + i], As[i * dv + j], num);
+    D[e] = KV[r * dkv + dk + j] - num / den[r];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < dk * dv; e += kUpdThreads) {
+    const int i = e / dv, j = e % dv;
+    float s = 0.f;
+    for (int r = 0; r < n; ++r) s = fmaf(KV[r * dkv + i], D[r * dv + j], s);
+    A[e] = As[e] + s;
+  }
+  for (int i = threadIdx.x; i < dk; i += kUpdThreads) {
+    float s = 0.f;
+    for (int r = 0; r < n; ++r) s += KV[r * dkv + i];
+    z[i] = zs[i] + s;
+  }
+  if (a.trace && threadIdx.x == 0) {
+    int* t = a.trace + 3 * (a.trace_base + blockIdx.x);
+    t[0] = a.step;
+    t[1] = c.l;
+    t[2] = c.s;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st) {
+  if (a.G <= 0 || a.M <= 0) return cudaSuccess;
+  if (a.dk % 32 || a.dv % 32 || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
+  const size_t smem = (static_cast<size_t>(a.dk) * a.dv + a.dk) * sizeof(float);
+  dim3 grid((a.M + kReadRows - 1) / kReadRows, a.G);
+  if (bf16) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(mem_read_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mem_read_kernel<__nv_bfloat16><<<grid, kReadWarps * 32, smem, st>>>(a);
+  } else {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(mem_read_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mem_read_kernel<float><<<grid, kReadWarps * 32, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
+  if (a.G <= 0) return cudaSuccess;
+  if (a.n * a.dkv > kKvThreads * kKvMaxOut) return cudaErrorInvalidValue;
+  const size_t smem = (static_cast<size_t>(a.n) * kMemKvSplit + static_cast<size_t>(kMemKvSplit) * (a.dkv + 1)) *
+                      sizeof(float);
+  dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G);
+  if (bf16) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(mem_kv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mem_kv_kernel<__nv_bfloat16><<<grid, kKvThreads, smem, st>>>(a);
+  } else {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(mem_kv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    mem_kv_kernel<float><<<grid, kKvThreads, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st) {
+  if (a.G <= 0) return cudaSuccess;
+  const size_t smem = (static_cast<size_t>(a.n) * (a.dk + a.dv) + static_cast<size_t>(a.dk) * a.dv + a.dk + a.n +
+                       static_cast<size_t>(a.n) * a.dv) *
+                      sizeof(float);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(mem_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  mem_update_kernel<<<a.G, kUpdThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace rmt

@@ -1,0 +1,116 @@
+// Row-streaming kernels (HBM-bound): RMSNorm, layer-0 input assembly, segment output.
+#include "common.cuh"
+#include "launch.h"
+
+namespace rmt {
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ void store(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+  static __device__ __forceinline__ float4 load(const float* p) { return *reinterpret_cast<const float4*>(p); }
+};
+template <> struct Vec4<__nv_bfloat16> {
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+  static __device__ __forceinline__ float4 load(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+  }
+};
+
+// RMSNorm: one warp per row, y = x * rsqrt(mean(x^2) + eps) * g, statistics in fp32.
+constexpr int kRmsWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a) {
+  const Cell c = a.cells[blockIdx.y];
+  const int row = blockIdx.x * kRmsWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= a.M) return;
+  const float* x = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row) * a.d;
+  T* y = static_cast<T*>(a.y) + (static_cast<size_t>(cell_index(a.y_mode, a.L, c)) * a.M + row) * a.d;
+  const T* g = static_cast<const T*>(a.g) + static_cast<size_t>(c.l) * a.d;
+  float ss = 0.f;
+  for (int k = lane * 4; k < a.d; k += 128) {
+    const float4 v = Vec4<float>::load(x + k);
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / static_cast<float>(a.d) + a.eps);
+  for (int k = lane * 4; k < a.d; k += 128) {
+    const float4 v = Vec4<float>::load(x + k);
+    const float4 gv = Vec4<T>::load(g + k);
+    Vec4<T>::store(y + k, make_float4(v.x * r * gv.x, v.y * r * gv.y, v.z * r * gv.z, v.w * r * gv.w));
+  }
+}
+
+// Layer-0 input of segment s: embeddings of the segment, then the memory tokens.
+template <typename T>
+__global__ void assemble_kernel(const T* emb, const T* mem, float* x, __nv_bfloat16* xb, int seg, int d, int s) {
+  const int r = blockIdx.x;
+  const T* src = r < seg ? emb + (static_cast<size_t>(s) * seg + r) * d : mem + static_cast<size_t>(r - seg) * d;
+  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
+    const float4 v = Vec4<T>::load(src + k);
+    Vec4<float>::store(x + static_cast<size_t>(r) * d + k, v);
+    if (xb) Vec4<__nv_bfloat16>::store(xb + static_cast<size_t>(r) * d + k, v);
+  }
+}
+
+template <typename T>
+__global__ void emit_kernel(const float* x, T* out, int seg, int d, int s) {
+  const int r = blockIdx.x;
+  T* dst = out + (static_cast<size_t>(s) * seg + r) * d;
+  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(x + static_cast<size_t>(r) * d + k));
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
+  if (a.G <= 0 || a.M <= 0) return cudaSuccess;
+  if (a.d % 4) return cudaErrorInvalidValue;
+  dim3 grid((a.M + kRmsWarps - 1) / kRmsWarps, a.G);
+  if (bf16)
+    rmsnorm_kernel<__nv_bfloat16><<<grid, kRmsWarps * 32, 0, st>>>(a);
+  else
+    rmsnorm_kernel<float><<<grid, kRmsWarps * 32, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __nv_bfloat16* xb_slot, int seg, int n_mem,
+                            int d, int s, bool bf16, cudaStream_t st) {
+  if (d % 4) return cudaErrorInvalidValue;
+  const int threads = d >= 1024 ? 256 : 128;
+  if (bf16)
+    assemble_kernel<__nv_bfloat16><<<seg + n_mem, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(emb),
+                                                                     static_cast<const __nv_bfloat16*>(mem), x_slot,
+                                                                     xb_slot, seg, d, s);
+  else
+    assemble_kernel<float><<<seg + n_mem, threads, 0, st>>>(static_cast<const float*>(emb),
+                                                            static_cast<const float*>(mem), x_slot, xb_slot, seg, d, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, bool bf16, cudaStream_t st) {
+  if (d % 4) return cudaErrorInvalidValue;
+  const int threads = d >= 1024 ? 256 : 128;
+  if (bf16)
+    emit_kernel<__nv_bfloat16><<<seg, threads, 0, st>>>(x_slot, static_cast<__nv_bfloat16*>(out), seg, d, s);
+  else
+    emit_kernel<float><<<seg, threads, 0, st>>>(x_slot, static_cast<float*>(out), seg, d, s);
+  return cudaGetLastError();
+}
+
+}  // namespace rmt

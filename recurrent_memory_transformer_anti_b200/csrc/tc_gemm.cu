@@ -1,0 +1,442 @@
+// Grouped GEMM on 5th-generation tensor cores (sm_100a): Y_g = epi(X_g . W_l(g)^T).
+//
+// "Architecture Overview" of the diagonal-batching skill page: GroupedGEMM operations
+// batch the matrix products of all layers on one diagonal into a single launch, each
+// group with its own layer's weights. Here a group is one (layer, segment) cell; its
+// weight is slice l of a [L, N, K] stack, addressed through the third coordinate of one
+// TMA tensor map (no per-group pointer copies).
+//
+// Design (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0      one thread issues TMA loads of A (128 x 64) and B (BN x 64) bf16 tiles,
+//               128-byte swizzled, into a STAGES-deep shared-memory ring;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into
+//               one of two TMEM accumulators and commits to mbarriers;
+//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (one row per thread),
+//               fused RoPE / SwiGLU / residual add / cast, stores to global memory.
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
+// Every wait is bounded (see sm100.cuh); on a timeout the CTA drains its in-flight copies
+// and MMAs, frees TMEM, records the failure in the error word and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace rmt {
+
+template <int BN>
+struct TcCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+namespace {
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Store 32 consecutive fp32 values as bf16 (64 bytes, four 16-byte stores).
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  }
+}
+
+__device__ __forceinline__ void store32_f32(float* dst, const float* v) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// Plain / residual epilogue of one 32-column chunk of one row.
+template <int EPI>
+__device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]);
+  const EpiParams& ep = a.ep;
+  if constexpr (EPI == kEpiStoreF32) {
+    const size_t idx = cell_index(ep.out_mode, a.L, c);
+    store32_f32(static_cast<float*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
+  } else if constexpr (EPI == kEpiStoreAct) {
+    const size_t idx = cell_index(ep.out_mode, a.L, c);
+    store32_bf16(static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
+  } else if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+    const size_t si = cell_index(ep.src_mode, a.L, c), di = cell_index(ep.dst_mode, a.L, c);
+    const float4* src = reinterpret_cast<const float4*>(ep.x + (si * a.M + row) * ep.ldx + col);
+    float* dst = ep.x + (di * a.M + row) * ep.ldx + col;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 s = src[q];
+      v[4 * q] += s.x;
+      v[4 * q + 1] += s.y;
+      v[4 * q + 2] += s.z;
+      v[4 * q + 3] += s.w;
+    }
+    store32_f32(dst, v);
+    if constexpr (EPI == kEpiResidCast) store32_bf16(ep.xb + (di * a.M + row) * ep.ldx + col, v);
+  }
+}
+
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0) {
+  const bool valid = row < a.M;
+  const EpiParams& ep = a.ep;
+  if constexpr (EPI == kEpiRope) {
+    const int dh = ep.head_dim, half = dh >> 1;
+    const size_t idx = cell_index(ep.out_mode, a.L, c);
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
+    for (int h0 = 0; h0 < BN; h0 += dh) {
+      const bool rot = (n0 + h0) < ep.rope_cols;
+      if (half >= 32) {
+        for (int p = 0; p < half; p += 32) {
+          uint32_t lo[32], hi[32];
+          sm100::tmem_ld32(tacc + h0 + p, lo);
+          sm100::tmem_ld32(tacc + h0 + half + p, hi);
+          sm100::tmem_wait_ld();
+          if (valid) {
+            float x1[32], x2[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float a1 = u2f(lo[j]), a2 = u2f(hi[j]);
+              if (rot) {
+                const float2 cs = ep.rope[(size_t)row * half + p + j];
+                x1[j] = a1 * cs.x - a2 * cs.y;
+                x2[j] = a2 * cs.x + a1 * cs.y;
+              } else {
+                x1[j] = a1;
+                x2[j] = a2;
+              }
+            }
+            store32_bf16(orow + n0 + h0 + p, x1);
+            store32_bf16(orow + n0 + h0 + half + p, x2);
+          }
+        }
+      } else {  // head_dim 32: both halves of the head in one 32-column chunk
+        uint32_t r[32];
+        sm100::tmem_ld32(tacc + h0, r);
+        sm100::tmem_wait_ld();
+        if (valid) {
+          float x[32];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a1 = u2f(r[j]), a2 = u2f(r[j + 16]);
+            if (rot) {
+              const float2 cs = ep.rope[(size_t)row * 16 + j];
+              x[j] = a1 * cs.x - a2 * cs.y;
+              x[j + 16] = a2 * cs.x + a1 * cs.y;
+            } else {
+              x[j] = a1;
+              x[j + 16] = a2;
+            }
+          }
+          store32_bf16(orow + n0 + h0, x);
+        }
+      }
+    }
+  } else if constexpr (EPI == kEpiSwiGLU) {
+    const size_t idx = cell_index(ep.out_mode, a.L, c);
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
+#pragma unroll 1
+    for (int b0 = 0; b0 < BN; b0 += 2 * kSwiGLUBlock) {
+#pragma unroll 1
+      for (int p = 0; p < kSwiGLUBlock; p += 32) {
+        uint32_t g[32], u[32];
+        sm100::tmem_ld32(tacc + b0 + p, g);
+        sm100::tmem_ld32(tacc + b0 + kSwiGLUBlock + p, u);
+        sm100::tmem_wait_ld();
+        if (valid) {
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j])) * u2f(u[j]);
+          store32_bf16(orow + (n0 + b0) / 2 + p, y);
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      uint32_t r[32];
+      sm100::tmem_ld32(tacc + cc, r);
+      sm100::tmem_wait_ld();
+      if (valid) epi_chunk<EPI>(a, c, row, n0 + cc, r);
+    }
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcGemmArgs args) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = sm100::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES + 8 * (2 * C::STAGES + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      sm100::mbar_init(full_bar(s), 1);
+      sm100::mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(tfull_bar(a), 1);
+      sm100::mbar_init(tempty_bar(a), 4);
+    }
+    sm100::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+    sm100::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tmA);
+    sm100::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), C::TMEM_COLS);
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int mt = (args.M + C::BM - 1) / C::BM;
+  const int nt = args.N / BN;
+  const int kbn = args.K / C::BK;
+  const int tiles = args.G * mt * nt;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int g = t / (mt * nt), r = t % (mt * nt);
+        const int n_tile = r / mt, m_tile = r % mt;
+        const Cell c = args.cells[g];
+        const int a3 = cell_index(args.a_mode, args.L, c);
+        for (int kb = 0; kb < kbn; ++kb) {
+          if (!sm100::mbar_wait(empty_bar(stage), ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + stage * C::STAGE_BYTES;
+          sm100::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          sm100::tma_load_3d(sa, &tmA, kb * C::BK, m_tile * C::BM, a3, full_bar(stage));
+          sm100::tma_load_3d(sa + C::A_BYTES, &tmB, kb * C::BK, n_tile * BN, c.l, full_bar(stage));
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        if (args.err) atomicOr(args.err, kErrTimeoutProducer);
+        // let the copies already in flight land before the CTA's shared memory goes away
+        for (long j = issued - 1; j >= 0 && j >= issued - C::STAGES; --j)
+          sm100::mbar_wait_drain(full_bar(static_cast<int>(j % C::STAGES)), static_cast<uint32_t>((j / C::STAGES) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_bf16_f32(C::BM, BN);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        if (!sm100::mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < kbn; ++kb) {
+          if (!sm100::mbar_wait(full_bar(stage), ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t sa = base + stage * C::STAGE_BYTES;
+          const uint64_t adesc = sm100::smem_desc_k128(sa);
+          const uint64_t bdesc = sm100::smem_desc_k128(sa + C::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k) {
+            // advance 16 bf16 (32 bytes) along K inside the swizzled 128-byte rows
+            sm100::mma_bf16(d_tmem, adesc + 2ull * k, bdesc + 2ull * k, idesc, (kb | k) != 0);
+          }
+          sm100::mma_commit(empty_bar(stage));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::mma_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      if (!ok) {
+        if (args.err) atomicOr(args.err, kErrTimeoutMma);
+        sm100::mma_commit(drain_bar);
+        sm100::mbar_wait_drain(drain_bar, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
+      if (!ok) {
+        if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
+        break;
+      }
+      sm100::tc_fence_after();
+      const int g = t / (mt * nt), r = t % (mt * nt);
+      const int n_tile = r / mt, m_tile = r % mt;
+      const Cell c = args.cells[g];
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      epilogue_tile<BN, EPI>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN);
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+int sm_count_cached() {
+  static int count[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+  return count[dev];
+}
+
+template <int BN, int EPI>
+cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
+  using C = TcCfg<BN>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int mt = (args.M + C::BM - 1) / C::BM;
+  const long tiles = static_cast<long>(args.G) * mt * (args.N / BN);
+  if (tiles <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
+  tc_gemm_kernel<BN, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(ta, tb, args);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
+  switch (args.epi) {
+    case kEpiStoreF32: return launch_bn_epi<BN, kEpiStoreF32>(ta, tb, args, st);
+    case kEpiStoreAct: return launch_bn_epi<BN, kEpiStoreAct>(ta, tb, args, st);
+    case kEpiResid: return launch_bn_epi<BN, kEpiResid>(ta, tb, args, st);
+    case kEpiResidCast: return launch_bn_epi<BN, kEpiResidCast>(ta, tb, args, st);
+    case kEpiRope:
+      if constexpr (BN >= 64) return launch_bn_epi<BN, kEpiRope>(ta, tb, args, st);
+      break;
+    case kEpiSwiGLU:
+      if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU>(ta, tb, args, st);
+      break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                       uint32_t box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode || !base || inner % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int tc_pick_bn(int N, int epi, int head_dim) {
+  const int cands[4] = {256, 128, 64, 32};
+  for (int bn : cands) {
+    if (N % bn) continue;
+    if (epi == kEpiSwiGLU && bn < 128) continue;
+    if (epi == kEpiRope && (bn < 64 || bn % head_dim)) continue;
+    return bn;
+  }
+  return 0;
+}
+
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn,
+                           cudaStream_t st) {
+  if (args.K % 64 != 0 || args.M <= 0) return cudaErrorInvalidValue;
+  switch (bn) {
+    case 256: return launch_bn<256>(ta, tb, args, st);
+    case 128: return launch_bn<128>(ta, tb, args, st);
+    case 64: return launch_bn<64>(ta, tb, args, st);
+    case 32: return launch_bn<32>(ta, tb, args, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rmt

@@ -1,0 +1,161 @@
+"""Kernel-level parity on the GPU, through the C ABI, against the oracle's functions (numpy,
+float64) and, for the grouped GEMM, against a float64 matmul of the same bf16 operands."""
+import numpy as np
+import pytest
+import torch
+
+from armt_synthetic import round_to_bf16
+from oracle import armt
+from recurrent_memory_transformer_anti_b200 import rmt
+from tests.gpu_util import normwise, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_ok):
+    torch.backends.cuda.matmul.allow_tf32 = False
+    yield
+
+
+def rng(seed):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+# ----------------------------------------------------------------------- grouped GEMM
+
+GEMM_CASES = [(g, 1040, n, 2048) for n in (2048, 8192) for g in (1, 2, 4, 8, 16)] + [
+    (3, 528, 256, 512), (2, 2064, 128, 128), (1, 100, 64, 64), (5, 16, 320, 192), (2, 1040, 64, 2048),
+    (2, 1040, 2048, 64), (1, 129, 192, 8192)]
+
+
+@pytest.mark.parametrize("G,M,N,K", GEMM_CASES)
+def test_grouped_gemm_matches_matmul(G, M, N, K):
+    r = rng(100 + G * 7 + N)
+    a = torch.from_numpy(r.standard_normal((G, M, K), dtype=np.float32)).to(torch.bfloat16).cuda()
+    b = torch.from_numpy(r.standard_normal((G, N, K), dtype=np.float32) * np.float32(0.02)).to(torch.bfloat16).cuda()
+    c = torch.full((G, M, N), float("nan"), device="cuda")
+    rmt.rmt_grouped_gemm_bf16(a, b, c, G, M, N, K, "f32")
+    rmt.rmt_sync(None)
+    ref = torch.bmm(a.double(), b.double().transpose(1, 2))
+    err = ((c.double() - ref).abs().max() / ref.abs().max()).item()
+    assert err < 1e-5, err
+    cb = torch.empty((G, M, N), device="cuda", dtype=torch.bfloat16)
+    rmt.rmt_grouped_gemm_bf16(a, b, cb, G, M, N, K, "bf16")
+    rmt.rmt_sync(None)
+    err_b = ((cb.double() - ref).abs().max() / ref.abs().max()).item()
+    assert err_b < 8e-3, err_b
+
+
+def test_grouped_gemm_each_group_uses_its_own_weight():
+    G, M, N, K = 4, 200, 128, 128
+    a = torch.ones((G, M, K), device="cuda", dtype=torch.bfloat16)
+    b = torch.stack([torch.full((N, K), float(g + 1) / 64, device="cuda") for g in range(G)]).to(torch.bfloat16)
+    c = torch.empty((G, M, N), device="cuda")
+    rmt.rmt_grouped_gemm_bf16(a, b, c, G, M, N, K, "f32")
+    rmt.rmt_sync(None)
+    for g in range(G):
+        assert torch.all(c[g] == 2.0 * (g + 1)), g
+
+
+# -------------------------------------------------------------------------- attention
+
+ATTN_CASES = [("bf16", 2, 1040, 32, 8, 64), ("bf16", 3, 208, 4, 2, 64), ("bf16", 2, 300, 4, 1, 128),
+              ("bf16", 2, 72, 4, 4, 32), ("bf16", 1, 1, 2, 1, 64), ("bf16", 1, 65, 2, 2, 64),
+              ("f32", 2, 72, 4, 4, 32), ("f32", 2, 208, 4, 2, 64), ("f32", 1, 130, 2, 1, 128)]
+
+
+@pytest.mark.parametrize("dtype,G,M,H,Hkv,dh", ATTN_CASES)
+def test_attention_matches_oracle(dtype, G, M, H, Hkv, dh):
+    r = rng(200 + M + H)
+    qkv = r.standard_normal((G, M, (H + 2 * Hkv) * dh), dtype=np.float32)
+    if dtype == "bf16":
+        qkv = round_to_bf16(qkv)
+    t = rmt.storage(qkv, dtype, "cuda")
+    out = torch.empty((G, M, H * dh), device="cuda", dtype=t.dtype)
+    rmt.rmt_attention(t, out, G, M, H, Hkv, dh, dtype)
+    rmt.rmt_sync(None)
+    got = to_np(out)
+    for g in range(G):
+        x = qkv[g].astype(np.float64)
+        q = x[:, :H * dh].reshape(M, H, dh)
+        k = x[:, H * dh:(H + Hkv) * dh].reshape(M, Hkv, dh)
+        v = x[:, (H + Hkv) * dh:].reshape(M, Hkv, dh)
+        ref = armt.causal_gqa_attention(q, k, v).reshape(M, H * dh)
+        tol = 1.2e-2 if dtype == "bf16" else 2e-5
+        assert normwise(got[g], ref) < tol
+
+
+# ------------------------------------------------------------------------------ memory
+
+@pytest.mark.parametrize("dtype,G,M,dk,dv", [("f32", 3, 1040, 64, 64), ("bf16", 3, 1040, 64, 64),
+                                             ("f32", 2, 72, 32, 32), ("f32", 2, 77, 128, 128),
+                                             ("f32", 2, 50, 32, 96), ("bf16", 4, 130, 128, 64)])
+def test_memory_read_matches_oracle(dtype, G, M, dk, dv):
+    r = rng(300 + M + dk)
+    q = r.standard_normal((G, M, dk), dtype=np.float32)
+    A = r.standard_normal((G, dk, dv), dtype=np.float32)
+    z = r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)
+    out = torch.empty((G, M, dv), device="cuda", dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+    tq, tA, tz = (torch.from_numpy(x).cuda() for x in (q, A, z))
+    rmt.rmt_memory_read(tq, tA, tz, out, G, M, dk, dv, 1e-6, dtype)
+    rmt.rmt_sync(None)
+    got = to_np(out)
+    for g in range(G):
+        ref = armt.memory_read(q[g].astype(np.float64), A[g].astype(np.float64), z[g].astype(np.float64), 1e-6)
+        assert normwise(got[g], ref) < (8e-3 if dtype == "bf16" else 1e-5)
+
+
+@pytest.mark.parametrize("G,n,dk,dv", [(5, 16, 64, 64), (3, 8, 32, 32), (2, 16, 128, 128), (2, 64, 64, 32),
+                                       (1, 1, 32, 64)])
+def test_memory_update_matches_oracle(G, n, dk, dv):
+    r = rng(400 + n + dk)
+    k = r.standard_normal((G, n, dk), dtype=np.float32)
+    v = r.standard_normal((G, n, dv), dtype=np.float32)
+    A = r.standard_normal((G, dk, dv), dtype=np.float32)
+    z = r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)
+    tk, tv, tA, tz = (torch.from_numpy(x).cuda() for x in (k, v, A, z))
+    rmt.rmt_memory_update(tk, tv, tA, tz, G, n, dk, dv, 1e-6)
+    rmt.rmt_sync(None)
+    for g in range(G):
+        rA, rz = armt.memory_update(k[g].astype(np.float64), v[g].astype(np.float64), A[g].astype(np.float64),
+                                    z[g].astype(np.float64), 1e-6)
+        assert normwise(to_np(tA[g]), rA) < 1e-5
+        assert normwise(to_np(tz[g]), rz) < 1e-6
+
+
+def test_memory_write_then_read_orthonormal_keys_on_gpu():
+    """phi(k_i) = e_i (k = 0 on the diagonal, -1000 elsewhere): after one write from an empty
+    memory, the read of k_j returns v_j / (1 + eps)."""
+    dk = dv = 64
+    eps = 1e-6
+    k = np.full((1, dk, dk), -1000.0, np.float32)
+    for i in range(dk):
+        k[0, i, i] = 0.0
+    v = rng(7).standard_normal((1, dk, dv), dtype=np.float32)
+    tk, tv = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()
+    A = torch.zeros((1, dk, dv), device="cuda")
+    z = torch.zeros((1, dk), device="cuda")
+    rmt.rmt_memory_update(tk, tv, A, z, 1, dk, dk, dv, eps)
+    o = torch.empty((1, dk, dv), device="cuda")
+    rmt.rmt_memory_read(tk, A, z, o, 1, dk, dk, dv, eps, "f32")
+    rmt.rmt_sync(None)
+    assert torch.all(z == 1.0)
+    np.testing.assert_allclose(to_np(o)[0], v[0] / (1 + eps), rtol=2e-7, atol=1e-7)
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+
+@pytest.mark.parametrize("dtype,rows,d", [("f32", 1040, 2048), ("bf16", 1040, 2048), ("f32", 7, 128),
+                                          ("bf16", 33, 3072)])
+def test_rmsnorm_matches_oracle(dtype, rows, d):
+    r = rng(500 + rows)
+    x = r.standard_normal((rows, d), dtype=np.float32) * 3
+    g = 1 + 0.1 * r.standard_normal(d, dtype=np.float32)
+    if dtype == "bf16":
+        g = round_to_bf16(g)
+    y = torch.empty((rows, d), device="cuda", dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+    rmt.rmt_rmsnorm(torch.from_numpy(x).cuda(), rmt.storage(g, dtype, "cuda"), y, rows, d, 1e-5, dtype)
+    rmt.rmt_sync(None)
+    ref = armt.rms_norm(x.astype(np.float64), g.astype(np.float64), 1e-5)
+    assert normwise(to_np(y), ref) < (5e-3 if dtype == "bf16" else 2e-6)

@@ -57,3 +57,14 @@ def test_diagonals_golden_table():
 def test_sequential_steps():
     t = armt.schedule_triples(3, 2, "sequential")
     np.testing.assert_array_equal(t, [[0, 0, 0], [1, 1, 0], [2, 2, 0], [3, 0, 1], [4, 1, 1], [5, 2, 1]])
+
+
+def test_bf16_rounding_of_the_input_generator():
+    """The fast (torch) rounding used for inputs equals round-to-nearest-even on the bits."""
+    from armt_synthetic import bf16_bits, bf16_bits_to_f32, round_to_bf16
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(100000).astype(np.float32) * s for s in (1e-3, 1.0, 1e3)])
+    x = np.concatenate([x, np.array([0.0, -0.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], np.float32)])
+    np.testing.assert_array_equal(round_to_bf16(x).view(np.uint32), bf16_bits_to_f32(bf16_bits(x)).view(np.uint32))
+    # ties go to even: 1 + 2^-8 sits halfway between 1 and 1 + 2^-7
+    assert round_to_bf16(np.array([1.0 + 2.0 ** -8], np.float32))[0] == 1.0
