@@ -196,6 +196,16 @@ rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void*
 rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G,
                              int32_t n, int32_t dk, int32_t dv, float eps, void* stream);
 
+/* Memory write from n rows per group (a layer's memory-token outputs):
+ *   k = y W_mk^T, v = y W_mv^T, then the delta-rule update above (phi applied to k).
+ * y [G, n, d] fp32; w_mkv [G, dk + dv, d] in dtype (the dk rows of W_mk, then the dv rows
+ * of W_mv); A [G, dk, dv] and z [G, dk] fp32, updated in place. The projection is split
+ * along d in blocks of 64 columns whose partial sums go to a library-owned device scratch
+ * buffer (grown with cudaMalloc on demand) and are added in a fixed order.
+ * n <= 64, n*(dk+dv) <= 4096; dk, dv multiples of 32, <= 128. */
+rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n,
+                            int32_t d, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
+
 /* RMSNorm of fp32 rows into dtype: y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g.
  * x [rows, d] fp32, g [d] and y [rows, d] in dtype. d % 4 == 0. */
 rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int32_t d, float eps,

@@ -109,6 +109,29 @@ rmt_status device_scratch(int G, const Cell** cells, int** err) {
   return RMT_OK;
 }
 
+// Split-K partial sums of rmt_memory_write, grown on demand (one buffer per device).
+struct PartialScratch {
+  float* p = nullptr;
+  size_t cap = 0;
+};
+PartialScratch g_part_scratch[64];
+
+rmt_status partial_scratch(size_t floats, float** out) {
+  int dev = 0;
+  RMT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RMT_EINVAL, "device index out of range");
+  PartialScratch& s = g_part_scratch[dev];
+  if (floats > s.cap) {
+    float* p = nullptr;
+    if (cudaMalloc(&p, floats * sizeof(float)) != cudaSuccess) return fail(RMT_ENOMEM, "scratch allocation failed");
+    if (s.p) cudaFree(s.p);
+    s.p = p;
+    s.cap = floats;
+  }
+  *out = s.p;
+  return RMT_OK;
+}
+
 }  // namespace
 
 struct rmt_handle {
@@ -421,7 +444,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_MEMKV, 2 * g * n * (dk + dv) * dd,
                   g * (n * dd * 4 + (dk + dv) * dd * es + h->nsplit * n * (dk + dv) * 4), st, [&] {
-                    MemKvArgs a{h->x, M, d, c.seg_len, c.n_mem, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
+                    MemKvArgs a{h->x, M, d, c.seg_len, c.n_mem, kOutSlot, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
                     return launch_mem_kv(a, h->bf16, st);
                   });
   if (e != cudaSuccess) return e;
@@ -777,6 +800,26 @@ rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int
   RMT_TRY(device_scratch(1, &cells, nullptr));
   RmsArgs a{x, g, y, rows, d, eps, 1, cells, kByLayer, kByLayer, 1};
   RMT_CUDA(launch_rmsnorm(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
+rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n, int32_t d,
+                            int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream) {
+  if (!y || !w_mkv || !A || !z) return fail(RMT_EINVAL, "null pointer");
+  if (G <= 0 || n <= 0 || n > 64 || d <= 0 || dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128 ||
+      n * (dk + dv) > 4096)
+    return fail(RMT_EINVAL, "bad sizes");
+  if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(G, &cells, nullptr));
+  const int nsplit = (d + kMemKvSplit - 1) / kMemKvSplit;
+  float* part = nullptr;
+  RMT_TRY(partial_scratch(size_t(G) * nsplit * n * (dk + dv), &part));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MemKvArgs ka{y, n, d, 0, n, kByLayer, w_mkv, part, dk + dv, G, cells, G};
+  RMT_CUDA(launch_mem_kv(ka, dtype == RMT_BF16, st));
+  MemUpdateArgs ua{part, nsplit, nullptr, nullptr, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0};
+  RMT_CUDA(launch_mem_update(ua, st));
   return RMT_OK;
 }
 

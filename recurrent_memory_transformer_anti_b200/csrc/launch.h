@@ -79,8 +79,9 @@ cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st);
 // Y = rows row0 .. row0+n-1 of the cell's output slot.
 constexpr int kMemKvSplit = 64;  // d_model columns per split
 struct MemKvArgs {
-  const float* x;  // residual stream [n_slots, M, d]
+  const float* x;  // [*, M, d] fp32: the residual stream slots (forward) or caller rows
   int M, d, row0, n;
+  IndexMode x_mode;  // slice of x holding the cell's rows (kOutSlot in the forward)
   const void* w;   // [L, dkv, d] in T
   float* part;     // [L, nsplit, n, dkv] fp32
   int dkv;

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   const Cell c = a.cells[blockIdx.y];
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
-  const float* Y = a.x + (static_cast<size_t>(out_slot(a.L, c.l, c.s)) * a.M + a.row0) * a.d + k0;
+  const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + a.row0) * a.d + k0;
   const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
   for (int e = threadIdx.x; e < a.n * KS; e += kKvThreads) {
     const int r = e / KS, k = e % KS;

@@ -159,3 +159,26 @@ def test_rmsnorm_matches_oracle(dtype, rows, d):
     rmt.rmt_sync(None)
     ref = armt.rms_norm(x.astype(np.float64), g.astype(np.float64), 1e-5)
     assert normwise(to_np(y), ref) < (5e-3 if dtype == "bf16" else 2e-6)
+
+
+@pytest.mark.parametrize("dtype,G,n,d,dk,dv", [("bf16", 4, 16, 2048, 64, 64), ("f32", 3, 8, 128, 32, 32),
+                                               ("bf16", 2, 16, 3072, 128, 128), ("f32", 2, 5, 200, 32, 64)])
+def test_memory_write_matches_oracle(dtype, G, n, d, dk, dv):
+    """Key/value projection of n rows (split-K partials reduced in fixed order) + update."""
+    r = rng(600 + d + n)
+    y = r.standard_normal((G, n, d), dtype=np.float32)
+    w = r.standard_normal((G, dk + dv, d), dtype=np.float32) * np.float32(0.02)
+    if dtype == "bf16":
+        w = round_to_bf16(w)
+    A = r.standard_normal((G, dk, dv), dtype=np.float32)
+    z = r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)
+    tA, tz = torch.from_numpy(A).cuda(), torch.from_numpy(z).cuda()
+    rmt.rmt_memory_write(torch.from_numpy(y).cuda(), rmt.storage(w, dtype, "cuda"), tA, tz, G, n, d, dk, dv, 1e-6,
+                         dtype)
+    rmt.rmt_sync(None)
+    for g in range(G):
+        y64, w64 = y[g].astype(np.float64), w[g].astype(np.float64)
+        rA, rz = armt.memory_update(y64 @ w64[:dk].T, y64 @ w64[dk:].T, A[g].astype(np.float64),
+                                    z[g].astype(np.float64), 1e-6)
+        assert normwise(to_np(tA[g]), rA) < 2e-5
+        assert normwise(to_np(tz[g]), rz) < 2e-6
