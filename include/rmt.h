@@ -206,6 +206,23 @@ rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z,
 rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n,
                             int32_t d, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
 
+/* rmt_memory_write without any device allocation. The paper has no counterpart: this is
+ * for callers that cannot let a library call cudaMalloc, such as a serving engine or a
+ * caching allocator that has already claimed the device memory for its own pool (there a
+ * cudaMalloc can fail, and it synchronizes the whole device, stalling the caller's other
+ * streams). Same arguments and results as rmt_memory_write; the cell table and the split-K
+ * partial sums live in a fixed 8 MiB array in the library's device memory, which every GPU
+ * that loads the library holds until the process exits. Sizes whose partial sums need
+ * more than 8 MiB - 64 KiB (G*ceil(d/64)*n*(dk+dv)*4 bytes), or G > 8192, return
+ * RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture. All calls share the array, which keeps the last call's contents (every
+ * value a call reads is written earlier in the same call): calls that overlap on the GPU,
+ * e.g. on two streams, race and give wrong results. */
+rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv, float* A, float* z, int32_t G,
+                                    int32_t n, int32_t d, int32_t dk, int32_t dv, float eps, rmt_dtype dtype,
+                                    void* stream);
+
 /* RMSNorm of fp32 rows into dtype: y[r] = x[r] / sqrt(mean(x[r]^2) + eps) * g.
  * x [rows, d] fp32, g [d] and y [rows, d] in dtype. d % 4 == 0. */
 rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int32_t d, float eps,

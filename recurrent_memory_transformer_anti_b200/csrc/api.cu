@@ -134,6 +134,11 @@ rmt_status partial_scratch(size_t floats, float** out) {
 
 }  // namespace
 
+namespace rmt {
+// Lets other translation units of the library report through rmt_last_error().
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace rmt
+
 struct rmt_handle {
   rmt_cfg cfg{};
   int dev = 0;

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4
 
 EXPORTED = ("rmt_create", "rmt_forward", "rmt_schedule_table", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
-            "rmt_memory_update", "rmt_memory_write", "rmt_rmsnorm", "rmt_probe", "rmt_probe_read")
+            "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
+            "rmt_probe_read")
 
 KERNELS = ("assemble", "memq", "memread", "memo", "rmsnorm1", "qkv", "attention", "o", "rmsnorm2", "gateup", "down",
            "memkv", "memupdate", "emit")
@@ -69,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "rmt_memory_read": [vp, vp, vp, vp, i32, i32, i32, i32, f32, ctypes.c_int, vp],
         "rmt_memory_update": [vp, vp, vp, vp, i32, i32, i32, i32, f32, vp],
         "rmt_memory_write": [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, ctypes.c_int, vp],
+        "rmt_memory_write_noalloc": [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, ctypes.c_int, vp],
         "rmt_rmsnorm": [vp, vp, vp, i32, i32, f32, ctypes.c_int, vp],
         "rmt_probe": [vp, ctypes.c_uint32],
         "rmt_probe_read": [vp, ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
@@ -242,6 +244,12 @@ def rmt_memory_update(k, v, A, z, G, n, dk, dv, eps, stream=None) -> None:
 def rmt_memory_write(y, w_mkv, A, z, G, n, d, dk, dv, eps, dtype="f32", stream=None) -> None:
     _check(_lib.rmt_memory_write(_ptr(y), _ptr(w_mkv), _ptr(A), _ptr(z), G, n, d, dk, dv, eps, DTYPES[dtype],
                                  _stream(stream)), "rmt_memory_write")
+
+
+def rmt_memory_write_noalloc(y, w_mkv, A, z, G, n, d, dk, dv, eps, dtype="f32", stream=None) -> None:
+    """rmt_memory_write with its scratch in the library's fixed device array (no cudaMalloc)."""
+    _check(_lib.rmt_memory_write_noalloc(_ptr(y), _ptr(w_mkv), _ptr(A), _ptr(z), G, n, d, dk, dv, eps,
+                                         DTYPES[dtype], _stream(stream)), "rmt_memory_write_noalloc")
 
 
 def rmt_rmsnorm(x, g, y, rows, d, eps, dtype="f32", stream=None) -> None:

@@ -1,0 +1,53 @@
+"""rmt_memory_write_noalloc against rmt_memory_write, on the GPU through the C ABI.
+
+The allocation-free variant is for callers that cannot let a library call cudaMalloc,
+such as a serving engine or caching allocator that already owns the device's memory
+(there cudaMalloc can fail, and it synchronizes the device). It must give the results of
+the allocating entry point, call after call, although its scratch (cell table and split-K
+partial sums) lives in one fixed device array that every call reuses.
+"""
+import numpy as np
+import pytest
+import torch
+
+from armt_synthetic import round_to_bf16
+from recurrent_memory_transformer_anti_b200 import rmt
+
+pytestmark = pytest.mark.gpu
+
+
+def normwise(a, b):
+    a = a.double().cpu()
+    b = b.double().cpu()
+    return float((a - b).abs().max() / b.abs().max().clamp_min(1e-30))
+
+
+@pytest.mark.parametrize("dtype,G,n,d,dk,dv", [("bf16", 16, 16, 2048, 64, 64), ("f32", 3, 8, 200, 32, 32)])
+def test_noalloc_memory_write_matches_allocating_entry_point(cuda_ok, dtype, G, n, d, dk, dv):
+    r = np.random.Generator(np.random.PCG64(700 + d))
+    A0 = torch.from_numpy(r.standard_normal((G, dk, dv), dtype=np.float32)).cuda()
+    z0 = torch.from_numpy(r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)).cuda()
+    A_ref, z_ref = A0.clone(), z0.clone()
+    A_new, z_new = A0.clone(), z0.clone()
+    for _ in range(2):  # two calls in a row: the second reuses the scratch the first left behind
+        y = torch.from_numpy(r.standard_normal((G, n, d), dtype=np.float32)).cuda()
+        w = r.standard_normal((G, dk + dv, d), dtype=np.float32) * np.float32(0.02)
+        w = rmt.storage(round_to_bf16(w) if dtype == "bf16" else w, dtype, "cuda")
+        rmt.rmt_memory_write(y, w, A_ref, z_ref, G, n, d, dk, dv, 1e-6, dtype)
+        rmt.rmt_memory_write_noalloc(y, w, A_new, z_new, G, n, d, dk, dv, 1e-6, dtype)
+        rmt.rmt_sync(None)
+        assert normwise(A_new, A_ref) < 2e-5
+        assert normwise(z_new, z_ref) < 2e-6
+        assert normwise(A_new, A0) > 1e-6  # the state really moved
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
+    G, n, d, dk, dv = 64, 16, 2048, 128, 128  # 64*32*16*256*4 B = 32 MiB of partial sums > 8 MiB
+    y = torch.zeros((G, n, d), device="cuda")
+    w = torch.zeros((G, dk + dv, d), device="cuda")
+    A = torch.zeros((G, dk, dv), device="cuda")
+    z = torch.zeros((G, dk), device="cuda")
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_memory_write_noalloc(y, w, A, z, G, n, d, dk, dv, 1e-6, "f32")
+    assert ex.value.status == rmt.RMT_EINVAL
+    assert "scratch" in str(ex.value)
