@@ -40,9 +40,11 @@ N_SEGMENTS = 128
 WORKLOAD = "LLaMA-1B-shaped ARMT prefill of one 131,072-token sequence (128 x (1024 + 16 memory) tokens)"
 DATA = "synthetic: seeded N(0,1) embeddings, random-init N(0,0.02) weights"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes per launch of the gate/up GEMM measured by ncu (profiles/gateup_gemm_1b.md); None
-# until a capture of the current kernel exists.
-GATEUP_TRAFFIC_BYTES_PER_LAUNCH = None
+# DRAM bytes (read + write) per cell of the gate/up GEMM, from one ncu capture of a 2-cell
+# launch of the current kernel (profiles/gateup_gemm_1b.md). Traffic grows with the number of
+# cells (each cell brings its own layer's weights and activations), so a launch's traffic is
+# this figure times its cells. None when no capture of the current kernel exists.
+GATEUP_TRAFFIC_BYTES_PER_CELL = 80.74e6
 
 
 def parse():
@@ -297,7 +299,9 @@ def main() -> int:
                 "frac": achieved / peak if achieved else None,
                 "peak_source": f"bf16_tflops_sustained ({peak_src})",
                 "launches": probe["launches"], "kernel_ms_per_step": probe["ms"] / K,
-                "traffic": GATEUP_TRAFFIC_BYTES_PER_LAUNCH}
+                "traffic": (GATEUP_TRAFFIC_BYTES_PER_CELL * cfg.n_layers * S / probe["launches"] * K
+                            if GATEUP_TRAFFIC_BYTES_PER_CELL and probe["launches"] else None),
+                "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 2-cell launch)"}
 
     # ---- per-kernel breakdown of one forward (outside the timed region)
     rmt.rmt_probe(h, list(rmt.KERNELS))

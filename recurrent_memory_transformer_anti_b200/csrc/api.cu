@@ -162,7 +162,7 @@ struct rmt_handle {
   void* out_stage = nullptr;
   size_t out_stage_bytes = 0;
   std::map<std::pair<int, int>, Table> tables;
-  CUtensorMap tm_xb, tm_om, tm_h, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo;
+  CUtensorMap tm_xb, tm_om, tm_h, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
   std::vector<void*> allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
@@ -310,7 +310,8 @@ rmt_status build_maps(rmt_handle* h) {
             make_tmap_bf16_3d(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) &&
             make_tmap_bf16_3d(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
             make_tmap_bf16_3d(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) &&
-            make_tmap_bf16_3d(&h->tm_wd, h->w_d, F, d, L, h->bn_d);
+            make_tmap_bf16_3d(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
+            make_tmap_bf16_3d(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128);
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
 }
 
@@ -428,7 +429,8 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_ATTENTION, g * c.n_heads * 4.0 * c.head_dim * m * (m + 1) / 2,
                   g * (m * nq * es + m * hd * es), st, [&] {
-                    AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L};
+                    AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err};
+                    if (h->bf16 && attention_tc_supported(c.head_dim)) return launch_attention_tc(h->tm_qkv, a, st);
                     return launch_attention(a, h->bf16, st);
                   });
   if (e != cudaSuccess) return e;
@@ -765,8 +767,16 @@ rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32
   if (dh != 32 && dh != 64 && dh != 128) return fail(RMT_EINVAL, "dh must be 32, 64 or 128");
   if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
   const Cell* cells = nullptr;
-  RMT_TRY(device_scratch(G, &cells, nullptr));
-  AttnArgs a{qkv, out, M, H, Hkv, dh, G, cells, kByLayer, G};
+  int* err = nullptr;
+  RMT_TRY(device_scratch(G, &cells, &err));
+  AttnArgs a{qkv, out, M, H, Hkv, dh, G, cells, kByLayer, G, err};
+  if (dtype == RMT_BF16 && attention_tc_supported(dh)) {
+    CUtensorMap tm;
+    if (!make_tmap_bf16_3d(&tm, qkv, uint64_t(H + 2 * Hkv) * dh, M, G, 128))
+      return fail(RMT_EINVAL, "tensor map encoding failed (qkv must be 16-byte aligned)");
+    RMT_CUDA(launch_attention_tc(tm, a, static_cast<cudaStream_t>(stream)));
+    return RMT_OK;
+  }
   RMT_CUDA(launch_attention(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }

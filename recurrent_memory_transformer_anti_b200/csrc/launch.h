@@ -55,8 +55,13 @@ struct AttnArgs {
   const Cell* cells;
   IndexMode mode;  // slice index of both buffers
   int L;
+  int* err;        // device error word for bounded waits (tensor-core kernel), may be null
 };
+// mma.sync (bf16) or fp32 FMA kernels, any head_dim in {32, 64, 128}
 cudaError_t launch_attention(const AttnArgs& a, bool bf16, cudaStream_t st);
+// tcgen05 kernel (bf16, head_dim 64 or 128): tm_qkv maps qkv as [*, M, (H+2Hkv)dh], box 64 x 128
+bool attention_tc_supported(int dh);
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, cudaStream_t st);
 
 // ------------------------------------------------------------------ associative memory
 struct MemReadArgs {

@@ -92,57 +92,57 @@ __global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemRead
 
 // ------------------------------------------------------------------ key/value projection
 // CTA = one split of kMemKvSplit columns of d_model for one cell: the n memory rows and the
-// dkv weight rows of that split are staged in shared memory, then each thread forms up to
-// 16 of the n x dkv partial dot products.
-constexpr int kKvThreads = 256, kKvMaxOut = 16;
+// dkv weight rows of that split are staged in shared memory; each thread then forms a
+// 4 x 4 block of the n x dkv partial dot products (4 + 4 shared loads per 16 FMAs).
+constexpr int kKvThreads = 256;
 
 template <typename T>
 __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   extern __shared__ float sm[];
   constexpr int KS = kMemKvSplit;
-  float* Ys = sm;                // [n][KS]
-  float* Ws = sm + a.n * KS;     // [KS][dkv + 1]
-  const int ldw = a.dkv + 1;
+  const int n4 = (a.n + 3) & ~3;  // rows padded to a multiple of 4 (padding rows are zero)
+  float* Ys = sm;                 // [KS][n4]   (transposed: k-major)
+  float* Ws = sm + KS * n4;       // [KS][dkv]
   const Cell c = a.cells[blockIdx.y];
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
   const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + a.row0) * a.d + k0;
   const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
-  for (int e = threadIdx.x; e < a.n * KS; e += kKvThreads) {
+  for (int e = threadIdx.x; e < n4 * KS; e += kKvThreads) {
     const int r = e / KS, k = e % KS;
-    Ys[e] = k < kw ? Y[static_cast<size_t>(r) * a.d + k] : 0.f;
+    Ys[k * n4 + r] = (r < a.n && k < kw) ? Y[static_cast<size_t>(r) * a.d + k] : 0.f;
   }
   for (int e = threadIdx.x; e < a.dkv * KS; e += kKvThreads) {
     const int j = e / KS, k = e % KS;
-    Ws[k * ldw + j] = k < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k]) : 0.f;
+    Ws[k * a.dkv + j] = k < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k]) : 0.f;
   }
   __syncthreads();
-  const int nout = a.n * a.dkv;
-  float acc[kKvMaxOut];
-#pragma unroll
-  for (int i = 0; i < kKvMaxOut; ++i) acc[i] = 0.f;
-  for (int k = 0; k < KS; ++k) {
-#pragma unroll
-    for (int i = 0; i < kKvMaxOut; ++i) {
-      const int e = threadIdx.x + i * kKvThreads;
-      if (e < nout) {
-        const int r = e / a.dkv, j = e % a.dkv;
-        acc[i] = fmaf(Ys[r * KS + k], Ws[k * ldw + j], acc[i]);
-      }
-    }
-  }
   const int nsplit = (a.d + KS - 1) / KS;
+  const int nout = a.n * a.dkv;
   float* part = a.part + (static_cast<size_t>(c.l) * nsplit + split) * nout;
+  const int jt = a.dkv / 4, tiles = (n4 / 4) * jt;
+  for (int t = threadIdx.x; t < tiles; t += kKvThreads) {
+    const int r0 = (t / jt) * 4, j0 = (t % jt) * 4;
+    float acc[4][4] = {};
+#pragma unroll 4
+    for (int k = 0; k < KS; ++k) {
+      const float4 y = *reinterpret_cast<const float4*>(Ys + k * n4 + r0);
+      const float4 w = *reinterpret_cast<const float4*>(Ws + k * a.dkv + j0);
+      const float yv[4] = {y.x, y.y, y.z, y.w}, wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int i = 0; i < kKvMaxOut; ++i) {
-    const int e = threadIdx.x + i * kKvThreads;
-    if (e < nout) part[e] = acc[i];
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(yv[i], wv[q], acc[i][q]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (r0 + i < a.n) *reinterpret_cast<float4*>(part + (r0 + i) * a.dkv + j0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
   }
 }
 
 // --------------------------------------------------------------------------- update
 // CTA = one cell. Shared memory: raw k|v rows, phi(k), A, z, row denominators, V - v_bar.
-constexpr int kUpdThreads = 256;
+constexpr int kUpdThreads = 512;
 
 __global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdateArgs a) {
   extern __shared__ float sm[];
@@ -162,8 +162,10 @@ __global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdate
     float val;
     if (a.part) {
       const float* p = a.part + ki * a.nsplit * n * dkv + e;
+      const size_t stride = static_cast<size_t>(n) * dkv;
       val = 0.f;
-      for (int sp = 0; sp < a.nsplit; ++sp) val += p[static_cast<size_t>(sp) * n * dkv];
+#pragma unroll 8
+      for (int sp = 0; sp < a.nsplit; ++sp) val += p[sp * stride];
     } else {
       val = j < dk ? a.k[(ki * n + r) * dk + j] : a.v[(ki * n + r) * dv + (j - dk)];
     }
@@ -227,9 +229,9 @@ cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st) {
 
 cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (a.G <= 0) return cudaSuccess;
-  if (a.n * a.dkv > kKvThreads * kKvMaxOut) return cudaErrorInvalidValue;
-  const size_t smem = (static_cast<size_t>(a.n) * kMemKvSplit + static_cast<size_t>(kMemKvSplit) * (a.dkv + 1)) *
-                      sizeof(float);
+  if (a.n > 64 || a.dkv % 4) return cudaErrorInvalidValue;
+  const size_t n4 = (a.n + 3) & ~3;
+  const size_t smem = (n4 * kMemKvSplit + static_cast<size_t>(kMemKvSplit) * a.dkv) * sizeof(float);
   dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G);
   if (bf16) {
     if (smem > 48 * 1024)

@@ -11,8 +11,9 @@
 //               128-byte swizzled, into a STAGES-deep shared-memory ring;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, K=16) into
 //               one of two TMEM accumulators and commits to mbarriers;
-//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (one row per thread),
-//               fused RoPE / SwiGLU / residual add / cast, stores to global memory.
+//   warps 2-9   epilogue, two warpgroups each taking half of the tile's columns:
+//               tcgen05.ld of the finished accumulator (one row per thread), fused RoPE /
+//               SwiGLU / residual add / cast, stores to global memory.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 // Every wait is bounded (see sm100.cuh); on a timeout the CTA drains its in-flight copies
 // and MMAs, frees TMEM, records the failure in the error word and returns.
@@ -33,7 +34,7 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int BAR_BYTES = 128 * ((8 * (2 * STAGES + 5) + 16 + 127) / 128);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
 };
 
@@ -41,30 +42,23 @@ namespace {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Store 32 consecutive fp32 values as bf16 (64 bytes, four 16-byte stores).
-__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                      pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
-  }
-}
-
 __device__ __forceinline__ void store32_f32(float* dst, const float* v) {
   float4* d = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
-// Plain / residual epilogue of one 32-column chunk of one row.
+// The epilogue runs on two warpgroups; each owns every TMEM lane (one row per thread, four
+// warps covering the 128 rows) and half of the tile's columns, so twice the rows' bytes
+// are in flight for the memory-bound residual and RoPE epilogues.
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+
+// Epilogue of one 32-column chunk of one row (row per thread). `src` holds the residual
+// values of the chunk for the residual kinds (loaded by the caller before the TMEM wait).
 template <int EPI>
-__device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32],
+                                          const float4 (&src)[8]) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]);
@@ -76,55 +70,61 @@ __device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, 
     const size_t idx = cell_index(ep.out_mode, a.L, c);
     store32_bf16(static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
   } else if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
-    const size_t si = cell_index(ep.src_mode, a.L, c), di = cell_index(ep.dst_mode, a.L, c);
-    const float4* src = reinterpret_cast<const float4*>(ep.x + (si * a.M + row) * ep.ldx + col);
+    const size_t di = cell_index(ep.dst_mode, a.L, c);
     float* dst = ep.x + (di * a.M + row) * ep.ldx + col;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const float4 s = src[q];
-      v[4 * q] += s.x;
-      v[4 * q + 1] += s.y;
-      v[4 * q + 2] += s.z;
-      v[4 * q + 3] += s.w;
+      v[4 * q] += src[q].x;
+      v[4 * q + 1] += src[q].y;
+      v[4 * q + 2] += src[q].z;
+      v[4 * q + 3] += src[q].w;
     }
     store32_f32(dst, v);
     if constexpr (EPI == kEpiResidCast) store32_bf16(ep.xb + (di * a.M + row) * ep.ldx + col, v);
   }
 }
 
+// Epilogue of one tile row for column half `part` (0 or 1) of the tile.
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0) {
+__device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0, int part) {
   const bool valid = row < a.M;
   const EpiParams& ep = a.ep;
   if constexpr (EPI == kEpiRope) {
     const int dh = ep.head_dim, half = dh >> 1;
     const size_t idx = cell_index(ep.out_mode, a.L, c);
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
-    for (int h0 = 0; h0 < BN; h0 += dh) {
+    const int heads = BN / dh;
+    // rotation pairs (i, i + dh/2) of each head, in 32-wide units: heads * max(1, half/32)
+    const int per_head = half >= 32 ? half / 32 : 1;
+    const int units = heads * per_head;
+    const int u0 = part * units / 2, u1 = (part + 1) * units / 2;
+#pragma unroll 1
+    for (int u = u0; u < u1; ++u) {
+      const int h0 = (u / per_head) * dh;
       const bool rot = (n0 + h0) < ep.rope_cols;
       if (half >= 32) {
-        for (int p = 0; p < half; p += 32) {
-          uint32_t lo[32], hi[32];
-          sm100::tmem_ld32(tacc + h0 + p, lo);
-          sm100::tmem_ld32(tacc + h0 + half + p, hi);
-          sm100::tmem_wait_ld();
-          if (valid) {
-            float x1[32], x2[32];
+        const int p = (u % per_head) * 32;
+        uint32_t lo[32], hi[32];
+        sm100::tmem_ld32(tacc + h0 + p, lo);
+        sm100::tmem_ld32(tacc + h0 + half + p, hi);
+        sm100::tmem_wait_ld();
+        if (valid) {
+          float x1[32], x2[32];
+          const float2* cs = ep.rope + (size_t)row * half + p;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float a1 = u2f(lo[j]), a2 = u2f(hi[j]);
-              if (rot) {
-                const float2 cs = ep.rope[(size_t)row * half + p + j];
-                x1[j] = a1 * cs.x - a2 * cs.y;
-                x2[j] = a2 * cs.x + a1 * cs.y;
-              } else {
-                x1[j] = a1;
-                x2[j] = a2;
-              }
+          for (int j = 0; j < 32; ++j) {
+            const float a1 = u2f(lo[j]), a2 = u2f(hi[j]);
+            if (rot) {
+              const float2 t = cs[j];
+              x1[j] = a1 * t.x - a2 * t.y;
+              x2[j] = a2 * t.x + a1 * t.y;
+            } else {
+              x1[j] = a1;
+              x2[j] = a2;
             }
-            store32_bf16(orow + n0 + h0 + p, x1);
-            store32_bf16(orow + n0 + h0 + half + p, x2);
           }
+          store32_bf16(orow + n0 + h0 + p, x1);
+          store32_bf16(orow + n0 + h0 + half + p, x2);
         }
       } else {  // head_dim 32: both halves of the head in one 32-column chunk
         uint32_t r[32];
@@ -136,9 +136,9 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
           for (int j = 0; j < 16; ++j) {
             const float a1 = u2f(r[j]), a2 = u2f(r[j + 16]);
             if (rot) {
-              const float2 cs = ep.rope[(size_t)row * 16 + j];
-              x[j] = a1 * cs.x - a2 * cs.y;
-              x[j + 16] = a2 * cs.x + a1 * cs.y;
+              const float2 t = ep.rope[(size_t)row * 16 + j];
+              x[j] = a1 * t.x - a2 * t.y;
+              x[j + 16] = a2 * t.x + a1 * t.y;
             } else {
               x[j] = a1;
               x[j + 16] = a2;
@@ -151,35 +151,49 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
   } else if constexpr (EPI == kEpiSwiGLU) {
     const size_t idx = cell_index(ep.out_mode, a.L, c);
     __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
+    constexpr int per_blk = kSwiGLUBlock / 32;  // 32-wide output units per gate/up block pair
+    constexpr int units = (BN / (2 * kSwiGLUBlock)) * per_blk;
+    const int u0 = part * units / 2, u1 = (part + 1) * units / 2;
 #pragma unroll 1
-    for (int b0 = 0; b0 < BN; b0 += 2 * kSwiGLUBlock) {
-#pragma unroll 1
-      for (int p = 0; p < kSwiGLUBlock; p += 32) {
-        uint32_t g[32], u[32];
-        sm100::tmem_ld32(tacc + b0 + p, g);
-        sm100::tmem_ld32(tacc + b0 + kSwiGLUBlock + p, u);
-        sm100::tmem_wait_ld();
-        if (valid) {
-          float y[32];
+    for (int u = u0; u < u1; ++u) {
+      const int b0 = (u / per_blk) * 2 * kSwiGLUBlock, p = (u % per_blk) * 32;
+      uint32_t g[32], up[32];
+      sm100::tmem_ld32(tacc + b0 + p, g);
+      sm100::tmem_ld32(tacc + b0 + kSwiGLUBlock + p, up);
+      sm100::tmem_wait_ld();
+      if (valid) {
+        float y[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j])) * u2f(u[j]);
-          store32_bf16(orow + (n0 + b0) / 2 + p, y);
-        }
+        for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j])) * u2f(up[j]);
+        store32_bf16(orow + (n0 + b0) / 2 + p, y);
       }
     }
   } else {
+    constexpr int chunks = BN / 32;
+    const int c0 = part * chunks / 2, c1 = (part + 1) * chunks / 2;
+    const float* src_row = nullptr;
+    if constexpr (EPI == kEpiResid || EPI == kEpiResidCast)
+      src_row = ep.x + (static_cast<size_t>(cell_index(ep.src_mode, a.L, c)) * a.M + (valid ? row : 0)) * ep.ldx + n0;
 #pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
+    for (int cc = c0; cc < c1; ++cc) {
       uint32_t r[32];
-      sm100::tmem_ld32(tacc + cc, r);
+      float4 src[8];
+      sm100::tmem_ld32(tacc + cc * 32, r);
+      if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+        // residual loads go out before the TMEM wait so both latencies overlap
+        if (valid) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) src[q] = reinterpret_cast<const float4*>(src_row + cc * 32)[q];
+        }
+      }
       sm100::tmem_wait_ld();
-      if (valid) epi_chunk<EPI>(a, c, row, n0 + cc, r);
+      if (valid) epi_chunk<EPI>(a, c, row, n0 + cc * 32, r, src);
     }
   }
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcGemmArgs args) {
   using C = TcCfg<BN>;
@@ -204,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       sm100::mbar_init(tfull_bar(a), 1);
-      sm100::mbar_init(tempty_bar(a), 4);
+      sm100::mbar_init(tempty_bar(a), kEpiWarps);
     }
     sm100::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -308,7 +322,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 belong to this warp
+    const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31 belong to this warp
+    const int part = (warp - 2) / 4;     // column half of the tile handled by this warpgroup
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -322,7 +337,7 @@ __global__ void __launch_bounds__(192, 1)
       const int n_tile = r / mt, m_tile = r % mt;
       const Cell c = args.cells[g];
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_tile<BN, EPI>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN);
+      epilogue_tile<BN, EPI>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(tempty_bar(acc));
@@ -367,7 +382,7 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   const long tiles = static_cast<long>(args.G) * mt * (args.N / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
-  tc_gemm_kernel<BN, EPI><<<grid, 192, C::SMEM_BYTES, st>>>(ta, tb, args);
+  tc_gemm_kernel<BN, EPI><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, args);
   return cudaGetLastError();
 }
 
