@@ -200,7 +200,7 @@ rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z,
  *   k = y W_mk^T, v = y W_mv^T, then the delta-rule update above (phi applied to k).
  * y [G, n, d] fp32; w_mkv [G, dk + dv, d] in dtype (the dk rows of W_mk, then the dv rows
  * of W_mv); A [G, dk, dv] and z [G, dk] fp32, updated in place. The projection is split
- * along d in blocks of 64 columns whose partial sums go to a library-owned device scratch
+ * along d in blocks of 128 columns whose partial sums go to a library-owned device scratch
  * buffer (grown with cudaMalloc on demand) and are added in a fixed order.
  * n <= 64, n*(dk+dv) <= 4096; dk, dv multiples of 32, <= 128. */
 rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n,
@@ -213,7 +213,7 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
  * streams). Same arguments and results as rmt_memory_write; the cell table and the split-K
  * partial sums live in a fixed 8 MiB array in the library's device memory, which every GPU
  * that loads the library holds until the process exits. Sizes whose partial sums need
- * more than 8 MiB - 64 KiB (G*ceil(d/64)*n*(dk+dv)*4 bytes), or G > 8192, return
+ * more than 8 MiB - 64 KiB (G*ceil(d/128)*n*(dk+dv)*4 bytes), or G > 8192, return
  * RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress); make that first call before any
  * stream capture. All calls share the array, which keeps the last call's contents (every

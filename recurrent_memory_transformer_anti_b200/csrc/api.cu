@@ -150,8 +150,10 @@ struct rmt_handle {
   // activations and state
   float* x = nullptr;
   __nv_bfloat16* xb = nullptr;
-  void *hbuf = nullptr, *qkv = nullptr, *att = nullptr, *u = nullptr, *om = nullptr;
+  void *qkv = nullptr, *att = nullptr, *u = nullptr, *om = nullptr;
   float *qm = nullptr, *part = nullptr, *A = nullptr, *z = nullptr;
+  float *ss1 = nullptr, *ss2 = nullptr;  // per-row sums of squares for the folded RMSNorms
+  int ss_parts = 0;
   float2* rope = nullptr;
   int* err = nullptr;
   int* trace = nullptr;
@@ -162,7 +164,7 @@ struct rmt_handle {
   void* out_stage = nullptr;
   size_t out_stage_bytes = 0;
   std::map<std::pair<int, int>, Table> tables;
-  CUtensorMap tm_xb, tm_om, tm_h, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv;
+  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
   std::vector<void*> allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
@@ -302,7 +304,6 @@ rmt_status build_maps(rmt_handle* h) {
   h->bn_d = tc_pick_bn(c.d_model, kEpiResidCast, 0);
   bool ok = make_tmap_bf16_3d(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) &&
             make_tmap_bf16_3d(&h->tm_om, h->om, c.d_v, M, L, 128) &&
-            make_tmap_bf16_3d(&h->tm_h, h->hbuf, d, M, L, 128) &&
             make_tmap_bf16_3d(&h->tm_att, h->att, hd, M, L, 128) &&
             make_tmap_bf16_3d(&h->tm_u, h->u, F, M, L, 128) &&
             make_tmap_bf16_3d(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) &&
@@ -327,6 +328,10 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   ep.head_dim = c.head_dim;
   ep.rope_cols = (c.n_heads + c.n_kv_heads) * c.head_dim;
   ep.out_mode = ep.src_mode = ep.dst_mode = kByLayer;
+  ep.ss_parts = h->ss_parts;
+  ep.inv_d = 1.f / float(d);
+  ep.rms_eps = c.rms_eps;
+  const EpiKind resid = h->bf16 ? kEpiResidCast : kEpiResid;  // bf16: also refresh the bf16 copy
   int N = 0, K = 0;
   EpiKind epi = kEpiStoreF32;
   IndexMode amode = kByLayer;
@@ -340,28 +345,28 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       ep.out = h->qm, ep.ldo = c.d_k;
       a32 = h->x, w = h->w_mq, ta = &h->tm_xb, tb = &h->tm_wmq, bn = h->bn_mq;
       break;
-    case kProjMemO:
-      N = d, K = c.d_v, epi = kEpiResid;
-      ep.src_mode = kInSlot, ep.dst_mode = kOutSlot;
+    case kProjMemO:  // x_out = x_in + read-out; emits the row sums of squares of RMSNorm 1
+      N = d, K = c.d_v, epi = resid;
+      ep.src_mode = kInSlot, ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss1;
       a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
       break;
-    case kProjQkv:
-      N = h->Nqkv, K = d, epi = kEpiRope;
-      ep.out = h->qkv, ep.ldo = h->Nqkv;
-      a32 = static_cast<const float*>(h->hbuf), w = h->w_qkv, ta = &h->tm_h, tb = &h->tm_wqkv, bn = h->bn_qkv;
+    case kProjQkv:  // rows of x_out scaled by RMSNorm 1 (gain folded into the weight), then RoPE
+      N = h->Nqkv, K = d, epi = kEpiRope, amode = kOutSlot;
+      ep.out = h->qkv, ep.ldo = h->Nqkv, ep.ss_in = h->ss1;
+      a32 = h->x, w = h->w_qkv, ta = &h->tm_xb, tb = &h->tm_wqkv, bn = h->bn_qkv;
       break;
-    case kProjO:
-      N = d, K = hd, epi = kEpiResid;
-      ep.src_mode = ep.dst_mode = kOutSlot;
+    case kProjO:  // x_out += attention output; emits the row sums of squares of RMSNorm 2
+      N = d, K = hd, epi = resid;
+      ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss2;
       a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
       break;
-    case kProjGateUp:
-      N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU;
-      ep.out = h->u, ep.ldo = c.d_ff;
-      a32 = static_cast<const float*>(h->hbuf), w = h->w_gu, ta = &h->tm_h, tb = &h->tm_wgu, bn = h->bn_gu;
+    case kProjGateUp:  // rows of x_out scaled by RMSNorm 2 (gain folded into the weight), SwiGLU
+      N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU, amode = kOutSlot;
+      ep.out = h->u, ep.ldo = c.d_ff, ep.ss_in = h->ss2;
+      a32 = h->x, w = h->w_gu, ta = &h->tm_xb, tb = &h->tm_wgu, bn = h->bn_gu;
       break;
-    case kProjDown:
-      N = d, K = c.d_ff, epi = h->bf16 ? kEpiResidCast : kEpiResid;
+    case kProjDown:  // x_out += MLP output; the bf16 copy feeds the next layer's memory query
+      N = d, K = c.d_ff, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb;
       a32 = static_cast<const float*>(h->u), w = h->w_d, ta = &h->tm_u, tb = &h->tm_wd, bn = h->bn_d;
       break;
@@ -370,7 +375,8 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
     return launch_tc_gemm(*ta, *tb, a, bn, st);
   }
-  SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, K, amode, static_cast<const float*>(w), epi, ep};
+  const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
+  SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, lda, amode, static_cast<const float*>(w), epi, ep};
   return launch_simt_gemm(a, st);
 }
 
@@ -419,11 +425,6 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv, g * (m * dv * es + dd * dv * es + 2 * m * dd * 4), st,
                   [&] { return run_proj(h, kProjMemO, cells, G, st); });
   if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_RMSNORM1, 3 * g * m * dd, g * (m * dd * 4 + dd * es + m * dd * es), st, [&] {
-    RmsArgs a{h->x, h->g1, h->hbuf, M, d, c.rms_eps, G, cells, kOutSlot, kByLayer, L};
-    return launch_rmsnorm(a, h->bf16, st);
-  });
-  if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_QKV, 2 * g * m * nq * dd, g * (m * dd * es + nq * dd * es + m * nq * es), st,
                   [&] { return run_proj(h, kProjQkv, cells, G, st); });
   if (e != cudaSuccess) return e;
@@ -436,11 +437,6 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd, g * (m * hd * es + dd * hd * es + 2 * m * dd * 4), st,
                   [&] { return run_proj(h, kProjO, cells, G, st); });
-  if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_RMSNORM2, 3 * g * m * dd, g * (m * dd * 4 + dd * es + m * dd * es), st, [&] {
-    RmsArgs a{h->x, h->g2, h->hbuf, M, d, c.rms_eps, G, cells, kOutSlot, kByLayer, L};
-    return launch_rmsnorm(a, h->bf16, st);
-  });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_GATEUP, 2 * g * m * 2 * F * dd, g * (m * dd * es + 2 * F * dd * es + m * F * es), st,
                   [&] { return run_proj(h, kProjGateUp, cells, G, st); });
@@ -545,7 +541,9 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
       {&h->w_mkv, L * (dk + dv) * d * es}, {&h->g1, L * d * es},            {&h->g2, L * d * es},
       {&h->memtok, size_t(c.n_mem) * d * es},
       {reinterpret_cast<void**>(&h->x), n_slots(c.n_layers) * M * d * 4},
-      {&h->hbuf, L * M * d * es},        {&h->qkv, L * M * h->Nqkv * es},   {&h->att, L * M * hd * es},
+      {&h->qkv, L * M * h->Nqkv * es},   {&h->att, L * M * hd * es},
+      {reinterpret_cast<void**>(&h->ss1), L * M * (d / 16 + 1) * 4},
+      {reinterpret_cast<void**>(&h->ss2), L * M * (d / 16 + 1) * 4},
       {&h->u, L * M * F * es},           {&h->om, L * M * dv * es},
       {reinterpret_cast<void**>(&h->qm), L * M * dk * 4},
       {reinterpret_cast<void**>(&h->part), L * h->nsplit * size_t(c.n_mem) * (dk + dv) * 4},
@@ -564,6 +562,10 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   }
   rmt_status st = pack_weights(h, weights);
   if (st != RMT_OK) return bail(st);
+  // RMSNorm gains folded into the projections that consume the normalized rows
+  if (launch_scale_cols(h->w_qkv, h->g1, c.n_layers, h->Nqkv, c.d_model, h->bf16, 0) != cudaSuccess ||
+      launch_scale_cols(h->w_gu, h->g2, c.n_layers, 2 * c.d_ff, c.d_model, h->bf16, 0) != cudaSuccess)
+    return bail(fail(RMT_ECUDA, "gain folding failed"));
   // RoPE table: angle p * theta^(-2i/dh) at segment-local position p, in double precision
   {
     const int half = c.head_dim / 2;
@@ -580,6 +582,10 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
     return bail(fail(RMT_ECUDA, "cudaMemset failed"));
   if (h->bf16) {
     if ((st = build_maps(h)) != RMT_OK) return bail(st);
+    h->ss_parts = (c.d_model / h->bn_o) * 2;  // memo and O projections: N = d_model, two halves per tile
+    if (h->bn_mo != h->bn_o) return bail(fail(RMT_EINVAL, "inconsistent projection tiles"));
+  } else {
+    h->ss_parts = (c.d_model + 127) / 128;  // fp32 kernel: one block per 128-column tile
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return bail(fail(RMT_ECUDA, "weight packing failed"));
   *out = h;

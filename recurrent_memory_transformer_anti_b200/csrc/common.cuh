@@ -61,7 +61,23 @@ struct EpiParams {
   const float2* rope;    // [M, head_dim/2] (cos, sin)
   int rope_cols;         // columns (q and k heads) that get RoPE
   int head_dim;
+  // RMSNorm folded into the GEMMs around it. A residual epilogue with ss_out writes, per row,
+  // the sum of squares of the new residual over each of its column blocks:
+  // ss_out[(layer * M + row) * ss_parts + block]. A RoPE or SwiGLU epilogue with ss_in scales
+  // each accumulator row by rsqrt(sum of that row's ss_parts blocks, in block order,
+  // * inv_d + rms_eps); the RMSNorm gain is folded into the weight columns at pack time.
+  float* ss_out;
+  const float* ss_in;
+  int ss_parts;
+  float inv_d, rms_eps;
 };
+
+// RMSNorm row scale from the per-block sums of squares of one row (fixed summation order).
+__device__ __forceinline__ float rms_row_scale(const float* ss_row, int parts, float inv_d, float eps) {
+  float s = 0.f;
+  for (int t = 0; t < parts; ++t) s += ss_row[t];
+  return rsqrtf(s * inv_d + eps);
+}
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 

@@ -82,7 +82,7 @@ cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st);
 // Partial products of the memory-token rows with [W_mk; W_mv], split along d_model so the
 // reduction order is fixed: part[l][split][r][j] = sum_{k in split} Y[r][k] W_mkv[l][j][k],
 // Y = rows row0 .. row0+n-1 of the cell's output slot.
-constexpr int kMemKvSplit = 64;  // d_model columns per split
+constexpr int kMemKvSplit = 128;  // d_model columns per split
 struct MemKvArgs {
   const float* x;  // [*, M, d] fp32: the residual stream slots (forward) or caller rows
   int M, d, row0, n;
@@ -131,6 +131,8 @@ struct RmsArgs {
 };
 cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st);
 
+// W[l][n][k] *= g[l][k] for l < L (an RMSNorm gain folded into the next projection).
+cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, cudaStream_t st);
 // Layer-0 input of segment s: rows 0..seg-1 from emb, rows seg..M-1 from the memory tokens.
 cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __nv_bfloat16* xb_slot, int seg, int n_mem,
                             int d, int s, bool bf16, cudaStream_t st);

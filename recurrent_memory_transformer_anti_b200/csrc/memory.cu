@@ -19,9 +19,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ----------------------------------------------------------------------------- read
-// CTA = 128 rows of one cell, 8 warps x 16 rows, 4 rows in flight per warp. A and z sit in
-// shared memory; lane j owns output columns j, j+32, ...; q_i reaches all lanes by shuffle.
-constexpr int kReadRows = 128, kReadWarps = 8, kReadBatch = 4;
+// CTA = 32 rows of one cell, 8 warps x 4 rows, all 4 rows of a warp in flight together.
+// A and z sit in shared memory; lane j owns output columns j, j+32, ...; q_i reaches all
+// lanes by shuffle. Small CTAs keep many warps resident: the work per row is a chain of
+// shuffles and FMAs, so latency, not bandwidth, sets the pace.
+constexpr int kReadRows = 32, kReadWarps = 8, kReadBatch = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemReadArgs a) {

@@ -76,7 +76,28 @@ __global__ void emit_kernel(const float* x, T* out, int seg, int d, int s) {
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(x + static_cast<size_t>(r) * d + k));
 }
 
+// W[l][n][k] *= g[l][k]: folds an RMSNorm gain into the weight that consumes its output.
+template <typename T>
+__global__ void scale_cols_kernel(T* w, const T* g, int N, int K) {
+  T* wl = w + static_cast<size_t>(blockIdx.y) * N * K;
+  const T* gl = g + static_cast<size_t>(blockIdx.y) * K;
+  const size_t n = static_cast<size_t>(N) * K;
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x)
+    wl[e] = from_f32<T>(to_f32<T>(wl[e]) * to_f32<T>(gl[e % K]));
+}
+
 }  // namespace
+
+cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, cudaStream_t st) {
+  dim3 grid(1024, L);
+  if (bf16)
+    scale_cols_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<__nv_bfloat16*>(w),
+                                                           static_cast<const __nv_bfloat16*>(g), N, K);
+  else
+    scale_cols_kernel<float><<<grid, 256, 0, st>>>(static_cast<float*>(w), static_cast<const float*>(g), N, K);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;

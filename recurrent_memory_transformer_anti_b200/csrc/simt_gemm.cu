@@ -58,6 +58,15 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
   __syncthreads();
 
   const EpiParams& ep = a.ep;
+  __shared__ float rs[BM];  // folded RMSNorm row scales (RoPE and SwiGLU epilogues)
+  if ((a.epi == kEpiRope || a.epi == kEpiSwiGLU) && t < BM) {
+    const int row = m0 + t;
+    rs[t] = (ep.ss_in && row < a.M)
+                ? rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                                ep.rms_eps)
+                : 1.f;
+  }
+  __syncthreads();
   if (a.epi == kEpiSwiGLU) {
     // output column j of this tile pair: gate at block-start + p, up at block-start + 64 + p
     float* out = static_cast<float*>(ep.out) + static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * a.M * ep.ldo;
@@ -66,7 +75,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
       const int blk = j / kSwiGLUBlock, p = j % kSwiGLUBlock;
       const int cg = blk * 2 * kSwiGLUBlock + p;
       if (m0 + r >= a.M || n0 + cg >= a.N) continue;
-      out[static_cast<size_t>(m0 + r) * ep.ldo + n0 / 2 + j] = silu_f(Cs[r][cg]) * Cs[r][cg + kSwiGLUBlock];
+      out[static_cast<size_t>(m0 + r) * ep.ldo + n0 / 2 + j] = silu_f(Cs[r][cg] * rs[r]) * (Cs[r][cg + kSwiGLUBlock] * rs[r]);
     }
     return;
   }
@@ -83,10 +92,11 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
         break;
       }
       case kEpiRope: {
+        v *= rs[r];
         if (col < ep.rope_cols) {
           const int half = ep.head_dim >> 1, i = col % ep.head_dim;
           const float2 cs = ep.rope[static_cast<size_t>(row) * half + (i % half)];
-          v = i < half ? v * cs.x - Cs[r][cc + half] * cs.y : v * cs.x + Cs[r][cc - half] * cs.y;
+          v = i < half ? v * cs.x - Cs[r][cc + half] * rs[r] * cs.y : v * cs.x + Cs[r][cc - half] * rs[r] * cs.y;
         }
         float* out = static_cast<float*>(ep.out) + static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * a.M * ep.ldo;
         out[static_cast<size_t>(row) * ep.ldo + col] = v;
@@ -96,11 +106,21 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
       case kEpiResidCast: {
         const float* src = ep.x + static_cast<size_t>(cell_index(ep.src_mode, a.L, c)) * a.M * ep.ldx;
         float* dst = ep.x + static_cast<size_t>(cell_index(ep.dst_mode, a.L, c)) * a.M * ep.ldx;
-        dst[static_cast<size_t>(row) * ep.ldx + col] = src[static_cast<size_t>(row) * ep.ldx + col] + v;
+        const float y = src[static_cast<size_t>(row) * ep.ldx + col] + v;
+        dst[static_cast<size_t>(row) * ep.ldx + col] = y;
+        Cs[r][cc] = y;  // kept for the row sums of squares below
         break;
       }
       default:
         break;
+    }
+  }
+  if ((a.epi == kEpiResid || a.epi == kEpiResidCast) && ep.ss_out) {
+    __syncthreads();
+    if (t < BM && m0 + t < a.M) {
+      float ss = 0.f;
+      for (int cc = 0; cc < BN && n0 + cc < a.N; ++cc) ss = fmaf(Cs[t][cc], Cs[t][cc], ss);
+      ep.ss_out[(static_cast<size_t>(c.l) * a.M + m0 + t) * ep.ss_parts + blockIdx.x] = ss;
     }
   }
 }

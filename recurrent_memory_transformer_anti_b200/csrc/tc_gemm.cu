@@ -57,8 +57,8 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 // Epilogue of one 32-column chunk of one row (row per thread). `src` holds the residual
 // values of the chunk for the residual kinds (loaded by the caller before the TMEM wait).
 template <int EPI>
-__device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32],
-                                          const float4 (&src)[8]) {
+__device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32],
+                                           const float4 (&src)[8]) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]);
@@ -81,7 +81,12 @@ __device__ __forceinline__ void epi_chunk(const TcGemmArgs& a, Cell c, int row, 
     }
     store32_f32(dst, v);
     if constexpr (EPI == kEpiResidCast) store32_bf16(ep.xb + (di * a.M + row) * ep.ldx + col, v);
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+    return ss;
   }
+  return 0.f;
 }
 
 // Epilogue of one tile row for column half `part` (0 or 1) of the tile.
@@ -89,6 +94,12 @@ template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0, int part) {
   const bool valid = row < a.M;
   const EpiParams& ep = a.ep;
+  float rs = 1.f;  // folded RMSNorm scale of this row (RoPE and SwiGLU epilogues)
+  if constexpr (EPI == kEpiRope || EPI == kEpiSwiGLU) {
+    if (ep.ss_in && valid)
+      rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                         ep.rms_eps);
+  }
   if constexpr (EPI == kEpiRope) {
     const int dh = ep.head_dim, half = dh >> 1;
     const size_t idx = cell_index(ep.out_mode, a.L, c);
@@ -113,7 +124,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
           const float2* cs = ep.rope + (size_t)row * half + p;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float a1 = u2f(lo[j]), a2 = u2f(hi[j]);
+            const float a1 = u2f(lo[j]) * rs, a2 = u2f(hi[j]) * rs;
             if (rot) {
               const float2 t = cs[j];
               x1[j] = a1 * t.x - a2 * t.y;
@@ -134,7 +145,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
           float x[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float a1 = u2f(r[j]), a2 = u2f(r[j + 16]);
+            const float a1 = u2f(r[j]) * rs, a2 = u2f(r[j + 16]) * rs;
             if (rot) {
               const float2 t = ep.rope[(size_t)row * 16 + j];
               x[j] = a1 * t.x - a2 * t.y;
@@ -164,7 +175,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
       if (valid) {
         float y[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j])) * u2f(up[j]);
+        for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j]) * rs) * (u2f(up[j]) * rs);
         store32_bf16(orow + (n0 + b0) / 2 + p, y);
       }
     }
@@ -174,6 +185,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
     const float* src_row = nullptr;
     if constexpr (EPI == kEpiResid || EPI == kEpiResidCast)
       src_row = ep.x + (static_cast<size_t>(cell_index(ep.src_mode, a.L, c)) * a.M + (valid ? row : 0)) * ep.ldx + n0;
+    float ss = 0.f;
 #pragma unroll 1
     for (int cc = c0; cc < c1; ++cc) {
       uint32_t r[32];
@@ -187,7 +199,11 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         }
       }
       sm100::tmem_wait_ld();
-      if (valid) epi_chunk<EPI>(a, c, row, n0 + cc * 32, r, src);
+      if (valid) ss += epi_chunk<EPI>(a, c, row, n0 + cc * 32, r, src);
+    }
+    if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+      if (ep.ss_out && valid)
+        ep.ss_out[(static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
     }
   }
 }

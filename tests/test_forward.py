@@ -149,3 +149,22 @@ def test_1b_shape_bench_configuration(cuda_ok):
         assert normwise(g, r) < BF16_TOL, name
     assert np.isfinite(full_d[0]).all() and np.isfinite(full_d[1]).all()
     rmt.rmt_destroy(h)
+
+
+@pytest.mark.parametrize("name,S,tol", [("tiny", 3, F32_TOL), ("small-bf16", 3, BF16_TOL)])
+def test_random_rmsnorm_gains_match_oracle(cuda_ok, name, S, tol):
+    """Gains far from 1 exercise the folding of each RMSNorm gain into the next projection."""
+    from armt_synthetic import make_weights, round_to_bf16
+    cfg = CONFIGS[name]
+    w = make_weights(cfg, seed=9)
+    rng = np.random.default_rng(10)
+    for key in ("g_attn", "g_mlp"):
+        g = [np.abs(1 + 0.5 * rng.standard_normal(cfg.d_model)).astype(np.float32) for _ in range(cfg.n_layers)]
+        w[key] = [round_to_bf16(x) for x in g] if cfg.dtype == "bf16" else g
+    w, h = build(cfg, weights=w)
+    emb = embeddings(cfg, S, seed=11)
+    got = forward(h, cfg, emb, S, "diagonal")
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32)
+    for g_, r, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g_, r) < tol, what
+    rmt.rmt_destroy(h)

@@ -42,7 +42,7 @@ def test_noalloc_memory_write_matches_allocating_entry_point(cuda_ok, dtype, G, 
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
-    G, n, d, dk, dv = 64, 16, 2048, 128, 128  # 64*32*16*256*4 B = 32 MiB of partial sums > 8 MiB
+    G, n, d, dk, dv = 64, 16, 2048, 128, 128  # 64*16*16*256*4 B = 16 MiB of partial sums > 8 MiB
     y = torch.zeros((G, n, d), device="cuda")
     w = torch.zeros((G, dk + dv, d), device="cuda")
     A = torch.zeros((G, dk, dv), device="cuda")
