@@ -149,7 +149,7 @@ struct rmt_handle {
        *w_mkv = nullptr, *g1 = nullptr, *g2 = nullptr, *memtok = nullptr;
   // activations and state
   float* x = nullptr;
-  __nv_bfloat16* xb = nullptr;
+  __half* xb = nullptr;  // bf16 mode: f16 operand copy of the residual stream
   void *qkv = nullptr, *att = nullptr, *u = nullptr, *om = nullptr;
   float *qm = nullptr, *part = nullptr, *A = nullptr, *z = nullptr;
   float *ss1 = nullptr, *ss2 = nullptr;  // per-row sums of squares for the folded RMSNorms
@@ -302,17 +302,15 @@ rmt_status build_maps(rmt_handle* h) {
   h->bn_o = tc_pick_bn(c.d_model, kEpiResid, 0);
   h->bn_gu = tc_pick_bn(2 * c.d_ff, kEpiSwiGLU, 0);
   h->bn_d = tc_pick_bn(c.d_model, kEpiResidCast, 0);
-  bool ok = make_tmap_bf16_3d(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) &&
-            make_tmap_bf16_3d(&h->tm_om, h->om, c.d_v, M, L, 128) &&
-            make_tmap_bf16_3d(&h->tm_att, h->att, hd, M, L, 128) &&
-            make_tmap_bf16_3d(&h->tm_u, h->u, F, M, L, 128) &&
-            make_tmap_bf16_3d(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) &&
-            make_tmap_bf16_3d(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->bn_mo) &&
-            make_tmap_bf16_3d(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) &&
-            make_tmap_bf16_3d(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
-            make_tmap_bf16_3d(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) &&
-            make_tmap_bf16_3d(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
-            make_tmap_bf16_3d(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128);
+  auto map = [](CUtensorMap* m, const void* p, uint64_t inner, uint64_t rows, uint64_t depth, uint32_t box) {
+    return make_tmap_16_3d(m, p, inner, rows, depth, box, true);
+  };
+  bool ok = map(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) && map(&h->tm_om, h->om, c.d_v, M, L, 128) &&
+            map(&h->tm_att, h->att, hd, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
+            map(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) && map(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->bn_mo) &&
+            map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) && map(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
+            map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) && map(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
+            map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128);
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
 }
 
@@ -373,7 +371,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   }
   if (h->bf16) {
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
-    return launch_tc_gemm(*ta, *tb, a, bn, st);
+    return launch_tc_gemm(*ta, *tb, a, bn, /*f16=*/true, st);
   }
   const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
   SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, lda, amode, static_cast<const float*>(w), epi, ep};
@@ -419,7 +417,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk), g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es),
                   st, [&] {
                     MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
-                    return launch_mem_read(a, h->bf16, st);
+                    return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st);
                   });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv, g * (m * dv * es + dd * dv * es + 2 * m * dd * 4), st,
@@ -431,8 +429,9 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   e = launch_kind(h, RMT_K_ATTENTION, g * c.n_heads * 4.0 * c.head_dim * m * (m + 1) / 2,
                   g * (m * nq * es + m * hd * es), st, [&] {
                     AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err};
-                    if (h->bf16 && attention_tc_supported(c.head_dim)) return launch_attention_tc(h->tm_qkv, a, st);
-                    return launch_attention(a, h->bf16, st);
+                    if (h->bf16 && attention_tc_supported(c.head_dim))
+                      return launch_attention_tc(h->tm_qkv, a, /*f16=*/true, st);
+                    return launch_attention(a, h->bf16 ? kElemF16 : kElemF32, st);
                   });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd, g * (m * hd * es + dd * hd * es + 2 * m * dd * 4), st,
@@ -557,14 +556,26 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
     if (!*e.p) return bail(fail(RMT_ENOMEM, "device allocation failed"));
   }
   if (h->bf16) {
-    h->xb = static_cast<__nv_bfloat16*>(h->alloc(n_slots(c.n_layers) * M * d * 2));
+    h->xb = static_cast<__half*>(h->alloc(n_slots(c.n_layers) * M * d * 2));
     if (!h->xb) return bail(fail(RMT_ENOMEM, "device allocation failed"));
   }
   rmt_status st = pack_weights(h, weights);
   if (st != RMT_OK) return bail(st);
+  // bf16 mode: the tensor-core operands are f16 (3 more mantissa bits than bf16, same MMA
+  // rate); the bf16 weight values convert exactly (bar magnitudes below 2^-17).
+  if (h->bf16) {
+    const size_t L_ = c.n_layers, d_ = c.d_model, hd_ = size_t(c.n_heads) * c.head_dim, F_ = c.d_ff;
+    const struct {
+      void* p;
+      size_t n;
+    } ops[] = {{h->w_qkv, L_ * h->Nqkv * d_}, {h->w_o, L_ * d_ * hd_},       {h->w_gu, L_ * 2 * F_ * d_},
+               {h->w_d, L_ * d_ * F_},        {h->w_mq, L_ * c.d_k * d_},    {h->w_mo, L_ * d_ * c.d_v}};
+    for (const auto& o : ops)
+      if (launch_bf16_to_f16(o.p, o.n, 0) != cudaSuccess) return bail(fail(RMT_ECUDA, "weight conversion failed"));
+  }
   // RMSNorm gains folded into the projections that consume the normalized rows
-  if (launch_scale_cols(h->w_qkv, h->g1, c.n_layers, h->Nqkv, c.d_model, h->bf16, 0) != cudaSuccess ||
-      launch_scale_cols(h->w_gu, h->g2, c.n_layers, 2 * c.d_ff, c.d_model, h->bf16, 0) != cudaSuccess)
+  if (launch_scale_cols(h->w_qkv, h->g1, c.n_layers, h->Nqkv, c.d_model, h->bf16, h->bf16, 0) != cudaSuccess ||
+      launch_scale_cols(h->w_gu, h->g2, c.n_layers, 2 * c.d_ff, c.d_model, h->bf16, h->bf16, 0) != cudaSuccess)
     return bail(fail(RMT_ECUDA, "gain folding failed"));
   // RoPE table: angle p * theta^(-2i/dh) at segment-local position p, in double precision
   {
@@ -762,7 +773,7 @@ rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t 
   ep.ldo = N;
   ep.out_mode = kByLayer;
   TcGemmArgs a{M, N, K, G, cells, G, kByLayer, static_cast<EpiKind>(epi), ep, err};
-  RMT_CUDA(launch_tc_gemm(ta, tb, a, bn, static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(launch_tc_gemm(ta, tb, a, bn, /*f16=*/false, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }
 
@@ -780,10 +791,10 @@ rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32
     CUtensorMap tm;
     if (!make_tmap_bf16_3d(&tm, qkv, uint64_t(H + 2 * Hkv) * dh, M, G, 128))
       return fail(RMT_EINVAL, "tensor map encoding failed (qkv must be 16-byte aligned)");
-    RMT_CUDA(launch_attention_tc(tm, a, static_cast<cudaStream_t>(stream)));
+    RMT_CUDA(launch_attention_tc(tm, a, /*f16=*/false, static_cast<cudaStream_t>(stream)));
     return RMT_OK;
   }
-  RMT_CUDA(launch_attention(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(launch_attention(a, dtype == RMT_BF16 ? kElemBF16 : kElemF32, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }
 
@@ -796,7 +807,7 @@ rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void*
   const Cell* cells = nullptr;
   RMT_TRY(device_scratch(G, &cells, nullptr));
   MemReadArgs a{q, A, z, o, M, dk, dv, eps, G, cells, kByLayer, kByLayer, G};
-  RMT_CUDA(launch_mem_read(a, dtype == RMT_BF16, static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(launch_mem_read(a, dtype == RMT_BF16 ? kElemBF16 : kElemF32, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }
 

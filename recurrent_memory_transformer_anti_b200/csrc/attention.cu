@@ -5,9 +5,10 @@
 // only through the associative memory (arXiv 2506.05229 abstract: recurrent memory
 // transformers process a long input segment by segment).
 //
-// bf16: flash-attention style, 64 query rows per CTA (16 per warp), key/value tiles of
-// 64 rows double-buffered with cp.async, QK^T and PV on mma.sync m16n8k16 (bf16 in, fp32
-// accumulate), online softmax in fp32 registers.
+// 16-bit (bf16 or f16): flash-attention style, 64 query rows per CTA (16 per warp),
+// key/value tiles of 64 rows double-buffered with cp.async, QK^T and PV on mma.sync
+// m16n8k16 (16-bit in, fp32 accumulate), online softmax in fp32 registers. Used for
+// head_dim 32 (the tensor-core kernel covers 64 and 128).
 // fp32: one thread per query row, key/value chunks staged in shared memory.
 #include "common.cuh"
 #include "launch.h"
@@ -40,20 +41,24 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
                : "r"(a));
 }
 
+template <typename OpT>
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  if constexpr (OpFormat<OpT>::value == 1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
 }
 
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// ------------------------------------------------------------------------ bf16 kernel
+// ---------------------------------------------------------------------- 16-bit kernel
 
 template <int HD>
 struct AttnSmem {
@@ -62,13 +67,13 @@ struct AttnSmem {
   static constexpr int BYTES = (BQ * LDS + 4 * TILE) * 2;
 };
 
-template <int HD>
-__global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
+template <int HD, typename OpT>
+__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   using S = AttnSmem<HD>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __nv_bfloat16* Qs = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* Ks = Qs + S::BQ * S::LDS;  // [2][BKV][LDS]
-  __nv_bfloat16* Vs = Ks + 2 * S::TILE;     // [2][BKV][LDS]
+  OpT* Qs = reinterpret_cast<OpT*>(smem_raw);
+  OpT* Ks = Qs + S::BQ * S::LDS;  // [2][BKV][LDS]
+  OpT* Vs = Ks + 2 * S::TILE;     // [2][BKV][LDS]
 
   const int nqt = (a.M + S::BQ - 1) / S::BQ;
   const int qt = nqt - 1 - blockIdx.x;  // longest rows first
@@ -77,10 +82,10 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
   const int rep = a.H / a.Hkv, kvh = h / rep;
   const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.H * HD;
   const size_t slice = cell_index(a.mode, a.L, c);
-  const __nv_bfloat16* base = static_cast<const __nv_bfloat16*>(a.qkv) + slice * a.M * ldq;
-  const __nv_bfloat16* qsrc = base + h * HD;
-  const __nv_bfloat16* ksrc = base + (a.H + kvh) * HD;
-  const __nv_bfloat16* vsrc = base + (a.H + a.Hkv + kvh) * HD;
+  const OpT* base = static_cast<const OpT*>(a.qkv) + slice * a.M * ldq;
+  const OpT* qsrc = base + h * HD;
+  const OpT* ksrc = base + (a.H + kvh) * HD;
+  const OpT* vsrc = base + (a.H + a.Hkv + kvh) * HD;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q0 = qt * S::BQ;
   constexpr int CH = HD / 8;  // 16-byte chunks per row
@@ -128,8 +133,8 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
       for (int kk = 0; kk < HD / 16; ++kk)
         ldsm_x4(qf[kk], Qs + (warp * 16 + (lane & 15)) * S::LDS + kk * 16 + (lane >> 4) * 8);
     }
-    const __nv_bfloat16* Kb = Ks + buf * S::TILE;
-    const __nv_bfloat16* Vb = Vs + buf * S::TILE;
+    const OpT* Kb = Ks + buf * S::TILE;
+    const OpT* Vb = Vs + buf * S::TILE;
 
     float s[8][4];
 #pragma unroll
@@ -140,8 +145,8 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
       for (int nb = 0; nb < 8; nb += 2) {
         uint32_t b[4];
         ldsm_x4(b, Kb + (nb * 8 + (lane >> 4) * 8 + (lane & 7)) * S::LDS + kk * 16 + ((lane >> 3) & 1) * 8);
-        mma16816(s[nb], qf[kk], b[0], b[1]);
-        mma16816(s[nb + 1], qf[kk], b[2], b[3]);
+        mma16816<OpT>(s[nb], qf[kk], b[0], b[1]);
+        mma16816<OpT>(s[nb + 1], qf[kk], b[2], b[3]);
       }
     }
     // scale, causal mask (and rows of the cell's ragged end), running max
@@ -195,16 +200,16 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
 #pragma unroll
     for (int kk = 0; kk < S::BKV / 16; ++kk) {
       uint32_t pa[4];
-      pa[0] = pack2(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack2(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      pa[0] = pack2<OpT>(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack2<OpT>(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack2<OpT>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack2<OpT>(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
       for (int nd = 0; nd < HD / 8; nd += 2) {
         uint32_t b[4];
         ldsm_x4_t(b, Vb + (kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)) * S::LDS + nd * 8 + (lane >> 4) * 8);
-        mma16816(o[nd], pa, b[0], b[1]);
-        mma16816(o[nd + 1], pa, b[2], b[3]);
+        mma16816<OpT>(o[nd], pa, b[0], b[1]);
+        mma16816<OpT>(o[nd + 1], pa, b[2], b[3]);
       }
     }
     __syncthreads();
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
     lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 1);
     lrow[r] += __shfl_xor_sync(0xffffffffu, lrow[r], 2);
   }
-  __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(a.out) + slice * a.M * ldo + h * HD;
+  OpT* obase = static_cast<OpT*>(a.out) + slice * a.M * ldo + h * HD;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int row = qrow0 + r * 8;
@@ -223,7 +228,7 @@ __global__ void __launch_bounds__(128) attn_bf16_kernel(const AttnArgs a) {
     const float inv = 1.f / lrow[r];
     uint32_t* dst = reinterpret_cast<uint32_t*>(obase + static_cast<size_t>(row) * ldo);
 #pragma unroll
-    for (int nd = 0; nd < HD / 8; ++nd) dst[(nd * 8 + 2 * tq) >> 1] = pack2(o[nd][2 * r] * inv, o[nd][2 * r + 1] * inv);
+    for (int nd = 0; nd < HD / 8; ++nd) dst[(nd * 8 + 2 * tq) >> 1] = pack2<OpT>(o[nd][2 * r] * inv, o[nd][2 * r + 1] * inv);
   }
 }
 
@@ -281,20 +286,20 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
   for (int i = 0; i < HD; ++i) dst[i] = o[i] * inv;
 }
 
-template <int HD>
-cudaError_t launch_bf16(const AttnArgs& a, cudaStream_t st) {
+template <int HD, typename OpT>
+cudaError_t launch_mma(const AttnArgs& a, cudaStream_t st) {
   using S = AttnSmem<HD>;
   static bool attr[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!attr[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+    cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel<HD, OpT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
     if (e != cudaSuccess) return e;
     attr[dev] = true;
   }
   dim3 grid((a.M + S::BQ - 1) / S::BQ, a.H, a.G);
-  attn_bf16_kernel<HD><<<grid, 128, S::BYTES, st>>>(a);
+  attn_mma_kernel<HD, OpT><<<grid, 128, S::BYTES, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -305,15 +310,25 @@ cudaError_t launch_f32(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int HD>
+cudaError_t launch_typed(const AttnArgs& a, ElemType t, cudaStream_t st) {
+  switch (t) {
+    case kElemF32: return launch_f32<HD>(a, st);
+    case kElemBF16: return launch_mma<HD, __nv_bfloat16>(a, st);
+    case kElemF16: return launch_mma<HD, __half>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-cudaError_t launch_attention(const AttnArgs& a, bool bf16, cudaStream_t st) {
+cudaError_t launch_attention(const AttnArgs& a, ElemType t, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;
   if (a.Hkv <= 0 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
   switch (a.dh) {
-    case 32: return bf16 ? launch_bf16<32>(a, st) : launch_f32<32>(a, st);
-    case 64: return bf16 ? launch_bf16<64>(a, st) : launch_f32<64>(a, st);
-    case 128: return bf16 ? launch_bf16<128>(a, st) : launch_f32<128>(a, st);
+    case 32: return launch_typed<32>(a, t, st);
+    case 64: return launch_typed<64>(a, t, st);
+    case 128: return launch_typed<128>(a, t, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -55,7 +55,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
-template <int HD>
+template <int HD, typename OpT>
 __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
   using C = TaCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
@@ -137,8 +137,8 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t tS = tmem_base, tO = tmem_base + 128;
-      constexpr uint32_t idS = sm100::idesc_bf16_f32(128, 128);
-      constexpr uint32_t idO = sm100::idesc_bf16_f32_bmn(128, HD);
+      constexpr uint32_t idS = sm100::idesc_f32acc(128, 128, OpFormat<OpT>::value);
+      constexpr uint32_t idO = sm100::idesc_f32acc_bmn(128, HD, OpFormat<OpT>::value);
       bool ok = sm100::mbar_wait(bar(kQFull), 0, abort_flag);
       auto issue_s = [&](int j) -> bool {
         if (!sm100::mbar_wait(bar(kKFull), j & 1, abort_flag)) return false;
@@ -207,21 +207,26 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
       sm100::mbar_arrive(bar(kSFree));
       const int k0 = j * 128;
       const bool need_mask = (j == qt) || (k0 + 128 > a.M);
-      float mx = -INFINITY;  // max of the raw scores (the scale is positive)
+      // causal mask (and the cell's ragged end) only on the tiles that need it
+      if (need_mask) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kv = k0 + 32 * q4 + i;
+            if (kv > qrow || kv >= a.M) s[q4][i] = __float_as_uint(-INFINITY);
+          }
+        }
+      }
+      // row max and row sum over 4 independent partials (short dependency chains)
+      float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float v = u2f(s[q4][i]);
-          if (need_mask) {
-            const int kv = k0 + 32 * q4 + i;
-            if (kv > qrow || kv >= a.M) v = -INFINITY;
-          }
-          s[q4][i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int i = 0; i < 32; ++i) mxp[i & 3] = fmaxf(mxp[i & 3], u2f(s[q4][i]));
       }
-      mx *= sl2;
+      float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+      mx *= sl2;  // max of the scaled scores (the scale is positive)
       float corr = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -231,16 +236,17 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
         m_use = mx;
         rescale = true;
       }
-      float sum = 0.f;
+      float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float p = ex2(fmaf(u2f(s[q4][i]), sl2, -m_use));
-          sum += p;
+          sp[i & 3] += p;
           s[q4][i] = __float_as_uint(p);
         }
       }
+      const float sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
       l = l * corr + sum;
       if (j > 0) {
         // P of tile j-1 must be consumed (and O final for it) before P and O change
@@ -264,10 +270,10 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         const int q4 = ch >> 2, i0 = (ch & 3) * 8;
-        const uint4 w = make_uint4(pack_bf16(u2f(s[q4][i0]), u2f(s[q4][i0 + 1])),
-                                   pack_bf16(u2f(s[q4][i0 + 2]), u2f(s[q4][i0 + 3])),
-                                   pack_bf16(u2f(s[q4][i0 + 4]), u2f(s[q4][i0 + 5])),
-                                   pack_bf16(u2f(s[q4][i0 + 6]), u2f(s[q4][i0 + 7])));
+        const uint4 w = make_uint4(pack2<OpT>(u2f(s[q4][i0]), u2f(s[q4][i0 + 1])),
+                                   pack2<OpT>(u2f(s[q4][i0 + 2]), u2f(s[q4][i0 + 3])),
+                                   pack2<OpT>(u2f(s[q4][i0 + 4]), u2f(s[q4][i0 + 5])),
+                                   pack2<OpT>(u2f(s[q4][i0 + 6]), u2f(s[q4][i0 + 7])));
         *reinterpret_cast<uint4*>(P + (ch >> 3) * C::SUB + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) = w;
       }
       sm100::fence_async_smem();
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
       sm100::tc_fence_after();
       const float inv = 1.f / l;
       const int ldo = a.H * HD;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.out) + (static_cast<size_t>(slice) * a.M + qrow) * ldo + h * HD;
+      OpT* dst = static_cast<OpT*>(a.out) + (static_cast<size_t>(slice) * a.M + qrow) * ldo + h * HD;
 #pragma unroll 1
       for (int oc = 0; oc < HD / 32; ++oc) {
         uint32_t o[32];
@@ -289,7 +295,7 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = u2f(o[i]) * inv;
-          store32_bf16(dst + 32 * oc, v);
+          store32_16(dst + 32 * oc, v);
         }
       }
     } else if (lane == 0 && a.err) {
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(192, HD == 64 ? 2 : 1) attn_tc_kernel(const __
   }
 }
 
-template <int HD>
+template <int HD, typename OpT>
 cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st) {
   using C = TaCfg<HD>;
   static bool attr[64] = {false};
@@ -313,12 +319,12 @@ cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st)
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!attr[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, OpT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr[dev] = true;
   }
   dim3 grid((a.M + 127) / 128, a.H, a.G);
-  attn_tc_kernel<HD><<<grid, 192, C::SMEM, st>>>(tm, a);
+  attn_tc_kernel<HD, OpT><<<grid, 192, C::SMEM, st>>>(tm, a);
   return cudaGetLastError();
 }
 
@@ -326,11 +332,11 @@ cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st)
 
 bool attention_tc_supported(int dh) { return dh == 64 || dh == 128; }
 
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, bool f16, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;
   if (a.Hkv <= 0 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
-  if (a.dh == 64) return launch_hd<64>(tm_qkv, a, st);
-  if (a.dh == 128) return launch_hd<128>(tm_qkv, a, st);
+  if (a.dh == 64) return f16 ? launch_hd<64, __half>(tm_qkv, a, st) : launch_hd<64, __nv_bfloat16>(tm_qkv, a, st);
+  if (a.dh == 128) return f16 ? launch_hd<128, __half>(tm_qkv, a, st) : launch_hd<128, __nv_bfloat16>(tm_qkv, a, st);
   return cudaErrorInvalidValue;
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -57,7 +58,7 @@ struct EpiParams {
   float* x;              // residual stream base ([n_slots, M, ldx] fp32)
   int ldx;
   IndexMode src_mode, dst_mode;
-  __nv_bfloat16* xb;     // bf16 copy of the residual stream ([n_slots, M, ldx]) or null
+  void* xb;              // operand-type copy of the residual stream ([n_slots, M, ldx]) or null
   const float2* rope;    // [M, head_dim/2] (cos, sin)
   int rope_cols;         // columns (q and k heads) that get RoPE
   int head_dim;
@@ -84,25 +85,42 @@ __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
 
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+// Two fp32 values rounded to a 16-bit type and packed into one 32-bit word (low half first).
+template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 
-// Store 32 consecutive fp32 values as bf16 (64 bytes, four 16-byte stores).
-__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) {
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) { return pack2<__nv_bfloat16>(a, b); }
+
+// Store 32 consecutive fp32 values as a 16-bit type (64 bytes, four 16-byte stores).
+template <typename T>
+__device__ __forceinline__ void store32_16(T* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                      pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+    d[q] = make_uint4(pack2<T>(v[8 * q + 0], v[8 * q + 1]), pack2<T>(v[8 * q + 2], v[8 * q + 3]),
+                      pack2<T>(v[8 * q + 4], v[8 * q + 5]), pack2<T>(v[8 * q + 6], v[8 * q + 7]));
   }
 }
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) { store32_16(dst, v); }
+
+// Tensor-core operand format code of the instruction descriptor (kind::f16): f16 0, bf16 1.
+template <typename T> struct OpFormat;
+template <> struct OpFormat<__half> { static constexpr uint32_t value = 0; };
+template <> struct OpFormat<__nv_bfloat16> { static constexpr uint32_t value = 1; };
 
 // phi(x) = elu(x) + 1
 __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : expf(x); }

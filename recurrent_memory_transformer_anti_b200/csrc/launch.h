@@ -8,6 +8,9 @@
 
 namespace rmt {
 
+// Element type of a buffer handed to a kernel.
+enum ElemType : int { kElemF32 = 0, kElemBF16 = 1, kElemF16 = 2 };
+
 // ------------------------------------------------------------------ grouped GEMMs
 // Group g computes rows 0..M-1 of cell cells[g]: Y = X . W^T with
 //   X = slice cell_index(a_mode, cells[g]) of a [*, M, K] stack,
@@ -23,11 +26,14 @@ struct TcGemmArgs {
   int* err;  // device error word (may be null)
 };
 
-// tensor-core path (bf16 operands in TMA tensor maps)
+// tensor-core path: 16-bit operands (f16 or bf16, one type per launch) in TMA tensor maps
+bool make_tmap_16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                     uint32_t box_rows, bool f16);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                        uint32_t box_rows);
 int tc_pick_bn(int N, int epi, int head_dim);  // 0 if no tile width fits
-cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn,
+// f16: operands (and 16-bit epilogue outputs) are f16, else bf16
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, bool f16,
                            cudaStream_t st);
 
 // fp32 FMA path (fp32 operands by pointer)
@@ -58,10 +64,10 @@ struct AttnArgs {
   int* err;        // device error word for bounded waits (tensor-core kernel), may be null
 };
 // mma.sync (bf16) or fp32 FMA kernels, any head_dim in {32, 64, 128}
-cudaError_t launch_attention(const AttnArgs& a, bool bf16, cudaStream_t st);
-// tcgen05 kernel (bf16, head_dim 64 or 128): tm_qkv maps qkv as [*, M, (H+2Hkv)dh], box 64 x 128
+cudaError_t launch_attention(const AttnArgs& a, ElemType t, cudaStream_t st);
+// tcgen05 kernel (16-bit, head_dim 64 or 128): tm_qkv maps qkv as [*, M, (H+2Hkv)dh], box 64 x 128
 bool attention_tc_supported(int dh);
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, bool f16, cudaStream_t st);
 
 // ------------------------------------------------------------------ associative memory
 struct MemReadArgs {
@@ -77,7 +83,7 @@ struct MemReadArgs {
   IndexMode state_mode;  // slice of A and z
   int L;
 };
-cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_t st);
 
 // Partial products of the memory-token rows with [W_mk; W_mv], split along d_model so the
 // reduction order is fixed: part[l][split][r][j] = sum_{k in split} Y[r][k] W_mkv[l][j][k],
@@ -132,9 +138,13 @@ struct RmsArgs {
 cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st);
 
 // W[l][n][k] *= g[l][k] for l < L (an RMSNorm gain folded into the next projection).
-cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, cudaStream_t st);
-// Layer-0 input of segment s: rows 0..seg-1 from emb, rows seg..M-1 from the memory tokens.
-cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __nv_bfloat16* xb_slot, int seg, int n_mem,
+// W and g share the model's storage type (f32 or bf16), or W is f16 and g bf16 (w_f16).
+cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, bool w_f16, cudaStream_t st);
+// In-place bf16 -> f16 conversion of n elements (the values of a bf16 weight as f16 operands).
+cudaError_t launch_bf16_to_f16(void* p, size_t n, cudaStream_t st);
+// Layer-0 input of segment s: rows 0..seg-1 from emb, rows seg..M-1 from the memory tokens,
+// into the fp32 slot and (if xb_slot) an f16 copy.
+cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __half* xb_slot, int seg, int n_mem,
                             int d, int s, bool bf16, cudaStream_t st);
 // Segment output: rows 0..seg-1 of an fp32 slot, cast to T, to out + s*seg*d.
 cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, bool bf16, cudaStream_t st);

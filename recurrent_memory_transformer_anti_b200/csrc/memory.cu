@@ -212,21 +212,24 @@ __global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdate
 
 }  // namespace
 
-cudaError_t launch_mem_read(const MemReadArgs& a, bool bf16, cudaStream_t st) {
+template <typename T>
+cudaError_t launch_mem_read_t(const MemReadArgs& a, size_t smem, cudaStream_t st) {
+  if (smem > 48 * 1024) cudaFuncSetAttribute(mem_read_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((a.M + kReadRows - 1) / kReadRows, a.G);
+  mem_read_kernel<T><<<grid, kReadWarps * 32, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;
   if (a.dk % 32 || a.dv % 32 || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
   const size_t smem = (static_cast<size_t>(a.dk) * a.dv + a.dk) * sizeof(float);
-  dim3 grid((a.M + kReadRows - 1) / kReadRows, a.G);
-  if (bf16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(mem_read_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    mem_read_kernel<__nv_bfloat16><<<grid, kReadWarps * 32, smem, st>>>(a);
-  } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(mem_read_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    mem_read_kernel<float><<<grid, kReadWarps * 32, smem, st>>>(a);
+  switch (out_type) {
+    case kElemF32: return launch_mem_read_t<float>(a, smem, st);
+    case kElemBF16: return launch_mem_read_t<__nv_bfloat16>(a, smem, st);
+    case kElemF16: return launch_mem_read_t<__half>(a, smem, st);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {

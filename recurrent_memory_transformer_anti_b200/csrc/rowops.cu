@@ -16,6 +16,15 @@ template <> struct Vec4<float> {
   static __device__ __forceinline__ void store(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
   static __device__ __forceinline__ float4 load(const float* p) { return *reinterpret_cast<const float4*>(p); }
 };
+template <> struct Vec4<__half> {
+  static __device__ __forceinline__ void store(__half* p, float4 v) {
+    __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
 template <> struct Vec4<__nv_bfloat16> {
   static __device__ __forceinline__ void store(__nv_bfloat16* p, float4 v) {
     __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
@@ -59,13 +68,13 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a
 
 // Layer-0 input of segment s: embeddings of the segment, then the memory tokens.
 template <typename T>
-__global__ void assemble_kernel(const T* emb, const T* mem, float* x, __nv_bfloat16* xb, int seg, int d, int s) {
+__global__ void assemble_kernel(const T* emb, const T* mem, float* x, __half* xb, int seg, int d, int s) {
   const int r = blockIdx.x;
   const T* src = r < seg ? emb + (static_cast<size_t>(s) * seg + r) * d : mem + static_cast<size_t>(r - seg) * d;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
     const float4 v = Vec4<T>::load(src + k);
     Vec4<float>::store(x + static_cast<size_t>(r) * d + k, v);
-    if (xb) Vec4<__nv_bfloat16>::store(xb + static_cast<size_t>(r) * d + k, v);
+    if (xb) Vec4<__half>::store(xb + static_cast<size_t>(r) * d + k, v);
   }
 }
 
@@ -77,25 +86,42 @@ __global__ void emit_kernel(const float* x, T* out, int seg, int d, int s) {
 }
 
 // W[l][n][k] *= g[l][k]: folds an RMSNorm gain into the weight that consumes its output.
-template <typename T>
-__global__ void scale_cols_kernel(T* w, const T* g, int N, int K) {
-  T* wl = w + static_cast<size_t>(blockIdx.y) * N * K;
-  const T* gl = g + static_cast<size_t>(blockIdx.y) * K;
+template <typename WT, typename GT>
+__global__ void scale_cols_kernel(WT* w, const GT* g, int N, int K) {
+  WT* wl = w + static_cast<size_t>(blockIdx.y) * N * K;
+  const GT* gl = g + static_cast<size_t>(blockIdx.y) * K;
   const size_t n = static_cast<size_t>(N) * K;
   for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
        e += static_cast<size_t>(gridDim.x) * blockDim.x)
-    wl[e] = from_f32<T>(to_f32<T>(wl[e]) * to_f32<T>(gl[e % K]));
+    wl[e] = from_f32<WT>(to_f32<WT>(wl[e]) * to_f32<GT>(gl[e % K]));
+}
+
+__global__ void bf16_to_f16_kernel(uint16_t* p, size_t n) {
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float v = __uint_as_float(static_cast<uint32_t>(p[e]) << 16);
+    const __half hv = __float2half_rn(v);
+    p[e] = *reinterpret_cast<const uint16_t*>(&hv);
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, cudaStream_t st) {
+cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, bool w_f16, cudaStream_t st) {
   dim3 grid(1024, L);
-  if (bf16)
-    scale_cols_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<__nv_bfloat16*>(w),
-                                                           static_cast<const __nv_bfloat16*>(g), N, K);
+  if (bf16 && w_f16)
+    scale_cols_kernel<__half, __nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<__half*>(w),
+                                                                    static_cast<const __nv_bfloat16*>(g), N, K);
+  else if (bf16)
+    scale_cols_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<__nv_bfloat16*>(w),
+                                                                           static_cast<const __nv_bfloat16*>(g), N, K);
   else
-    scale_cols_kernel<float><<<grid, 256, 0, st>>>(static_cast<float*>(w), static_cast<const float*>(g), N, K);
+    scale_cols_kernel<float, float><<<grid, 256, 0, st>>>(static_cast<float*>(w), static_cast<const float*>(g), N, K);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_to_f16(void* p, size_t n, cudaStream_t st) {
+  bf16_to_f16_kernel<<<2048, 256, 0, st>>>(static_cast<uint16_t*>(p), n);
   return cudaGetLastError();
 }
 
@@ -110,7 +136,7 @@ cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __nv_bfloat16* xb_slot, int seg, int n_mem,
+cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __half* xb_slot, int seg, int n_mem,
                             int d, int s, bool bf16, cudaStream_t st) {
   if (d % 4) return cudaErrorInvalidValue;
   const int threads = d >= 1024 ? 256 : 128;

@@ -126,19 +126,21 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 accumulator.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
+// Instruction descriptor, kind::f16 with an fp32 accumulator: A and B both of format `fmt`
+// (0 = f16, 1 = bf16; the two operands of one MMA always share a type), both K-major.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int m, int n, uint32_t fmt) {
   return (1u << 4)                                   // D format: f32
-         | (1u << 7)                                 // A format: bf16
-         | (1u << 10)                                // B format: bf16
+         | (fmt << 7)                                // A format
+         | (fmt << 10)                               // B format
          | (static_cast<uint32_t>(n >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);    // M / 16
 }
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) { return idesc_f32acc(m, n, 1u); }
 
-// As idesc_bf16_f32, with B given MN-major (N contiguous in shared memory) instead of
+// As idesc_f32acc, with B given MN-major (N contiguous in shared memory) instead of
 // K-major. Used for the attention product P.V, where V is stored [kv rows][head dims].
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int m, int n) {
-  return idesc_bf16_f32(m, n) | (1u << 16);
+__host__ __device__ constexpr uint32_t idesc_f32acc_bmn(int m, int n, uint32_t fmt) {
+  return idesc_f32acc(m, n, fmt) | (1u << 16);
 }
 
 // Shared-memory descriptor of an MN-major operand with the 128-byte swizzle: rows of 128 B

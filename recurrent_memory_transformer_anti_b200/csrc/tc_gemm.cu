@@ -56,7 +56,7 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 // Epilogue of one 32-column chunk of one row (row per thread). `src` holds the residual
 // values of the chunk for the residual kinds (loaded by the caller before the TMEM wait).
-template <int EPI>
+template <int EPI, typename OpT>
 __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32],
                                            const float4 (&src)[8]) {
   float v[32];
@@ -68,7 +68,7 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
     store32_f32(static_cast<float*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
   } else if constexpr (EPI == kEpiStoreAct) {
     const size_t idx = cell_index(ep.out_mode, a.L, c);
-    store32_bf16(static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
+    store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
   } else if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
     const size_t di = cell_index(ep.dst_mode, a.L, c);
     float* dst = ep.x + (di * a.M + row) * ep.ldx + col;
@@ -80,7 +80,7 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
       v[4 * q + 3] += src[q].w;
     }
     store32_f32(dst, v);
-    if constexpr (EPI == kEpiResidCast) store32_bf16(ep.xb + (di * a.M + row) * ep.ldx + col, v);
+    if constexpr (EPI == kEpiResidCast) store32_16(static_cast<OpT*>(ep.xb) + (di * a.M + row) * ep.ldx + col, v);
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
@@ -90,7 +90,7 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
 }
 
 // Epilogue of one tile row for column half `part` (0 or 1) of the tile.
-template <int BN, int EPI>
+template <int BN, int EPI, typename OpT>
 __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0, int part) {
   const bool valid = row < a.M;
   const EpiParams& ep = a.ep;
@@ -103,7 +103,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
   if constexpr (EPI == kEpiRope) {
     const int dh = ep.head_dim, half = dh >> 1;
     const size_t idx = cell_index(ep.out_mode, a.L, c);
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
+    OpT* orow = static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo;
     const int heads = BN / dh;
     // rotation pairs (i, i + dh/2) of each head, in 32-wide units: heads * max(1, half/32)
     const int per_head = half >= 32 ? half / 32 : 1;
@@ -121,12 +121,14 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         sm100::tmem_wait_ld();
         if (valid) {
           float x1[32], x2[32];
-          const float2* cs = ep.rope + (size_t)row * half + p;
+          // (cos, sin) of two frequencies per 16-byte load
+          const float4* cs = reinterpret_cast<const float4*>(ep.rope + (size_t)row * half + p);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float a1 = u2f(lo[j]) * rs, a2 = u2f(hi[j]) * rs;
             if (rot) {
-              const float2 t = cs[j];
+              const float4 t4 = cs[j >> 1];
+              const float2 t = (j & 1) ? make_float2(t4.z, t4.w) : make_float2(t4.x, t4.y);
               x1[j] = a1 * t.x - a2 * t.y;
               x2[j] = a2 * t.x + a1 * t.y;
             } else {
@@ -134,8 +136,8 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
               x2[j] = a2;
             }
           }
-          store32_bf16(orow + n0 + h0 + p, x1);
-          store32_bf16(orow + n0 + h0 + half + p, x2);
+          store32_16(orow + n0 + h0 + p, x1);
+          store32_16(orow + n0 + h0 + half + p, x2);
         }
       } else {  // head_dim 32: both halves of the head in one 32-column chunk
         uint32_t r[32];
@@ -155,13 +157,13 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
               x[j + 16] = a2;
             }
           }
-          store32_bf16(orow + n0 + h0, x);
+          store32_16(orow + n0 + h0, x);
         }
       }
     }
   } else if constexpr (EPI == kEpiSwiGLU) {
     const size_t idx = cell_index(ep.out_mode, a.L, c);
-    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(ep.out) + (idx * a.M + row) * ep.ldo;
+    OpT* orow = static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo;
     constexpr int per_blk = kSwiGLUBlock / 32;  // 32-wide output units per gate/up block pair
     constexpr int units = (BN / (2 * kSwiGLUBlock)) * per_blk;
     const int u0 = part * units / 2, u1 = (part + 1) * units / 2;
@@ -176,7 +178,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         float y[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j]) * rs) * (u2f(up[j]) * rs);
-        store32_bf16(orow + (n0 + b0) / 2 + p, y);
+        store32_16(orow + (n0 + b0) / 2 + p, y);
       }
     }
   } else {
@@ -199,7 +201,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         }
       }
       sm100::tmem_wait_ld();
-      if (valid) ss += epi_chunk<EPI>(a, c, row, n0 + cc * 32, r, src);
+      if (valid) ss += epi_chunk<EPI, OpT>(a, c, row, n0 + cc * 32, r, src);
     }
     if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
       if (ep.ss_out && valid)
@@ -208,7 +210,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, typename OpT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcGemmArgs args) {
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = sm100::idesc_bf16_f32(C::BM, BN);
+      constexpr uint32_t idesc = sm100::idesc_f32acc(C::BM, BN, OpFormat<OpT>::value);
       int stage = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       bool ok = true;
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int n_tile = r / mt, m_tile = r % mt;
       const Cell c = args.cells[g];
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_tile<BN, EPI>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
+      epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(tempty_bar(acc));
@@ -381,7 +383,7 @@ int sm_count_cached() {
   return count[dev];
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, typename OpT>
 cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
   using C = TcCfg<BN>;
   static bool attr_set[64] = {false};
@@ -389,7 +391,7 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI, OpT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -398,23 +400,34 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   const long tiles = static_cast<long>(args.G) * mt * (args.N / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
-  tc_gemm_kernel<BN, EPI><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, args);
+  tc_gemm_kernel<BN, EPI, OpT><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, args);
   return cudaGetLastError();
 }
 
-template <int BN>
+template <int BN, typename OpT>
 cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
   switch (args.epi) {
-    case kEpiStoreF32: return launch_bn_epi<BN, kEpiStoreF32>(ta, tb, args, st);
-    case kEpiStoreAct: return launch_bn_epi<BN, kEpiStoreAct>(ta, tb, args, st);
-    case kEpiResid: return launch_bn_epi<BN, kEpiResid>(ta, tb, args, st);
-    case kEpiResidCast: return launch_bn_epi<BN, kEpiResidCast>(ta, tb, args, st);
+    case kEpiStoreF32: return launch_bn_epi<BN, kEpiStoreF32, OpT>(ta, tb, args, st);
+    case kEpiStoreAct: return launch_bn_epi<BN, kEpiStoreAct, OpT>(ta, tb, args, st);
+    case kEpiResid: return launch_bn_epi<BN, kEpiResid, OpT>(ta, tb, args, st);
+    case kEpiResidCast: return launch_bn_epi<BN, kEpiResidCast, OpT>(ta, tb, args, st);
     case kEpiRope:
-      if constexpr (BN >= 64) return launch_bn_epi<BN, kEpiRope>(ta, tb, args, st);
+      if constexpr (BN >= 64) return launch_bn_epi<BN, kEpiRope, OpT>(ta, tb, args, st);
       break;
     case kEpiSwiGLU:
-      if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU>(ta, tb, args, st);
+      if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU, OpT>(ta, tb, args, st);
       break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename OpT>
+cudaError_t launch_op(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, cudaStream_t st) {
+  switch (bn) {
+    case 256: return launch_bn<256, OpT>(ta, tb, args, st);
+    case 128: return launch_bn<128, OpT>(ta, tb, args, st);
+    case 64: return launch_bn<64, OpT>(ta, tb, args, st);
+    case 32: return launch_bn<32, OpT>(ta, tb, args, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -433,18 +446,23 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 }  // namespace
 
-bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
-                       uint32_t box_rows) {
+bool make_tmap_16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                     uint32_t box_rows, bool f16) {
   auto encode = get_encode_fn();
   if (!encode || !base || inner % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
   cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                       uint32_t box_rows) {
+  return make_tmap_16_3d(map, base, inner, rows, depth, box_rows, false);
 }
 
 int tc_pick_bn(int N, int epi, int head_dim) {
@@ -458,16 +476,10 @@ int tc_pick_bn(int N, int epi, int head_dim) {
   return 0;
 }
 
-cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn,
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, bool f16,
                            cudaStream_t st) {
   if (args.K % 64 != 0 || args.M <= 0) return cudaErrorInvalidValue;
-  switch (bn) {
-    case 256: return launch_bn<256>(ta, tb, args, st);
-    case 128: return launch_bn<128>(ta, tb, args, st);
-    case 64: return launch_bn<64>(ta, tb, args, st);
-    case 32: return launch_bn<32>(ta, tb, args, st);
-  }
-  return cudaErrorInvalidValue;
+  return f16 ? launch_op<__half>(ta, tb, args, bn, st) : launch_op<__nv_bfloat16>(ta, tb, args, bn, st);
 }
 
 }  // namespace rmt

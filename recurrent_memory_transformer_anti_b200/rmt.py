@@ -144,7 +144,7 @@ class Handle:
         self.cfg = cfg
 
     def __del__(self):
-        if getattr(self, "ptr", None):
+        if getattr(self, "ptr", None) and _lib is not None:  # the module may be torn down at exit
             _lib.rmt_destroy(self.ptr)
             self.ptr = None
 
