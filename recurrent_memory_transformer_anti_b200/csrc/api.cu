@@ -164,7 +164,7 @@ struct rmt_handle {
   void* out_stage = nullptr;
   size_t out_stage_bytes = 0;
   std::map<std::pair<int, int>, Table> tables;
-  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv;
+  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
   std::vector<void*> allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
@@ -310,7 +310,8 @@ rmt_status build_maps(rmt_handle* h) {
             map(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) && map(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->bn_mo) &&
             map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) && map(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
             map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) && map(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
-            map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128);
+            map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
+            make_tmap_f32_resid(&h->tm_x, h->x, d, M, n_slots(c.n_layers));
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
 }
 
@@ -371,7 +372,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   }
   if (h->bf16) {
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
-    return launch_tc_gemm(*ta, *tb, a, bn, /*f16=*/true, st);
+    return launch_tc_gemm(*ta, *tb, h->tm_x, a, bn, /*f16=*/true, st);
   }
   const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
   SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, lda, amode, static_cast<const float*>(w), epi, ep};
@@ -773,7 +774,7 @@ rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t 
   ep.ldo = N;
   ep.out_mode = kByLayer;
   TcGemmArgs a{M, N, K, G, cells, G, kByLayer, static_cast<EpiKind>(epi), ep, err};
-  RMT_CUDA(launch_tc_gemm(ta, tb, a, bn, /*f16=*/false, static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(launch_tc_gemm(ta, tb, ta, a, bn, /*f16=*/false, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }
 

@@ -32,9 +32,12 @@ bool make_tmap_16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                        uint32_t box_rows);
 int tc_pick_bn(int N, int epi, int head_dim);  // 0 if no tile width fits
-// f16: operands (and 16-bit epilogue outputs) are f16, else bf16
-cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, bool f16,
-                           cudaStream_t st);
+// Residual-stream map for the residual epilogues: fp32 [depth, rows, inner], 32 x 32 boxes.
+bool make_tmap_f32_resid(CUtensorMap* map, const float* base, uint64_t inner, uint64_t rows, uint64_t depth);
+// f16: operands (and 16-bit epilogue outputs) are f16, else bf16. tx: the residual-stream map
+// (read and written by the residual epilogues; any valid map otherwise).
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
+                           int bn, bool f16, cudaStream_t st);
 
 // fp32 FMA path (fp32 operands by pointer)
 struct SimtGemmArgs {

@@ -34,8 +34,12 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int BAR_BYTES = 128 * ((8 * (2 * STAGES + 5) + 16 + 127) / 128);
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int NBAR = 2 * STAGES + 5 + 8;  // ring, accumulators, drain, one per epilogue warp
+  static constexpr int BAR_BYTES = 1024 * ((8 * NBAR + 16 + 1023) / 1024);
+  static constexpr int EPI_BUF = 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 residual block
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + EPI_OFF + 8 * EPI_BUF;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 namespace {
@@ -210,10 +214,75 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
   }
 }
 
+// Residual epilogue of one warp (tile rows rowbase .. rowbase+31, one per lane) over its
+// column half, through TMA: each 32 x 32 block of the residual stream is loaded into the
+// warp's swizzled shared block, the accumulator rows are added in place, and the block is
+// stored back with one bulk copy; the operand-type copy goes out with plain stores.
+template <int BN, int EPI, typename OpT>
+__device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CUtensorMap* tmX, uint32_t tacc, Cell c,
+                                                   int rowbase, int n0, int part, int lane, uint8_t* buf,
+                                                   uint32_t buf_s, uint32_t rbar, uint32_t& rph,
+                                                   volatile int* abort_flag) {
+  const EpiParams& ep = a.ep;
+  if (rowbase >= a.M) return true;  // the whole block lies past the cell
+  const int row = rowbase + lane;
+  const bool valid = row < a.M;
+  const int src = cell_index(ep.src_mode, a.L, c), dst = cell_index(ep.dst_mode, a.L, c);
+  constexpr int chunks = BN / 32;
+  const int c0 = part * chunks / 2, c1 = (part + 1) * chunks / 2;
+  float4* rowp = reinterpret_cast<float4*>(buf + lane * 128);
+  float ss = 0.f;
+#pragma unroll 1
+  for (int cc = c0; cc < c1; ++cc) {
+    const int col = n0 + cc * 32;
+    if (lane == 0) {
+      sm100::bulk_wait_read_all();  // the previous store has read the block
+      sm100::mbar_arrive_expect_tx(rbar, 32 * 32 * 4);
+      sm100::tma_load_3d(buf_s, tmX, col, rowbase, src, rbar);
+    }
+    uint32_t r[32];
+    sm100::tmem_ld32(tacc + cc * 32, r);
+    sm100::tmem_wait_ld();
+    if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar, rph, abort_flag))) {
+      if (lane == 0) sm100::mbar_wait_drain(rbar, rph);  // let the load land before the block is reused
+      return false;
+    }
+    rph ^= 1u;
+    float y[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 xv = rowp[q ^ (lane & 7)];  // 128-byte swizzle: chunk q of row r sits at q ^ (r % 8)
+      xv.x += u2f(r[4 * q]);
+      xv.y += u2f(r[4 * q + 1]);
+      xv.z += u2f(r[4 * q + 2]);
+      xv.w += u2f(r[4 * q + 3]);
+      rowp[q ^ (lane & 7)] = xv;
+      y[4 * q] = xv.x;
+      y[4 * q + 1] = xv.y;
+      y[4 * q + 2] = xv.z;
+      y[4 * q + 3] = xv.w;
+    }
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss = fmaf(y[j], y[j], ss);
+      if constexpr (EPI == kEpiResidCast)
+        store32_16(static_cast<OpT*>(ep.xb) + ((size_t)dst * a.M + row) * ep.ldx + col, y);
+    }
+    sm100::fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      sm100::tma_store_3d(tmX, buf_s, col, rowbase, dst);
+      sm100::bulk_commit();
+    }
+  }
+  if (ep.ss_out && valid) ep.ss_out[(static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
+  return true;
+}
+
 template <int BN, int EPI, typename OpT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmX, const TcGemmArgs args) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = sm100::smem_u32(smem_raw);
@@ -225,7 +294,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES + 8 * (2 * C::STAGES + 5));
+  auto resid_bar = [&](int w) { return bar0 + 8u * (2 * C::STAGES + 5 + w); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -239,6 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::mbar_init(tempty_bar(a), kEpiWarps);
     }
     sm100::mbar_init(drain_bar, 1);
+    for (int w = 0; w < kEpiWarps; ++w) sm100::mbar_init(resid_bar(w), 1);
     *abort_flag = 0;
     sm100::fence_barrier_init();
     sm100::fence_proxy_async_smem();
@@ -342,10 +413,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31 belong to this warp
     const int part = (warp - 2) / 4;     // column half of the tile handled by this warpgroup
+    const int ew = warp - 2;
+    uint8_t* rbuf = smem + C::EPI_OFF + ew * C::EPI_BUF;
+    const uint32_t rbuf_s = base + C::EPI_OFF + ew * C::EPI_BUF;
+    uint32_t rph = 0;
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      const bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
+      bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
       if (!ok) {
         if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
         break;
@@ -355,7 +430,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int n_tile = r / mt, m_tile = r % mt;
       const Cell c = args.cells[g];
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
+      if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+        ok = epilogue_resid_tma<BN, EPI, OpT>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
+                                              lane, rbuf, rbuf_s, resid_bar(ew), rph, abort_flag);
+        if (!ok) {
+          if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
+          break;
+        }
+      } else {
+        epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
+      }
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(tempty_bar(acc));
@@ -364,6 +448,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         aph ^= 1u;
       }
     }
+    if (lane == 0) sm100::bulk_wait_all();  // residual stores complete before the CTA leaves
   }
 
   sm100::tc_fence_before();
@@ -384,7 +469,8 @@ int sm_count_cached() {
 }
 
 template <int BN, int EPI, typename OpT>
-cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
+cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
+                          cudaStream_t st) {
   using C = TcCfg<BN>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -400,34 +486,36 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   const long tiles = static_cast<long>(args.G) * mt * (args.N / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
-  tc_gemm_kernel<BN, EPI, OpT><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, args);
+  tc_gemm_kernel<BN, EPI, OpT><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, tx, args);
   return cudaGetLastError();
 }
 
 template <int BN, typename OpT>
-cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, cudaStream_t st) {
+cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
+                      cudaStream_t st) {
   switch (args.epi) {
-    case kEpiStoreF32: return launch_bn_epi<BN, kEpiStoreF32, OpT>(ta, tb, args, st);
-    case kEpiStoreAct: return launch_bn_epi<BN, kEpiStoreAct, OpT>(ta, tb, args, st);
-    case kEpiResid: return launch_bn_epi<BN, kEpiResid, OpT>(ta, tb, args, st);
-    case kEpiResidCast: return launch_bn_epi<BN, kEpiResidCast, OpT>(ta, tb, args, st);
+    case kEpiStoreF32: return launch_bn_epi<BN, kEpiStoreF32, OpT>(ta, tb, tx, args, st);
+    case kEpiStoreAct: return launch_bn_epi<BN, kEpiStoreAct, OpT>(ta, tb, tx, args, st);
+    case kEpiResid: return launch_bn_epi<BN, kEpiResid, OpT>(ta, tb, tx, args, st);
+    case kEpiResidCast: return launch_bn_epi<BN, kEpiResidCast, OpT>(ta, tb, tx, args, st);
     case kEpiRope:
-      if constexpr (BN >= 64) return launch_bn_epi<BN, kEpiRope, OpT>(ta, tb, args, st);
+      if constexpr (BN >= 64) return launch_bn_epi<BN, kEpiRope, OpT>(ta, tb, tx, args, st);
       break;
     case kEpiSwiGLU:
-      if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU, OpT>(ta, tb, args, st);
+      if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU, OpT>(ta, tb, tx, args, st);
       break;
   }
   return cudaErrorInvalidValue;
 }
 
 template <typename OpT>
-cudaError_t launch_op(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, cudaStream_t st) {
+cudaError_t launch_op(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
+                      int bn, cudaStream_t st) {
   switch (bn) {
-    case 256: return launch_bn<256, OpT>(ta, tb, args, st);
-    case 128: return launch_bn<128, OpT>(ta, tb, args, st);
-    case 64: return launch_bn<64, OpT>(ta, tb, args, st);
-    case 32: return launch_bn<32, OpT>(ta, tb, args, st);
+    case 256: return launch_bn<256, OpT>(ta, tb, tx, args, st);
+    case 128: return launch_bn<128, OpT>(ta, tb, tx, args, st);
+    case 64: return launch_bn<64, OpT>(ta, tb, tx, args, st);
+    case 32: return launch_bn<32, OpT>(ta, tb, tx, args, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -476,10 +564,23 @@ int tc_pick_bn(int N, int epi, int head_dim) {
   return 0;
 }
 
-cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& args, int bn, bool f16,
-                           cudaStream_t st) {
+bool make_tmap_f32_resid(CUtensorMap* map, const float* base, uint64_t inner, uint64_t rows, uint64_t depth) {
+  auto encode = get_encode_fn();
+  if (!encode || !base || inner % 32 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {inner * 4, inner * rows * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
+                           int bn, bool f16, cudaStream_t st) {
   if (args.K % 64 != 0 || args.M <= 0) return cudaErrorInvalidValue;
-  return f16 ? launch_op<__half>(ta, tb, args, bn, st) : launch_op<__nv_bfloat16>(ta, tb, args, bn, st);
+  return f16 ? launch_op<__half>(ta, tb, tx, args, bn, st) : launch_op<__nv_bfloat16>(ta, tb, tx, args, bn, st);
 }
 
 }  // namespace rmt
