@@ -155,6 +155,7 @@ struct rmt_handle {
   float *ss1 = nullptr, *ss2 = nullptr;  // per-row sums of squares for the folded RMSNorms
   int ss_parts = 0;
   float2* rope = nullptr;
+  __half2* rope_h = nullptr;  // (cos, sin) as f16 pairs for the tensor-core RoPE epilogue
   int* err = nullptr;
   int* trace = nullptr;
   size_t trace_cap = 0;
@@ -164,7 +165,7 @@ struct rmt_handle {
   void* out_stage = nullptr;
   size_t out_stage_bytes = 0;
   std::map<std::pair<int, int>, Table> tables;
-  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x;
+  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
   std::vector<void*> allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
@@ -311,7 +312,8 @@ rmt_status build_maps(rmt_handle* h) {
             map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) && map(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
             map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) && map(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
-            make_tmap_f32_resid(&h->tm_x, h->x, d, M, n_slots(c.n_layers));
+            make_tmap_f32_resid(&h->tm_x, h->x, d, M, n_slots(c.n_layers)) &&
+            (c.head_dim < 64 || map(&h->tm_rope, h->rope_h, c.head_dim, M, 1, 32));
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
 }
 
@@ -371,8 +373,10 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       break;
   }
   if (h->bf16) {
+    const bool rope_tma = p == kProjQkv && c.head_dim >= 64;
+    ep.rope_tma = rope_tma;
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
-    return launch_tc_gemm(*ta, *tb, h->tm_x, a, bn, /*f16=*/true, st);
+    return launch_tc_gemm(*ta, *tb, rope_tma ? h->tm_rope : h->tm_x, a, bn, /*f16=*/true, st);
   }
   const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
   SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, lda, amode, static_cast<const float*>(w), epi, ep};
@@ -550,6 +554,7 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
       {reinterpret_cast<void**>(&h->A), L * dk * dv * 4},
       {reinterpret_cast<void**>(&h->z), L * dk * 4},
       {reinterpret_cast<void**>(&h->rope), M * (c.head_dim / 2) * sizeof(float2)},
+      {reinterpret_cast<void**>(&h->rope_h), M * (c.head_dim / 2) * sizeof(__half2)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
   };
   for (auto& e : plan) {
@@ -587,7 +592,10 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
         const double ang = double(p) * std::pow(double(c.rope_theta), -2.0 * i / c.head_dim);
         tab[p * half + i] = make_float2(float(std::cos(ang)), float(std::sin(ang)));
       }
-    if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess)
+    std::vector<__half2> tab_h(tab.size());
+    for (size_t i = 0; i < tab.size(); ++i) tab_h[i] = __floats2half2_rn(tab[i].x, tab[i].y);
+    if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(h->rope_h, tab_h.data(), tab_h.size() * sizeof(__half2), cudaMemcpyHostToDevice) != cudaSuccess)
       return bail(fail(RMT_ECUDA, "rope table upload failed"));
   }
   if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(h->x, 0, n_slots(c.n_layers) * M * d * 4) != cudaSuccess)

@@ -62,6 +62,7 @@ struct EpiParams {
   const float2* rope;    // [M, head_dim/2] (cos, sin)
   int rope_cols;         // columns (q and k heads) that get RoPE
   int head_dim;
+  int rope_tma;          // tensor-core kernel: (cos, sin) come as f16 pairs through the tx map
   // RMSNorm folded into the GEMMs around it. A residual epilogue with ss_out writes, per row,
   // the sum of squares of the new residual over each of its column blocks:
   // ss_out[(layer * M + row) * ss_parts + block]. A RoPE or SwiGLU epilogue with ss_in scales

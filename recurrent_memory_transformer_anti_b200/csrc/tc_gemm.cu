@@ -279,6 +279,78 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
   return true;
 }
 
+// RoPE epilogue of one warp (tile rows rowbase .. rowbase+31, one per lane) over its share
+// of the tile's heads. The (cos, sin) pairs of the warp's 32 rows and 32 frequencies come
+// into the warp's shared block with one TMA load (f16 pairs, 128-byte rows, swizzled) and
+// are reused for every head of the tile; units are ordered frequency block first, so a
+// warp loads each block once per tile. Only for head_dim >= 64.
+template <int BN, typename OpT>
+__device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUtensorMap* tmR, uint32_t tacc, Cell c,
+                                                  int rowbase, int n0, int part, int lane, const uint8_t* buf,
+                                                  uint32_t buf_s, uint32_t rbar, uint32_t& rph,
+                                                  volatile int* abort_flag) {
+  const EpiParams& ep = a.ep;
+  if (rowbase >= a.M) return true;
+  const int row = rowbase + lane;
+  const bool valid = row < a.M;
+  const int dh = ep.head_dim, half = dh >> 1;
+  const int heads = BN / dh, per_head = half / 32, units = heads * per_head;
+  const int u0 = part * units / 2, u1 = (part + 1) * units / 2;
+  float rs = 1.f;
+  if (ep.ss_in && valid)
+    rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                       ep.rms_eps);
+  const size_t idx = cell_index(ep.out_mode, a.L, c);
+  OpT* orow = static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo;
+  const uint4* rowp = reinterpret_cast<const uint4*>(buf + lane * 128);
+  int loaded = -1;
+#pragma unroll 1
+  for (int u = u0; u < u1; ++u) {
+    const int pb = u / heads, h0 = (u % heads) * dh, p = pb * 32;
+    const bool rot = (n0 + h0) < ep.rope_cols;
+    if (rot && pb != loaded) {
+      if (lane == 0) {
+        sm100::mbar_arrive_expect_tx(rbar, 32 * 32 * 4);
+        sm100::tma_load_3d(buf_s, tmR, 2 * p, rowbase, 0, rbar);
+      }
+      if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar, rph, abort_flag))) {
+        if (lane == 0) sm100::mbar_wait_drain(rbar, rph);
+        return false;
+      }
+      rph ^= 1u;
+      loaded = pb;
+    }
+    uint32_t lo[32], hi[32];
+    sm100::tmem_ld32(tacc + h0 + p, lo);
+    sm100::tmem_ld32(tacc + h0 + half + p, hi);
+    sm100::tmem_wait_ld();
+    if (valid) {
+      float x1[32], x2[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of the row holds frequencies 4q .. 4q+3
+        const uint4 w = rowp[q ^ (lane & 7)];
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * q + e;
+          const float a1 = u2f(lo[j]) * rs, a2 = u2f(hi[j]) * rs;
+          if (rot) {
+            const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&wv[e]));
+            x1[j] = a1 * t.x - a2 * t.y;
+            x2[j] = a2 * t.x + a1 * t.y;
+          } else {
+            x1[j] = a1;
+            x2[j] = a2;
+          }
+        }
+      }
+      store32_16(orow + n0 + h0 + p, x1);
+      store32_16(orow + n0 + h0 + half + p, x2);
+    }
+  }
+  return true;
+}
+
 template <int BN, int EPI, typename OpT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -433,6 +505,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
         ok = epilogue_resid_tma<BN, EPI, OpT>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
                                               lane, rbuf, rbuf_s, resid_bar(ew), rph, abort_flag);
+        if (!ok) {
+          if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
+          break;
+        }
+      } else if (EPI == kEpiRope && args.ep.rope_tma) {
+        ok = epilogue_rope_tma<BN, OpT>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part, lane,
+                                        rbuf, rbuf_s, resid_bar(ew), rph, abort_flag);
         if (!ok) {
           if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
           break;
