@@ -170,8 +170,9 @@ const char* rmt_last_error(void);
  *   C[g] = A[g] . B[g]^T for g in 0..G-1, bf16 inputs, fp32 accumulation.
  * A [G, M, K] bf16, B [G, N, K] bf16 (a distinct weight per group, [out, in]),
  * C [G, M, N] in out_dtype (RMT_F32 or RMT_BF16). Needs K % 64 == 0 and N % 64 == 0;
- * M is arbitrary (ragged last tile). Pointers 16-byte aligned. "Architecture Overview":
- * GroupedGEMM operations batched across layers within a diagonal. */
+ * M is arbitrary (ragged last tile). Pointers 16-byte aligned. When N % 256 == 0 the
+ * product runs on CTA pairs (2-SM MMAs, tokens along the MMA's N), else on single CTAs.
+ * "Architecture Overview": GroupedGEMM operations batched across layers within a diagonal. */
 rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t G, int32_t M,
                                  int32_t N, int32_t K, rmt_dtype out_dtype, void* stream);
 

@@ -166,7 +166,12 @@ struct rmt_handle {
   size_t out_stage_bytes = 0;
   std::map<std::pair<int, int>, Table> tables;
   CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
+  // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
+  CUtensorMap tp_xb, tp_om, tp_att, tp_u;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
+  // bf16 mode: projections that run on the CTA-pair GEMM (decided before packing, which
+  // depends on it for the RoPE and SwiGLU row orders)
+  bool pair_mo = false, pair_qkv = false, pair_o = false, pair_gu = false, pair_d = false;
   std::vector<void*> allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
   struct ProbeRec {
@@ -271,16 +276,33 @@ rmt_status pack_weights(rmt_handle* h, const rmt_weights* w) {
     return static_cast<char*>(base) + (l * elems_per_layer + off) * es;
   };
   const size_t nqkv = size_t(h->Nqkv);
+  // pair packing of a rotated projection: rows p and p + dh/2 of each head go to 2p, 2p + 1
+  auto copy_rope_pairs = [&](char* dst, const void* src, size_t heads, const char* what) -> rmt_status {
+    if (!src) return fail(RMT_EINVAL, std::string("null weight pointer: ") + what);
+    const size_t row = d * es, dh = c.head_dim, half = dh / 2;
+    for (size_t hh = 0; hh < heads; ++hh) {
+      const char* s0 = static_cast<const char*>(src) + hh * dh * row;
+      char* d0 = dst + hh * dh * row;
+      RMT_CUDA(cudaMemcpy2D(d0, 2 * row, s0, row, row, half, cudaMemcpyDefault));
+      RMT_CUDA(cudaMemcpy2D(d0 + row, 2 * row, s0 + half * row, row, row, half, cudaMemcpyDefault));
+    }
+    return RMT_OK;
+  };
   for (size_t l = 0; l < L; ++l) {
-    RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l), w->wq[l], hd * d * es, "wq"));
-    RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, hd * d), w->wk[l], kvd * d * es, "wk"));
+    if (h->pair_qkv) {
+      RMT_TRY(copy_rope_pairs(at(h->w_qkv, nqkv * d, l), w->wq[l], c.n_heads, "wq"));
+      RMT_TRY(copy_rope_pairs(at(h->w_qkv, nqkv * d, l, hd * d), w->wk[l], c.n_kv_heads, "wk"));
+    } else {
+      RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l), w->wq[l], hd * d * es, "wq"));
+      RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, hd * d), w->wk[l], kvd * d * es, "wk"));
+    }
     RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, (hd + kvd) * d), w->wv[l], kvd * d * es, "wv"));
     RMT_TRY(copy_in(at(h->w_o, d * hd, l), w->wo[l], d * hd * es, "wo"));
-    // gate/up interleaved in blocks of kSwiGLUBlock rows: [g0 u0 g1 u1 ...]
+    // gate/up interleaved: row by row for the pair GEMM, else in blocks of kSwiGLUBlock rows
     if (!w->w_gate[l] || !w->w_up[l]) return fail(RMT_EINVAL, "null w_gate/w_up");
-    const size_t blk = size_t(kSwiGLUBlock) * d * es;
-    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l), 2 * blk, w->w_gate[l], blk, blk, F / kSwiGLUBlock, cudaMemcpyDefault));
-    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l) + blk, 2 * blk, w->w_up[l], blk, blk, F / kSwiGLUBlock,
+    const size_t rows = h->pair_gu ? 1 : kSwiGLUBlock, blk = rows * d * es;
+    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l), 2 * blk, w->w_gate[l], blk, blk, F / rows, cudaMemcpyDefault));
+    RMT_CUDA(cudaMemcpy2D(at(h->w_gu, 2 * F * d, l) + blk, 2 * blk, w->w_up[l], blk, blk, F / rows,
                           cudaMemcpyDefault));
     RMT_TRY(copy_in(at(h->w_d, d * F, l), w->w_down[l], d * F * es, "w_down"));
     RMT_TRY(copy_in(at(h->w_mq, dk * d, l), w->w_mq[l], dk * d * es, "w_mq"));
@@ -306,11 +328,19 @@ rmt_status build_maps(rmt_handle* h) {
   auto map = [](CUtensorMap* m, const void* p, uint64_t inner, uint64_t rows, uint64_t depth, uint32_t box) {
     return make_tmap_16_3d(m, p, inner, rows, depth, box, true);
   };
+  // weight boxes: 128 rows per CTA on the pair GEMM, else the tile width
+  const uint32_t pb = static_cast<uint32_t>(pair_token_tile(static_cast<int>(M)) / 2);
+  const bool any_pair = h->pair_mo || h->pair_qkv || h->pair_o || h->pair_gu || h->pair_d;
   bool ok = map(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) && map(&h->tm_om, h->om, c.d_v, M, L, 128) &&
             map(&h->tm_att, h->att, hd, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
-            map(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) && map(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->bn_mo) &&
-            map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->bn_qkv) && map(&h->tm_wo, h->w_o, hd, d, L, h->bn_o) &&
-            map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->bn_gu) && map(&h->tm_wd, h->w_d, F, d, L, h->bn_d) &&
+            map(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) &&
+            map(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->pair_mo ? 128 : h->bn_mo) &&
+            map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->pair_qkv ? 128 : h->bn_qkv) &&
+            map(&h->tm_wo, h->w_o, hd, d, L, h->pair_o ? 128 : h->bn_o) &&
+            map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->pair_gu ? 128 : h->bn_gu) &&
+            map(&h->tm_wd, h->w_d, F, d, L, h->pair_d ? 128 : h->bn_d) &&
+            (!any_pair || (map(&h->tp_xb, h->xb, d, M, n_slots(c.n_layers), pb) && map(&h->tp_om, h->om, c.d_v, M, L, pb) &&
+                           map(&h->tp_att, h->att, hd, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
             make_tmap_f32_resid(&h->tm_x, h->x, d, M, n_slots(c.n_layers)) &&
             (c.head_dim < 64 || map(&h->tm_rope, h->rope_h, c.head_dim, M, 1, 32));
@@ -338,8 +368,9 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   IndexMode amode = kByLayer;
   const float* a32 = nullptr;
   const void* w = nullptr;
-  const CUtensorMap *ta = nullptr, *tb = nullptr;
+  const CUtensorMap *ta = nullptr, *tb = nullptr, *tp = nullptr;
   int bn = 0;
+  bool pair = false;
   switch (p) {
     case kProjMemQ:
       N = c.d_k, K = d, epi = kEpiStoreF32, amode = kInSlot;
@@ -350,27 +381,36 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       N = d, K = c.d_v, epi = resid;
       ep.src_mode = kInSlot, ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss1;
       a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
+      tp = &h->tp_om, pair = h->pair_mo;
       break;
     case kProjQkv:  // rows of x_out scaled by RMSNorm 1 (gain folded into the weight), then RoPE
       N = h->Nqkv, K = d, epi = kEpiRope, amode = kOutSlot;
       ep.out = h->qkv, ep.ldo = h->Nqkv, ep.ss_in = h->ss1;
       a32 = h->x, w = h->w_qkv, ta = &h->tm_xb, tb = &h->tm_wqkv, bn = h->bn_qkv;
+      tp = &h->tp_xb, pair = h->pair_qkv;
       break;
     case kProjO:  // x_out += attention output; emits the row sums of squares of RMSNorm 2
       N = d, K = hd, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss2;
       a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
+      tp = &h->tp_att, pair = h->pair_o;
       break;
     case kProjGateUp:  // rows of x_out scaled by RMSNorm 2 (gain folded into the weight), SwiGLU
       N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU, amode = kOutSlot;
       ep.out = h->u, ep.ldo = c.d_ff, ep.ss_in = h->ss2;
       a32 = h->x, w = h->w_gu, ta = &h->tm_xb, tb = &h->tm_wgu, bn = h->bn_gu;
+      tp = &h->tp_xb, pair = h->pair_gu;
       break;
     case kProjDown:  // x_out += MLP output; the bf16 copy feeds the next layer's memory query
       N = d, K = c.d_ff, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb;
       a32 = static_cast<const float*>(h->u), w = h->w_d, ta = &h->tm_u, tb = &h->tm_wd, bn = h->bn_d;
+      tp = &h->tp_u, pair = h->pair_d;
       break;
+  }
+  if (h->bf16 && pair) {
+    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
+    return launch_tc_pair_gemm(*tb, *tp, a, /*f16=*/true, st);
   }
   if (h->bf16) {
     const bool rope_tma = p == kProjQkv && c.head_dim >= 64;
@@ -564,6 +604,16 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   if (h->bf16) {
     h->xb = static_cast<__half*>(h->alloc(n_slots(c.n_layers) * M * d * 2));
     if (!h->xb) return bail(fail(RMT_ENOMEM, "device allocation failed"));
+  }
+  if (h->bf16) {
+    const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
+    // the memory read-out projection (K = d_v) is a pure stream over the residual; it stays on
+    // the single-CTA kernel, whose residual epilogue moves whole blocks through TMA
+    h->pair_mo = false;
+    h->pair_qkv = tc_pair_supported(Mi, h->Nqkv, di, kEpiRope, c.head_dim);
+    h->pair_o = tc_pair_supported(Mi, di, hdi, kEpiResidCast, 0);
+    h->pair_gu = tc_pair_supported(Mi, 2 * Fi, di, kEpiSwiGLU, 0);
+    h->pair_d = tc_pair_supported(Mi, di, Fi, kEpiResidCast, 0);
   }
   rmt_status st = pack_weights(h, weights);
   if (st != RMT_OK) return bail(st);
@@ -774,14 +824,21 @@ rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t 
   RMT_TRY(device_scratch(G, &cells, &err));
   CUtensorMap ta, tb;
   const int epi = out_dtype == RMT_F32 ? kEpiStoreF32 : kEpiStoreAct;
-  const int bn = tc_pick_bn(N, epi, 0);
-  if (!make_tmap_bf16_3d(&ta, A, K, M, G, 128) || !make_tmap_bf16_3d(&tb, B, K, N, G, bn))
-    return fail(RMT_EINVAL, "tensor map encoding failed (pointers must be 16-byte aligned)");
   EpiParams ep{};
   ep.out = C;
   ep.ldo = N;
   ep.out_mode = kByLayer;
   TcGemmArgs a{M, N, K, G, cells, G, kByLayer, static_cast<EpiKind>(epi), ep, err};
+  if (tc_pair_supported(M, N, K, epi, 0)) {  // widths in multiples of 256: CTA-pair kernel
+    if (!make_tmap_bf16_3d(&ta, A, K, M, G, static_cast<uint32_t>(pair_token_tile(M) / 2)) ||
+        !make_tmap_bf16_3d(&tb, B, K, N, G, 128))
+      return fail(RMT_EINVAL, "tensor map encoding failed (pointers must be 16-byte aligned)");
+    RMT_CUDA(launch_tc_pair_gemm(tb, ta, a, /*f16=*/false, static_cast<cudaStream_t>(stream)));
+    return RMT_OK;
+  }
+  const int bn = tc_pick_bn(N, epi, 0);
+  if (!make_tmap_bf16_3d(&ta, A, K, M, G, 128) || !make_tmap_bf16_3d(&tb, B, K, N, G, bn))
+    return fail(RMT_EINVAL, "tensor map encoding failed (pointers must be 16-byte aligned)");
   RMT_CUDA(launch_tc_gemm(ta, tb, ta, a, bn, /*f16=*/false, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
 }

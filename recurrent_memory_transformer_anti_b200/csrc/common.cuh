@@ -51,6 +51,17 @@ enum EpiKind : int {
 
 constexpr int kSwiGLUBlock = 64;
 
+// Token tile of the CTA-pair GEMM (tokens along the MMA's N): the cell's M rows split into
+// ceil(M / 256) near-equal tiles, each rounded up to a multiple of 16 (M = 1040 gives 5 x 208,
+// no padding). The pair kernel packs its projections differently from the other GEMMs:
+// RoPE partners (i, i + head_dim/2) of each rotated head sit on adjacent weight rows
+// (2p, 2p + 1), and gate/up rows alternate (gate_j at 2j, up_j at 2j + 1).
+__host__ __device__ inline int pair_token_tile(int M) {
+  const int n = (M + 255) / 256;
+  const int t = (M + n - 1) / n;
+  return (t + 15) / 16 * 16;
+}
+
 struct EpiParams {
   void* out;             // kEpiStore*, kEpiRope, kEpiSwiGLU output (stacked [*, M, ldo])
   int ldo;               // output row stride (elements)

@@ -39,6 +39,13 @@ bool make_tmap_f32_resid(CUtensorMap* map, const float* base, uint64_t inner, ui
 cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
                            int bn, bool f16, cudaStream_t st);
 
+// CTA-pair path (features along M, tokens along N): tw maps the [L, N, K] weights with
+// 128-row boxes, tx the [*, M, K] activations with pair_token_tile(M)/2-row boxes. RoPE and
+// SwiGLU expect the pair packing described with pair_token_tile.
+bool tc_pair_supported(int M, int N, int K, int epi, int head_dim);
+cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, bool f16,
+                                cudaStream_t st);
+
 // fp32 FMA path (fp32 operands by pointer)
 struct SimtGemmArgs {
   int M, N, K;

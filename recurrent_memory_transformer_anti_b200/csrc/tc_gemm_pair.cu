@@ -1,0 +1,550 @@
+// Grouped GEMM on CTA pairs (tcgen05.mma.cta_group::2, sm_100a), transposed orientation.
+//
+// "Architecture Overview" of the diagonal-batching skill page: the products of all layers on
+// one diagonal run as one GroupedGEMM launch, each group (one (layer, segment) cell) with its
+// own layer's weights. This kernel computes each group's Y^T = W_l . X^T: output features run
+// along the MMA's M (256 per CTA pair, 128 per CTA) and the cell's tokens along N, in tiles of
+// pair_token_tile(M) tokens. Two things follow from that orientation:
+//   * a cell of M = 1040 rows needs no padding tile (N is any multiple of 16 up to 256);
+//   * one TMEM lane holds one output feature over consecutive tokens, so each epilogue
+//     instruction of a warp reads or writes 32 consecutive features of one token row.
+// The pair halves the bytes each SM fetches per MMA: each CTA loads 128 weight rows and half
+// of the token rows, and the MMA reads the other token half from the peer's shared memory.
+//
+// Roles per CTA (320 threads, one CTA per SM, persistent over pair tiles):
+//   warp 0      one thread issues the TMA loads of this CTA's weight half (128 rows) and token
+//               half (NT/2 rows), 128 K-columns per ring stage (two 64-column swizzle blocks);
+//               both CTAs' byte counts complete on the even CTA's barrier, which the even CTA
+//               arms for the pair;
+//   warp 1      TMEM (512 columns: two accumulators 256 apart); in the even CTA one thread
+//               issues the pair MMAs (M = 256, N = tile tokens, K = 16), 8 per stage, and
+//               releases each stage to both CTAs with one commit;
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (32 features) over one
+//               half of the tile's tokens, 16 or 32 tokens per step, with the global loads
+//               a step needs issued before its TMEM wait.
+// Every wait is bounded (see sm100.cuh); on a timeout the CTA records it in the error word,
+// stops issuing work and meets its peer at the final cluster barrier before freeing TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace rmt {
+namespace {
+
+// Shared memory: [barriers 1 KB][sums of squares 8 KB][row scales 2 KB][ring], 1024-aligned.
+// A ring stage holds two 64-column blocks, each this CTA's weight half (16 KB) and token half
+// (NT/2 rows of 128 B, rounded to 1 KB); the ring takes as many stages as fit (3 at NT = 208).
+// Fewer, wider stages beat more, narrower ones: each commit stalls the MMA pipe for a while.
+// Each stage is released by one commit that arrives on the empty barriers of both CTAs.
+struct PairCfg {
+  static constexpr int FM = 128;               // weight rows (output features) per CTA
+  static constexpr int BK = 64;                // K-columns per swizzle block
+  static constexpr int W_BYTES = FM * BK * 2;  // 16 KB
+  static constexpr int MAX_STAGES = 8;
+  static constexpr int ACC_COLS = 256;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int NBAR = 2 * MAX_STAGES + 2 + 2 + 2 + 1;  // ring, tfull, tempty, warpgroup sync, drain
+  static constexpr int BAR_BYTES = 1024;
+  static constexpr int RED_OFF = BAR_BYTES;  // [2 acc][2 wg][4 quarters][128] fp32
+  static constexpr int RED_BYTES = 2 * 2 * 4 * 128 * 4;
+  static constexpr int RS_OFF = RED_OFF + RED_BYTES;  // [2 acc][2 wg][128] fp32 row scales
+  static constexpr int RS_BYTES = 2 * 2 * 128 * 4;
+  static constexpr int RING_OFF = RS_OFF + RS_BYTES;
+  static constexpr int SMEM_BYTES = 232448;  // the per-block maximum; the ring fills the rest
+  static constexpr int RING_BYTES = SMEM_BYTES - 1024 - RING_OFF;
+  static_assert(8 * NBAR + 16 <= BAR_BYTES, "barrier area");
+  static_assert(RING_OFF % 1024 == 0, "ring alignment");
+  __host__ __device__ static int x_bytes(int NT) { return ((NT / 2) * BK * 2 + 1023) / 1024 * 1024; }
+  __host__ __device__ static int block_bytes(int NT) { return W_BYTES + x_bytes(NT); }
+  __host__ __device__ static int stages(int NT) {
+    const int s = RING_BYTES / (2 * block_bytes(NT));
+    return s < MAX_STAGES ? s : MAX_STAGES;
+  }
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// silu(x) = x / (1 + e^-x) with the fast exponential and division intrinsics (relative error
+// of a few 1e-7; for x below about -87 the quotient is 0, the limit of silu): the epilogue
+// shares issue slots with the MMA issuer, so its instruction count shows in the GEMM's time.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// Per-token sums of s[0..15] over the warp's 32 lanes (15 + 1 shuffles, fixed order): token t
+// ends up in lanes 2t and 2t + 1.
+__device__ __forceinline__ float warp_sum16_transposed(float (&s)[16], int lane) {
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    const bool hi = lane & (2 * o);
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float keep = hi ? s[o + k] : s[k];
+      const float give = hi ? s[k] : s[o + k];
+      s[k] = keep + __shfl_xor_sync(0xffffffffu, give, 2 * o);
+    }
+  }
+  return s[0] + __shfl_xor_sync(0xffffffffu, s[0], 1);
+}
+
+// RMSNorm row scale from one row of per-block sums of squares, with every load of the row in
+// flight at once when the row is a whole number of 16-byte vectors (at most 32 blocks).
+__device__ __forceinline__ float row_scale(const float* ss_row, int parts, float inv_d, float eps) {
+  if ((parts & 3) == 0 && parts <= 32) {
+    const float4* p = reinterpret_cast<const float4*>(ss_row);
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 4 * i < parts ? p[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s = (((s + v[i].x) + v[i].y) + v[i].z) + v[i].w;
+    return rsqrtf(s * inv_d + eps);
+  }
+  return rms_row_scale(ss_row, parts, inv_d, eps);
+}
+
+// Epilogue of one warp: its 32 features (f = this lane's output column) over tokens
+// tok0 .. tok0 + cnt - 1 of the cell (cnt a multiple of 8, at most 128), accumulator columns
+// from tacc. A step covers 32 columns; columns past cnt (at most 24) are read, not stored.
+template <int EPI, typename OpT>
+__device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint32_t tacc, int tok0, int cnt, int f,
+                                              int lane, const float* rs, float* red) {
+  const EpiParams& ep = a.ep;
+  const int M = a.M;
+  const int lim = min(cnt, M - tok0);  // valid tokens of this warp's range
+  if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+    // 16 tokens per step; the next step's residual loads go out before this step's TMEM wait
+    const size_t si = cell_index(ep.src_mode, a.L, c), di = cell_index(ep.dst_mode, a.L, c);
+    const float* src = ep.x + (si * M + tok0) * ep.ldx + f;
+    float* dst = ep.x + (di * M + tok0) * ep.ldx + f;
+    OpT* xb = nullptr;
+    if constexpr (EPI == kEpiResidCast) xb = static_cast<OpT*>(ep.xb) + (di * M + tok0) * ep.ldx + f;
+    const bool want_ss = ep.ss_out != nullptr;
+    float xs[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) xs[j] = j < lim ? src[static_cast<size_t>(j) * ep.ldx] : 0.f;
+#pragma unroll 1
+    for (int j0 = 0; j0 < cnt; j0 += 16) {
+      uint32_t r[16];
+      sm100::tmem_ld16(tacc + j0, r);
+      float xn[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) xn[j] = j0 + 16 + j < lim ? src[static_cast<size_t>(j0 + 16 + j) * ep.ldx] : 0.f;
+      sm100::tmem_wait_ld();
+      float sq[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float y = xs[j] + u2f(r[j]);
+        if (j0 + j < lim) {
+          dst[static_cast<size_t>(j0 + j) * ep.ldx] = y;
+          if constexpr (EPI == kEpiResidCast) xb[static_cast<size_t>(j0 + j) * ep.ldx] = from_f32<OpT>(y);
+        }
+        sq[j] = j0 + j < lim ? y * y : 0.f;
+        xs[j] = xn[j];
+      }
+      if (want_ss) {
+        const float s = warp_sum16_transposed(sq, lane);
+        if ((lane & 1) == 0 && j0 + (lane >> 1) < cnt) red[j0 + (lane >> 1)] = s;
+      }
+    }
+  } else if constexpr (EPI == kEpiStoreF32 || EPI == kEpiStoreAct) {
+    const size_t o0 = (cell_index(ep.out_mode, a.L, c) * static_cast<size_t>(M) + tok0) * ep.ldo + f;
+#pragma unroll 1
+    for (int j0 = 0; j0 < cnt; j0 += 32) {
+      uint32_t r[32];
+      sm100::tmem_ld32(tacc + j0, r);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j0 + j < lim) {
+          const size_t o = o0 + static_cast<size_t>(j0 + j) * ep.ldo;
+          if constexpr (EPI == kEpiStoreF32)
+            static_cast<float*>(ep.out)[o] = u2f(r[j]);
+          else
+            static_cast<OpT*>(ep.out)[o] = from_f32<OpT>(u2f(r[j]));
+        }
+      }
+    }
+  } else if constexpr (EPI == kEpiRope) {
+    // lanes 2p and 2p + 1 of a rotated head hold the pair (x_p, x_{p + dh/2}). The angle of
+    // token t is t * theta_p: each step reads (cos, sin) at its first token from the table and
+    // advances one token at a time by the rotation of position 1 (complex multiplication in
+    // fp32; 31 steps add a few units of 1e-6 of error), so a step needs two table reads.
+    const int dh = ep.head_dim, hh = dh >> 1;
+    const int i = f % dh, p = i >> 1;
+    const bool odd = i & 1, rot = f < ep.rope_cols;
+    OpT* out = static_cast<OpT*>(ep.out) + (static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * M + tok0) * ep.ldo + f;
+    const float2 step = (rot && M > 1) ? ep.rope[hh + p] : make_float2(1.f, 0.f);
+#pragma unroll 1
+    for (int j0 = 0; j0 < cnt; j0 += 32) {
+      float2 cs = (rot && j0 < lim) ? ep.rope[static_cast<size_t>(tok0 + j0) * hh + p] : make_float2(1.f, 0.f);
+      uint32_t r[32];
+      sm100::tmem_ld32(tacc + j0, r);
+      sm100::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float x = u2f(r[j]) * rs[j0 + j];
+        const float other = __shfl_xor_sync(0xffffffffu, x, 1);
+        const float y = odd ? fmaf(x, cs.x, other * cs.y) : fmaf(x, cs.x, -other * cs.y);
+        if (j0 + j < lim) out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
+        cs = make_float2(fmaf(cs.x, step.x, -cs.y * step.y), fmaf(cs.y, step.x, cs.x * step.y));
+      }
+    }
+  } else if constexpr (EPI == kEpiSwiGLU) {
+    // even lanes hold gate_j, odd lanes up_j (j = f / 2); after one exchange the even lane
+    // finishes tokens 0..15 of the step and the odd lane tokens 16..31
+    const bool odd = lane & 1;
+    OpT* out = static_cast<OpT*>(ep.out) + (static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * M + tok0) * ep.ldo +
+               (f >> 1);
+#pragma unroll 1
+    for (int j0 = 0; j0 < cnt; j0 += 32) {
+      uint32_t r[32];
+      sm100::tmem_ld32(tacc + j0, r);
+      sm100::tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]) * rs[j0 + j];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float got = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[16 + j], 1);
+        const float g = odd ? got : v[j], u = odd ? v[16 + j] : got;
+        const int t = j0 + (odd ? 16 : 0) + j;
+        if (t < lim) out[static_cast<size_t>(t) * ep.ldo] = from_f32<OpT>(silu_fast(g) * u);
+      }
+    }
+  }
+}
+
+template <int EPI, typename OpT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                        const TcGemmArgs args) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = sm100::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bar0 = base;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::MAX_STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::MAX_STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::MAX_STAGES + 2 + a); };
+  auto wg_bar = [&](int w) { return bar0 + 8u * (2 * C::MAX_STAGES + 4 + w); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::MAX_STAGES + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int M = args.M;
+  const int NT = pair_token_tile(M);
+  const int STAGES = C::stages(NT);
+  const uint32_t BLK = static_cast<uint32_t>(C::block_bytes(NT));
+  const uint32_t ring = base + C::RING_OFF;
+
+  const uint32_t rank = sm100::cluster_ctarank();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      sm100::mbar_init(full_bar(s), 1);
+      sm100::mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      sm100::mbar_init(tfull_bar(a), 1);
+      sm100::mbar_init(tempty_bar(a), 2 * C::EPI_WARPS);  // the epilogue warps of both CTAs
+      sm100::mbar_init(wg_bar(a), 4);
+    }
+    sm100::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+    sm100::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tmW);
+    sm100::tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) sm100::tmem_alloc_pair(sm100::smem_u32(tmem_slot), C::TMEM_COLS);
+  sm100::tc_fence_before();
+  sm100::cluster_sync();  // both CTAs' barriers initialised and TMEM allocated before any remote use
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int ntt = (M + NT - 1) / NT;
+  const int npair = args.N / 256;
+  const int kblk = args.K / C::BK;  // 64-column blocks
+  const int kst = (kblk + 1) / 2;   // ring stages per tile (the last may hold one block)
+  const int tiles = args.G * npair * ntt;
+  const int cl = static_cast<int>(sm100::cluster_id_x()), ncl = static_cast<int>(sm100::cluster_count_x());
+  // tokens of token tile tt (the last one rounded up to 16; rows past M read as zeros)
+  auto tile_tokens = [&](int tt) {
+    const int rem = M - tt * NT;
+    return rem >= NT ? NT : ((rem + 15) & ~15);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t blk_tx = 2u * (C::W_BYTES + static_cast<uint32_t>(NT / 2) * C::BK * 2);  // one block, both CTAs
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      auto acquire = [&]() { return sm100::mbar_wait(empty_bar(stage), ph ^ 1u, abort_flag); };
+      for (int t = cl; t < tiles && ok; t += ncl) {
+        const int g = t / (npair * ntt), r = t % (npair * ntt);
+        const int fp = r / ntt, tt = r % ntt;
+        const Cell c = args.cells[g];
+        const int a3 = cell_index(args.a_mode, args.L, c);
+        const int wrow = fp * 256 + static_cast<int>(rank) * C::FM;
+        const int xrow = tt * NT + static_cast<int>(rank) * (tile_tokens(tt) / 2);
+        for (int ks = 0; ks < kst; ++ks) {
+          if (!acquire()) {
+            ok = false;
+            break;
+          }
+          const int nb = (2 * ks + 1 < kblk) ? 2 : 1;
+          if (rank == 0) sm100::mbar_arrive_expect_tx(full_bar(stage), static_cast<uint32_t>(nb) * blk_tx);
+          const uint32_t sa = ring + static_cast<uint32_t>(stage) * 2u * BLK;
+          const uint32_t fb = sm100::mapa_shared(full_bar(stage), 0);
+          for (int b = 0; b < nb; ++b) {
+            sm100::tma_load_3d_pair(sa + b * BLK, &tmW, (2 * ks + b) * C::BK, wrow, c.l, fb);
+            sm100::tma_load_3d_pair(sa + b * BLK + C::W_BYTES, &tmX, (2 * ks + b) * C::BK, xrow, a3, fb);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // every stage's last fill consumed: no MMA can still read this CTA's ring and no commit
+      // can still arrive on it
+      for (int i = 0; i < STAGES && ok; ++i) {
+        ok = acquire();
+        if (++stage == STAGES) {
+          stage = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) {
+        if (args.err) atomicOr(args.err, kErrTimeoutProducer);
+        // copies already issued complete on the even CTA's barriers, which this CTA cannot
+        // wait on: give them a millisecond to land before shared memory can be released
+        const uint64_t t0 = sm100::global_timer_ns();
+        while (sm100::global_timer_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc0 = sm100::idesc_f32acc(256, 0, OpFormat<OpT>::value);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      bool ok = true;
+      for (int t = cl; t < tiles && ok; t += ncl) {
+        const int tt = (t % (npair * ntt)) % ntt;
+        const uint32_t idesc = idesc0 | (static_cast<uint32_t>(tile_tokens(tt) >> 3) << 17);
+        if (!sm100::mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::ACC_COLS);
+        for (int ks = 0; ks < kst; ++ks) {
+          if (!sm100::mbar_wait(full_bar(stage), ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const int nb = (2 * ks + 1 < kblk) ? 2 : 1;
+          const uint32_t sa = ring + static_cast<uint32_t>(stage) * 2u * BLK;
+          for (int b = 0; b < nb; ++b) {
+            const uint64_t adesc = sm100::smem_desc_k128(sa + b * BLK);
+            const uint64_t bdesc = sm100::smem_desc_k128(sa + b * BLK + C::W_BYTES);
+#pragma unroll
+            for (int k = 0; k < C::BK / 16; ++k)
+              sm100::mma_pair(d_tmem, adesc + 2ull * k, bdesc + 2ull * k, idesc, (ks | b | k) != 0);
+          }
+          sm100::mma_commit_pair_cta_mask(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::mma_commit_pair_cta_mask(tfull_bar(acc), 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      if (!ok) {
+        if (args.err) atomicOr(args.err, kErrTimeoutMma);
+        sm100::mma_commit_pair(sm100::mapa_shared(drain_bar, 0));
+        sm100::mbar_wait_drain(drain_bar, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;    // TMEM lanes 32 * quarter .. +31 belong to this warp
+    const int wg = (warp - 2) >> 2;  // token half of the tile handled by this warpgroup
+    const int wq = (warp - 2) & 3;   // this warp's rank inside its warpgroup
+    const int ew = warp - 2;
+    float* red_all = reinterpret_cast<float*>(smem + C::RED_OFF);
+    float* rs_all = reinterpret_cast<float*>(smem + C::RS_OFF);
+    const uint32_t tempty_lead0 = sm100::mapa_shared(tempty_bar(0), 0);
+    const uint32_t tempty_lead1 = sm100::mapa_shared(tempty_bar(1), 0);
+    const EpiParams& ep = args.ep;
+    int acc = 0;
+    uint32_t aph = 0, wph = 0;
+    // the four warps of this warpgroup meet (bounded); false on a timeout
+    auto wg_sync = [&]() {
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(wg_bar(wg));
+      const bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(wg_bar(wg), wph, abort_flag));
+      wph ^= 1u;
+      if (!ok && lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
+      return ok;
+    };
+    for (int t = cl; t < tiles; t += ncl) {
+      const int g = t / (npair * ntt), r = t % (npair * ntt);
+      const int fp = r / ntt, tt = r % ntt;
+      const Cell c = args.cells[g];
+      const int nt = tile_tokens(tt), cnt = nt / 2;
+      const int tok0 = tt * NT + wg * cnt;
+      const int fcta = fp * 256 + static_cast<int>(rank) * C::FM;  // first feature of this CTA
+      const int f = fcta + quarter * 32 + lane;
+      float* rs = rs_all + (acc * 2 + wg) * 128;
+      if constexpr (EPI == kEpiRope || EPI == kEpiSwiGLU) {
+        // folded RMSNorm: each warp computes the row scales of 32 of the warpgroup's tokens,
+        // ahead of the accumulator wait, and the warpgroup shares them
+        const int k = wq * 32 + lane, tok = tok0 + k;
+        if (k < cnt)
+          rs[k] = (ep.ss_in && tok < M)
+                      ? row_scale(ep.ss_in + (static_cast<size_t>(c.l) * M + tok) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                                  ep.rms_eps)
+                      : 1.f;
+        if (!wg_sync()) break;
+      }
+      if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+        // warm L2 with the residual rows of this CTA's next tile (its rows of 128 features)
+        const int tn = t + ncl;
+        if (tn < tiles) {
+          const int gn = tn / (npair * ntt), rn = tn % (npair * ntt);
+          const int fpn = rn / ntt, ttn = rn % ntt;
+          const Cell cn = args.cells[gn];
+          const int k = ew * 32 + lane, ntn = tile_tokens(ttn);
+          if (k < ntn && ttn * NT + k < M) {
+            const size_t si = cell_index(ep.src_mode, args.L, cn);
+            sm100::prefetch_l2_bulk(ep.x + (si * M + ttn * NT + k) * ep.ldx + fpn * 256 + rank * C::FM, C::FM * 4);
+          }
+        }
+      }
+      bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
+      if (!ok) {
+        if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
+        break;
+      }
+      sm100::tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(acc * C::ACC_COLS + wg * cnt);
+      float* red = red_all + ((acc * 2 + wg) * 4 + quarter) * 128;
+      pair_epilogue<EPI, OpT>(args, c, tacc, tok0, cnt, f, lane, rs, red);
+      // accumulator drained: release it to the even CTA's MMA issuer
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive_cluster(acc ? tempty_lead1 : tempty_lead0);
+      if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
+        if (ep.ss_out) {
+          // the four warps of this warpgroup hold 32-feature sums of the same tokens: combine
+          // them in quarter order into one partial per (token, 128-feature block)
+          if (!wg_sync()) break;
+          const float* rb = red_all + (acc * 2 + wg) * 4 * 128;
+          const int k = wq * 32 + lane;
+          const int tok = tok0 + k;
+          if (k < cnt && tok < M)
+            ep.ss_out[(static_cast<size_t>(c.l) * M + tok) * ep.ss_parts + fcta / C::FM] =
+                ((rb[k] + rb[128 + k]) + rb[256 + k]) + rb[384 + k];
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        aph ^= 1u;
+      }
+    }
+  }
+
+  sm100::tc_fence_before();
+  sm100::cluster_sync();  // no remote arrival or MMA can still target either CTA after this
+  sm100::tc_fence_after();
+  if (warp == 1) sm100::tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+}
+
+int max_pair_clusters(const void* fn) {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cached[dev]) {
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sms / 2;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int EPI, typename OpT>
+cudaError_t launch_pair_epi(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  const void* fn = reinterpret_cast<const void*>(tc_pair_gemm_kernel<EPI, OpT>);
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int NT = pair_token_tile(args.M);
+  const long tiles = static_cast<long>(args.G) * (args.N / 256) * ((args.M + NT - 1) / NT);
+  if (tiles <= 0) return cudaSuccess;
+  const int maxc = max_pair_clusters(fn);
+  const int clusters = static_cast<int>(tiles < maxc ? tiles : maxc);
+  tc_pair_gemm_kernel<EPI, OpT><<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tw, tx, args);
+  return cudaGetLastError();
+}
+
+template <typename OpT>
+cudaError_t launch_pair_op(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, cudaStream_t st) {
+  switch (args.epi) {
+    case kEpiStoreF32: return launch_pair_epi<kEpiStoreF32, OpT>(tw, tx, args, st);
+    case kEpiStoreAct: return launch_pair_epi<kEpiStoreAct, OpT>(tw, tx, args, st);
+    case kEpiResidCast: return launch_pair_epi<kEpiResidCast, OpT>(tw, tx, args, st);
+    case kEpiRope: return launch_pair_epi<kEpiRope, OpT>(tw, tx, args, st);
+    case kEpiSwiGLU: return launch_pair_epi<kEpiSwiGLU, OpT>(tw, tx, args, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool tc_pair_supported(int M, int N, int K, int epi, int head_dim) {
+  if (M <= 0 || N <= 0 || N % 256 != 0 || K <= 0 || K % 64 != 0) return false;
+  if (epi == kEpiResid) return false;  // 16-bit operands always refresh the operand copy (kEpiResidCast)
+  if (epi == kEpiRope && (head_dim <= 0 || head_dim % 2 != 0)) return false;
+  return pair_token_tile(M) <= 256;
+}
+
+cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, bool f16,
+                                cudaStream_t st) {
+  if (!tc_pair_supported(args.M, args.N, args.K, args.epi, args.ep.head_dim)) return cudaErrorInvalidValue;
+  return f16 ? launch_pair_op<__half>(tw, tx, args, st) : launch_pair_op<__nv_bfloat16>(tw, tx, args, st);
+}
+
+}  // namespace rmt

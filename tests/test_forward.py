@@ -169,3 +169,30 @@ def test_random_rmsnorm_gains_match_oracle(cuda_ok, name, S, tol):
     for g_, r, what in zip(got, ref, ("out", "A", "z")):
         assert normwise(g_, r) < tol, what
     rmt.rmt_destroy(h)
+
+
+MIXED_CONFIGS = {
+    # d_model 192: memo, QKV, O and down stay on single-CTA tiles, gate/up runs on CTA pairs
+    "mixed-tiles": dict(n_layers=3, d_model=192, n_heads=3, n_kv_heads=1, head_dim=64, d_ff=384, seg_len=100,
+                        n_mem=8, d_k=64, d_v=64),
+    # head_dim 128 on CTA pairs; 158 rows per cell end in a ragged token tile
+    "pairs-dh128": dict(n_layers=3, d_model=256, n_heads=2, n_kv_heads=1, head_dim=128, d_ff=512, seg_len=150,
+                        n_mem=8, d_k=64, d_v=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MIXED_CONFIGS))
+def test_bf16_tile_paths_match_oracle(cuda_ok, name):
+    import dataclasses
+    cfg = dataclasses.replace(CONFIGS["small-bf16"], **MIXED_CONFIGS[name])
+    w, h = build(cfg)
+    S = 3
+    emb = embeddings(cfg, S, seed=12)
+    got = forward(h, cfg, emb, S, "diagonal")
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32)
+    for g_, r, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g_, r) < BF16_TOL, what
+    seq = forward(h, cfg, emb, S, "sequential")
+    for a, b in zip(got, seq):
+        np.testing.assert_array_equal(a, b)
+    rmt.rmt_destroy(h)

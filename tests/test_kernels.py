@@ -24,9 +24,12 @@ def rng(seed):
 
 # ----------------------------------------------------------------------- grouped GEMM
 
+# N % 256 == 0 runs on CTA pairs (tokens along the MMA's N, ragged last token tile), other
+# widths on single CTAs (ragged last row tile)
 GEMM_CASES = [(g, 1040, n, 2048) for n in (2048, 8192) for g in (1, 2, 4, 8, 16)] + [
     (3, 528, 256, 512), (2, 2064, 128, 128), (1, 100, 64, 64), (5, 16, 320, 192), (2, 1040, 64, 2048),
-    (2, 1040, 2048, 64), (1, 129, 192, 8192)]
+    (2, 1040, 2048, 64), (1, 129, 192, 8192), (2, 2064, 256, 128), (1, 1, 256, 64), (3, 100, 512, 192),
+    (1, 257, 256, 64), (4, 17, 768, 128), (2, 1040, 16384, 128)]
 
 
 @pytest.mark.parametrize("G,M,N,K", GEMM_CASES)
@@ -47,8 +50,9 @@ def test_grouped_gemm_matches_matmul(G, M, N, K):
     assert err_b < 8e-3, err_b
 
 
-def test_grouped_gemm_each_group_uses_its_own_weight():
-    G, M, N, K = 4, 200, 128, 128
+@pytest.mark.parametrize("N", [128, 256])
+def test_grouped_gemm_each_group_uses_its_own_weight(N):
+    G, M, K = 4, 200, 128
     a = torch.ones((G, M, K), device="cuda", dtype=torch.bfloat16)
     b = torch.stack([torch.full((N, K), float(g + 1) / 64, device="cuda") for g in range(G)]).to(torch.bfloat16)
     c = torch.empty((G, M, N), device="cuda")
