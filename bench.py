@@ -56,6 +56,9 @@ def parse():
     p.add_argument("--segments", type=int, default=N_SEGMENTS)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-sequential", action="store_true")
+    p.add_argument("--microbench", choices=["gemm", "memory"], default=None,
+                   help="kernel-level sweeps instead of the forward: one JSON line per configuration")
+    p.add_argument("--reps", type=int, default=10, help="timed repetitions per microbench configuration")
     return p.parse_args()
 
 
@@ -220,6 +223,96 @@ def cpu_baseline(cfg, w, emb) -> dict:
                       "is the same for every segment"}
 
 
+def run_microbench(args, local: int) -> int:
+    """Kernel-level sweeps through the C ABI on synthetic inputs. Each repetition is timed
+    alone with CUDA events after L2 is flushed (a 256 MB write), and the median is reported."""
+    import torch
+
+    from recurrent_memory_transformer_anti_b200 import rmt
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+
+    def median_ms(fn, reps=max(1, args.reps)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    def emit(kind, config, ms, work, unit, peak, peak_name):
+        rate = work / (ms / 1e3) / 1e12 if unit == "TFLOP/s" else work / (ms / 1e3) / 1e9
+        print(json.dumps({"microbench": kind, "config": config, "ms": ms, "achieved": rate, "unit": unit,
+                          "peak": peak, "frac": rate / peak, "peak_source": f"{peak_name} ({peak_src})"}), flush=True)
+
+    if args.microbench == "gemm":
+        # grouped GEMM sweep: M = 1040 rows per group, K = 2048, a distinct weight per group
+        M, K = 1040, 2048
+        for N in (2048, 8192):
+            for G in (1, 2, 4, 8, 16):
+                a = torch.randn(G, M, K, device=dev, generator=gen).to(torch.bfloat16)
+                b = (torch.randn(G, N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+                c = torch.empty(G, M, N, device=dev, dtype=torch.bfloat16)
+                ms = median_ms(lambda: rmt.rmt_grouped_gemm_bf16(a, b, c, G, M, N, K, "bf16"))
+                emit("grouped_gemm_bf16", {"G": G, "M": M, "N": N, "K": K,
+                                           "kernel": "CTA pairs" if N % 256 == 0 else "single CTAs"},
+                     ms, 2.0 * G * M * N * K, "TFLOP/s", peaks["bf16_tflops"], "bf16_tflops")
+                del a, b, c
+        return 0
+
+    # memory-path kernels: the diagonal's size (G = 16 cells) and about 10^6 rows (HBM-bound)
+    dk = dv = 64
+    n, d, eps, hbm = 16, 2048, 1e-6, peaks["hbm_gbs"]
+    for G, M in ((16, 1040), (1024, 1040)):
+        q = torch.randn(G, M, dk, device=dev, generator=gen)
+        A = torch.randn(G, dk, dv, device=dev, generator=gen) * 0.1
+        z = torch.rand(G, dk, device=dev, generator=gen) + 1.0
+        o = torch.empty(G, M, dv, device=dev, dtype=torch.bfloat16)
+        ms = median_ms(lambda: rmt.rmt_memory_read(q, A, z, o, G, M, dk, dv, eps, "bf16"))
+        emit("memory_read", {"G": G, "M": M, "dk": dk, "dv": dv, "rows": G * M}, ms,
+             G * (M * dk * 4 + dk * dv * 4 + dk * 4 + M * dv * 2), "GB/s", hbm, "hbm_gbs")
+        del q, A, z, o
+    for G in (16, 16384):
+        k = torch.randn(G, n, dk, device=dev, generator=gen)
+        v = torch.randn(G, n, dv, device=dev, generator=gen)
+        A = torch.zeros(G, dk, dv, device=dev)
+        z = torch.zeros(G, dk, device=dev)
+        ms = median_ms(lambda: rmt.rmt_memory_update(k, v, A, z, G, n, dk, dv, eps))
+        emit("memory_update", {"G": G, "n": n, "dk": dk, "dv": dv}, ms,
+             G * (n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), "GB/s", hbm, "hbm_gbs")
+        del k, v, A, z
+    for G in (16, 2048):
+        y = torch.randn(G, n, d, device=dev, generator=gen)
+        wkv = (torch.randn(G, dk + dv, d, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+        A = torch.zeros(G, dk, dv, device=dev)
+        z = torch.zeros(G, dk, device=dev)
+        ms = median_ms(lambda: rmt.rmt_memory_write(y, wkv, A, z, G, n, d, dk, dv, eps, "bf16"))
+        emit("memory_write", {"G": G, "n": n, "d": d, "dk": dk, "dv": dv}, ms,
+             G * (n * d * 4 + (dk + dv) * d * 2 + 2 * (dk * dv + dk) * 4), "GB/s", hbm, "hbm_gbs")
+        del y, wkv, A, z
+    for rows in (16 * 1040, 131072):
+        x = torch.randn(rows, d, device=dev, generator=gen)
+        g = torch.ones(d, device=dev, dtype=torch.bfloat16)
+        y = torch.empty(rows, d, device=dev, dtype=torch.bfloat16)
+        ms = median_ms(lambda: rmt.rmt_rmsnorm(x, g, y, rows, d, 1e-5, "bf16"))
+        emit("rmsnorm", {"rows": rows, "d": d}, ms, rows * d * (4 + 2) + d * 2, "GB/s", hbm, "hbm_gbs")
+        del x, g, y
+    return 0
+
+
 def main() -> int:
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -227,6 +320,8 @@ def main() -> int:
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.microbench:
+        return run_microbench(args, local)
 
     import torch
     import torch.distributed as dist
@@ -308,8 +403,10 @@ def main() -> int:
     run("diagonal", 1)
     rmt.rmt_sync(h, stream)
     breakdown = {}
+    step_flops = 0.0
     for k in rmt.KERNELS:
         r = rmt.rmt_probe_read(h, k)
+        step_flops += r["flops"]
         if r["launches"]:
             breakdown[k] = {"ms": round(r["ms"], 3), "launches": r["launches"],
                             "tflops": round(r["flops"] / r["ms"] / 1e9, 1) if r["ms"] > 0 and r["flops"] else None,
@@ -365,6 +462,11 @@ def main() -> int:
                        "batch": 1, "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (weights 1.96 GB, embeddings 0.54 GB): no flush"},
             "roofline": roofline,
+            "path": {"algorithmic_tflop_per_step": step_flops / 1e12,
+                     "achieved_tflops": step_flops / (ms / 1e3) / 1e12,
+                     "frac_of_burst": step_flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "frac_of_sustained": step_flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+                     "note": "every kernel's algorithmic flops (GEMMs, causal attention, memory read/write) over the step"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": probe["all_launches"],
