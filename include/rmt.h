@@ -106,6 +106,18 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
 rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule,
                        void* out_hidden, float* out_A, float* out_z, void* stream);
 
+/* rmt_forward starting from a given memory state instead of zeros: in_A [n_layers, d_k, d_v]
+ * and in_z [n_layers, d_k] fp32, device or host, both given or both NULL (NULL: zeros, as
+ * rmt_forward). The state after segment s depends only on the segments up to s, so a
+ * sequence may be prefilled in chunks: running segments 0..S1-1, then resuming with the
+ * state it returned over segments S1..S-1, gives the same bits as one run over 0..S-1.
+ * in_A / in_z may alias out_A / out_z. Other arguments, errors and ordering as rmt_forward.
+ * Streaming continuation of the recurrent memory (the pages' recurrence carries only A and z
+ * from one segment to the next). */
+rmt_status rmt_forward_resume(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule,
+                              const float* in_A, const float* in_z, void* out_hidden, float* out_A, float* out_z,
+                              void* stream);
+
 /* The execution order as int32 triples (step, layer, segment), one per cell, n_layers*
  * n_segments of them: steps ascend; within a diagonal step layers ascend. Host memory,
  * cap = capacity of out_dls in int32 elements (>= 3*L*S). Needs no GPU. */

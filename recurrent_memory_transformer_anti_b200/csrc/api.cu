@@ -48,6 +48,16 @@ bool is_host_ptr(const void* p) {
   return attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged;
 }
 
+// Page-locked (or registered) host memory: asynchronous copies from and to it overlap kernels.
+bool is_pinned_host_ptr(const void* p) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return attr.type == cudaMemoryTypeHost;
+}
+
 struct Table {
   std::vector<Cell> cells;  // host copy, execution order
   std::vector<int> off, cnt;
@@ -164,6 +174,19 @@ struct rmt_handle {
   size_t emb_stage_bytes = 0;
   void* out_stage = nullptr;
   size_t out_stage_bytes = 0;
+  // per-segment host<->device copies for page-locked host buffers, overlapped with the steps
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> copy_events;  // [0]: forward start, [1]: copies done, then 2 per segment
+  bool copy_resources(size_t n_segments) {
+    if (!h2d && cudaStreamCreateWithFlags(&h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (!d2h && cudaStreamCreateWithFlags(&d2h, cudaStreamNonBlocking) != cudaSuccess) return false;
+    while (copy_events.size() < 2 + 2 * n_segments) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+      copy_events.push_back(e);
+    }
+    return true;
+  }
   std::map<std::pair<int, int>, Table> tables;
   CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
   // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
@@ -216,6 +239,11 @@ struct rmt_handle {
     emb_stage = out_stage = nullptr;
     for (cudaEvent_t e : probe_pool) cudaEventDestroy(e);
     probe_pool.clear();
+    for (cudaEvent_t e : copy_events) cudaEventDestroy(e);
+    copy_events.clear();
+    if (h2d) cudaStreamDestroy(h2d);
+    if (d2h) cudaStreamDestroy(d2h);
+    h2d = d2h = nullptr;
     probe_recs.clear();
     probe_used = 0;
   }
@@ -662,9 +690,12 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   return RMT_OK;
 }
 
-rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, void* out_hidden,
-                       float* out_A, float* out_z, void* stream) {
+namespace {
+
+rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, const float* in_A,
+                        const float* in_z, void* out_hidden, float* out_A, float* out_z, void* stream) {
   if (!h) return fail(RMT_EINVAL, "null handle");
+  if ((in_A == nullptr) != (in_z == nullptr)) return fail(RMT_EINVAL, "in_A and in_z must both be given or both be NULL");
   if (!emb || !out_hidden) return fail(RMT_EINVAL, "emb and out_hidden must not be null");
   if (n_segments <= 0) return fail(RMT_EINVAL, "n_segments must be positive");
   if (schedule != RMT_DIAGONAL && schedule != RMT_SEQUENTIAL) return fail(RMT_EINVAL, "unknown schedule");
@@ -672,6 +703,12 @@ rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_s
   const rmt_cfg& c = h->cfg;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t io_bytes = size_t(n_segments) * c.seg_len * c.d_model * h->es;
+  const size_t seg_bytes = size_t(c.seg_len) * c.d_model * h->es;
+  // page-locked host buffers: one copy per segment on side streams, each segment's input just
+  // ahead of the step that assembles it and its output right after the step that emits it
+  const bool in_pinned = is_pinned_host_ptr(emb), out_pinned = is_pinned_host_ptr(out_hidden);
+  if ((in_pinned || out_pinned) && !h->copy_resources(size_t(n_segments)))
+    return fail(RMT_ECUDA, "copy stream or event creation failed");
   const void* emb_dev = emb;
   if (is_host_ptr(emb)) {
     if (h->emb_stage_bytes < io_bytes) {
@@ -681,7 +718,19 @@ rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_s
       if (cudaMalloc(&h->emb_stage, io_bytes) != cudaSuccess) return fail(RMT_ENOMEM, "staging allocation failed");
       h->emb_stage_bytes = io_bytes;
     }
-    RMT_CUDA(cudaMemcpyAsync(h->emb_stage, emb, io_bytes, cudaMemcpyHostToDevice, st));
+    if (in_pinned) {
+      // the staging buffer may still be read by an earlier forward on `st`
+      RMT_CUDA(cudaEventRecord(h->copy_events[0], st));
+      RMT_CUDA(cudaStreamWaitEvent(h->h2d, h->copy_events[0], 0));
+      for (int s = 0; s < n_segments; ++s) {
+        RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(h->emb_stage) + s * seg_bytes,
+                                 static_cast<const char*>(emb) + s * seg_bytes, seg_bytes, cudaMemcpyHostToDevice,
+                                 h->h2d));
+        RMT_CUDA(cudaEventRecord(h->copy_events[2 + 2 * s], h->h2d));
+      }
+    } else {
+      RMT_CUDA(cudaMemcpyAsync(h->emb_stage, emb, io_bytes, cudaMemcpyHostToDevice, st));
+    }
     emb_dev = h->emb_stage;
   }
   void* out_dev = out_hidden;
@@ -719,18 +768,52 @@ rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_s
     h->trace_cap = ncell;
   }
   const size_t L = c.n_layers;
-  RMT_CUDA(cudaMemsetAsync(h->A, 0, L * c.d_k * c.d_v * sizeof(float), st));
-  RMT_CUDA(cudaMemsetAsync(h->z, 0, L * c.d_k * sizeof(float), st));
+  if (in_A) {  // continue from the caller's state (the state after an earlier run's last segment)
+    RMT_CUDA(cudaMemcpyAsync(h->A, in_A, L * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
+    RMT_CUDA(cudaMemcpyAsync(h->z, in_z, L * c.d_k * sizeof(float), cudaMemcpyDefault, st));
+  } else {
+    RMT_CUDA(cudaMemsetAsync(h->A, 0, L * c.d_k * c.d_v * sizeof(float), st));
+    RMT_CUDA(cudaMemsetAsync(h->z, 0, L * c.d_k * sizeof(float), st));
+  }
+  const bool split_in = in_pinned && emb_dev != emb, split_out = out_host && out_pinned;
   for (int step = 0; step < int(t.off.size()); ++step) {
+    const Cell first = t.cells[t.off[step]], last = t.cells[t.off[step] + t.cnt[step] - 1];
+    if (split_in && first.l == 0) RMT_CUDA(cudaStreamWaitEvent(st, h->copy_events[2 + 2 * first.s], 0));
     cudaError_t e = enqueue_step(h, t, step, emb_dev, out_dev, st);
     if (e != cudaSuccess) return fail(RMT_ECUDA, std::string("launch failed: ") + cudaGetErrorString(e));
+    if (split_out && last.l == int(L) - 1) {
+      cudaEvent_t done = h->copy_events[3 + 2 * last.s];
+      RMT_CUDA(cudaEventRecord(done, st));
+      RMT_CUDA(cudaStreamWaitEvent(h->d2h, done, 0));
+      RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(out_hidden) + last.s * seg_bytes,
+                               static_cast<const char*>(out_dev) + last.s * seg_bytes, seg_bytes,
+                               cudaMemcpyDeviceToHost, h->d2h));
+    }
   }
-  if (out_host) RMT_CUDA(cudaMemcpyAsync(out_hidden, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
+  if (split_out) {
+    RMT_CUDA(cudaEventRecord(h->copy_events[1], h->d2h));
+    RMT_CUDA(cudaStreamWaitEvent(st, h->copy_events[1], 0));
+  } else if (out_host) {
+    RMT_CUDA(cudaMemcpyAsync(out_hidden, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
+  }
   if (out_A) RMT_CUDA(cudaMemcpyAsync(out_A, h->A, L * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
   if (out_z) RMT_CUDA(cudaMemcpyAsync(out_z, h->z, L * c.d_k * sizeof(float), cudaMemcpyDefault, st));
   h->traced_cells = int(ncell);
   RMT_CUDA(cudaGetLastError());
   return RMT_OK;
+}
+
+}  // namespace
+
+rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, void* out_hidden,
+                       float* out_A, float* out_z, void* stream) {
+  return forward_impl(h, emb, n_segments, schedule, nullptr, nullptr, out_hidden, out_A, out_z, stream);
+}
+
+rmt_status rmt_forward_resume(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule,
+                              const float* in_A, const float* in_z, void* out_hidden, float* out_A, float* out_z,
+                              void* stream) {
+  return forward_impl(h, emb, n_segments, schedule, in_A, in_z, out_hidden, out_A, out_z, stream);
 }
 
 rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap) {

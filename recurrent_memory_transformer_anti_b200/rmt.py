@@ -21,7 +21,7 @@ SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
 DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16}
 STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE"}
 
-EXPORTED = ("rmt_create", "rmt_forward", "rmt_schedule_table", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
+EXPORTED = ("rmt_create", "rmt_forward", "rmt_forward_resume", "rmt_schedule_table", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
             "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
             "rmt_probe_read")
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
     sigs = {
         "rmt_create": [ctypes.POINTER(rmt_weights), ctypes.POINTER(rmt_cfg), ctypes.POINTER(vp)],
         "rmt_forward": [vp, vp, i32, ctypes.c_int, vp, vp, vp, vp],
+        "rmt_forward_resume": [vp, vp, i32, ctypes.c_int, vp, vp, vp, vp, vp, vp],
         "rmt_schedule_table": [i32, i32, ctypes.c_int, p32, sz],
         "rmt_get_schedule": [vp, i32, ctypes.c_int, p32, sz],
         "rmt_get_trace": [vp, p32, sz],
@@ -172,6 +173,13 @@ def rmt_forward(h: Handle, emb, n_segments: int, schedule, out_hidden, out_A=Non
     sch = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
     _check(_lib.rmt_forward(h.ptr, _ptr(emb), int(n_segments), sch, _ptr(out_hidden), _ptr(out_A), _ptr(out_z),
                             _stream(stream)), "rmt_forward")
+
+
+def rmt_forward_resume(h: Handle, emb, n_segments: int, schedule, in_A, in_z, out_hidden, out_A=None, out_z=None,
+                       stream=None) -> None:
+    sch = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    _check(_lib.rmt_forward_resume(h.ptr, _ptr(emb), int(n_segments), sch, _ptr(in_A), _ptr(in_z), _ptr(out_hidden),
+                                   _ptr(out_A), _ptr(out_z), _stream(stream)), "rmt_forward_resume")
 
 
 def rmt_schedule_table(n_layers: int, n_segments: int, schedule) -> np.ndarray:

@@ -95,6 +95,32 @@ def test_host_buffers_give_the_same_bits(tiny):
         np.testing.assert_array_equal(a, b)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small-bf16"])
+def test_pinned_host_buffers_give_the_same_bits(cuda_ok, name):
+    """Page-locked host buffers take the overlapped path: one copy per segment on side
+    streams, ordered against the steps by events. Two back-to-back forwards on the same
+    staging buffers check that a forward's copies wait for the previous one."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    S = 4
+    emb = embeddings(cfg, S, seed=16)
+    emb2 = embeddings(cfg, S, seed=17)
+    for schedule in ("diagonal", "sequential"):
+        refs = [forward(h, cfg, x, S, schedule) for x in (emb, emb2)]
+        e_host = [rmt.storage(x, cfg.dtype).pin_memory() for x in (emb, emb2)]
+        outs = [torch.empty_like(e).pin_memory() for e in e_host]
+        As = [torch.empty(cfg.n_layers, cfg.d_k, cfg.d_v).pin_memory() for _ in e_host]
+        zs = [torch.empty(cfg.n_layers, cfg.d_k).pin_memory() for _ in e_host]
+        for i in range(2):  # enqueued back to back, synchronized once
+            rmt.rmt_forward(h, e_host[i], S, schedule, outs[i], As[i], zs[i])
+        rmt.rmt_sync(h)
+        for i in range(2):
+            np.testing.assert_array_equal(refs[i][0], outs[i].float().numpy())
+            np.testing.assert_array_equal(refs[i][1], As[i].numpy())
+            np.testing.assert_array_equal(refs[i][2], zs[i].numpy())
+    rmt.rmt_destroy(h)
+
+
 def test_forward_argument_errors(tiny):
     cfg, w, h = tiny
     e = torch.zeros(cfg.seg_len, cfg.d_model, device="cuda")
@@ -195,4 +221,60 @@ def test_bf16_tile_paths_match_oracle(cuda_ok, name):
     seq = forward(h, cfg, emb, S, "sequential")
     for a, b in zip(got, seq):
         np.testing.assert_array_equal(a, b)
+    rmt.rmt_destroy(h)
+
+
+def _resume(h, cfg, emb, n_segments, A0, z0, schedule="diagonal"):
+    """rmt_forward_resume on device buffers from a state (A0, z0); returns (out, A, z) as numpy."""
+    e = rmt.storage(emb, cfg.dtype, device="cuda")
+    out = torch.empty_like(e)
+    A = torch.empty(cfg.n_layers, cfg.d_k, cfg.d_v, device="cuda")
+    z = torch.empty(cfg.n_layers, cfg.d_k, device="cuda")
+    rmt.rmt_forward_resume(h, e, n_segments, schedule, A0, z0, out, A, z)
+    rmt.rmt_sync(h)
+    return out.float().cpu().numpy(), A.cpu().numpy(), z.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,S1,S2", [("tiny", 3, 2), ("small-bf16", 2, 3)])
+def test_resume_in_chunks_equals_one_run_bitwise(cuda_ok, name, S1, S2):
+    """Prefilling in two chunks (the second resumed from the state the first returned) gives
+    the bits of one run: the state after a segment depends only on the segments before it."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    S, n1 = S1 + S2, S1 * cfg.seg_len
+    emb = embeddings(cfg, S, seed=13)
+    full = forward(h, cfg, emb, S, "diagonal")
+    first = forward(h, cfg, emb[:n1], S1, "diagonal")
+    np.testing.assert_array_equal(first[0], full[0][:n1])
+    A1 = torch.from_numpy(first[1]).cuda()
+    z1 = torch.from_numpy(first[2]).cuda()
+    for schedule in ("diagonal", "sequential"):
+        second = _resume(h, cfg, emb[n1:], S2, A1, z1, schedule)
+        np.testing.assert_array_equal(second[0], full[0][n1:])
+        np.testing.assert_array_equal(second[1], full[1])
+        np.testing.assert_array_equal(second[2], full[2])
+    # host state buffers give the same bits
+    host = _resume(h, cfg, emb[n1:], S2, torch.from_numpy(first[1]), torch.from_numpy(first[2]))
+    np.testing.assert_array_equal(host[0], full[0][n1:])
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_forward_resume(h, rmt.storage(emb[:cfg.seg_len], cfg.dtype, device="cuda"), 1, "diagonal", A1, None,
+                               torch.empty(cfg.seg_len, cfg.d_model, device="cuda"))
+    assert ex.value.status == rmt.RMT_EINVAL
+    rmt.rmt_destroy(h)
+
+
+@pytest.mark.parametrize("name,tol", [("tiny", F32_TOL), ("small-bf16", BF16_TOL)])
+def test_resume_from_a_given_state_matches_oracle(cuda_ok, name, tol):
+    """Both sides start from the same seeded synthetic state (z > 0, as a sum of phi values)."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    rng = np.random.default_rng(14)
+    A0 = (0.1 * rng.standard_normal((cfg.n_layers, cfg.d_k, cfg.d_v))).astype(np.float32)
+    z0 = (1.0 + np.abs(rng.standard_normal((cfg.n_layers, cfg.d_k)))).astype(np.float32)
+    S = 3
+    emb = embeddings(cfg, S, seed=15)
+    got = _resume(h, cfg, emb, S, torch.from_numpy(A0).cuda(), torch.from_numpy(z0).cuda())
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32, A0=A0, z0=z0)
+    for g_, r, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g_, r) < tol, what
     rmt.rmt_destroy(h)
