@@ -69,6 +69,8 @@ struct AttnSmem {
 
 template <int HD, typename OpT>
 __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   using S = AttnSmem<HD>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   OpT* Qs = reinterpret_cast<OpT*>(smem_raw);
@@ -236,6 +238,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
 
 template <int HD>
 __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   constexpr int BQ = 64, CK = 32;
   __shared__ float Kc[CK][HD];
   __shared__ float Vc[CK][HD];
@@ -299,14 +303,16 @@ cudaError_t launch_mma(const AttnArgs& a, cudaStream_t st) {
     attr[dev] = true;
   }
   dim3 grid((a.M + S::BQ - 1) / S::BQ, a.H, a.G);
-  attn_mma_kernel<HD, OpT><<<grid, 128, S::BYTES, st>>>(a);
+  const cudaError_t e = launch_pdl(attn_mma_kernel<HD, OpT>, grid, dim3(128), S::BYTES, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int HD>
 cudaError_t launch_f32(const AttnArgs& a, cudaStream_t st) {
   dim3 grid((a.M + 63) / 64, a.H, a.G);
-  attn_f32_kernel<HD><<<grid, 64, 0, st>>>(a);
+  const cudaError_t e = launch_pdl(attn_f32_kernel<HD>, grid, dim3(64), 0, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

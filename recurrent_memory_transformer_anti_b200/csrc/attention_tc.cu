@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();  // this CTA holds its TMEM: the next kernel may be scheduled
+  pdl_wait();     // q, k, v come from the previous kernel of the stream
 
   if (warp == 0) {
     if (lane == 0) {
@@ -409,7 +411,8 @@ cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st)
   const long items = static_cast<long>((a.M + 127) / 128) * a.H * a.G;
   const long cap = static_cast<long>(sms[dev] > 0 ? sms[dev] : 148) * C::CTAS_PER_SM;
   const int grid = static_cast<int>(items < cap ? items : cap);
-  attn_tc_kernel<HD, OpT><<<grid, 192, C::SMEM, st>>>(tm, a);
+  const cudaError_t e = launch_pdl(attn_tc_kernel<HD, OpT>, dim3(grid), dim3(192), C::SMEM, st, tm, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -16,6 +16,17 @@ enum : int {
   kErrBadArgs = 8,
 };
 
+// Programmatic dependent launch. The forward launches its kernels with programmatic stream
+// serialization, so a kernel may be scheduled while the previous one in the stream is still
+// finishing. pdl_wait() blocks until every earlier kernel of the stream has completed and its
+// writes are visible: each kernel calls it before its first global-memory access to data
+// another kernel writes or reads. pdl_trigger() lets the next kernel be scheduled once every
+// CTA of this grid has issued it (or exited); kernels that allocate TMEM issue it only after
+// the allocation, so that an early dependent CTA can never hold TMEM this grid still needs.
+// Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // One (layer, segment) cell of the grid.
 struct Cell {
   int l, s;

@@ -27,6 +27,8 @@ constexpr int kReadRows = 32, kReadWarps = 8, kReadBatch = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemReadArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ float sm[];
   const int dk = a.dk, dv = a.dv, nk = dk >> 5, nv = dv >> 5;
   float* As = sm;            // [dk][dv]
@@ -100,6 +102,8 @@ constexpr int kKvThreads = 256;
 
 template <typename T>
 __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ float sm[];
   constexpr int KS = kMemKvSplit;
   const int n4 = (a.n + 3) & ~3;  // rows padded to a multiple of 4 (padding rows are zero)
@@ -147,6 +151,8 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
 constexpr int kUpdThreads = 512;
 
 __global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdateArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ float sm[];
   const int n = a.n, dk = a.dk, dv = a.dv, dkv = dk + dv;
   float* KV = sm;              // [n][dkv]: phi(k) in columns < dk, v after
@@ -216,7 +222,8 @@ template <typename T>
 cudaError_t launch_mem_read_t(const MemReadArgs& a, size_t smem, cudaStream_t st) {
   if (smem > 48 * 1024) cudaFuncSetAttribute(mem_read_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((a.M + kReadRows - 1) / kReadRows, a.G);
-  mem_read_kernel<T><<<grid, kReadWarps * 32, smem, st>>>(a);
+  const cudaError_t e = launch_pdl(mem_read_kernel<T>, grid, dim3(kReadWarps * 32), smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -241,11 +248,11 @@ cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(mem_kv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    mem_kv_kernel<__nv_bfloat16><<<grid, kKvThreads, smem, st>>>(a);
+    return launch_pdl(mem_kv_kernel<__nv_bfloat16>, grid, dim3(kKvThreads), smem, st, a);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(mem_kv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    mem_kv_kernel<float><<<grid, kKvThreads, smem, st>>>(a);
+    return launch_pdl(mem_kv_kernel<float>, grid, dim3(kKvThreads), smem, st, a);
   }
   return cudaGetLastError();
 }
@@ -258,7 +265,8 @@ cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st) {
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(mem_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  mem_update_kernel<<<a.G, kUpdThreads, smem, st>>>(a);
+  const cudaError_t e = launch_pdl(mem_update_kernel, dim3(a.G), dim3(kUpdThreads), smem, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

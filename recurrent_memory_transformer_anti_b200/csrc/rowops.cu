@@ -69,6 +69,8 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a
 // Layer-0 input of segment s: embeddings of the segment, then the memory tokens.
 template <typename T>
 __global__ void assemble_kernel(const T* emb, const T* mem, float* x, __half* xb, int seg, int d, int s) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   const int r = blockIdx.x;
   const T* src = r < seg ? emb + (static_cast<size_t>(s) * seg + r) * d : mem + static_cast<size_t>(r - seg) * d;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
@@ -80,6 +82,8 @@ __global__ void assemble_kernel(const T* emb, const T* mem, float* x, __half* xb
 
 template <typename T>
 __global__ void emit_kernel(const float* x, T* out, int seg, int d, int s) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   const int r = blockIdx.x;
   T* dst = out + (static_cast<size_t>(s) * seg + r) * d;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(x + static_cast<size_t>(r) * d + k));
@@ -141,12 +145,12 @@ cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __h
   if (d % 4) return cudaErrorInvalidValue;
   const int threads = d >= 1024 ? 256 : 128;
   if (bf16)
-    assemble_kernel<__nv_bfloat16><<<seg + n_mem, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(emb),
-                                                                     static_cast<const __nv_bfloat16*>(mem), x_slot,
-                                                                     xb_slot, seg, d, s);
+    return launch_pdl(assemble_kernel<__nv_bfloat16>, dim3(seg + n_mem), dim3(threads), 0, st,
+                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x_slot, xb_slot,
+                      seg, d, s);
   else
-    assemble_kernel<float><<<seg + n_mem, threads, 0, st>>>(static_cast<const float*>(emb),
-                                                            static_cast<const float*>(mem), x_slot, xb_slot, seg, d, s);
+    return launch_pdl(assemble_kernel<float>, dim3(seg + n_mem), dim3(threads), 0, st, static_cast<const float*>(emb),
+                      static_cast<const float*>(mem), x_slot, xb_slot, seg, d, s);
   return cudaGetLastError();
 }
 
@@ -154,9 +158,11 @@ cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, b
   if (d % 4) return cudaErrorInvalidValue;
   const int threads = d >= 1024 ? 256 : 128;
   if (bf16)
-    emit_kernel<__nv_bfloat16><<<seg, threads, 0, st>>>(x_slot, static_cast<__nv_bfloat16*>(out), seg, d, s);
+    return launch_pdl(emit_kernel<__nv_bfloat16>, dim3(seg), dim3(threads), 0, st, x_slot,
+                      static_cast<__nv_bfloat16*>(out), seg, d, s);
   else
-    emit_kernel<float><<<seg, threads, 0, st>>>(x_slot, static_cast<float*>(out), seg, d, s);
+    return launch_pdl(emit_kernel<float>, dim3(seg), dim3(threads), 0, st, x_slot, static_cast<float*>(out), seg, d,
+                      s);
   return cudaGetLastError();
 }
 

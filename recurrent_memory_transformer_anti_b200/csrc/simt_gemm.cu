@@ -12,6 +12,8 @@ namespace {
 constexpr int BM = 64, BN = 128, BK = 16, NT = 256;
 
 __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
   __shared__ float As[BK][BM];
   __shared__ float Bs[BK][BN];
   __shared__ float Cs[BM][BN + 1];
@@ -131,7 +133,8 @@ cudaError_t launch_simt_gemm(const SimtGemmArgs& a, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0 || a.N <= 0) return cudaSuccess;
   if (a.epi == kEpiRope && (BN % a.ep.head_dim != 0)) return cudaErrorInvalidValue;
   dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM, a.G);
-  simt_gemm_kernel<<<grid, NT, 0, st>>>(a);
+  const cudaError_t e = launch_pdl(simt_gemm_kernel, grid, dim3(NT), 0, st, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -395,6 +395,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();  // this CTA holds its TMEM: the next kernel may be scheduled
+  pdl_wait();     // operands and residuals come from the previous kernels of the stream
 
   const int mt = (args.M + C::BM - 1) / C::BM;
   const int nt = args.N / BN;
@@ -565,7 +567,9 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   const long tiles = static_cast<long>(args.G) * mt * (args.N / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
-  tc_gemm_kernel<BN, EPI, OpT><<<grid, kGemmThreads, C::SMEM_BYTES, st>>>(ta, tb, tx, args);
+  const cudaError_t e =
+      launch_pdl(tc_gemm_kernel<BN, EPI, OpT>, dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st, ta, tb, tx, args);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

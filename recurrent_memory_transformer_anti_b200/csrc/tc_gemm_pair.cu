@@ -268,6 +268,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   sm100::cluster_sync();  // both CTAs' barriers initialised and TMEM allocated before any remote use
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();  // this CTA holds its TMEM: the next kernel may be scheduled
+  pdl_wait();     // operands and residuals come from the previous kernels of the stream
 
   const int ntt = (M + NT - 1) / NT;
   const int npair = args.N / 256;
@@ -516,7 +518,9 @@ cudaError_t launch_pair_epi(const CUtensorMap& tw, const CUtensorMap& tx, const 
   if (tiles <= 0) return cudaSuccess;
   const int maxc = max_pair_clusters(fn);
   const int clusters = static_cast<int>(tiles < maxc ? tiles : maxc);
-  tc_pair_gemm_kernel<EPI, OpT><<<2 * clusters, PairCfg::THREADS, PairCfg::SMEM_BYTES, st>>>(tw, tx, args);
+  const cudaError_t e = launch_pdl(tc_pair_gemm_kernel<EPI, OpT>, dim3(2 * clusters), dim3(PairCfg::THREADS),
+                                   PairCfg::SMEM_BYTES, st, tw, tx, args);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
