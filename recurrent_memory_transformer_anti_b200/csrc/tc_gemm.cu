@@ -26,19 +26,25 @@
 
 namespace rmt {
 
-template <int BN>
+// NBUF: 32 x 32 residual blocks per epilogue warp (two keep the next block's load in flight).
+// Each epilogue warp also has a 32 x 32 staging block for the 16-bit copy of the residual.
+template <int BN, int NBUF = 2>
 struct TcCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int EPI_BUF = NBUF * 32 * 32 * 4;  // per epilogue warp: NBUF 32 x 32 fp32 residual blocks
+  static constexpr int XS_ROW = 80;             // staging row: 64 B of 16-bit values + 16 B of padding
+  static constexpr int XS_BUF = 32 * XS_ROW;     // per epilogue warp
+  static constexpr int RING_BUDGET = 232448 - 1024 - 2048 - 8 * EPI_BUF - 8 * XS_BUF;
+  static constexpr int STAGES = (RING_BUDGET / STAGE_BYTES) > 8 ? 8 : (RING_BUDGET / STAGE_BYTES);
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int NBAR = 2 * STAGES + 5 + 8;  // ring, accumulators, drain, one per epilogue warp
+  static constexpr int NBAR = 2 * STAGES + 5 + 8 * NBUF;  // ring, accumulators, drain, NBUF per epilogue warp
   static constexpr int BAR_BYTES = 1024 * ((8 * NBAR + 16 + 1023) / 1024);
-  static constexpr int EPI_BUF = 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 residual block
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES + BAR_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + EPI_OFF + 8 * EPI_BUF;
+  static constexpr int XS_OFF = EPI_OFF + 8 * EPI_BUF;
+  static constexpr int SMEM_BYTES = 1024 + XS_OFF + 8 * XS_BUF;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -215,39 +221,51 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
 }
 
 // Residual epilogue of one warp (tile rows rowbase .. rowbase+31, one per lane) over its
-// column half, through TMA: each 32 x 32 block of the residual stream is loaded into the
-// warp's swizzled shared block, the accumulator rows are added in place, and the block is
-// stored back with one bulk copy; the operand-type copy goes out with plain stores.
-template <int BN, int EPI, typename OpT>
+// column half, through TMA: each 32 x 32 block of the residual stream is loaded into one of
+// the warp's NBUF swizzled shared blocks, the accumulator rows are added in place, and the
+// block is stored back with one bulk copy; the operand-type copy goes out with plain stores.
+// Up to NBUF block loads are in flight: a block is refilled with chunk k + NBUF as soon as the
+// store of chunk k has read it. rbar is block 0's barrier (block b's is 8 b bytes further);
+// bit b of rph is block b's phase.
+template <int BN, int EPI, typename OpT, int NBUF>
 __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CUtensorMap* tmX, uint32_t tacc, Cell c,
                                                    int rowbase, int n0, int part, int lane, uint8_t* buf,
                                                    uint32_t buf_s, uint32_t rbar, uint32_t& rph,
-                                                   volatile int* abort_flag) {
+                                                   volatile int* abort_flag, uint8_t* xstage) {
   const EpiParams& ep = a.ep;
   if (rowbase >= a.M) return true;  // the whole block lies past the cell
   const int row = rowbase + lane;
   const bool valid = row < a.M;
   const int src = cell_index(ep.src_mode, a.L, c), dst = cell_index(ep.dst_mode, a.L, c);
-  constexpr int chunks = BN / 32;
+  constexpr int chunks = BN / 32, BLK = 32 * 32 * 4;
   const int c0 = part * chunks / 2, c1 = (part + 1) * chunks / 2;
-  float4* rowp = reinterpret_cast<float4*>(buf + lane * 128);
+  uint32_t pend = 0;  // blocks whose load is in flight (lane 0's view)
+  auto issue = [&](int cc, int b) {
+    sm100::bulk_wait_read_all();  // the last store from block b has read it
+    sm100::mbar_arrive_expect_tx(rbar + 8u * b, BLK);
+    sm100::tma_load_3d(buf_s + b * BLK, tmX, n0 + cc * 32, rowbase, src, rbar + 8u * b);
+    pend |= 1u << b;
+  };
+  if (lane == 0)
+    for (int j = 0; j < NBUF && c0 + j < c1; ++j) issue(c0 + j, j);
   float ss = 0.f;
 #pragma unroll 1
   for (int cc = c0; cc < c1; ++cc) {
+    const int b = (cc - c0) % NBUF;
     const int col = n0 + cc * 32;
-    if (lane == 0) {
-      sm100::bulk_wait_read_all();  // the previous store has read the block
-      sm100::mbar_arrive_expect_tx(rbar, 32 * 32 * 4);
-      sm100::tma_load_3d(buf_s, tmX, col, rowbase, src, rbar);
-    }
     uint32_t r[32];
     sm100::tmem_ld32(tacc + cc * 32, r);
     sm100::tmem_wait_ld();
-    if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar, rph, abort_flag))) {
-      if (lane == 0) sm100::mbar_wait_drain(rbar, rph);  // let the load land before the block is reused
+    if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar + 8u * b, (rph >> b) & 1u, abort_flag))) {
+      if (lane == 0) {  // let every load in flight land before the blocks are reused
+        for (int x = 0; x < NBUF; ++x)
+          if (pend & (1u << x)) sm100::mbar_wait_drain(rbar + 8u * x, (rph >> x) & 1u);
+      }
       return false;
     }
-    rph ^= 1u;
+    rph ^= 1u << b;
+    pend &= ~(1u << b);
+    float4* rowp = reinterpret_cast<float4*>(buf + b * BLK + lane * 128);
     float y[32];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -265,14 +283,32 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
     if (valid) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) ss = fmaf(y[j], y[j], ss);
-      if constexpr (EPI == kEpiResidCast)
-        store32_16(static_cast<OpT*>(ep.xb) + ((size_t)dst * a.M + row) * ep.ldx + col, y);
+    }
+    if constexpr (EPI == kEpiResidCast) {
+      // the 16-bit copy: stage the warp's 32 x 32 block, then store it row by row, each
+      // instruction covering 8 rows x 64 contiguous bytes
+      uint4* mine = reinterpret_cast<uint4*>(xstage + lane * 80);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        mine[q] = make_uint4(pack2<OpT>(y[8 * q], y[8 * q + 1]), pack2<OpT>(y[8 * q + 2], y[8 * q + 3]),
+                             pack2<OpT>(y[8 * q + 4], y[8 * q + 5]), pack2<OpT>(y[8 * q + 6], y[8 * q + 7]));
+      __syncwarp();
+      OpT* xb = static_cast<OpT*>(ep.xb) + ((size_t)dst * a.M + rowbase) * ep.ldx + col + (lane & 3) * 8;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r2 = (lane >> 2) + 8 * k;
+        if (rowbase + r2 < a.M)
+          *reinterpret_cast<uint4*>(xb + static_cast<size_t>(r2) * ep.ldx) =
+              *reinterpret_cast<const uint4*>(xstage + r2 * 80 + (lane & 3) * 16);
+      }
+      __syncwarp();
     }
     sm100::fence_async_smem();
     __syncwarp();
     if (lane == 0) {
-      sm100::tma_store_3d(tmX, buf_s, col, rowbase, dst);
+      sm100::tma_store_3d(tmX, buf_s + b * BLK, col, rowbase, dst);
       sm100::bulk_commit();
+      if (cc + NBUF < c1) issue(cc + NBUF, b);
     }
   }
   if (ep.ss_out && valid) ep.ss_out[(static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
@@ -313,8 +349,8 @@ __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUt
         sm100::mbar_arrive_expect_tx(rbar, 32 * 32 * 4);
         sm100::tma_load_3d(buf_s, tmR, 2 * p, rowbase, 0, rbar);
       }
-      if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar, rph, abort_flag))) {
-        if (lane == 0) sm100::mbar_wait_drain(rbar, rph);
+      if (!__all_sync(0xffffffffu, sm100::mbar_wait(rbar, rph & 1u, abort_flag))) {
+        if (lane == 0) sm100::mbar_wait_drain(rbar, rph & 1u);
         return false;
       }
       rph ^= 1u;
@@ -351,11 +387,11 @@ __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUt
   return true;
 }
 
-template <int BN, int EPI, typename OpT>
+template <int BN, int EPI, typename OpT, int NBUF>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmX, const TcGemmArgs args) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, NBUF>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = sm100::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -366,7 +402,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
-  auto resid_bar = [&](int w) { return bar0 + 8u * (2 * C::STAGES + 5 + w); };
+  auto resid_bar = [&](int w) { return bar0 + 8u * (2 * C::STAGES + 5 + NBUF * w); };  // and the NBUF-1 after it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE_BYTES + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -381,7 +417,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       sm100::mbar_init(tempty_bar(a), kEpiWarps);
     }
     sm100::mbar_init(drain_bar, 1);
-    for (int w = 0; w < kEpiWarps; ++w) sm100::mbar_init(resid_bar(w), 1);
+    for (int w = 0; w < NBUF * kEpiWarps; ++w) sm100::mbar_init(resid_bar(0) + 8u * w, 1);
     *abort_flag = 0;
     sm100::fence_barrier_init();
     sm100::fence_proxy_async_smem();
@@ -505,8 +541,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const Cell c = args.cells[g];
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
-        ok = epilogue_resid_tma<BN, EPI, OpT>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
-                                              lane, rbuf, rbuf_s, resid_bar(ew), rph, abort_flag);
+        ok = epilogue_resid_tma<BN, EPI, OpT, NBUF>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
+                                                    lane, rbuf, rbuf_s, resid_bar(ew), rph, abort_flag,
+                                                    smem + C::XS_OFF + ew * C::XS_BUF);
         if (!ok) {
           if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
           break;
@@ -549,16 +586,16 @@ int sm_count_cached() {
   return count[dev];
 }
 
-template <int BN, int EPI, typename OpT>
+template <int BN, int EPI, typename OpT, int NBUF = 2>
 cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
                           cudaStream_t st) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, NBUF>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI, OpT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI, OpT, NBUF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -568,7 +605,7 @@ cudaError_t launch_bn_epi(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sm_count_cached() ? tiles : sm_count_cached());
   const cudaError_t e =
-      launch_pdl(tc_gemm_kernel<BN, EPI, OpT>, dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st, ta, tb, tx, args);
+      launch_pdl(tc_gemm_kernel<BN, EPI, OpT, NBUF>, dim3(grid), dim3(kGemmThreads), C::SMEM_BYTES, st, ta, tb, tx, args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
