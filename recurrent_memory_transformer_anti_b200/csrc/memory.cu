@@ -96,8 +96,11 @@ __global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemRead
 
 // ------------------------------------------------------------------ key/value projection
 // CTA = one split of kMemKvSplit columns of d_model for one cell: the n memory rows and the
-// dkv weight rows of that split are staged in shared memory; each thread then forms a
-// 4 x 4 block of the n x dkv partial dot products (4 + 4 shared loads per 16 FMAs).
+// dkv weight rows of that split are staged in shared memory, k-major; each thread then forms
+// a 4-row x 2-column block of the n x dkv partial dot products over the split, k ascending.
+// Staging reads 16-byte vectors: one lane takes 8 consecutive columns of one weight row (4 of
+// one memory row) and writes them down a column of the k-major block, so the lanes of a warp
+// write consecutive words.
 constexpr int kKvThreads = 256;
 
 template <typename T>
@@ -107,42 +110,74 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   extern __shared__ float sm[];
   constexpr int KS = kMemKvSplit;
   const int n4 = (a.n + 3) & ~3;  // rows padded to a multiple of 4 (padding rows are zero)
-  float* Ys = sm;                 // [KS][n4]   (transposed: k-major)
+  float* Ys = sm;                 // [KS][n4]
   float* Ws = sm + KS * n4;       // [KS][dkv]
   const Cell c = a.cells[blockIdx.y];
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
   const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + a.row0) * a.d + k0;
   const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
-  for (int e = threadIdx.x; e < n4 * KS; e += kKvThreads) {
-    const int r = e / KS, k = e % KS;
-    Ys[k * n4 + r] = (r < a.n && k < kw) ? Y[static_cast<size_t>(r) * a.d + k] : 0.f;
+  // 16-byte vectors only where every row start is 16-byte aligned
+  const bool y_vec = (a.d % 4 == 0) && (reinterpret_cast<uintptr_t>(a.x) % 16 == 0);
+  const bool w_vec = sizeof(T) == 2 && (a.d % 8 == 0) && (reinterpret_cast<uintptr_t>(a.w) % 16 == 0);
+  // memory rows: one lane per (row, 4 columns), rows fastest
+  for (int e = threadIdx.x; e < n4 * (KS / 4); e += kKvThreads) {
+    const int r = e % n4, k = 4 * (e / n4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < a.n) {
+      const float* yr = Y + static_cast<size_t>(r) * a.d + k;
+      if (y_vec && k + 3 < kw) {
+        v = *reinterpret_cast<const float4*>(yr);
+      } else {
+        if (k < kw) v.x = yr[0];
+        if (k + 1 < kw) v.y = yr[1];
+        if (k + 2 < kw) v.z = yr[2];
+        if (k + 3 < kw) v.w = yr[3];
+      }
+    }
+    Ys[(k + 0) * n4 + r] = v.x;
+    Ys[(k + 1) * n4 + r] = v.y;
+    Ys[(k + 2) * n4 + r] = v.z;
+    Ys[(k + 3) * n4 + r] = v.w;
   }
-  for (int e = threadIdx.x; e < a.dkv * KS; e += kKvThreads) {
-    const int j = e / KS, k = e % KS;
-    Ws[k * a.dkv + j] = k < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k]) : 0.f;
+  // weight rows: one lane per (row, 8 columns), rows fastest
+  for (int e = threadIdx.x; e < a.dkv * (KS / 8); e += kKvThreads) {
+    const int j = e % a.dkv, k = 8 * (e / a.dkv);
+    float w8[8];
+    if (w_vec && k + 7 < kw) {
+      const uint4 u = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(j) * a.d + k);
+      const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) w8[t] = to_f32<T>(h[t]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) w8[t] = k + t < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k + t]) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) Ws[(k + t) * a.dkv + j] = w8[t];
   }
   __syncthreads();
   const int nsplit = (a.d + KS - 1) / KS;
   const int nout = a.n * a.dkv;
   float* part = a.part + (static_cast<size_t>(c.l) * nsplit + split) * nout;
-  const int jt = a.dkv / 4, tiles = (n4 / 4) * jt;
+  const int jt = a.dkv / 2, tiles = (n4 / 4) * jt;
   for (int t = threadIdx.x; t < tiles; t += kKvThreads) {
-    const int r0 = (t / jt) * 4, j0 = (t % jt) * 4;
-    float acc[4][4] = {};
-#pragma unroll 4
+    const int r0 = (t / jt) * 4, j0 = (t % jt) * 2;
+    float acc[4][2] = {};
+#pragma unroll 8
     for (int k = 0; k < KS; ++k) {
       const float4 y = *reinterpret_cast<const float4*>(Ys + k * n4 + r0);
-      const float4 w = *reinterpret_cast<const float4*>(Ws + k * a.dkv + j0);
-      const float yv[4] = {y.x, y.y, y.z, y.w}, wv[4] = {w.x, w.y, w.z, w.w};
+      const float2 w = *reinterpret_cast<const float2*>(Ws + k * a.dkv + j0);
+      const float yv[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(yv[i], wv[q], acc[i][q]);
+      for (int i = 0; i < 4; ++i) {
+        acc[i][0] = fmaf(yv[i], w.x, acc[i][0]);
+        acc[i][1] = fmaf(yv[i], w.y, acc[i][1]);
+      }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (r0 + i < a.n) *reinterpret_cast<float4*>(part + (r0 + i) * a.dkv + j0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      if (r0 + i < a.n) *reinterpret_cast<float2*>(part + (r0 + i) * a.dkv + j0) = make_float2(acc[i][0], acc[i][1]);
   }
 }
 

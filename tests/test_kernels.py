@@ -165,8 +165,10 @@ def test_rmsnorm_matches_oracle(dtype, rows, d):
     assert normwise(to_np(y), ref) < (5e-3 if dtype == "bf16" else 2e-6)
 
 
+# bf16 widths that are not a multiple of 8 take the scalar staging path (no 16-byte vectors)
 @pytest.mark.parametrize("dtype,G,n,d,dk,dv", [("bf16", 4, 16, 2048, 64, 64), ("f32", 3, 8, 128, 32, 32),
-                                               ("bf16", 2, 16, 3072, 128, 128), ("f32", 2, 5, 200, 32, 64)])
+                                               ("bf16", 2, 16, 3072, 128, 128), ("f32", 2, 5, 200, 32, 64),
+                                               ("bf16", 2, 16, 100, 32, 32), ("bf16", 2, 7, 260, 32, 64)])
 def test_memory_write_matches_oracle(dtype, G, n, d, dk, dv):
     """Key/value projection of n rows (split-K partials reduced in fixed order) + update."""
     r = rng(600 + d + n)
