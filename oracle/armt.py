@@ -30,6 +30,10 @@ layer equations):
   theta = 500000 at segment-local positions, causal GQA attention over the segment and
   memory tokens, SwiGLU MLP; no biases.
 * memory tokens are appended after each segment's tokens at layer 0; state starts at 0.
+* a sequence whose length is not a multiple of the segment length ends in a shorter
+  segment (the sketch in P1 "Implementation" cuts with ceil division); its memory tokens
+  follow its last token, and its memory write reads the cell's last n_mem rows.
+* a batch is a set of independent sequences, each with its own memory state.
 * the output is the last layer's rows of the segment tokens.
 
 Arithmetic runs in the dtype given (float32 or float64); RoPE angles and their cos/sin
@@ -42,8 +46,8 @@ import math
 import numpy as np
 
 __all__ = ["phi", "silu", "rms_norm", "rope", "causal_gqa_attention", "memory_read",
-           "memory_update", "armt_cell", "forward", "diagonals", "sequential_steps",
-           "schedule_triples"]
+           "memory_update", "armt_cell", "forward", "forward_tokens", "forward_batch", "diagonals",
+           "sequential_steps", "schedule_triples", "schedule_quads"]
 
 
 # ----------------------------------------------------------------------------- schedule
@@ -77,6 +81,33 @@ def schedule_triples(n_layers: int, n_segments: int, schedule: str) -> np.ndarra
     steps = diagonals(n_layers, n_segments) if schedule == "diagonal" else sequential_steps(n_layers, n_segments)
     rows = [(t, l, s) for t, cells in enumerate(steps) for (l, s) in cells]
     return np.asarray(rows, dtype=np.int32).reshape(-1, 3)
+
+
+def schedule_quads(n_layers: int, n_segments: list, schedule: str) -> np.ndarray:
+    """Schedule of a batch whose sequence b has n_segments[b] segments, as int32 rows
+    (step, sequence, layer, segment) in execution order.
+
+    [P1 "Implementation": the input is a [B, T, D] batch; one diagonal step runs the cell
+    (l, s) for the whole batch.] Diagonal: step d holds every (b, l, s) with l + s = d, layers
+    ascending and, within a layer, sequences ascending; steps without a cell are dropped.
+    Sequential: one cell per step, sequence by sequence, each in the single-sequence order.
+    """
+    rows = []
+    if schedule == "diagonal":
+        step = 0
+        for d in range(n_layers + max(n_segments) - 1):
+            cells = [(b, l, d - l) for l in range(n_layers) for b in range(len(n_segments))
+                     if 0 <= d - l < n_segments[b]]
+            if cells:
+                rows += [(step, b, l, s) for (b, l, s) in cells]
+                step += 1
+    else:
+        step = 0
+        for b, nb in enumerate(n_segments):
+            for (cell,) in sequential_steps(n_layers, nb):
+                rows.append((step, b) + cell)
+                step += 1
+    return np.asarray(rows, dtype=np.int32).reshape(-1, 4)
 
 
 # ------------------------------------------------------------------ elementwise pieces
@@ -184,8 +215,8 @@ def armt_cell(x: np.ndarray, lw: dict, A: np.ndarray, z: np.ndarray, cfg) -> tup
     h = rms_norm(x, lw["g_mlp"], cfg.rms_eps)
     u = silu(h @ lw["w_gate"].T) * (h @ lw["w_up"].T)
     x = x + u @ lw["w_down"].T
-    # memory write from this layer's memory-token output rows
-    y = x[cfg.seg_len:]
+    # memory write from this layer's memory-token output rows (the cell's last n_mem rows)
+    y = x[m - cfg.n_mem:]
     A, z = memory_update(y @ lw["w_mk"].T, y @ lw["w_mv"].T, A, z, cfg.mem_eps)
     return x, A, z
 
@@ -194,25 +225,50 @@ def layer_weights(weights: dict, l: int, dtype) -> dict:
     return {k: np.asarray(v[l], dtype=dtype) for k, v in weights.items() if k != "mem_tokens"}
 
 
-def forward(cfg, weights: dict, emb: np.ndarray, n_segments: int, dtype=np.float32,
-            A0=None, z0=None):
-    """Sequential ARMT prefill over n_segments segments of emb [n_segments*seg_len, d].
+def forward_tokens(cfg, weights: dict, emb: np.ndarray, dtype=np.float32, A0=None, z0=None):
+    """Sequential ARMT prefill of one sequence of T = emb.shape[0] tokens.
 
-    Cell (l, s) takes layer l-1's output for segment s (for l = 0: the segment's
-    embeddings followed by the memory tokens) and layer l's memory state after segment
-    s-1 (zeros before segment 0). Returns (out [n_segments*seg_len, d], A [L, dk, dv],
-    z [L, dk]) in `dtype`.
+    [P1 "Implementation": the sequence is cut into ceil(T / segment_length) segments, each
+    ending at min(start + segment_length, T).] So every segment holds seg_len tokens except
+    possibly the last, which holds the rest; each segment is followed by the memory tokens.
+    Cell (l, s) takes layer l-1's output for segment s (for l = 0: the segment's embeddings
+    followed by the memory tokens) and layer l's memory state after segment s-1 (A0, z0, or
+    zeros, before segment 0). Returns (out [T, d], A [L, dk, dv], z [L, dk]) in `dtype`.
     """
     L, seg = cfg.n_layers, cfg.seg_len
     emb = np.asarray(emb, dtype=dtype)
+    T = emb.shape[0]
     mem = np.asarray(weights["mem_tokens"], dtype=dtype)
     lws = [layer_weights(weights, l, dtype) for l in range(L)]
     A = [np.zeros((cfg.d_k, cfg.d_v), dtype) if A0 is None else np.array(A0[l], dtype) for l in range(L)]
     z = [np.zeros(cfg.d_k, dtype) if z0 is None else np.array(z0[l], dtype) for l in range(L)]
-    out = np.empty((n_segments * seg, cfg.d_model), dtype)
-    for s in range(n_segments):
-        x = np.concatenate([emb[s * seg:(s + 1) * seg], mem], axis=0)
+    out = np.empty((T, cfg.d_model), dtype)
+    for s in range(-(-T // seg)):
+        lo, hi = s * seg, min((s + 1) * seg, T)
+        x = np.concatenate([emb[lo:hi], mem], axis=0)
         for l in range(L):
             x, A[l], z[l] = armt_cell(x, lws[l], A[l], z[l], cfg)
-        out[s * seg:(s + 1) * seg] = x[:seg]
+        out[lo:hi] = x[:hi - lo]
     return out, np.stack(A), np.stack(z)
+
+
+def forward(cfg, weights: dict, emb: np.ndarray, n_segments: int, dtype=np.float32,
+            A0=None, z0=None):
+    """Sequential ARMT prefill over n_segments full segments of emb [n_segments*seg_len, d].
+
+    Returns (out [n_segments*seg_len, d], A [L, dk, dv], z [L, dk]) in `dtype`.
+    """
+    return forward_tokens(cfg, weights, np.asarray(emb)[:n_segments * cfg.seg_len], dtype, A0, z0)
+
+
+def forward_batch(cfg, weights: dict, embs: list, dtype=np.float32, A0=None, z0=None):
+    """A batch of independent sequences (embs[b]: [T_b, d]), each run by forward_tokens with
+    its own memory state (A0[b], z0[b] or zeros). Returns ([out_b], A [B, L, dk, dv],
+    z [B, L, dk])."""
+    outs, As, zs = [], [], []
+    for b, e in enumerate(embs):
+        o, A, z = forward_tokens(cfg, weights, e, dtype, None if A0 is None else A0[b], None if z0 is None else z0[b])
+        outs.append(o)
+        As.append(A)
+        zs.append(z)
+    return outs, np.stack(As), np.stack(zs)

@@ -248,6 +248,64 @@ def test_forward_matches_torch_reference_model():
     assert np.abs(got[1]).max() > 0.1
 
 
+def _torch_forward_tokens(cfg, w, emb):
+    """The torch reference model over one sequence of any length: its last segment, if
+    short, runs as a segment of a model whose segment length is that segment's length."""
+    L, seg, T = cfg.n_layers, cfg.seg_len, emb.shape[0]
+    A = [np.zeros((cfg.d_k, cfg.d_v)) for _ in range(L)]
+    z = [np.zeros(cfg.d_k) for _ in range(L)]
+    outs = []
+    for lo in range(0, T, seg):
+        part = emb[lo:lo + seg]
+        c = cfg.with_(seg_len=part.shape[0])
+        x = np.concatenate([part, w["mem_tokens"]]).astype(np.float64)
+        for l in range(L):
+            lw = {k: v[l] for k, v in w.items() if k != "mem_tokens"}
+            x, A[l], z[l] = _torch_cell(x, lw, A[l], z[l], c)
+        outs.append(x[:part.shape[0]])
+    return np.concatenate(outs), np.stack(A), np.stack(z)
+
+
+@pytest.mark.parametrize("extra", [1, 5, 11])
+def test_short_last_segment_matches_torch_reference_model(extra):
+    cfg = SMALL
+    w = _random_gains(make_weights(cfg, seed=34, std=0.2), 35)
+    emb = make_embeddings(cfg, 3, seed=36)[:2 * cfg.seg_len + extra]
+    got = armt.forward_tokens(cfg, w, emb, dtype=np.float64)
+    ref = _torch_forward_tokens(cfg, w, emb)
+    assert got[0].shape == (2 * cfg.seg_len + extra, cfg.d_model)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-10, atol=1e-11)
+
+
+def test_short_sequence_is_one_segment_of_its_own_length():
+    """A sequence shorter than a segment gives the result of a model whose segments are
+    exactly that long (memory tokens at positions T .. T + n_mem - 1)."""
+    cfg = SMALL
+    w = make_weights(cfg, seed=37, std=0.2)
+    emb = make_embeddings(cfg, 1, seed=38)[:7]
+    got = armt.forward_tokens(cfg, w, emb, dtype=np.float64)
+    ref = armt.forward(cfg.with_(seg_len=7), w, emb, 1, dtype=np.float64)
+    for g, r in zip(got, ref):
+        np.testing.assert_array_equal(g, r)
+    # and the memory rows are the cell's last rows, not rows seg_len.. of a full segment
+    full = armt.forward(cfg, w, make_embeddings(cfg, 1, seed=38), 1, dtype=np.float64)
+    assert np.abs(full[1] - got[1]).max() > 1e-6
+
+
+def test_batch_entries_are_the_sequences_alone():
+    cfg = SMALL
+    w = make_weights(cfg, seed=39, std=0.2)
+    embs = [make_embeddings(cfg, 3, seed=40 + b)[:n] for b, n in enumerate([2 * cfg.seg_len + 3, cfg.seg_len, 4])]
+    outs, A, z = armt.forward_batch(cfg, w, embs, dtype=np.float64)
+    assert A.shape == (3, cfg.n_layers, cfg.d_k, cfg.d_v) and z.shape == (3, cfg.n_layers, cfg.d_k)
+    for b, e in enumerate(embs):
+        ref = _torch_forward_tokens(cfg, w, e)
+        np.testing.assert_allclose(outs[b], ref[0], rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(A[b], ref[1], rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(z[b], ref[2], rtol=1e-10, atol=1e-11)
+
+
 # -------------------------------------------------------------- recurrence invariants
 
 def test_later_segments_do_not_change_earlier_outputs():

@@ -68,3 +68,40 @@ def test_bf16_rounding_of_the_input_generator():
     np.testing.assert_array_equal(round_to_bf16(x).view(np.uint32), bf16_bits_to_f32(bf16_bits(x)).view(np.uint32))
     # ties go to even: 1 + 2^-8 sits halfway between 1 and 1 + 2^-7
     assert round_to_bf16(np.array([1.0 + 2.0 ** -8], np.float32))[0] == 1.0
+
+
+def brute_force_batch(L, S):
+    """All cells (b, l, s) of a batch grouped by l + s, each group ordered by (l, b)."""
+    cells = [(b, l, s) for b, n in enumerate(S) for l in range(L) for s in range(n)]
+    cells.sort(key=lambda c: (c[1] + c[2], c[1], c[0]))
+    groups = {}
+    for b, l, s in cells:
+        groups.setdefault(l + s, []).append((b, l, s))
+    return [groups[k] for k in sorted(groups)]
+
+
+@pytest.mark.parametrize("S", [[1], [3, 1], [2, 5, 2], [4, 4], [1, 1, 1, 7]])
+@pytest.mark.parametrize("L", [1, 2, 5])
+def test_batch_diagonals_brute_force(L, S):
+    q = armt.schedule_quads(L, S, "diagonal")
+    got = [[tuple(r[1:]) for r in q if r[0] == t] for t in range(q[:, 0].max() + 1)]
+    assert got == brute_force_batch(L, S)
+    assert len(q) == L * sum(S) and len({tuple(r[1:]) for r in q}) == len(q)
+    where = {tuple(r[1:]): r[0] for r in q}
+    for (b, l, s), t in where.items():
+        if l > 0:
+            assert where[(b, l - 1, s)] < t
+        if s > 0:
+            assert where[(b, l, s - 1)] < t
+    # at most one cell per (sequence, layer) in a step: each state is updated in place
+    for t in range(q[:, 0].max() + 1):
+        bl = [(r[1], r[2]) for r in q if r[0] == t]
+        assert len(set(bl)) == len(bl)
+    # one sequence: the single-sequence schedule with a zero sequence column
+    if len(S) == 1:
+        np.testing.assert_array_equal(q[:, [0, 2, 3]], armt.schedule_triples(L, S[0], "diagonal"))
+
+
+def test_batch_sequential_order():
+    q = armt.schedule_quads(2, [2, 1], "sequential")
+    np.testing.assert_array_equal(q, [[0, 0, 0, 0], [1, 0, 1, 0], [2, 0, 0, 1], [3, 0, 1, 1], [4, 1, 0, 0], [5, 1, 1, 0]])
