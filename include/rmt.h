@@ -89,9 +89,16 @@ typedef struct {
 typedef struct rmt_handle rmt_handle;
 
 /* Validate cfg, copy and pack the weights into library-owned device memory (on the
- * current CUDA device), allocate activations and state. Synchronous. The caller may free
- * its weight buffers when this returns. *out is set only on RMT_OK. */
+ * current CUDA device), allocate activations and state for one sequence. Synchronous. The
+ * caller may free its weight buffers when this returns. *out is set only on RMT_OK. */
 rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle** out);
+
+/* Size the handle's activations and memory state for up to max_batch sequences per forward
+ * (rmt_create sizes them for one). Synchronizes the device and reallocates when max_batch is
+ * above the current size; a smaller max_batch is a no-op. A forward with a larger batch does
+ * this itself, so calling it first keeps later forwards free of device allocations.
+ * RMT_ENOMEM leaves the handle without activations until a later reservation succeeds. */
+rmt_status rmt_reserve(rmt_handle* h, int32_t max_batch);
 
 /* ARMT prefill of n_segments segments (batch 1).
  *   emb        [n_segments*seg_len, d_model] in cfg.dtype, device or host.
@@ -118,6 +125,29 @@ rmt_status rmt_forward_resume(rmt_handle* h, const void* emb, int32_t n_segments
                               const float* in_A, const float* in_z, void* out_hidden, float* out_A, float* out_z,
                               void* stream);
 
+/* Batched, variable-length ARMT prefill ("Implementation" of the diagonal-batching skill
+ * page: a [B, T, D] input cut into ceil(T / seg_len) segments, the last one ending at T).
+ *   batch      number of sequences, >= 1.
+ *   n_tokens   host array [batch]: tokens of each sequence, each >= 1. Sequence b has
+ *              ceil(n_tokens[b] / seg_len) segments; its last segment holds the remaining
+ *              r = n_tokens[b] - (segments - 1) * seg_len tokens, followed as every segment by
+ *              the n_mem memory tokens (positions r .. r + n_mem - 1 of that segment).
+ *   emb        [sum(n_tokens), d_model] in cfg.dtype, device or host: the sequences packed one
+ *              after another (equal lengths T: the row-major [batch, T, d_model] tensor).
+ *   out_hidden same shape and packing: the last layer's hidden states at the token rows.
+ *   in_A/in_z  [batch, n_layers, d_k, d_v] / [batch, n_layers, d_k] fp32 initial states,
+ *              device or host, both given or both NULL (zeros); may alias out_A / out_z.
+ *   out_A/out_z the same shapes, or NULL: each sequence's state after its last segment.
+ * Sequences do not interact: each result is that of the sequence run alone. RMT_DIAGONAL
+ * puts every cell (b, l, s) with l + s = d of all sequences into step d (layers ascending,
+ * then sequences); RMT_SEQUENTIAL runs one cell per step, sequences outermost, then segments,
+ * then layers. Both give the same bits. Grows the activations (rmt_reserve) when batch is
+ * above the reserved size. RMT_EINVAL on a non-positive batch or length, or more than 2^30
+ * tokens. Other behaviour as rmt_forward. */
+rmt_status rmt_forward_batch(rmt_handle* h, const void* emb, int32_t batch, const int32_t* n_tokens,
+                             rmt_schedule schedule, const float* in_A, const float* in_z, void* out_hidden,
+                             float* out_A, float* out_z, void* stream);
+
 /* The execution order as int32 triples (step, layer, segment), one per cell, n_layers*
  * n_segments of them: steps ascend; within a diagonal step layers ascend. Host memory,
  * cap = capacity of out_dls in int32 elements (>= 3*L*S). Needs no GPU. */
@@ -126,8 +156,15 @@ rmt_status rmt_schedule_table(int32_t n_layers, int32_t n_segments, rmt_schedule
 rmt_status rmt_get_schedule(const rmt_handle* h, int32_t n_segments, rmt_schedule schedule,
                             int32_t* out_dls, size_t cap);
 
+/* The execution order of rmt_forward_batch as int32 quadruples (step, sequence, layer,
+ * segment), one per cell; n_segments is a host array [batch] (>= 1 each) and cap the capacity
+ * of out_dbls in int32 elements (>= 4 * n_layers * sum(n_segments)). Needs no GPU. */
+rmt_status rmt_schedule_table_batch(int32_t n_layers, int32_t batch, const int32_t* n_segments,
+                                    rmt_schedule schedule, int32_t* out_dbls, size_t cap);
+
 /* The (step, layer, segment) triples the device recorded for each cell during the last
- * forward, in schedule-table order (written by the memory-update kernel of each cell).
+ * forward, in schedule-table order (written by the memory-update kernel of each cell); after
+ * rmt_forward_batch, the order of rmt_schedule_table_batch without its sequence column.
  * Synchronizes the device. RMT_ESTATE before the first forward. */
 rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap);
 

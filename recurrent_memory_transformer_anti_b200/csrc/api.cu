@@ -13,7 +13,9 @@
 // Each kernel does the same arithmetic for a cell whatever else shares its launch, so the
 // two schedules give identical bits ("Dependency Preservation" in "Architecture
 // Overview"; arXiv 2506.05229 abstract: a pure run-time reordering with exact recurrence).
+#include <climits>
 #include <cmath>
+#include <cstdint>
 #include <cstring>
 #include <map>
 #include <string>
@@ -61,28 +63,76 @@ bool is_pinned_host_ptr(const void* p) {
 struct Table {
   std::vector<Cell> cells;  // host copy, execution order
   std::vector<int> off, cnt;
+  // per step: its first n_first cells are of layer 0 (assembled from the embeddings) and its
+  // last n_last cells of layer L-1 (emitted)
+  std::vector<int> n_first, n_last;
+  std::vector<int> seg_base;  // per sequence: ordinal of its first segment among all segments
   Cell* dev = nullptr;
 };
 
-void build_table(int L, int S, rmt_schedule sch, Table& t) {
+// Execution order of the cells (b, l, s) of a batch, sequence b having S[b] segments.
+// Diagonal: step d holds every cell with l + s = d, in ascending layer and, within a layer,
+// ascending sequence; steps with no cell are skipped. Sequential: one cell per step,
+// sequences outermost, then segments, then layers. Only l, s and b are set.
+void order_cells(int L, const std::vector<int>& S, rmt_schedule sch, Table& t) {
   t.cells.clear();
   t.off.clear();
   t.cnt.clear();
+  t.n_first.clear();
+  t.n_last.clear();
+  const int B = static_cast<int>(S.size());
+  int smax = 0;
+  for (int sb : S) smax = sb > smax ? sb : smax;
+  auto push_step = [&](size_t begin) {
+    const int n = static_cast<int>(t.cells.size() - begin);
+    int nf = 0, nl = 0;
+    while (nf < n && t.cells[begin + nf].l == 0) ++nf;
+    while (nl < n && t.cells[t.cells.size() - 1 - nl].l == L - 1) ++nl;
+    t.off.push_back(static_cast<int>(begin));
+    t.cnt.push_back(n);
+    t.n_first.push_back(nf);
+    t.n_last.push_back(nl);
+  };
   if (sch == RMT_DIAGONAL) {
-    for (int d = 0; d <= L + S - 2; ++d) {
-      const int lo = d - S + 1 > 0 ? d - S + 1 : 0, hi = d < L - 1 ? d : L - 1;
-      if (lo > hi) continue;
-      t.off.push_back(static_cast<int>(t.cells.size()));
-      for (int l = lo; l <= hi; ++l) t.cells.push_back(Cell{l, d - l});
-      t.cnt.push_back(hi - lo + 1);
+    for (int d = 0; d <= L + smax - 2; ++d) {
+      const size_t begin = t.cells.size();
+      for (int l = 0; l < L && l <= d; ++l)
+        for (int b = 0; b < B; ++b)
+          if (d - l < S[b]) t.cells.push_back(Cell{l, d - l, b, 0, 0, 0, 0, 0});
+      if (t.cells.size() > begin) push_step(begin);
     }
   } else {
-    for (int s = 0; s < S; ++s)
-      for (int l = 0; l < L; ++l) {
-        t.off.push_back(static_cast<int>(t.cells.size()));
-        t.cells.push_back(Cell{l, s});
-        t.cnt.push_back(1);
-      }
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < S[b]; ++s)
+        for (int l = 0; l < L; ++l) {
+          const size_t begin = t.cells.size();
+          t.cells.push_back(Cell{l, s, b, 0, 0, 0, 0, 0});
+          push_step(begin);
+        }
+  }
+}
+
+// The full cell table of a batch whose sequence b holds T[b] tokens (packed one after
+// another): ceil(T[b] / seg) segments, the last one possibly short.
+void build_table(int L, int seg, int n_mem, const std::vector<int>& T, rmt_schedule sch, Table& t) {
+  std::vector<int> S(T.size()), base(T.size());
+  t.seg_base.assign(T.size(), 0);
+  int rows = 0, segs = 0;
+  for (size_t b = 0; b < T.size(); ++b) {
+    S[b] = (T[b] + seg - 1) / seg;
+    base[b] = rows;
+    t.seg_base[b] = segs;
+    rows += T[b];
+    segs += S[b];
+  }
+  order_cells(L, S, sch, t);
+  for (Cell& c : t.cells) {
+    const int tokens = T[c.b] - c.s * seg;
+    c.m = (tokens < seg ? tokens : seg) + n_mem;
+    c.k = c.b * L + c.l;
+    c.xin = c.b * n_slots(L) + in_slot(L, c.l, c.s);
+    c.xout = c.b * n_slots(L) + out_slot(L, c.l, c.s);
+    c.t0 = base[c.b] + c.s * seg;
   }
 }
 
@@ -106,7 +156,7 @@ rmt_status device_scratch(int G, const Cell** cells, int** err) {
   if (G > s.cap) {
     const int cap = G > 4096 ? G : 4096;
     std::vector<Cell> h(cap);
-    for (int g = 0; g < cap; ++g) h[g] = Cell{g, 0};
+    for (int g = 0; g < cap; ++g) h[g] = identity_cell(g);
     Cell* p = nullptr;
     if (cudaMalloc(&p, sizeof(Cell) * cap) != cudaSuccess) return fail(RMT_ENOMEM, "cell table allocation failed");
     RMT_CUDA(cudaMemcpy(p, h.data(), sizeof(Cell) * cap, cudaMemcpyHostToDevice));
@@ -187,7 +237,7 @@ struct rmt_handle {
     }
     return true;
   }
-  std::map<std::pair<int, int>, Table> tables;
+  std::map<std::pair<std::vector<int>, int>, Table> tables;  // keyed by (token counts, schedule)
   CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
   // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
   CUtensorMap tp_xb, tp_om, tp_att, tp_u;
@@ -196,6 +246,9 @@ struct rmt_handle {
   // depends on it for the RoPE and SwiGLU row orders)
   bool pair_mo = false, pair_qkv = false, pair_o = false, pair_gu = false, pair_d = false;
   std::vector<void*> allocs;
+  // activations and memory state, sized for cap_b sequences (rmt_reserve)
+  int cap_b = 0;
+  std::vector<void*> act_allocs;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
   struct ProbeRec {
     int kind;
@@ -226,9 +279,28 @@ struct rmt_handle {
     allocs.push_back(p);
     return p;
   }
+  void* act_alloc(size_t bytes) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    act_allocs.push_back(p);
+    return p;
+  }
+  void free_acts() {
+    for (void* p : act_allocs) cudaFree(p);
+    act_allocs.clear();
+    cap_b = 0;
+    x = nullptr;
+    xb = nullptr;
+    qkv = att = u = om = nullptr;
+    qm = part = A = z = ss1 = ss2 = nullptr;
+  }
   void release() {
     for (void* p : allocs) cudaFree(p);
     allocs.clear();
+    free_acts();
     for (auto& kv : tables)
       if (kv.second.dev) cudaFree(kv.second.dev);
     tables.clear();
@@ -346,7 +418,10 @@ rmt_status pack_weights(rmt_handle* h, const rmt_weights* w) {
 
 rmt_status build_maps(rmt_handle* h) {
   const rmt_cfg& c = h->cfg;
-  const uint64_t L = c.n_layers, d = c.d_model, hd = uint64_t(c.n_heads) * c.head_dim, F = c.d_ff, M = h->M;
+  // stacks of the cap_b sequences: residual slots [cap_b * n_slots], layer scratch [cap_b * L]
+  const uint64_t L = uint64_t(h->cap_b) * c.n_layers, d = c.d_model, hd = uint64_t(c.n_heads) * c.head_dim,
+                 F = c.d_ff, M = h->M, NS = uint64_t(h->cap_b) * n_slots(c.n_layers);
+  const uint64_t LW = c.n_layers;  // weight stacks
   h->bn_mq = tc_pick_bn(c.d_k, kEpiStoreF32, 0);
   h->bn_mo = tc_pick_bn(c.d_model, kEpiResid, 0);
   h->bn_qkv = tc_pick_bn(h->Nqkv, kEpiRope, c.head_dim);
@@ -359,20 +434,80 @@ rmt_status build_maps(rmt_handle* h) {
   // weight boxes: 128 rows per CTA on the pair GEMM, else the tile width
   const uint32_t pb = static_cast<uint32_t>(pair_token_tile(static_cast<int>(M)) / 2);
   const bool any_pair = h->pair_mo || h->pair_qkv || h->pair_o || h->pair_gu || h->pair_d;
-  bool ok = map(&h->tm_xb, h->xb, d, M, n_slots(c.n_layers), 128) && map(&h->tm_om, h->om, c.d_v, M, L, 128) &&
+  bool ok = map(&h->tm_xb, h->xb, d, M, NS, 128) && map(&h->tm_om, h->om, c.d_v, M, L, 128) &&
             map(&h->tm_att, h->att, hd, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
-            map(&h->tm_wmq, h->w_mq, d, c.d_k, L, h->bn_mq) &&
-            map(&h->tm_wmo, h->w_mo, c.d_v, d, L, h->pair_mo ? 128 : h->bn_mo) &&
-            map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, L, h->pair_qkv ? 128 : h->bn_qkv) &&
-            map(&h->tm_wo, h->w_o, hd, d, L, h->pair_o ? 128 : h->bn_o) &&
-            map(&h->tm_wgu, h->w_gu, d, 2 * F, L, h->pair_gu ? 128 : h->bn_gu) &&
-            map(&h->tm_wd, h->w_d, F, d, L, h->pair_d ? 128 : h->bn_d) &&
-            (!any_pair || (map(&h->tp_xb, h->xb, d, M, n_slots(c.n_layers), pb) && map(&h->tp_om, h->om, c.d_v, M, L, pb) &&
+            map(&h->tm_wmq, h->w_mq, d, c.d_k, LW, h->bn_mq) &&
+            map(&h->tm_wmo, h->w_mo, c.d_v, d, LW, h->pair_mo ? 128 : h->bn_mo) &&
+            map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, LW, h->pair_qkv ? 128 : h->bn_qkv) &&
+            map(&h->tm_wo, h->w_o, hd, d, LW, h->pair_o ? 128 : h->bn_o) &&
+            map(&h->tm_wgu, h->w_gu, d, 2 * F, LW, h->pair_gu ? 128 : h->bn_gu) &&
+            map(&h->tm_wd, h->w_d, F, d, LW, h->pair_d ? 128 : h->bn_d) &&
+            (!any_pair || (map(&h->tp_xb, h->xb, d, M, NS, pb) && map(&h->tp_om, h->om, c.d_v, M, L, pb) &&
                            map(&h->tp_att, h->att, hd, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
-            make_tmap_f32_resid(&h->tm_x, h->x, d, M, n_slots(c.n_layers)) &&
+            make_tmap_f32_resid(&h->tm_x, h->x, d, M, NS) &&
             (c.head_dim < 64 || map(&h->tm_rope, h->rope_h, c.head_dim, M, 1, 32));
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
+}
+
+// (Re)allocate the activations, the layer scratch and the memory state for B sequences and
+// rebuild the tensor maps over them. Waits for the device first: earlier forwards may still
+// use the old buffers.
+rmt_status reserve_acts(rmt_handle* h, int B) {
+  if (B <= h->cap_b) return RMT_OK;
+  RMT_CUDA(cudaDeviceSynchronize());
+  h->free_acts();
+  const rmt_cfg& c = h->cfg;
+  const size_t nb = B, L = c.n_layers, d = c.d_model, M = h->M, es = h->es, hd = size_t(c.n_heads) * c.head_dim,
+               F = c.d_ff, dk = c.d_k, dv = c.d_v, BL = nb * L;
+  struct {
+    void** p;
+    size_t bytes;
+  } plan[] = {
+      {reinterpret_cast<void**>(&h->x), nb * n_slots(c.n_layers) * M * d * 4},
+      {&h->qkv, BL * M * h->Nqkv * es},   {&h->att, BL * M * hd * es},
+      {reinterpret_cast<void**>(&h->ss1), BL * M * (d / 16 + 1) * 4},
+      {reinterpret_cast<void**>(&h->ss2), BL * M * (d / 16 + 1) * 4},
+      {&h->u, BL * M * F * es},           {&h->om, BL * M * dv * es},
+      {reinterpret_cast<void**>(&h->qm), BL * M * dk * 4},
+      {reinterpret_cast<void**>(&h->part), BL * h->nsplit * size_t(c.n_mem) * (dk + dv) * 4},
+      {reinterpret_cast<void**>(&h->A), BL * dk * dv * 4},
+      {reinterpret_cast<void**>(&h->z), BL * dk * 4},
+  };
+  for (auto& e : plan) {
+    *e.p = h->act_alloc(e.bytes);
+    if (!*e.p) {
+      h->free_acts();
+      return fail(RMT_ENOMEM, "activation allocation failed");
+    }
+  }
+  if (h->bf16) {
+    h->xb = static_cast<__half*>(h->act_alloc(nb * n_slots(c.n_layers) * M * d * 2));
+    if (!h->xb) {
+      h->free_acts();
+      return fail(RMT_ENOMEM, "activation allocation failed");
+    }
+  }
+  if (cudaMemset(h->x, 0, nb * n_slots(c.n_layers) * M * d * 4) != cudaSuccess) {
+    h->free_acts();
+    return fail(RMT_ECUDA, "cudaMemset failed");
+  }
+  h->cap_b = B;
+  if (h->bf16) {
+    rmt_status st = build_maps(h);
+    if (st != RMT_OK) {
+      h->free_acts();
+      return st;
+    }
+    h->ss_parts = (c.d_model / h->bn_o) * 2;  // memo and O projections: N = d_model, two halves per tile
+    if (h->bn_mo != h->bn_o) {
+      h->free_acts();
+      return fail(RMT_EINVAL, "inconsistent projection tiles");
+    }
+  } else {
+    h->ss_parts = (c.d_model + 127) / 128;  // fp32 kernel: one block per 128-column tile
+  }
+  return RMT_OK;
 }
 
 enum Proj { kProjMemQ, kProjMemO, kProjQkv, kProjO, kProjGateUp, kProjDown };
@@ -470,17 +605,24 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   const rmt_cfg& c = h->cfg;
   const int L = c.n_layers, d = c.d_model, M = h->M, G = t.cnt[step], off = t.off[step];
   const Cell* cells = t.dev + off;
-  const Cell first = t.cells[off], last = t.cells[off + G - 1];
-  const size_t slot_elems = size_t(M) * d;
-  // algorithmic work per launch (flops; bytes that must cross HBM at least once)
-  const double g = G, m = M, dd = d, es = h->es, dk = c.d_k, dv = c.d_v, hd = double(c.n_heads) * c.head_dim,
+  const int n_first = t.n_first[step], n_last = t.n_last[step];
+  // algorithmic work per launch (flops; bytes that must cross HBM at least once), over the
+  // valid rows of the step's cells: g * m = their rows, pairs = their causal (query, key) pairs
+  double rows = 0, pairs = 0, rows_first = 0, rows_last = 0;
+  for (int i = 0; i < G; ++i) {
+    const double mc = cell_rows(t.cells[off + i], M);
+    rows += mc;
+    pairs += mc * (mc + 1) / 2;
+    if (i < n_first) rows_first += mc;
+    if (i >= G - n_last) rows_last += mc - c.n_mem;
+  }
+  const double g = G, m = rows / G, dd = d, es = h->es, dk = c.d_k, dv = c.d_v, hd = double(c.n_heads) * c.head_dim,
                nq = h->Nqkv, F = c.d_ff, n = c.n_mem, ea = h->bf16 ? 2.0 : 4.0;
   cudaError_t e;
-  if (first.l == 0) {
-    const int sl = in_slot(L, 0, first.s);
-    e = launch_kind(h, RMT_K_ASSEMBLE, 0, m * dd * (es + 4 + (h->bf16 ? 2 : 0)), st, [&] {
-      return launch_assemble(emb, h->memtok, h->x + sl * slot_elems, h->bf16 ? h->xb + sl * slot_elems : nullptr,
-                             c.seg_len, c.n_mem, d, first.s, h->bf16, st);
+  if (n_first > 0) {
+    e = launch_kind(h, RMT_K_ASSEMBLE, 0, rows_first * dd * (es + 4 + (h->bf16 ? 2 : 0)), st, [&] {
+      return launch_assemble(cells, n_first, emb, h->memtok, h->x, h->bf16 ? h->xb : nullptr, M, c.n_mem, d, h->bf16,
+                             st);
     });
     if (e != cudaSuccess) return e;
   }
@@ -499,7 +641,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   e = launch_kind(h, RMT_K_QKV, 2 * g * m * nq * dd, g * (m * dd * es + nq * dd * es + m * nq * es), st,
                   [&] { return run_proj(h, kProjQkv, cells, G, st); });
   if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_ATTENTION, g * c.n_heads * 4.0 * c.head_dim * m * (m + 1) / 2,
+  e = launch_kind(h, RMT_K_ATTENTION, c.n_heads * 4.0 * c.head_dim * pairs,
                   g * (m * nq * es + m * hd * es), st, [&] {
                     AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err};
                     if (h->bf16 && attention_tc_supported(c.head_dim))
@@ -519,7 +661,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_MEMKV, 2 * g * n * (dk + dv) * dd,
                   g * (n * dd * 4 + (dk + dv) * dd * es + h->nsplit * n * (dk + dv) * 4), st, [&] {
-                    MemKvArgs a{h->x, M, d, c.seg_len, c.n_mem, kOutSlot, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
+                    MemKvArgs a{h->x, M, d, c.n_mem, kOutSlot, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
                     return launch_mem_kv(a, h->bf16, st);
                   });
   if (e != cudaSuccess) return e;
@@ -530,9 +672,9 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                     return launch_mem_update(a, st);
                   });
   if (e != cudaSuccess) return e;
-  if (last.l == L - 1) {
-    e = launch_kind(h, RMT_K_EMIT, 0, double(c.seg_len) * dd * (4 + es), st, [&] {
-      return launch_emit(h->x + out_slot(L, L - 1, last.s) * slot_elems, out, c.seg_len, d, last.s, h->bf16, st);
+  if (n_last > 0) {
+    e = launch_kind(h, RMT_K_EMIT, 0, rows_last * dd * (4 + es), st, [&] {
+      return launch_emit(cells + G - n_last, n_last, h->x, out, M, c.n_mem, d, h->bf16, st);
     });
     if (e != cudaSuccess) return e;
   }
@@ -566,7 +708,7 @@ rmt_status rmt_schedule_table(int32_t n_layers, int32_t n_segments, rmt_schedule
   const size_t need = 3 * size_t(n_layers) * size_t(n_segments);
   if (cap < need) return fail(RMT_EINVAL, "out_dls capacity below 3*n_layers*n_segments");
   Table t;
-  build_table(n_layers, n_segments, schedule, t);
+  order_cells(n_layers, std::vector<int>{n_segments}, schedule, t);
   size_t k = 0;
   for (size_t step = 0; step < t.off.size(); ++step)
     for (int i = 0; i < t.cnt[step]; ++i) {
@@ -574,6 +716,32 @@ rmt_status rmt_schedule_table(int32_t n_layers, int32_t n_segments, rmt_schedule
       out_dls[k++] = int32_t(step);
       out_dls[k++] = c.l;
       out_dls[k++] = c.s;
+    }
+  return RMT_OK;
+}
+
+rmt_status rmt_schedule_table_batch(int32_t n_layers, int32_t batch, const int32_t* n_segments, rmt_schedule schedule,
+                                    int32_t* out_dbls, size_t cap) {
+  if (n_layers <= 0 || batch <= 0 || !n_segments) return fail(RMT_EINVAL, "n_layers and batch must be positive");
+  if (schedule != RMT_DIAGONAL && schedule != RMT_SEQUENTIAL) return fail(RMT_EINVAL, "unknown schedule");
+  if (!out_dbls) return fail(RMT_EINVAL, "out_dbls is null");
+  std::vector<int> S(n_segments, n_segments + batch);
+  size_t cells = 0;
+  for (int v : S) {
+    if (v <= 0) return fail(RMT_EINVAL, "every sequence needs at least one segment");
+    cells += size_t(v) * size_t(n_layers);
+  }
+  if (cap < 4 * cells) return fail(RMT_EINVAL, "out_dbls capacity below 4 * cells");
+  Table t;
+  order_cells(n_layers, S, schedule, t);
+  size_t k = 0;
+  for (size_t step = 0; step < t.off.size(); ++step)
+    for (int i = 0; i < t.cnt[step]; ++i) {
+      const Cell c = t.cells[t.off[step] + i];
+      out_dbls[k++] = int32_t(step);
+      out_dbls[k++] = c.b;
+      out_dbls[k++] = c.l;
+      out_dbls[k++] = c.s;
     }
   return RMT_OK;
 }
@@ -612,15 +780,6 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
       {&h->w_d, L * d * F * es},         {&h->w_mq, L * dk * d * es},       {&h->w_mo, L * d * dv * es},
       {&h->w_mkv, L * (dk + dv) * d * es}, {&h->g1, L * d * es},            {&h->g2, L * d * es},
       {&h->memtok, size_t(c.n_mem) * d * es},
-      {reinterpret_cast<void**>(&h->x), n_slots(c.n_layers) * M * d * 4},
-      {&h->qkv, L * M * h->Nqkv * es},   {&h->att, L * M * hd * es},
-      {reinterpret_cast<void**>(&h->ss1), L * M * (d / 16 + 1) * 4},
-      {reinterpret_cast<void**>(&h->ss2), L * M * (d / 16 + 1) * 4},
-      {&h->u, L * M * F * es},           {&h->om, L * M * dv * es},
-      {reinterpret_cast<void**>(&h->qm), L * M * dk * 4},
-      {reinterpret_cast<void**>(&h->part), L * h->nsplit * size_t(c.n_mem) * (dk + dv) * 4},
-      {reinterpret_cast<void**>(&h->A), L * dk * dv * 4},
-      {reinterpret_cast<void**>(&h->z), L * dk * 4},
       {reinterpret_cast<void**>(&h->rope), M * (c.head_dim / 2) * sizeof(float2)},
       {reinterpret_cast<void**>(&h->rope_h), M * (c.head_dim / 2) * sizeof(__half2)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
@@ -628,10 +787,6 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   for (auto& e : plan) {
     *e.p = h->alloc(e.bytes);
     if (!*e.p) return bail(fail(RMT_ENOMEM, "device allocation failed"));
-  }
-  if (h->bf16) {
-    h->xb = static_cast<__half*>(h->alloc(n_slots(c.n_layers) * M * d * 2));
-    if (!h->xb) return bail(fail(RMT_ENOMEM, "device allocation failed"));
   }
   if (h->bf16) {
     const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
@@ -676,15 +831,8 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
         cudaMemcpy(h->rope_h, tab_h.data(), tab_h.size() * sizeof(__half2), cudaMemcpyHostToDevice) != cudaSuccess)
       return bail(fail(RMT_ECUDA, "rope table upload failed"));
   }
-  if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess || cudaMemset(h->x, 0, n_slots(c.n_layers) * M * d * 4) != cudaSuccess)
-    return bail(fail(RMT_ECUDA, "cudaMemset failed"));
-  if (h->bf16) {
-    if ((st = build_maps(h)) != RMT_OK) return bail(st);
-    h->ss_parts = (c.d_model / h->bn_o) * 2;  // memo and O projections: N = d_model, two halves per tile
-    if (h->bn_mo != h->bn_o) return bail(fail(RMT_EINVAL, "inconsistent projection tiles"));
-  } else {
-    h->ss_parts = (c.d_model + 127) / 128;  // fp32 kernel: one block per 128-column tile
-  }
+  if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return bail(fail(RMT_ECUDA, "cudaMemset failed"));
+  if ((st = reserve_acts(h, 1)) != RMT_OK) return bail(st);
   if (cudaDeviceSynchronize() != cudaSuccess) return bail(fail(RMT_ECUDA, "weight packing failed"));
   *out = h;
   return RMT_OK;
@@ -692,23 +840,59 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
 
 namespace {
 
-rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, const float* in_A,
-                        const float* in_z, void* out_hidden, float* out_A, float* out_z, void* stream) {
+// Sequences of a forward: token counts, checked. A sequence needs at least one token; t0 of
+// every cell (an int) must stay in range.
+rmt_status check_lengths(int32_t batch, const int32_t* n_tokens, std::vector<int>& T, size_t& total) {
+  if (batch <= 0) return fail(RMT_EINVAL, "batch must be positive");
+  if (!n_tokens) return fail(RMT_EINVAL, "n_tokens is null");
+  T.assign(n_tokens, n_tokens + batch);
+  total = 0;
+  for (int v : T) {
+    if (v <= 0) return fail(RMT_EINVAL, "every sequence needs at least one token");
+    total += size_t(v);
+  }
+  if (total > size_t(INT32_MAX) / 2) return fail(RMT_EINVAL, "too many tokens");
+  return RMT_OK;
+}
+
+rmt_status forward_impl(rmt_handle* h, const void* emb, const std::vector<int>& T, size_t total_tokens,
+                        rmt_schedule schedule, const float* in_A, const float* in_z, void* out_hidden, float* out_A,
+                        float* out_z, void* stream) {
   if (!h) return fail(RMT_EINVAL, "null handle");
   if ((in_A == nullptr) != (in_z == nullptr)) return fail(RMT_EINVAL, "in_A and in_z must both be given or both be NULL");
   if (!emb || !out_hidden) return fail(RMT_EINVAL, "emb and out_hidden must not be null");
-  if (n_segments <= 0) return fail(RMT_EINVAL, "n_segments must be positive");
   if (schedule != RMT_DIAGONAL && schedule != RMT_SEQUENTIAL) return fail(RMT_EINVAL, "unknown schedule");
   DeviceGuard guard(h->dev);
   const rmt_cfg& c = h->cfg;
+  const int B = static_cast<int>(T.size());
+  RMT_TRY(reserve_acts(h, B));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t io_bytes = size_t(n_segments) * c.seg_len * c.d_model * h->es;
-  const size_t seg_bytes = size_t(c.seg_len) * c.d_model * h->es;
+  const size_t row_bytes = size_t(c.d_model) * h->es;
+  const size_t io_bytes = total_tokens * row_bytes;
+  const auto key = std::make_pair(T, int(schedule));
+  auto it = h->tables.find(key);
+  if (it == h->tables.end()) {
+    Table t;
+    build_table(c.n_layers, c.seg_len, c.n_mem, T, schedule, t);
+    if (cudaMalloc(&t.dev, sizeof(Cell) * t.cells.size()) != cudaSuccess)
+      return fail(RMT_ENOMEM, "cell table allocation failed");
+    if (cudaMemcpy(t.dev, t.cells.data(), sizeof(Cell) * t.cells.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(t.dev);
+      return fail(RMT_ECUDA, "cell table upload failed");
+    }
+    it = h->tables.emplace(key, std::move(t)).first;
+  }
+  const Table& t = it->second;
+  const size_t ncell = t.cells.size();
+  size_t n_segments = 0;
+  for (int v : T) n_segments += size_t((v + c.seg_len - 1) / c.seg_len);
   // page-locked host buffers: one copy per segment on side streams, each segment's input just
   // ahead of the step that assembles it and its output right after the step that emits it
   const bool in_pinned = is_pinned_host_ptr(emb), out_pinned = is_pinned_host_ptr(out_hidden);
-  if ((in_pinned || out_pinned) && !h->copy_resources(size_t(n_segments)))
+  if ((in_pinned || out_pinned) && !h->copy_resources(n_segments))
     return fail(RMT_ECUDA, "copy stream or event creation failed");
+  auto seg_ord = [&](const Cell& x) { return size_t(t.seg_base[x.b]) + size_t(x.s); };
+  auto seg_rows = [&](const Cell& x) { return size_t(x.m - c.n_mem); };
   const void* emb_dev = emb;
   if (is_host_ptr(emb)) {
     if (h->emb_stage_bytes < io_bytes) {
@@ -722,11 +906,14 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_
       // the staging buffer may still be read by an earlier forward on `st`
       RMT_CUDA(cudaEventRecord(h->copy_events[0], st));
       RMT_CUDA(cudaStreamWaitEvent(h->h2d, h->copy_events[0], 0));
-      for (int s = 0; s < n_segments; ++s) {
-        RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(h->emb_stage) + s * seg_bytes,
-                                 static_cast<const char*>(emb) + s * seg_bytes, seg_bytes, cudaMemcpyHostToDevice,
-                                 h->h2d));
-        RMT_CUDA(cudaEventRecord(h->copy_events[2 + 2 * s], h->h2d));
+      // segments in the order their layer-0 cells run
+      for (size_t i = 0; i < ncell; ++i) {
+        const Cell& x = t.cells[i];
+        if (x.l != 0) continue;
+        const size_t o = size_t(x.t0) * row_bytes;
+        RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(h->emb_stage) + o, static_cast<const char*>(emb) + o,
+                                 seg_rows(x) * row_bytes, cudaMemcpyHostToDevice, h->h2d));
+        RMT_CUDA(cudaEventRecord(h->copy_events[2 + 2 * seg_ord(x)], h->h2d));
       }
     } else {
       RMT_CUDA(cudaMemcpyAsync(h->emb_stage, emb, io_bytes, cudaMemcpyHostToDevice, st));
@@ -745,21 +932,6 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_
     }
     out_dev = h->out_stage;
   }
-  const auto key = std::make_pair(int(n_segments), int(schedule));
-  auto it = h->tables.find(key);
-  if (it == h->tables.end()) {
-    Table t;
-    build_table(c.n_layers, n_segments, schedule, t);
-    if (cudaMalloc(&t.dev, sizeof(Cell) * t.cells.size()) != cudaSuccess)
-      return fail(RMT_ENOMEM, "cell table allocation failed");
-    if (cudaMemcpy(t.dev, t.cells.data(), sizeof(Cell) * t.cells.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
-      cudaFree(t.dev);
-      return fail(RMT_ECUDA, "cell table upload failed");
-    }
-    it = h->tables.emplace(key, std::move(t)).first;
-  }
-  const Table& t = it->second;
-  const size_t ncell = t.cells.size();
   if (h->trace_cap < ncell) {
     if (h->trace) cudaFree(h->trace);
     h->trace = nullptr;
@@ -767,27 +939,32 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_
     if (cudaMalloc(&h->trace, 3 * sizeof(int) * ncell) != cudaSuccess) return fail(RMT_ENOMEM, "trace allocation failed");
     h->trace_cap = ncell;
   }
-  const size_t L = c.n_layers;
+  const size_t BL = size_t(B) * c.n_layers;
   if (in_A) {  // continue from the caller's state (the state after an earlier run's last segment)
-    RMT_CUDA(cudaMemcpyAsync(h->A, in_A, L * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
-    RMT_CUDA(cudaMemcpyAsync(h->z, in_z, L * c.d_k * sizeof(float), cudaMemcpyDefault, st));
+    RMT_CUDA(cudaMemcpyAsync(h->A, in_A, BL * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
+    RMT_CUDA(cudaMemcpyAsync(h->z, in_z, BL * c.d_k * sizeof(float), cudaMemcpyDefault, st));
   } else {
-    RMT_CUDA(cudaMemsetAsync(h->A, 0, L * c.d_k * c.d_v * sizeof(float), st));
-    RMT_CUDA(cudaMemsetAsync(h->z, 0, L * c.d_k * sizeof(float), st));
+    RMT_CUDA(cudaMemsetAsync(h->A, 0, BL * c.d_k * c.d_v * sizeof(float), st));
+    RMT_CUDA(cudaMemsetAsync(h->z, 0, BL * c.d_k * sizeof(float), st));
   }
   const bool split_in = in_pinned && emb_dev != emb, split_out = out_host && out_pinned;
   for (int step = 0; step < int(t.off.size()); ++step) {
-    const Cell first = t.cells[t.off[step]], last = t.cells[t.off[step] + t.cnt[step] - 1];
-    if (split_in && first.l == 0) RMT_CUDA(cudaStreamWaitEvent(st, h->copy_events[2 + 2 * first.s], 0));
+    const int off = t.off[step], G = t.cnt[step];
+    if (split_in)
+      for (int i = 0; i < t.n_first[step]; ++i)
+        RMT_CUDA(cudaStreamWaitEvent(st, h->copy_events[2 + 2 * seg_ord(t.cells[off + i])], 0));
     cudaError_t e = enqueue_step(h, t, step, emb_dev, out_dev, st);
     if (e != cudaSuccess) return fail(RMT_ECUDA, std::string("launch failed: ") + cudaGetErrorString(e));
-    if (split_out && last.l == int(L) - 1) {
-      cudaEvent_t done = h->copy_events[3 + 2 * last.s];
+    if (split_out && t.n_last[step] > 0) {
+      cudaEvent_t done = h->copy_events[3 + 2 * seg_ord(t.cells[off + G - 1])];
       RMT_CUDA(cudaEventRecord(done, st));
       RMT_CUDA(cudaStreamWaitEvent(h->d2h, done, 0));
-      RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(out_hidden) + last.s * seg_bytes,
-                               static_cast<const char*>(out_dev) + last.s * seg_bytes, seg_bytes,
-                               cudaMemcpyDeviceToHost, h->d2h));
+      for (int i = G - t.n_last[step]; i < G; ++i) {
+        const Cell& x = t.cells[off + i];
+        const size_t o = size_t(x.t0) * row_bytes;
+        RMT_CUDA(cudaMemcpyAsync(static_cast<char*>(out_hidden) + o, static_cast<const char*>(out_dev) + o,
+                                 seg_rows(x) * row_bytes, cudaMemcpyDeviceToHost, h->d2h));
+      }
     }
   }
   if (split_out) {
@@ -796,8 +973,8 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_
   } else if (out_host) {
     RMT_CUDA(cudaMemcpyAsync(out_hidden, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
   }
-  if (out_A) RMT_CUDA(cudaMemcpyAsync(out_A, h->A, L * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
-  if (out_z) RMT_CUDA(cudaMemcpyAsync(out_z, h->z, L * c.d_k * sizeof(float), cudaMemcpyDefault, st));
+  if (out_A) RMT_CUDA(cudaMemcpyAsync(out_A, h->A, BL * c.d_k * c.d_v * sizeof(float), cudaMemcpyDefault, st));
+  if (out_z) RMT_CUDA(cudaMemcpyAsync(out_z, h->z, BL * c.d_k * sizeof(float), cudaMemcpyDefault, st));
   h->traced_cells = int(ncell);
   RMT_CUDA(cudaGetLastError());
   return RMT_OK;
@@ -807,13 +984,34 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, int32_t n_segments, rmt_
 
 rmt_status rmt_forward(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule, void* out_hidden,
                        float* out_A, float* out_z, void* stream) {
-  return forward_impl(h, emb, n_segments, schedule, nullptr, nullptr, out_hidden, out_A, out_z, stream);
+  return rmt_forward_resume(h, emb, n_segments, schedule, nullptr, nullptr, out_hidden, out_A, out_z, stream);
 }
 
 rmt_status rmt_forward_resume(rmt_handle* h, const void* emb, int32_t n_segments, rmt_schedule schedule,
                               const float* in_A, const float* in_z, void* out_hidden, float* out_A, float* out_z,
                               void* stream) {
-  return forward_impl(h, emb, n_segments, schedule, in_A, in_z, out_hidden, out_A, out_z, stream);
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  if (n_segments <= 0) return fail(RMT_EINVAL, "n_segments must be positive");
+  if (int64_t(n_segments) * h->cfg.seg_len > INT32_MAX / 2) return fail(RMT_EINVAL, "too many tokens");
+  const int32_t tokens = n_segments * h->cfg.seg_len;
+  return rmt_forward_batch(h, emb, 1, &tokens, schedule, in_A, in_z, out_hidden, out_A, out_z, stream);
+}
+
+rmt_status rmt_forward_batch(rmt_handle* h, const void* emb, int32_t batch, const int32_t* n_tokens,
+                             rmt_schedule schedule, const float* in_A, const float* in_z, void* out_hidden,
+                             float* out_A, float* out_z, void* stream) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  std::vector<int> T;
+  size_t total = 0;
+  RMT_TRY(check_lengths(batch, n_tokens, T, total));
+  return forward_impl(h, emb, T, total, schedule, in_A, in_z, out_hidden, out_A, out_z, stream);
+}
+
+rmt_status rmt_reserve(rmt_handle* h, int32_t max_batch) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  if (max_batch <= 0) return fail(RMT_EINVAL, "max_batch must be positive");
+  DeviceGuard guard(h->dev);
+  return reserve_acts(h, max_batch);
 }
 
 rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap) {
@@ -997,7 +1195,7 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
   float* part = nullptr;
   RMT_TRY(partial_scratch(size_t(G) * nsplit * n * (dk + dv), &part));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  MemKvArgs ka{y, n, d, 0, n, kByLayer, w_mkv, part, dk + dv, G, cells, G};
+  MemKvArgs ka{y, n, d, n, kByLayer, w_mkv, part, dk + dv, G, cells, G};
   RMT_CUDA(launch_mem_kv(ka, dtype == RMT_BF16, st));
   MemUpdateArgs ua{part, nsplit, nullptr, nullptr, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0};
   RMT_CUDA(launch_mem_update(ua, st));

@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const int qt = nqt - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y;
   const Cell c = a.cells[blockIdx.z];
+  const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
   const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.H * HD;
   const size_t slice = cell_index(a.mode, a.L, c);
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
     }
     // scale, causal mask (and rows of the cell's ragged end), running max
     const int k0 = kt * S::BKV;
-    const bool need_mask = (kt == qt) || (k0 + S::BKV > a.M);
+    const bool need_mask = (kt == qt) || (k0 + S::BKV > kvlim);
     float mx[2] = {mrow[0], mrow[1]};
 #pragma unroll
     for (int nb = 0; nb < 8; ++nb) {
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
         if (need_mask) {
           const int kv = k0 + nb * 8 + 2 * tq + (e & 1);
           const int qr = qrow0 + (e >> 1) * 8;
-          if (kv > qr || kv >= a.M) v = -INFINITY;
+          if (kv > qr || kv >= kvlim) v = -INFINITY;
         }
         s[nb][e] = v;
         mx[e >> 1] = fmaxf(mx[e >> 1], v);
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
   __shared__ float Vc[CK][HD];
   const int qc = blockIdx.x, h = blockIdx.y;
   const Cell c = a.cells[blockIdx.z];
+  const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
   const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.H * HD;
   const size_t slice = cell_index(a.mode, a.L, c);
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
     o[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int last = min(a.M, (qc + 1) * BQ);  // keys 0..last-1 can be seen by this block
+  const int last = min(kvlim, (qc + 1) * BQ);  // keys 0..last-1 can be seen by this block
   for (int k0 = 0; k0 < last; k0 += CK) {
     __syncthreads();
     for (int e = threadIdx.x; e < CK * HD; e += BQ) {
@@ -271,7 +273,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
     if (!valid) continue;
     for (int r = 0; r < CK; ++r) {
       const int kr = k0 + r;
-      if (kr > row) break;
+      if (kr > row || kr >= kvlim) break;
       float sc = 0.f;
 #pragma unroll
       for (int i = 0; i < HD; ++i) sc = fmaf(q[i], Kc[r][i], sc);

@@ -275,6 +275,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       decode(it, qt, h, g);
       const Cell c = a.cells[g];
       const int slice = cell_index(a.mode, a.L, c);
+      const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
       const int qrow = qt * 128 + r;
       float m_use = 0.f, l = 0.f;
       for (int j = 0; j <= qt; ++j, ++t) {
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
         sm100::tc_fence_before();
         sm100::mbar_arrive(bar(kSFree));
         const int k0 = j * 128;
-        const bool need_mask = (j == qt) || (k0 + 128 > a.M);
+        const bool need_mask = (j == qt) || (k0 + 128 > kvlim);
         // causal mask (and the cell's ragged end) only on the tiles that need it
         if (need_mask) {
 #pragma unroll
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int kv = k0 + 32 * q4 + i;
-              if (kv > qrow || kv >= a.M) s[q4][i] = __float_as_uint(-INFINITY);
+              if (kv > qrow || kv >= kvlim) s[q4][i] = __float_as_uint(-INFINITY);
             }
           }
         }

@@ -27,12 +27,24 @@ enum : int {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// One (layer, segment) cell of the grid.
+// One (layer, segment) cell of the grid of one sequence of the batch, with the indices the
+// kernels need precomputed on the host:
+//   l      layer: selects the weights
+//   s      segment of the sequence (recorded by the trace)
+//   b      sequence of the batch
+//   m      valid rows of the cell: the segment's tokens, then its n_mem memory tokens
+//          (M for every segment but a short last one). Rows m..M-1 are padding: they start
+//          as zeros, no valid row reads them (attention masks keys >= m; the memory write
+//          reads rows m-n_mem..m-1) and they are never emitted.
+//   k      per-(sequence, layer) index: memory state A, z and the layer scratch buffers
+//   xin    residual slot the cell reads, xout the slot it writes
+//   t0     row of the segment's first token in the packed embeddings / outputs
 struct Cell {
-  int l, s;
+  int l, s, b, m, k, xin, xout, t0;
 };
 
-// Activation slots. The residual stream of cell (l, s) lives in a [M, d] fp32 slot:
+// Activation slots of one sequence, each an [M, d] fp32 residual block; sequence b owns
+// slots b*n_slots(L) .. (b+1)*n_slots(L)-1.
 //   output slot  : ((l + s) % 2) * L + l            (written by cell (l, s))
 //   input slot   : output slot of (l-1, s), or 2L + s % 2 for layer 0 (embeddings + memory)
 // Cell (l, s) runs on diagonal l + s; its input was written on diagonal l + s - 1 and is
@@ -46,9 +58,15 @@ constexpr int n_slots(int L) { return 2 * L + 2; }
 // How a kernel turns a cell into an index of a stacked [*, M, cols] buffer.
 enum IndexMode : int { kByLayer = 0, kInSlot = 1, kOutSlot = 2 };
 
-__device__ __forceinline__ int cell_index(IndexMode mode, int L, Cell c) {
-  return mode == kByLayer ? c.l : (mode == kInSlot ? in_slot(L, c.l, c.s) : out_slot(L, c.l, c.s));
+__host__ __device__ inline int cell_index(IndexMode mode, int /*L*/, Cell c) {
+  return mode == kByLayer ? c.k : (mode == kInSlot ? c.xin : c.xout);
 }
+
+// Rows of the cell that hold tokens (keys past them are masked), given the buffer's M.
+__host__ __device__ inline int cell_rows(const Cell& c, int M) { return c.m < M ? c.m : M; }
+
+// Cell g of the kernel-level entry points: group g uses slice g of every stacked operand.
+__host__ __device__ inline Cell identity_cell(int g) { return Cell{g, 0, 0, 0x7fffffff, g, g, g, 0}; }
 
 // GEMM epilogues shared by the tensor-core and the fp32 kernels.
 enum EpiKind : int {

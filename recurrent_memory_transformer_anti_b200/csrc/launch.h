@@ -122,7 +122,7 @@ cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_
 constexpr int kMemKvSplit = 128;  // d_model columns per split
 struct MemKvArgs {
   const float* x;  // [*, M, d] fp32: the residual stream slots (forward) or caller rows
-  int M, d, row0, n;
+  int M, d, n;     // the n rows read are the cell's last n valid rows (cell_rows(c, M) - n ..)
   IndexMode x_mode;  // slice of x holding the cell's rows (kOutSlot in the forward)
   const void* w;   // [L, dkv, d] in T
   float* part;     // [L, nsplit, n, dkv] fp32
@@ -173,11 +173,13 @@ cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st);
 cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool bf16, bool w_f16, cudaStream_t st);
 // In-place bf16 -> f16 conversion of n elements (the values of a bf16 weight as f16 operands).
 cudaError_t launch_bf16_to_f16(void* p, size_t n, cudaStream_t st);
-// Layer-0 input of segment s: rows 0..seg-1 from emb, rows seg..M-1 from the memory tokens,
-// into the fp32 slot and (if xb_slot) an f16 copy.
-cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __half* xb_slot, int seg, int n_mem,
-                            int d, int s, bool bf16, cudaStream_t st);
-// Segment output: rows 0..seg-1 of an fp32 slot, cast to T, to out + s*seg*d.
-cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, bool bf16, cudaStream_t st);
+// Layer-0 inputs of the G cells (all of layer 0): in slot c.xin of x (and of xb, if given),
+// rows 0..m-n_mem-1 from emb rows c.t0.., rows m-n_mem..m-1 from the memory tokens, rows
+// m..M-1 zero (m = cell_rows(c, M)).
+cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
+                            int n_mem, int d, bool bf16, cudaStream_t st);
+// Segment outputs of the G cells: rows 0..m-n_mem-1 of slot c.xout, cast to T, to out rows c.t0...
+cudaError_t launch_emit(const Cell* cells, int G, const float* x, void* out, int M, int n_mem, int d, bool bf16,
+                        cudaStream_t st);
 
 }  // namespace rmt

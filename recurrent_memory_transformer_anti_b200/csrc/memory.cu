@@ -115,7 +115,9 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   const Cell c = a.cells[blockIdx.y];
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
-  const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + a.row0) * a.d + k0;
+  // the cell's memory rows are its last n valid rows
+  const int row0 = cell_rows(c, a.M) - a.n;
+  const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row0) * a.d + k0;
   const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
   // 16-byte vectors only where every row start is 16-byte aligned
   const bool y_vec = (a.d % 4 == 0) && (reinterpret_cast<uintptr_t>(a.x) % 16 == 0);
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   __syncthreads();
   const int nsplit = (a.d + KS - 1) / KS;
   const int nout = a.n * a.dkv;
-  float* part = a.part + (static_cast<size_t>(c.l) * nsplit + split) * nout;
+  float* part = a.part + (static_cast<size_t>(c.k) * nsplit + split) * nout;
   const int jt = a.dkv / 2, tiles = (n4 / 4) * jt;
   for (int t = threadIdx.x; t < tiles; t += kKvThreads) {
     const int r0 = (t / jt) * 4, j0 = (t % jt) * 2;

@@ -18,7 +18,7 @@ using rmt::Cell;
 // Scratch for rmt_memory_write_noalloc: the cell table, then the partial sums. Every GPU
 // that loads the library holds these 8 MiB until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
-constexpr size_t kNoAllocCellBytes = 64 << 10;  // room for 8192 cells
+constexpr size_t kNoAllocCellBytes = 256 << 10;  // room for 8192 cells
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch, looked up once per device (host code cannot use the
@@ -27,7 +27,7 @@ void* g_noalloc_addr[64] = {};
 
 __global__ void fill_cells_kernel(Cell* cells, int G) {
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g < G) cells[g] = Cell{g, 0};
+  if (g < G) cells[g] = rmt::identity_cell(g);
 }
 
 }  // namespace
@@ -72,7 +72,7 @@ extern "C" rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv
   fill_cells_kernel<<<(G + 255) / 256, 256, 0, st>>>(cells, G);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) {
-    rmt::MemKvArgs ka{y, n, d, 0, n, rmt::kByLayer, w_mkv, part, dk + dv, G, cells, G};
+    rmt::MemKvArgs ka{y, n, d, n, rmt::kByLayer, w_mkv, part, dk + dv, G, cells, G};
     e = rmt::launch_mem_kv(ka, dtype == RMT_BF16, st);
   }
   if (e == cudaSuccess) {

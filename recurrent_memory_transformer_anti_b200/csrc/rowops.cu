@@ -66,27 +66,37 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a
   }
 }
 
-// Layer-0 input of segment s: embeddings of the segment, then the memory tokens.
+// Layer-0 input of cell blockIdx.y (row blockIdx.x of M): the segment's tokens from the packed
+// embeddings, then the memory tokens, then zero padding up to M.
 template <typename T>
-__global__ void assemble_kernel(const T* emb, const T* mem, float* x, __half* xb, int seg, int d, int s) {
+__global__ void assemble_kernel(const Cell* cells, const T* emb, const T* mem, float* x, __half* xb, int M, int n_mem,
+                                int d) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
-  const int r = blockIdx.x;
-  const T* src = r < seg ? emb + (static_cast<size_t>(s) * seg + r) * d : mem + static_cast<size_t>(r - seg) * d;
+  const Cell c = cells[blockIdx.y];
+  const int r = blockIdx.x, m = cell_rows(c, M), seg = m - n_mem;
+  const T* src = r < seg ? emb + (static_cast<size_t>(c.t0) + r) * d
+                         : (r < m ? mem + static_cast<size_t>(r - seg) * d : nullptr);
+  const size_t row = (static_cast<size_t>(c.xin) * M + r) * d;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
-    const float4 v = Vec4<T>::load(src + k);
-    Vec4<float>::store(x + static_cast<size_t>(r) * d + k, v);
-    if (xb) Vec4<__half>::store(xb + static_cast<size_t>(r) * d + k, v);
+    const float4 v = src ? Vec4<T>::load(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+    Vec4<float>::store(x + row + k, v);
+    if (xb) Vec4<__half>::store(xb + row + k, v);
   }
 }
 
+// Output rows of cell blockIdx.y: its segment's tokens (row blockIdx.x), cast to T, to the
+// packed output at the segment's first token.
 template <typename T>
-__global__ void emit_kernel(const float* x, T* out, int seg, int d, int s) {
+__global__ void emit_kernel(const Cell* cells, const float* x, T* out, int M, int n_mem, int d) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
+  const Cell c = cells[blockIdx.y];
   const int r = blockIdx.x;
-  T* dst = out + (static_cast<size_t>(s) * seg + r) * d;
-  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(x + static_cast<size_t>(r) * d + k));
+  if (r >= cell_rows(c, M) - n_mem) return;
+  const float* src = x + (static_cast<size_t>(c.xout) * M + r) * d;
+  T* dst = out + (static_cast<size_t>(c.t0) + r) * d;
+  for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(src + k));
 }
 
 // W[l][n][k] *= g[l][k]: folds an RMSNorm gain into the weight that consumes its output.
@@ -140,30 +150,28 @@ cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_assemble(const void* emb, const void* mem, float* x_slot, __half* xb_slot, int seg, int n_mem,
-                            int d, int s, bool bf16, cudaStream_t st) {
+cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
+                            int n_mem, int d, bool bf16, cudaStream_t st) {
   if (d % 4) return cudaErrorInvalidValue;
+  if (G <= 0) return cudaSuccess;
   const int threads = d >= 1024 ? 256 : 128;
   if (bf16)
-    return launch_pdl(assemble_kernel<__nv_bfloat16>, dim3(seg + n_mem), dim3(threads), 0, st,
-                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x_slot, xb_slot,
-                      seg, d, s);
-  else
-    return launch_pdl(assemble_kernel<float>, dim3(seg + n_mem), dim3(threads), 0, st, static_cast<const float*>(emb),
-                      static_cast<const float*>(mem), x_slot, xb_slot, seg, d, s);
-  return cudaGetLastError();
+    return launch_pdl(assemble_kernel<__nv_bfloat16>, dim3(M, G), dim3(threads), 0, st, cells,
+                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d);
+  return launch_pdl(assemble_kernel<float>, dim3(M, G), dim3(threads), 0, st, cells, static_cast<const float*>(emb),
+                    static_cast<const float*>(mem), x, xb, M, n_mem, d);
 }
 
-cudaError_t launch_emit(const float* x_slot, void* out, int seg, int d, int s, bool bf16, cudaStream_t st) {
+cudaError_t launch_emit(const Cell* cells, int G, const float* x, void* out, int M, int n_mem, int d, bool bf16,
+                        cudaStream_t st) {
   if (d % 4) return cudaErrorInvalidValue;
+  if (G <= 0) return cudaSuccess;
   const int threads = d >= 1024 ? 256 : 128;
   if (bf16)
-    return launch_pdl(emit_kernel<__nv_bfloat16>, dim3(seg), dim3(threads), 0, st, x_slot,
-                      static_cast<__nv_bfloat16*>(out), seg, d, s);
-  else
-    return launch_pdl(emit_kernel<float>, dim3(seg), dim3(threads), 0, st, x_slot, static_cast<float*>(out), seg, d,
-                      s);
-  return cudaGetLastError();
+    return launch_pdl(emit_kernel<__nv_bfloat16>, dim3(M - n_mem, G), dim3(threads), 0, st, cells, x,
+                      static_cast<__nv_bfloat16*>(out), M, n_mem, d);
+  return launch_pdl(emit_kernel<float>, dim3(M - n_mem, G), dim3(threads), 0, st, cells, x, static_cast<float*>(out), M,
+                    n_mem, d);
 }
 
 }  // namespace rmt

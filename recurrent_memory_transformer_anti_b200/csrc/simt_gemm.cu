@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
   if ((a.epi == kEpiRope || a.epi == kEpiSwiGLU) && t < BM) {
     const int row = m0 + t;
     rs[t] = (ep.ss_in && row < a.M)
-                ? rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                ? rms_row_scale(ep.ss_in + (static_cast<size_t>(c.k) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
                                 ep.rms_eps)
                 : 1.f;
   }
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
     if (t < BM && m0 + t < a.M) {
       float ss = 0.f;
       for (int cc = 0; cc < BN && n0 + cc < a.N; ++cc) ss = fmaf(Cs[t][cc], Cs[t][cc], ss);
-      ep.ss_out[(static_cast<size_t>(c.l) * a.M + m0 + t) * ep.ss_parts + blockIdx.x] = ss;
+      ep.ss_out[(static_cast<size_t>(c.k) * a.M + m0 + t) * ep.ss_parts + blockIdx.x] = ss;
     }
   }
 }

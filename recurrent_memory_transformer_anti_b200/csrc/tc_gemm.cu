@@ -107,7 +107,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
   float rs = 1.f;  // folded RMSNorm scale of this row (RoPE and SwiGLU epilogues)
   if constexpr (EPI == kEpiRope || EPI == kEpiSwiGLU) {
     if (ep.ss_in && valid)
-      rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+      rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.k) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
                          ep.rms_eps);
   }
   if constexpr (EPI == kEpiRope) {
@@ -215,7 +215,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
     }
     if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
       if (ep.ss_out && valid)
-        ep.ss_out[(static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
+        ep.ss_out[(static_cast<size_t>(c.k) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
     }
   }
 }
@@ -311,7 +311,7 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
       if (cc + NBUF < c1) issue(cc + NBUF, b);
     }
   }
-  if (ep.ss_out && valid) ep.ss_out[(static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
+  if (ep.ss_out && valid) ep.ss_out[(static_cast<size_t>(c.k) * a.M + row) * ep.ss_parts + (n0 / BN) * 2 + part] = ss;
   return true;
 }
 
@@ -334,7 +334,7 @@ __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUt
   const int u0 = part * units / 2, u1 = (part + 1) * units / 2;
   float rs = 1.f;
   if (ep.ss_in && valid)
-    rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.l) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+    rs = rms_row_scale(ep.ss_in + (static_cast<size_t>(c.k) * a.M + row) * ep.ss_parts, ep.ss_parts, ep.inv_d,
                        ep.rms_eps);
   const size_t idx = cell_index(ep.out_mode, a.L, c);
   OpT* orow = static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo;

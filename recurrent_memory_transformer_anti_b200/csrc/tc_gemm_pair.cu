@@ -420,7 +420,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         const int k = wq * 32 + lane, tok = tok0 + k;
         if (k < cnt)
           rs[k] = (ep.ss_in && tok < M)
-                      ? row_scale(ep.ss_in + (static_cast<size_t>(c.l) * M + tok) * ep.ss_parts, ep.ss_parts, ep.inv_d,
+                      ? row_scale(ep.ss_in + (static_cast<size_t>(c.k) * M + tok) * ep.ss_parts, ep.ss_parts, ep.inv_d,
                                   ep.rms_eps)
                       : 1.f;
         if (!wg_sync()) break;
@@ -462,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           const int k = wq * 32 + lane;
           const int tok = tok0 + k;
           if (k < cnt && tok < M)
-            ep.ss_out[(static_cast<size_t>(c.l) * M + tok) * ep.ss_parts + fcta / C::FM] =
+            ep.ss_out[(static_cast<size_t>(c.k) * M + tok) * ep.ss_parts + fcta / C::FM] =
                 ((rb[k] + rb[128 + k]) + rb[256 + k]) + rb[384 + k];
         }
       }

@@ -21,7 +21,8 @@ SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
 DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16}
 STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE"}
 
-EXPORTED = ("rmt_create", "rmt_forward", "rmt_forward_resume", "rmt_schedule_table", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
+EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "rmt_forward_batch", "rmt_schedule_table",
+            "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
             "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
             "rmt_probe_read")
@@ -61,7 +62,10 @@ def _load() -> ctypes.CDLL:
         "rmt_create": [ctypes.POINTER(rmt_weights), ctypes.POINTER(rmt_cfg), ctypes.POINTER(vp)],
         "rmt_forward": [vp, vp, i32, ctypes.c_int, vp, vp, vp, vp],
         "rmt_forward_resume": [vp, vp, i32, ctypes.c_int, vp, vp, vp, vp, vp, vp],
+        "rmt_forward_batch": [vp, vp, i32, p32, ctypes.c_int, vp, vp, vp, vp, vp, vp],
+        "rmt_reserve": [vp, i32],
         "rmt_schedule_table": [i32, i32, ctypes.c_int, p32, sz],
+        "rmt_schedule_table_batch": [i32, i32, p32, ctypes.c_int, p32, sz],
         "rmt_get_schedule": [vp, i32, ctypes.c_int, p32, sz],
         "rmt_get_trace": [vp, p32, sz],
         "rmt_sync": [vp, vp],
@@ -180,6 +184,29 @@ def rmt_forward_resume(h: Handle, emb, n_segments: int, schedule, in_A, in_z, ou
     sch = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
     _check(_lib.rmt_forward_resume(h.ptr, _ptr(emb), int(n_segments), sch, _ptr(in_A), _ptr(in_z), _ptr(out_hidden),
                                    _ptr(out_A), _ptr(out_z), _stream(stream)), "rmt_forward_resume")
+
+
+def rmt_forward_batch(h: Handle, emb, n_tokens, schedule, out_hidden, in_A=None, in_z=None, out_A=None, out_z=None,
+                      stream=None) -> None:
+    sch = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    nt = np.ascontiguousarray(np.asarray(n_tokens, dtype=np.int32).reshape(-1))
+    _check(_lib.rmt_forward_batch(h.ptr, _ptr(emb), int(nt.size), nt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                  sch, _ptr(in_A), _ptr(in_z), _ptr(out_hidden), _ptr(out_A), _ptr(out_z),
+                                  _stream(stream)), "rmt_forward_batch")
+
+
+def rmt_reserve(h: Handle, max_batch: int) -> None:
+    _check(_lib.rmt_reserve(h.ptr, int(max_batch)), "rmt_reserve")
+
+
+def rmt_schedule_table_batch(n_layers: int, n_segments, schedule) -> np.ndarray:
+    sch = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    ns = np.ascontiguousarray(np.asarray(n_segments, dtype=np.int32).reshape(-1))
+    out = np.zeros(4 * n_layers * int(ns.sum()), np.int32)
+    _check(_lib.rmt_schedule_table_batch(n_layers, int(ns.size), ns.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), sch,
+                                         out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), out.size),
+           "rmt_schedule_table_batch")
+    return out.reshape(-1, 4)
 
 
 def rmt_schedule_table(n_layers: int, n_segments: int, schedule) -> np.ndarray:

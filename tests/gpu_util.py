@@ -39,3 +39,25 @@ def forward(h, cfg, emb, n_segments, schedule="diagonal"):
 
 def embeddings(cfg, n_segments, seed=1):
     return make_embeddings(cfg, n_segments, seed=seed)
+
+
+def forward_batch(h, cfg, embs, schedule="diagonal", in_A=None, in_z=None, host=False):
+    """rmt_forward_batch over the sequences embs[b] ([T_b, d] each), packed one after another.
+
+    host=True passes page-locked host buffers for the embeddings and the outputs. Returns
+    ([out_b] as float32 numpy, A [B, L, dk, dv], z [B, L, dk])."""
+    lens = [int(e.shape[0]) for e in embs]
+    e = rmt.storage(np.concatenate(embs), cfg.dtype, device="cuda")
+    if host:
+        e = e.cpu().pin_memory()
+    out = torch.empty_like(e)
+    if host:
+        out = out.pin_memory()
+    B = len(embs)
+    A = torch.empty(B, cfg.n_layers, cfg.d_k, cfg.d_v, device="cuda")
+    z = torch.empty(B, cfg.n_layers, cfg.d_k, device="cuda")
+    rmt.rmt_forward_batch(h, e, lens, schedule, out, in_A, in_z, A, z)
+    rmt.rmt_sync(h)
+    o = to_np(out)
+    starts = np.cumsum([0] + lens)
+    return [o[starts[b]:starts[b + 1]] for b in range(B)], to_np(A), to_np(z)

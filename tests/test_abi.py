@@ -36,6 +36,29 @@ def test_library_schedule_equals_oracle_enumeration(schedule):
                                           armt.schedule_triples(L, S, schedule))
 
 
+@pytest.mark.parametrize("schedule", ["diagonal", "sequential"])
+def test_library_batch_schedule_equals_oracle_enumeration(schedule):
+    rng = np.random.default_rng(5)
+    for L in (1, 2, 3, 16):
+        for _ in range(12):
+            S = [int(v) for v in rng.integers(1, 9, size=int(rng.integers(1, 5)))]
+            np.testing.assert_array_equal(rmt.rmt_schedule_table_batch(L, S, schedule),
+                                          armt.schedule_quads(L, S, schedule))
+
+
+def test_batch_schedule_argument_errors():
+    lib = rmt.lib()
+    buf = (ctypes.c_int32 * 64)()
+    ns = (ctypes.c_int32 * 2)(2, 1)
+    assert lib.rmt_schedule_table_batch(2, 2, ns, 0, buf, 64) == rmt.RMT_OK
+    assert lib.rmt_schedule_table_batch(2, 2, ns, 0, buf, 4 * 6 - 1) == rmt.RMT_EINVAL
+    assert lib.rmt_schedule_table_batch(2, 0, ns, 0, buf, 64) == rmt.RMT_EINVAL
+    assert lib.rmt_schedule_table_batch(2, 2, None, 0, buf, 64) == rmt.RMT_EINVAL
+    bad = (ctypes.c_int32 * 2)(2, 0)
+    assert lib.rmt_schedule_table_batch(2, 2, bad, 0, buf, 64) == rmt.RMT_EINVAL
+    assert lib.rmt_schedule_table_batch(2, 2, ns, 5, buf, 64) == rmt.RMT_EINVAL
+
+
 def test_schedule_of_the_131k_workload():
     t = rmt.rmt_schedule_table(16, 128, "diagonal")
     np.testing.assert_array_equal(t, armt.schedule_triples(16, 128, "diagonal"))

@@ -15,7 +15,7 @@ import torch
 from armt_synthetic import CONFIGS
 from oracle import armt
 from recurrent_memory_transformer_anti_b200 import rmt
-from tests.gpu_util import build, embeddings, forward, normwise
+from tests.gpu_util import build, embeddings, forward, forward_batch, normwise
 
 pytestmark = pytest.mark.gpu
 
@@ -278,3 +278,98 @@ def test_resume_from_a_given_state_matches_oracle(cuda_ok, name, tol):
     for g_, r, what in zip(got, ref, ("out", "A", "z")):
         assert normwise(g_, r) < tol, what
     rmt.rmt_destroy(h)
+
+
+# ------------------------------------------------ short last segments and batches
+
+@pytest.mark.parametrize("name,tol", [("tiny", F32_TOL), ("small-bf16", BF16_TOL)])
+@pytest.mark.parametrize("extra", [1, 37])
+def test_short_last_segment_matches_oracle(cuda_ok, name, tol, extra):
+    """2 full segments and a third of `extra` tokens: its memory tokens follow its last
+    token, keys past them are masked and its memory write reads its last n_mem rows."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    extra = min(extra, cfg.seg_len - 1)
+    emb = embeddings(cfg, 3, seed=16)[:2 * cfg.seg_len + extra]
+    got = forward_batch(h, cfg, [emb], "diagonal")
+    ref = armt.forward_tokens(cfg, w, emb, dtype=np.float32)
+    assert normwise(got[0][0], ref[0]) < tol
+    assert normwise(got[1][0], ref[1]) < tol
+    assert normwise(got[2][0], ref[2]) < tol
+    seq = forward_batch(h, cfg, [emb], "sequential")
+    np.testing.assert_array_equal(got[0][0], seq[0][0])
+    np.testing.assert_array_equal(got[1], seq[1])
+    # the full segments are those of a run without the short one
+    full = forward(h, cfg, emb[:2 * cfg.seg_len], 2, "diagonal")
+    np.testing.assert_array_equal(got[0][0][:2 * cfg.seg_len], full[0])
+    rmt.rmt_destroy(h)
+
+
+@pytest.mark.parametrize("name,tol", [("tiny", F32_TOL), ("small-bf16", BF16_TOL)])
+def test_batch_matches_oracle_and_each_sequence_alone(cuda_ok, name, tol):
+    """Sequences of different lengths (short last segments, one shorter than a segment) in
+    one batch: each result equals the oracle's and, bit for bit, the sequence run alone."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    seg = cfg.seg_len
+    lens = [3 * seg + 5, seg, 2 * seg - 1, 3]
+    embs = [embeddings(cfg, 4, seed=20 + b)[:n] for b, n in enumerate(lens)]
+    got = forward_batch(h, cfg, embs, "diagonal")
+    outs, A_ref, z_ref = armt.forward_batch(cfg, w, embs, dtype=np.float32)
+    for b in range(len(lens)):
+        assert got[0][b].shape == (lens[b], cfg.d_model)
+        assert normwise(got[0][b], outs[b]) < tol, b
+        assert normwise(got[1][b], A_ref[b]) < tol, b
+        assert normwise(got[2][b], z_ref[b]) < tol, b
+        alone = forward_batch(h, cfg, [embs[b]], "diagonal")
+        np.testing.assert_array_equal(got[0][b], alone[0][0])
+        np.testing.assert_array_equal(got[1][b], alone[1][0])
+        np.testing.assert_array_equal(got[2][b], alone[2][0])
+    seq = forward_batch(h, cfg, embs, "sequential")
+    for b in range(len(lens)):
+        np.testing.assert_array_equal(got[0][b], seq[0][b])
+    np.testing.assert_array_equal(got[1], seq[1])
+    np.testing.assert_array_equal(got[2], seq[2])
+    # the device trace is the batch schedule without its sequence column
+    segs = [-(-n // seg) for n in lens]
+    trace = rmt.rmt_get_trace(h, cfg.n_layers * sum(segs))
+    np.testing.assert_array_equal(trace, armt.schedule_quads(cfg.n_layers, segs, "sequential")[:, [0, 2, 3]])
+    rmt.rmt_destroy(h)
+
+
+def test_batch_with_initial_states_and_pinned_host_buffers(cuda_ok):
+    cfg = CONFIGS["small-bf16"]
+    w, h = build(cfg)
+    rmt.rmt_reserve(h, 3)
+    seg = cfg.seg_len
+    lens = [2 * seg + 9, seg + 1, 2 * seg]
+    embs = [embeddings(cfg, 3, seed=30 + b)[:n] for b, n in enumerate(lens)]
+    rng = np.random.default_rng(31)
+    A0 = (0.1 * rng.standard_normal((3, cfg.n_layers, cfg.d_k, cfg.d_v))).astype(np.float32)
+    z0 = (1.0 + np.abs(rng.standard_normal((3, cfg.n_layers, cfg.d_k)))).astype(np.float32)
+    dev = forward_batch(h, cfg, embs, "diagonal", torch.from_numpy(A0).cuda(), torch.from_numpy(z0).cuda())
+    pinned = forward_batch(h, cfg, embs, "diagonal", torch.from_numpy(A0), torch.from_numpy(z0), host=True)
+    outs, A_ref, z_ref = armt.forward_batch(cfg, w, embs, dtype=np.float32, A0=A0, z0=z0)
+    for b in range(3):
+        np.testing.assert_array_equal(dev[0][b], pinned[0][b])
+        assert normwise(dev[0][b], outs[b]) < BF16_TOL, b
+        assert normwise(dev[1][b], A_ref[b]) < BF16_TOL, b
+    np.testing.assert_array_equal(dev[1], pinned[1])
+    np.testing.assert_array_equal(dev[2], pinned[2])
+    rmt.rmt_destroy(h)
+
+
+def test_batch_argument_errors(tiny):
+    cfg, w, h = tiny
+    e = rmt.storage(embeddings(cfg, 1), cfg.dtype, device="cuda")
+    out = torch.empty_like(e)
+    for lens in ([], [0], [cfg.seg_len, -3]):
+        with pytest.raises(rmt.RmtError) as ex:
+            rmt.rmt_forward_batch(h, e, lens, "diagonal", out)
+        assert ex.value.status == rmt.RMT_EINVAL
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_reserve(h, 0)
+    assert ex.value.status == rmt.RMT_EINVAL
+    # the handle is still usable
+    rmt.rmt_forward_batch(h, e, [cfg.seg_len], "diagonal", out)
+    rmt.rmt_sync(h)
