@@ -56,7 +56,7 @@ def parse():
     p.add_argument("--segments", type=int, default=N_SEGMENTS)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-sequential", action="store_true")
-    p.add_argument("--microbench", choices=["gemm", "memory"], default=None,
+    p.add_argument("--microbench", choices=["gemm", "memory", "attention"], default=None,
                    help="kernel-level sweeps instead of the forward: one JSON line per configuration")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions per microbench configuration")
     return p.parse_args()
@@ -271,6 +271,20 @@ def run_microbench(args, local: int) -> int:
                                            "kernel": "CTA pairs" if N % 256 == 0 else "single CTAs"},
                      ms, 2.0 * G * M * N * K, "TFLOP/s", peaks["bf16_tflops"], "bf16_tflops")
                 del a, b, c
+        return 0
+
+    if args.microbench == "attention":
+        # segment-local causal GQA attention of the 1B shape: 32 query / 8 key-value heads of
+        # 64, M = 1040 rows per cell, G = 16 cells (one full diagonal); causal flops
+        # 4 * dh * M (M + 1) / 2 per head and cell
+        M, H, Hkv, dh = 1040, 32, 8, 64
+        for G in (1, 16):
+            qkv = (torch.randn(G, M, (H + 2 * Hkv) * dh, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+            out = torch.empty(G, M, H * dh, device=dev, dtype=torch.bfloat16)
+            ms = median_ms(lambda: rmt.rmt_attention(qkv, out, G, M, H, Hkv, dh, "bf16"))
+            emit("attention", {"G": G, "M": M, "H": H, "Hkv": Hkv, "dh": dh}, ms,
+                 G * H * 4.0 * dh * M * (M + 1) / 2, "TFLOP/s", peaks["bf16_tflops"], "bf16_tflops")
+            del qkv, out
         return 0
 
     # memory-path kernels: the diagonal's size (G = 16 cells) and about 10^6 rows (HBM-bound)

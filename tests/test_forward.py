@@ -178,6 +178,31 @@ def test_1b_shape_bench_configuration(cuda_ok):
     rmt.rmt_destroy(h)
 
 
+@pytest.mark.parametrize("name", ["3b-512", "3b-2048"])
+def test_3b_shape_full_size(cuda_ok, name):
+    """The LLaMA-3B-shaped workloads at 131,072 tokens (28 layers, d 3072, 24/8 heads of 128,
+    d_k = d_v = 128, segments of 512 or 2048 + 16 tokens; the 2064-row cells end in a ragged
+    token tile). DIAGONAL equals SEQUENTIAL bit for bit at the full size; the first segment
+    of the full run equals a one-segment run bit for bit, and that run (hidden states and the
+    28 layers' memory states) matches the oracle within the bf16 tolerance."""
+    cfg = CONFIGS[name]
+    w, h = build(cfg)
+    S = 131072 // cfg.seg_len
+    emb = embeddings(cfg, S)
+    full_d = forward(h, cfg, emb, S, "diagonal")
+    full_s = forward(h, cfg, emb, S, "sequential")
+    for a, b in zip(full_d, full_s):
+        np.testing.assert_array_equal(a, b)
+    assert np.isfinite(full_d[0]).all() and np.isfinite(full_d[1]).all()
+    del full_s
+    part = forward(h, cfg, emb[:cfg.seg_len], 1, "diagonal")
+    np.testing.assert_array_equal(full_d[0][:cfg.seg_len], part[0])
+    rmt.rmt_destroy(h)
+    ref = armt.forward(cfg, w, emb[:cfg.seg_len], 1, dtype=np.float32)
+    for g, r, what in zip(part, ref, ("out", "A", "z")):
+        assert normwise(g, r) < BF16_TOL, what
+
+
 @pytest.mark.parametrize("name,S,tol", [("tiny", 3, F32_TOL), ("small-bf16", 3, BF16_TOL)])
 def test_random_rmsnorm_gains_match_oracle(cuda_ok, name, S, tol):
     """Gains far from 1 exercise the folding of each RMSNorm gain into the next projection."""
