@@ -245,6 +245,9 @@ struct rmt_handle {
   // bf16 mode: projections that run on the CTA-pair GEMM (decided before packing, which
   // depends on it for the RoPE and SwiGLU row orders)
   bool pair_mo = false, pair_qkv = false, pair_o = false, pair_gu = false, pair_d = false;
+  // bf16 mode with d_k = d_v = 64: the memory read runs in the mem-q GEMM's epilogue (the
+  // query never goes to memory) and has no launch of its own
+  bool fuse_read = false;
   std::vector<void*> allocs;
   // activations and memory state, sized for cap_b sequences (rmt_reserve)
   int cap_b = 0;
@@ -539,6 +542,11 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       N = c.d_k, K = d, epi = kEpiStoreF32, amode = kInSlot;
       ep.out = h->qm, ep.ldo = c.d_k;
       a32 = h->x, w = h->w_mq, ta = &h->tm_xb, tb = &h->tm_wmq, bn = h->bn_mq;
+      if (h->fuse_read) {  // o = phi(q) A / (phi(q) . z + eps) straight from the accumulator
+        epi = kEpiMemRead;
+        ep.out = h->om, ep.ldo = c.d_v;
+        ep.mem_A = h->A, ep.mem_z = h->z, ep.mem_dv = c.d_v, ep.mem_eps = c.mem_eps;
+      }
       break;
     case kProjMemO:  // x_out = x_in + read-out; emits the row sums of squares of RMSNorm 1
       N = d, K = c.d_v, epi = resid;
@@ -626,15 +634,22 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
     });
     if (e != cudaSuccess) return e;
   }
-  e = launch_kind(h, RMT_K_MEMQ, 2 * g * m * dk * dd, g * (m * dd * ea + dk * dd * es + m * dk * 4), st,
-                  [&] { return run_proj(h, kProjMemQ, cells, G, st); });
-  if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk), g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es),
-                  st, [&] {
-                    MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
-                    return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st);
-                  });
-  if (e != cudaSuccess) return e;
+  if (h->fuse_read) {  // mem-q GEMM with the memory read in its epilogue
+    e = launch_kind(h, RMT_K_MEMQ, g * m * (2 * dk * dd + 2 * dk * dv + 2 * dk),
+                    g * (m * dd * ea + dk * dd * es + dk * dv * 4 + dk * 4 + m * dv * es), st,
+                    [&] { return run_proj(h, kProjMemQ, cells, G, st); });
+    if (e != cudaSuccess) return e;
+  } else {
+    e = launch_kind(h, RMT_K_MEMQ, 2 * g * m * dk * dd, g * (m * dd * ea + dk * dd * es + m * dk * 4), st,
+                    [&] { return run_proj(h, kProjMemQ, cells, G, st); });
+    if (e != cudaSuccess) return e;
+    e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk),
+                    g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es), st, [&] {
+                      MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
+                      return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st);
+                    });
+    if (e != cudaSuccess) return e;
+  }
   e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv, g * (m * dv * es + dd * dv * es + 2 * m * dd * 4), st,
                   [&] { return run_proj(h, kProjMemO, cells, G, st); });
   if (e != cudaSuccess) return e;
@@ -793,6 +808,7 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
     // the memory read-out projection (K = d_v) is a pure stream over the residual; it stays on
     // the single-CTA kernel, whose residual epilogue moves whole blocks through TMA
     h->pair_mo = false;
+    h->fuse_read = c.d_k == 64 && c.d_v == 64 && tc_pick_bn(c.d_k, kEpiStoreF32, 0) == 64;
     h->pair_qkv = tc_pair_supported(Mi, h->Nqkv, di, kEpiRope, c.head_dim);
     h->pair_o = tc_pair_supported(Mi, di, hdi, kEpiResidCast, 0);
     h->pair_gu = tc_pair_supported(Mi, 2 * Fi, di, kEpiSwiGLU, 0);

@@ -76,6 +76,7 @@ enum EpiKind : int {
   kEpiResidCast = 3,  // as kEpiResid, and also xb(bf16)[dst] = bf16(result)
   kEpiRope = 4,       // out(T) = RoPE(acc) for columns < rope_cols, acc elsewhere
   kEpiSwiGLU = 5,     // out(T)[:, j] = silu(gate_j) * up_j, gate/up interleaved in blocks of 64
+  kEpiMemRead = 6,    // out(T) = phi(acc) A / (phi(acc) . z + eps): the memory read of the query rows
 };
 
 constexpr int kSwiGLUBlock = 64;
@@ -112,6 +113,13 @@ struct EpiParams {
   const float* ss_in;
   int ss_parts;
   float inv_d, rms_eps;
+  // kEpiMemRead: the accumulator row is the raw memory query q (d_k = the tile width); the
+  // epilogue writes o = phi(q) A / (phi(q) . z + mem_eps) (d_v = mem_dv columns) to out,
+  // with A [d_k][d_v] and z [d_k] fp32 of state slice cell_index(kByLayer).
+  const float* mem_A;
+  const float* mem_z;
+  int mem_dv;
+  float mem_eps;
 };
 
 // RMSNorm row scale from the per-block sums of squares of one row (fixed summation order).

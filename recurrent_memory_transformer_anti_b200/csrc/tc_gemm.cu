@@ -387,6 +387,68 @@ __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUt
   return true;
 }
 
+// Memory-read epilogue: stage this warp's half of the cell's A (columns part*dv/2 .. +dv/2,
+// row-major [dk][dv/2]) and z into the warp's own shared block, before the accumulator wait.
+// Each warp holds a private copy, so only the warp itself must be done with the previous one.
+template <int BN>
+__device__ __forceinline__ void stage_mem_state(const TcGemmArgs& a, Cell c, int part, int lane, float* As, float* zs) {
+  const EpiParams& ep = a.ep;
+  const int dv = ep.mem_dv, hv = dv / 2;
+  const size_t si = cell_index(kByLayer, a.L, c);
+  const float* A = ep.mem_A + si * BN * dv + part * hv;
+  __syncwarp();  // the warp's previous tile has read its copy
+  for (int e = lane; e < BN * hv / 4; e += 32) {
+    const int i = e / (hv / 4), j4 = e % (hv / 4);
+    reinterpret_cast<float4*>(As)[e] = *reinterpret_cast<const float4*>(A + static_cast<size_t>(i) * dv + 4 * j4);
+  }
+  for (int i = lane; i < BN; i += 32) zs[i] = ep.mem_z[si * BN + i];
+  __syncwarp();
+}
+
+// Memory-read epilogue of one row (row per thread), output columns part*dv/2 .. +dv/2: the
+// query row is the accumulator (BN = d_k columns); o = phi(q) A / (phi(q) . z + eps) with
+// both sums over i ascending in fp32.
+template <int BN, typename OpT>
+__device__ __forceinline__ void epilogue_mem_read(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int part,
+                                                  const float* As, const float* zs) {
+  const EpiParams& ep = a.ep;
+  constexpr int HV = 32;  // output columns per thread (d_v = 64)
+  float fq[BN];
+#pragma unroll
+  for (int c32 = 0; c32 < BN / 32; ++c32) {
+    uint32_t r[32];
+    sm100::tmem_ld32(tacc + 32 * c32, r);
+    sm100::tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) fq[32 * c32 + j] = phi_f(u2f(r[j]));
+  }
+  if (row >= a.M) return;
+  float den = 0.f;
+#pragma unroll
+  for (int i = 0; i < BN; ++i) den = fmaf(fq[i], zs[i], den);
+  den += ep.mem_eps;
+  float acc[HV];
+#pragma unroll
+  for (int j = 0; j < HV; ++j) acc[j] = 0.f;
+#pragma unroll
+  for (int i = 0; i < BN; ++i) {  // fully unrolled: fq stays in registers
+    const float4* Ai = reinterpret_cast<const float4*>(As + i * HV);
+#pragma unroll
+    for (int j4 = 0; j4 < HV / 4; ++j4) {
+      const float4 av = Ai[j4];
+      acc[4 * j4] = fmaf(fq[i], av.x, acc[4 * j4]);
+      acc[4 * j4 + 1] = fmaf(fq[i], av.y, acc[4 * j4 + 1]);
+      acc[4 * j4 + 2] = fmaf(fq[i], av.z, acc[4 * j4 + 2]);
+      acc[4 * j4 + 3] = fmaf(fq[i], av.w, acc[4 * j4 + 3]);
+    }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int j = 0; j < HV; ++j) acc[j] *= inv;
+  const size_t idx = cell_index(ep.out_mode, a.L, c);
+  store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + part * HV, acc);
+}
+
 template <int BN, int EPI, typename OpT, int NBUF>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -530,15 +592,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int g = t / (mt * nt), r = t % (mt * nt);
+      const int n_tile = r / mt, m_tile = r % mt;
+      const Cell c = args.cells[g];
+      if constexpr (EPI == kEpiMemRead)
+        stage_mem_state<BN>(args, c, part, lane, reinterpret_cast<float*>(rbuf),
+                            reinterpret_cast<float*>(smem + C::XS_OFF + ew * C::XS_BUF));
       bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
       if (!ok) {
         if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
         break;
       }
       sm100::tc_fence_after();
-      const int g = t / (mt * nt), r = t % (mt * nt);
-      const int n_tile = r / mt, m_tile = r % mt;
-      const Cell c = args.cells[g];
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
         ok = epilogue_resid_tma<BN, EPI, OpT, NBUF>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
@@ -555,6 +620,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
           break;
         }
+      } else if constexpr (EPI == kEpiMemRead) {
+        epilogue_mem_read<BN, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, part,
+                                   reinterpret_cast<const float*>(rbuf),
+                                   reinterpret_cast<const float*>(smem + C::XS_OFF + ew * C::XS_BUF));
       } else {
         epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
       }
@@ -623,6 +692,11 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
       break;
     case kEpiSwiGLU:
       if constexpr (BN >= 128) return launch_bn_epi<BN, kEpiSwiGLU, OpT>(ta, tb, tx, args, st);
+      break;
+    case kEpiMemRead:  // d_k = d_v = 64: each epilogue warp's copy of half of A fills its residual buffer
+      if constexpr (BN == 64) {
+        if (args.N == 64 && args.ep.mem_dv == 64) return launch_bn_epi<BN, kEpiMemRead, OpT>(ta, tb, tx, args, st);
+      }
       break;
   }
   return cudaErrorInvalidValue;
