@@ -141,6 +141,26 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------ reference arm
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value (a job takes as long as its slowest rank). Every rank
+    must call it, in the same order; `device` is where the backend reduces (cuda for nccl,
+    cpu for gloo)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job throughput of `world` replicas that each process units_per_rank units, with
+    ms the max-over-ranks time (units per second)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def run_reference(args, world: int, rank: int) -> int:
     """The oracle (numpy, strictly sequential) on the host cores: each step runs the next
     block of (layer, segment) cells of the same workload in sequential order, carrying the
@@ -377,12 +397,7 @@ def main() -> int:
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1) / n
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
 
     run("diagonal", W)
     rmt.rmt_sync(h, stream)
@@ -398,7 +413,7 @@ def main() -> int:
     rmt.rmt_sync(h, stream)
     rmt.rmt_probe(h, [])
     tokens = S * cfg.seg_len
-    value = world * tokens / (ms / 1e3)
+    value = job_throughput(tokens, ms, world)
 
     peaks, peak_src = load_peaks()
     achieved = probe["flops"] / (probe["ms"] / 1e3) / 1e12 if probe["ms"] > 0 else None
@@ -432,7 +447,7 @@ def main() -> int:
     if not args.no_sequential:
         run("sequential", 1)
         seq_ms = timed("sequential", max(1, min(K, 3)))
-        seq = {"ms_per_step": seq_ms, "tokens_per_s": world * tokens / (seq_ms / 1e3),
+        seq = {"ms_per_step": seq_ms, "tokens_per_s": job_throughput(tokens, seq_ms, world),
                "diagonal_speedup": seq_ms / ms}
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
@@ -452,13 +467,9 @@ def main() -> int:
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
     rmt.rmt_sync(h, stream)
-    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": job_throughput(tokens, e2e_ms, world), "unit": UNIT,
            "h2d_bytes_per_step": e_host.numel() * e_host.element_size(),
            "d2h_bytes_per_step": o_host.numel() * o_host.element_size() + A_host.numel() * 4 + z_host.numel() * 4}
 
