@@ -46,7 +46,8 @@ import math
 import numpy as np
 
 __all__ = ["phi", "silu", "rms_norm", "rope", "causal_gqa_attention", "memory_read",
-           "memory_update", "armt_cell", "forward", "forward_tokens", "forward_batch", "diagonals",
+           "memory_update", "decoder_layer", "armt_cell", "forward", "forward_tokens", "forward_batch",
+           "full_attention_forward", "diagonals",
            "sequential_steps", "schedule_triples", "schedule_quads"]
 
 
@@ -194,16 +195,11 @@ def memory_update(k_raw: np.ndarray, v: np.ndarray, A: np.ndarray, z: np.ndarray
 
 # ------------------------------------------------------------------------------- model
 
-def armt_cell(x: np.ndarray, lw: dict, A: np.ndarray, z: np.ndarray, cfg) -> tuple:
-    """One (layer, segment) cell: x [M, d] is the layer input (segment rows, then memory rows).
-
-    lw holds this layer's matrices ([out, in]) and gains. Returns (layer output, A', z').
-    """
+def decoder_layer(x: np.ndarray, lw: dict, cfg) -> np.ndarray:
+    """The LLaMA decoder layer of a cell (no memory): x [m, d] at positions 0..m-1, causal
+    attention over its own rows. Returns the layer output [m, d]."""
     m = x.shape[0]
     hq, hkv, dh = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
-    # associative read at the layer input, projected back to d_model and added
-    o = memory_read(x @ lw["w_mq"].T, A, z, cfg.mem_eps)
-    x = x + o @ lw["w_mo"].T
     # attention block
     h = rms_norm(x, lw["g_attn"], cfg.rms_eps)
     q = rope((h @ lw["wq"].T).reshape(m, hq, dh), cfg.rope_theta)
@@ -214,7 +210,19 @@ def armt_cell(x: np.ndarray, lw: dict, A: np.ndarray, z: np.ndarray, cfg) -> tup
     # SwiGLU MLP block
     h = rms_norm(x, lw["g_mlp"], cfg.rms_eps)
     u = silu(h @ lw["w_gate"].T) * (h @ lw["w_up"].T)
-    x = x + u @ lw["w_down"].T
+    return x + u @ lw["w_down"].T
+
+
+def armt_cell(x: np.ndarray, lw: dict, A: np.ndarray, z: np.ndarray, cfg) -> tuple:
+    """One (layer, segment) cell: x [M, d] is the layer input (segment rows, then memory rows).
+
+    lw holds this layer's matrices ([out, in]) and gains. Returns (layer output, A', z').
+    """
+    m = x.shape[0]
+    # associative read at the layer input, projected back to d_model and added
+    o = memory_read(x @ lw["w_mq"].T, A, z, cfg.mem_eps)
+    x = x + o @ lw["w_mo"].T
+    x = decoder_layer(x, lw, cfg)
     # memory write from this layer's memory-token output rows (the cell's last n_mem rows)
     y = x[m - cfg.n_mem:]
     A, z = memory_update(y @ lw["w_mk"].T, y @ lw["w_mv"].T, A, z, cfg.mem_eps)
@@ -272,3 +280,14 @@ def forward_batch(cfg, weights: dict, embs: list, dtype=np.float32, A0=None, z0=
         As.append(A)
         zs.append(z)
     return outs, np.stack(As), np.stack(zs)
+
+
+def full_attention_forward(cfg, weights: dict, emb: np.ndarray, dtype=np.float32) -> np.ndarray:
+    """The comparison model of the ARMT paper [P2 abstract: ARMT with diagonal batching against
+    full-attention LLaMA-1B at 131,072 tokens]: the same decoder layers without the memory (no
+    memory tokens, no read or write), run over the whole sequence emb [T, d] as one causal
+    segment at positions 0..T-1. Returns the last layer's hidden states [T, d] in `dtype`."""
+    x = np.asarray(emb, dtype=dtype)
+    for l in range(cfg.n_layers):
+        x = decoder_layer(x, layer_weights(weights, l, dtype), cfg)
+    return x

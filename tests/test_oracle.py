@@ -306,6 +306,39 @@ def test_batch_entries_are_the_sequences_alone():
         np.testing.assert_allclose(z[b], ref[2], rtol=1e-10, atol=1e-11)
 
 
+def test_full_attention_model_matches_torch_layers():
+    """The comparison model: torch decoder layers over the whole sequence. With a zero memory
+    state the torch cell's read is exactly zero, and with n_mem = 0 it writes nothing."""
+    cfg = SMALL
+    w = _random_gains(make_weights(cfg, seed=24, std=0.2), 25)
+    T = 2 * cfg.seg_len + 7
+    emb = make_embeddings(cfg, 3, seed=26)[:T]
+    got = armt.full_attention_forward(cfg, w, emb, dtype=np.float64)
+    c = cfg.with_(seg_len=T, n_mem=0)
+    x = emb.astype(np.float64)
+    for l in range(cfg.n_layers):
+        lw = {k: v[l] for k, v in w.items() if k != "mem_tokens"}
+        x, _, _ = _torch_cell(x, lw, np.zeros((cfg.d_k, cfg.d_v)), np.zeros(cfg.d_k), c)
+    np.testing.assert_allclose(got, x, rtol=1e-10, atol=1e-11)
+
+
+def test_full_attention_equals_the_first_segment_of_the_armt():
+    """Before any memory is written the ARMT's read is exactly zero, and its memory tokens come
+    after the segment's tokens, which the causal mask hides from them: a sequence that fits in
+    one segment gets the same hidden states from both models."""
+    cfg = SMALL
+    w = make_weights(cfg, seed=27, std=0.2)
+    emb = make_embeddings(cfg, 1, seed=28)[:9]
+    full = armt.full_attention_forward(cfg, w, emb, dtype=np.float64)
+    armt_out, _, _ = armt.forward_tokens(cfg, w, emb, dtype=np.float64)
+    np.testing.assert_allclose(full, armt_out, rtol=1e-12, atol=1e-12)
+    # and a second segment does see the memory: the models part there
+    emb2 = make_embeddings(cfg, 2, seed=28)
+    full2 = armt.full_attention_forward(cfg, w, emb2[cfg.seg_len:], dtype=np.float64)
+    armt2, _, _ = armt.forward(cfg, w, emb2, 2, dtype=np.float64)
+    assert np.abs(full2 - armt2[cfg.seg_len:]).max() > 1e-6
+
+
 # -------------------------------------------------------------- recurrence invariants
 
 def test_later_segments_do_not_change_earlier_outputs():
