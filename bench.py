@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--segments", type=int, default=N_SEGMENTS)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-sequential", action="store_true")
+    p.add_argument("--no-full-attention", action="store_true",
+                   help="skip the full-attention comparison model (the decoder stack without memory over all tokens)")
     p.add_argument("--microbench", choices=["gemm", "memory", "attention"], default=None,
                    help="kernel-level sweeps instead of the forward: one JSON line per configuration")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions per microbench configuration")
@@ -450,6 +452,27 @@ def main() -> int:
         seq = {"ms_per_step": seq_ms, "tokens_per_s": job_throughput(tokens, seq_ms, world),
                "diagonal_speedup": seq_ms / ms}
 
+    # ---- the paper's comparison model on the same tokens: the decoder stack without the
+    # memory, causal over the whole sequence (arXiv 2506.05229 abstract reports 3.3x for ARMT
+    # with diagonal batching over full-attention LLaMA-1B at 131,072 tokens)
+    full = None
+    if not args.no_full_attention:
+        rmt.rmt_full_attention_forward(h, e, tokens, out, stream)  # allocates its activations
+        rmt.rmt_sync(h, stream)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rmt.rmt_full_attention_forward(h, e, tokens, out, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        full_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        rmt.rmt_sync(h, stream)
+        full = {"model": "the same 16-layer decoder without the associative memory, causal over all tokens",
+                "ms_per_step": full_ms, "tokens_per_s": job_throughput(tokens, full_ms, world),
+                "armt_diagonal_speedup": full_ms / ms, "pages_speedup": 3.3}
+
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     e_host = e.cpu().pin_memory()
     o_host = torch.empty_like(e_host).pin_memory()
@@ -497,6 +520,7 @@ def main() -> int:
             "gpu_launches": probe["all_launches"],
             "clocks": clocks,
             "sequential": seq,
+            "full_attention": full,
             "breakdown_one_step": breakdown,
         }
         print(json.dumps(line))

@@ -148,6 +148,20 @@ rmt_status rmt_forward_batch(rmt_handle* h, const void* emb, int32_t batch, cons
                              rmt_schedule schedule, const float* in_A, const float* in_z, void* out_hidden,
                              float* out_A, float* out_z, void* stream);
 
+/* The comparison model of the ARMT paper (arXiv 2506.05229 abstract: ARMT with diagonal
+ * batching against full-attention LLaMA-1B at 131,072 tokens): the handle's decoder stack
+ * without its associative memory -- no memory tokens, no memory read or write -- over one
+ * sequence of n_tokens, causal over all of them, RoPE at positions 0 .. n_tokens-1, on the
+ * handle's weights.
+ *   emb        [n_tokens, d_model] bf16, device or host.
+ *   out_hidden [n_tokens, d_model] bf16, device or host: the last layer's hidden states.
+ * bf16 handles only (RMT_EINVAL otherwise, or for n_tokens <= 0). The first call with a
+ * longer sequence allocates the activations for it (about 50 KB per token at the 1B shape)
+ * and synchronizes the device; RMT_ENOMEM if they do not fit. Asynchronous on `stream`
+ * otherwise; same ordering rules as rmt_forward. */
+rmt_status rmt_full_attention_forward(rmt_handle* h, const void* emb, int32_t n_tokens, void* out_hidden,
+                                      void* stream);
+
 /* The execution order as int32 triples (step, layer, segment), one per cell, n_layers*
  * n_segments of them: steps ascend; within a diagonal step layers ascend. Host memory,
  * cap = capacity of out_dls in int32 elements (>= 3*L*S). Needs no GPU. */

@@ -252,6 +252,18 @@ struct rmt_handle {
   // activations and memory state, sized for cap_b sequences (rmt_reserve)
   int cap_b = 0;
   std::vector<void*> act_allocs;
+  // full-attention forward (rmt_full_attention_forward): one causal segment of up to full_cap
+  // tokens, no memory; its own activations and tensor maps, allocated on first use
+  int full_cap = 0, full_T = 0;
+  std::vector<void*> full_allocs;
+  float* fx = nullptr;     // [2][T][d] residual slots (layer l reads slot l % 2, writes the other)
+  __half* fxb = nullptr;   // [2][T][d] f16 operand copies
+  void *fqkv = nullptr, *fatt = nullptr, *fu = nullptr;
+  float *fss1 = nullptr, *fss2 = nullptr;
+  float2* frope = nullptr;
+  __half2* frope_h = nullptr;
+  Cell* fcells = nullptr;  // [L]: cell l = layer l of the one segment
+  CUtensorMap fm_xb, fm_att, fm_u, fm_qkv, fm_x, fm_rope, fp_xb, fp_att, fp_u;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
   struct ProbeRec {
     int kind;
@@ -300,10 +312,23 @@ struct rmt_handle {
     qkv = att = u = om = nullptr;
     qm = part = A = z = ss1 = ss2 = nullptr;
   }
+  void free_full() {
+    for (void* p : full_allocs) cudaFree(p);
+    full_allocs.clear();
+    full_cap = full_T = 0;
+    fx = nullptr;
+    fxb = nullptr;
+    fqkv = fatt = fu = nullptr;
+    fss1 = fss2 = nullptr;
+    frope = nullptr;
+    frope_h = nullptr;
+    fcells = nullptr;
+  }
   void release() {
     for (void* p : allocs) cudaFree(p);
     allocs.clear();
     free_acts();
+    free_full();
     for (auto& kv : tables)
       if (kv.second.dev) cudaFree(kv.second.dev);
     tables.clear();
@@ -696,6 +721,125 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   return cudaSuccess;
 }
 
+// ------------------------------------------------ full-attention forward (comparison model)
+
+// Buffers, RoPE tables, cell table and tensor maps of the full-attention forward for T tokens
+// (reallocated when T exceeds the current capacity; the maps are rebuilt for every new T).
+rmt_status full_buffers(rmt_handle* h, int T) {
+  const rmt_cfg& c = h->cfg;
+  const size_t d = c.d_model, hd = size_t(c.n_heads) * c.head_dim, F = c.d_ff, half = c.head_dim / 2;
+  if (T > h->full_cap) {
+    RMT_CUDA(cudaDeviceSynchronize());  // an earlier full forward may still use the old buffers
+    h->free_full();
+    const size_t Tn = size_t(T);
+    struct {
+      void** p;
+      size_t bytes;
+    } plan[] = {
+        {reinterpret_cast<void**>(&h->fx), 2 * Tn * d * 4},      {reinterpret_cast<void**>(&h->fxb), 2 * Tn * d * 2},
+        {&h->fqkv, Tn * h->Nqkv * 2},                            {&h->fatt, Tn * hd * 2},
+        {&h->fu, Tn * F * 2},                                    {reinterpret_cast<void**>(&h->fss1), Tn * (d / 16 + 1) * 4},
+        {reinterpret_cast<void**>(&h->fss2), Tn * (d / 16 + 1) * 4},
+        {reinterpret_cast<void**>(&h->frope), Tn * half * sizeof(float2)},
+        {reinterpret_cast<void**>(&h->frope_h), Tn * half * sizeof(__half2)},
+        {reinterpret_cast<void**>(&h->fcells), size_t(c.n_layers) * sizeof(Cell)},
+    };
+    for (auto& e : plan) {
+      void* q = nullptr;
+      if (cudaMalloc(&q, e.bytes) != cudaSuccess) {
+        cudaGetLastError();
+        h->free_full();
+        return fail(RMT_ENOMEM, "full-attention buffer allocation failed");
+      }
+      h->full_allocs.push_back(q);
+      *e.p = q;
+    }
+    // RoPE angles p * theta^(-2i/dh) at positions 0..T-1, in double precision
+    std::vector<float2> tab(Tn * half);
+    std::vector<__half2> tab_h(Tn * half);
+    for (size_t q = 0; q < Tn; ++q)
+      for (size_t i = 0; i < half; ++i) {
+        const double ang = double(q) * std::pow(double(c.rope_theta), -2.0 * double(i) / c.head_dim);
+        tab[q * half + i] = make_float2(float(std::cos(ang)), float(std::sin(ang)));
+        tab_h[q * half + i] = __floats2half2_rn(tab[q * half + i].x, tab[q * half + i].y);
+      }
+    RMT_CUDA(cudaMemcpy(h->frope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    RMT_CUDA(cudaMemcpy(h->frope_h, tab_h.data(), tab_h.size() * sizeof(__half2), cudaMemcpyHostToDevice));
+    h->full_cap = T;
+  }
+  if (T != h->full_T) {
+    std::vector<Cell> cells(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) cells[l] = Cell{l, 0, 0, T, 0, l & 1, (l + 1) & 1, 0};
+    RMT_CUDA(cudaMemcpy(h->fcells, cells.data(), cells.size() * sizeof(Cell), cudaMemcpyHostToDevice));
+    auto map = [](CUtensorMap* m, const void* q, uint64_t inner, uint64_t rows, uint64_t depth, uint32_t box) {
+      return make_tmap_16_3d(m, q, inner, rows, depth, box, true);
+    };
+    const uint64_t Tu = uint64_t(T), pb = uint64_t(pair_token_tile(T) / 2);
+    const bool ok = map(&h->fm_xb, h->fxb, d, Tu, 2, 128) && map(&h->fm_att, h->fatt, hd, Tu, 1, 128) &&
+                    map(&h->fm_u, h->fu, F, Tu, 1, 128) && map(&h->fm_qkv, h->fqkv, h->Nqkv, Tu, 1, 128) &&
+                    map(&h->fp_xb, h->fxb, d, Tu, 2, uint32_t(pb)) && map(&h->fp_att, h->fatt, hd, Tu, 1, uint32_t(pb)) &&
+                    map(&h->fp_u, h->fu, F, Tu, 1, uint32_t(pb)) && make_tmap_f32_resid(&h->fm_x, h->fx, d, Tu, 2) &&
+                    (c.head_dim < 64 || map(&h->fm_rope, h->frope_h, c.head_dim, Tu, 1, 32));
+    if (!ok) return fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
+    h->full_T = T;
+  }
+  return RMT_OK;
+}
+
+// One projection of layer `cell` of the full-attention forward: the layer reads its input
+// slot for QKV; O adds the attention output to it into the output slot (and emits the RMSNorm
+// 2 statistics); gate/up reads the output slot; down adds the MLP output in place and emits
+// the RMSNorm 1 statistics of the next layer's input.
+cudaError_t run_proj_full(rmt_handle* h, Proj p, const Cell* cell, cudaStream_t st) {
+  const rmt_cfg& c = h->cfg;
+  const int d = c.d_model, hd = c.n_heads * c.head_dim, T = h->full_T;
+  EpiParams ep{};
+  ep.x = h->fx;
+  ep.ldx = d;
+  ep.rope = h->frope;
+  ep.head_dim = c.head_dim;
+  ep.rope_cols = (c.n_heads + c.n_kv_heads) * c.head_dim;
+  ep.out_mode = ep.src_mode = ep.dst_mode = kByLayer;
+  ep.ss_parts = h->ss_parts;
+  ep.inv_d = 1.f / float(d);
+  ep.rms_eps = c.rms_eps;
+  int N = 0, K = 0, bn = 0;
+  EpiKind epi = kEpiStoreAct;
+  IndexMode amode = kByLayer;
+  const CUtensorMap *ta = nullptr, *tb = nullptr, *tp = nullptr;
+  bool pair = false;
+  switch (p) {
+    case kProjQkv:
+      N = h->Nqkv, K = d, epi = kEpiRope, amode = kInSlot;
+      ep.out = h->fqkv, ep.ldo = h->Nqkv, ep.ss_in = h->fss1;
+      ta = &h->fm_xb, tb = &h->tm_wqkv, tp = &h->fp_xb, bn = h->bn_qkv, pair = h->pair_qkv;
+      break;
+    case kProjO:
+      N = d, K = hd, epi = kEpiResidCast;
+      ep.src_mode = kInSlot, ep.dst_mode = kOutSlot, ep.xb = h->fxb, ep.ss_out = h->fss2;
+      ta = &h->fm_att, tb = &h->tm_wo, tp = &h->fp_att, bn = h->bn_o, pair = h->pair_o;
+      break;
+    case kProjGateUp:
+      N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU, amode = kOutSlot;
+      ep.out = h->fu, ep.ldo = c.d_ff, ep.ss_in = h->fss2;
+      ta = &h->fm_xb, tb = &h->tm_wgu, tp = &h->fp_xb, bn = h->bn_gu, pair = h->pair_gu;
+      break;
+    case kProjDown:
+      N = d, K = c.d_ff, epi = kEpiResidCast;
+      ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->fxb, ep.ss_out = h->fss1;
+      ta = &h->fm_u, tb = &h->tm_wd, tp = &h->fp_u, bn = h->bn_d, pair = h->pair_d;
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  TcGemmArgs a{T, N, K, 1, cell, c.n_layers, amode, epi, ep, h->err};
+  if (pair && tc_pair_supported(T, N, K, epi, c.head_dim)) return launch_tc_pair_gemm(*tb, *tp, a, /*f16=*/true, st);
+  if (pair) return cudaErrorInvalidValue;  // the weights are packed for the CTA-pair kernel
+  const bool rope_tma = p == kProjQkv && c.head_dim >= 64;
+  a.ep.rope_tma = rope_tma;
+  return launch_tc_gemm(*ta, *tb, rope_tma ? h->fm_rope : h->fm_x, a, bn, /*f16=*/true, st);
+}
+
 struct DeviceGuard {
   int prev = -1;
   explicit DeviceGuard(int dev) {
@@ -1021,6 +1165,68 @@ rmt_status rmt_forward_batch(rmt_handle* h, const void* emb, int32_t batch, cons
   size_t total = 0;
   RMT_TRY(check_lengths(batch, n_tokens, T, total));
   return forward_impl(h, emb, T, total, schedule, in_A, in_z, out_hidden, out_A, out_z, stream);
+}
+
+rmt_status rmt_full_attention_forward(rmt_handle* h, const void* emb, int32_t n_tokens, void* out_hidden,
+                                      void* stream) {
+  if (!h) return fail(RMT_EINVAL, "null handle");
+  if (!emb || !out_hidden) return fail(RMT_EINVAL, "emb and out_hidden must not be null");
+  if (!h->bf16) return fail(RMT_EINVAL, "the full-attention forward needs a bf16 handle");
+  if (n_tokens <= 0) return fail(RMT_EINVAL, "n_tokens must be positive");
+  const rmt_cfg& c = h->cfg;
+  if (h->ss_parts > 32 || c.d_model % h->ss_parts || (c.d_model / h->ss_parts) % 4)
+    return fail(RMT_EINVAL, "d_model does not fit the RMSNorm statistics blocks");
+  DeviceGuard guard(h->dev);
+  RMT_TRY(full_buffers(h, n_tokens));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int L = c.n_layers, d = c.d_model, T = n_tokens;
+  const size_t io_bytes = size_t(T) * d * h->es;
+  const void* emb_dev = emb;
+  if (is_host_ptr(emb)) {
+    if (h->emb_stage_bytes < io_bytes) {
+      if (h->emb_stage) cudaFree(h->emb_stage);
+      h->emb_stage = nullptr;
+      h->emb_stage_bytes = 0;
+      if (cudaMalloc(&h->emb_stage, io_bytes) != cudaSuccess) return fail(RMT_ENOMEM, "staging allocation failed");
+      h->emb_stage_bytes = io_bytes;
+    }
+    RMT_CUDA(cudaMemcpyAsync(h->emb_stage, emb, io_bytes, cudaMemcpyHostToDevice, st));
+    emb_dev = h->emb_stage;
+  }
+  void* out_dev = out_hidden;
+  const bool out_host = is_host_ptr(out_hidden);
+  if (out_host) {
+    if (h->out_stage_bytes < io_bytes) {
+      if (h->out_stage) cudaFree(h->out_stage);
+      h->out_stage = nullptr;
+      h->out_stage_bytes = 0;
+      if (cudaMalloc(&h->out_stage, io_bytes) != cudaSuccess) return fail(RMT_ENOMEM, "staging allocation failed");
+      h->out_stage_bytes = io_bytes;
+    }
+    out_dev = h->out_stage;
+  }
+  auto launch_fail = [&](cudaError_t e) {
+    return fail(RMT_ECUDA, std::string("launch failed: ") + cudaGetErrorString(e));
+  };
+  // the input: the embeddings into slot 0 (fp32 and the f16 copy), and their RMSNorm statistics
+  cudaError_t e = launch_assemble(h->fcells, 1, emb_dev, h->memtok, h->fx, h->fxb, T, 0, d, true, st);
+  if (e == cudaSuccess) e = launch_row_ssq(h->fx, h->fss1, T, d, h->ss_parts, st);
+  if (e != cudaSuccess) return launch_fail(e);
+  for (int l = 0; l < L; ++l) {
+    const Cell* cell = h->fcells + l;
+    if ((e = run_proj_full(h, kProjQkv, cell, st)) != cudaSuccess) return launch_fail(e);
+    AttnArgs a{h->fqkv, h->fatt, T, c.n_heads, c.n_kv_heads, c.head_dim, 1, cell, kByLayer, L, h->err};
+    e = attention_tc_supported(c.head_dim) ? launch_attention_tc(h->fm_qkv, a, /*f16=*/true, st)
+                                           : launch_attention(a, kElemF16, st);
+    if (e != cudaSuccess) return launch_fail(e);
+    if ((e = run_proj_full(h, kProjO, cell, st)) != cudaSuccess) return launch_fail(e);
+    if ((e = run_proj_full(h, kProjGateUp, cell, st)) != cudaSuccess) return launch_fail(e);
+    if ((e = run_proj_full(h, kProjDown, cell, st)) != cudaSuccess) return launch_fail(e);
+  }
+  if ((e = launch_emit(h->fcells + L - 1, 1, h->fx, out_dev, T, 0, d, true, st)) != cudaSuccess) return launch_fail(e);
+  if (out_host) RMT_CUDA(cudaMemcpyAsync(out_hidden, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
+  RMT_CUDA(cudaGetLastError());
+  return RMT_OK;
 }
 
 rmt_status rmt_reserve(rmt_handle* h, int32_t max_batch) {

@@ -99,6 +99,27 @@ __global__ void emit_kernel(const Cell* cells, const float* x, T* out, int M, in
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) Vec4<T>::store(dst + k, Vec4<float>::load(src + k));
 }
 
+// Row sums of squares of an fp32 [M, d] block, per column block b of width w = d / parts
+// (ss[row * parts + b]): the RMSNorm statistics a folded projection reads. One warp per
+// block: each lane squares 4 consecutive columns per 128-column step, then a fixed butterfly
+// adds the lanes.
+__global__ void row_ssq_kernel(const float* x, float* ss, int d, int parts) {
+  pdl_trigger();
+  pdl_wait();  // inputs come from the previous kernels of the stream
+  const int row = blockIdx.x, b = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (b >= parts) return;
+  const int w = d / parts;
+  const float* xb = x + static_cast<size_t>(row) * d + static_cast<size_t>(b) * w;
+  float s = 0.f;
+  for (int k = lane * 4; k < w; k += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(xb + k);
+    s += ((v.x * v.x + v.y * v.y) + v.z * v.z) + v.w * v.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) ss[static_cast<size_t>(row) * parts + b] = s;
+}
+
 // W[l][n][k] *= g[l][k]: folds an RMSNorm gain into the weight that consumes its output.
 template <typename WT, typename GT>
 __global__ void scale_cols_kernel(WT* w, const GT* g, int N, int K) {
@@ -160,6 +181,12 @@ cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const voi
                       static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d);
   return launch_pdl(assemble_kernel<float>, dim3(M, G), dim3(threads), 0, st, cells, static_cast<const float*>(emb),
                     static_cast<const float*>(mem), x, xb, M, n_mem, d);
+}
+
+cudaError_t launch_row_ssq(const float* x, float* ss, int M, int d, int parts, cudaStream_t st) {
+  if (parts <= 0 || parts > 32 || d % parts || (d / parts) % 4) return cudaErrorInvalidValue;
+  if (M <= 0) return cudaSuccess;
+  return launch_pdl(row_ssq_kernel, dim3(M), dim3(32 * parts), 0, st, x, ss, d, parts);
 }
 
 cudaError_t launch_emit(const Cell* cells, int G, const float* x, void* out, int M, int n_mem, int d, bool bf16,

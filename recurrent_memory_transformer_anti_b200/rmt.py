@@ -21,7 +21,8 @@ SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
 DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16}
 STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE"}
 
-EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "rmt_forward_batch", "rmt_schedule_table",
+EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "rmt_forward_batch",
+            "rmt_full_attention_forward", "rmt_schedule_table",
             "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
             "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
@@ -64,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "rmt_forward_resume": [vp, vp, i32, ctypes.c_int, vp, vp, vp, vp, vp, vp],
         "rmt_forward_batch": [vp, vp, i32, p32, ctypes.c_int, vp, vp, vp, vp, vp, vp],
         "rmt_reserve": [vp, i32],
+        "rmt_full_attention_forward": [vp, vp, i32, vp, vp],
         "rmt_schedule_table": [i32, i32, ctypes.c_int, p32, sz],
         "rmt_schedule_table_batch": [i32, i32, p32, ctypes.c_int, p32, sz],
         "rmt_get_schedule": [vp, i32, ctypes.c_int, p32, sz],
@@ -193,6 +195,11 @@ def rmt_forward_batch(h: Handle, emb, n_tokens, schedule, out_hidden, in_A=None,
     _check(_lib.rmt_forward_batch(h.ptr, _ptr(emb), int(nt.size), nt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                                   sch, _ptr(in_A), _ptr(in_z), _ptr(out_hidden), _ptr(out_A), _ptr(out_z),
                                   _stream(stream)), "rmt_forward_batch")
+
+
+def rmt_full_attention_forward(h: Handle, emb, n_tokens: int, out_hidden, stream=None) -> None:
+    _check(_lib.rmt_full_attention_forward(h.ptr, _ptr(emb), int(n_tokens), _ptr(out_hidden), _stream(stream)),
+           "rmt_full_attention_forward")
 
 
 def rmt_reserve(h: Handle, max_batch: int) -> None:

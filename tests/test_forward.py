@@ -398,3 +398,63 @@ def test_batch_argument_errors(tiny):
     # the handle is still usable
     rmt.rmt_forward_batch(h, e, [cfg.seg_len], "diagonal", out)
     rmt.rmt_sync(h)
+
+
+# ------------------------------------------------ full-attention comparison model
+
+def _full(h, cfg, emb):
+    e = rmt.storage(emb, cfg.dtype, device="cuda")
+    out = torch.empty_like(e)
+    rmt.rmt_full_attention_forward(h, e, emb.shape[0], out)
+    rmt.rmt_sync(h)
+    return out.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("T", [1, 130, 455])
+def test_full_attention_matches_oracle(cuda_ok, T):
+    """The decoder stack without the memory, causal over T tokens (one or several query tiles
+    with a ragged tail), against the oracle's comparison model."""
+    cfg = CONFIGS["small-bf16"]
+    w, h = build(cfg)
+    emb = embeddings(cfg, 3, seed=40)[:T]
+    got = _full(h, cfg, emb)
+    ref = armt.full_attention_forward(cfg, w, emb, dtype=np.float32)
+    assert normwise(got, ref) < BF16_TOL
+    # a longer call reallocates; a shorter one after it reuses the buffers with the same bits
+    if T > 1:
+        _full(h, cfg, embeddings(cfg, 3, seed=41))
+        np.testing.assert_array_equal(_full(h, cfg, emb), got)
+    rmt.rmt_destroy(h)
+
+
+def test_full_attention_argument_errors(tiny, cuda_ok):
+    cfg, w, h = tiny  # an fp32 handle
+    e = rmt.storage(embeddings(cfg, 1), cfg.dtype, device="cuda")
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_full_attention_forward(h, e, cfg.seg_len, torch.empty_like(e))
+    assert ex.value.status == rmt.RMT_EINVAL
+    cfg2 = CONFIGS["small-bf16"]
+    w2, h2 = build(cfg2)
+    e2 = rmt.storage(embeddings(cfg2, 1), cfg2.dtype, device="cuda")
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_full_attention_forward(h2, e2, 0, torch.empty_like(e2))
+    assert ex.value.status == rmt.RMT_EINVAL
+    rmt.rmt_destroy(h2)
+
+
+def test_full_attention_1b_at_131k(cuda_ok):
+    """The comparison model at the bench's size: LLaMA-1B shape, 131,072 tokens, one causal
+    segment. The oracle cannot run it in seconds, so: the first 1024 rows equal a 1024-token
+    run bit for bit (a row never depends on later tokens, and both runs tile tokens by 256),
+    and that run matches the oracle within the bf16 tolerance."""
+    cfg = CONFIGS["1b"]
+    w, h = build(cfg)
+    T, P = 131072, 1024
+    emb = embeddings(cfg, T // cfg.seg_len)
+    full = _full(h, cfg, emb)
+    assert np.isfinite(full).all()
+    part = _full(h, cfg, emb[:P])
+    np.testing.assert_array_equal(full[:P], part)
+    rmt.rmt_destroy(h)
+    ref = armt.full_attention_forward(cfg, w, emb[:P], dtype=np.float32)
+    assert normwise(part, ref) < BF16_TOL
