@@ -381,8 +381,9 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
           store32_16(dst + 32 * oc, v);
         }
       }
+      // O read (the MMA warp reads none of the output stores: no release needed)
       sm100::tc_fence_before();
-      sm100::mbar_arrive(bar(kOFree));
+      sm100::mbar_arrive_relaxed(bar(kOFree));
     }
     if (!ok && lane == 0 && a.err) atomicOr(a.err, kErrTimeoutEpilogue);
   }

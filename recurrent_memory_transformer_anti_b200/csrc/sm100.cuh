@@ -38,6 +38,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Arrive without release semantics (orders none of this thread's earlier memory accesses):
+// for signals whose consumer reads nothing this thread wrote, e.g. "this warp's tcgen05.ld of a
+// TMEM range completed", given after its global stores, which the arrive then need not drain.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
@@ -310,6 +317,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 // Arrive once on an mbarrier anywhere in the cluster (cluster-scope release).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// Arrive on a cluster barrier without release semantics: orders none of this thread's earlier
+// memory accesses. For signals whose consumer reads nothing this thread wrote -- such as "this
+// warp's tcgen05.ld of an accumulator completed" (after tcgen05.wait::ld and
+// tcgen05.fence::before_thread_sync) -- so the arrive need not wait for earlier global stores.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 // 3-D tiled load into this CTA's shared memory whose byte count completes on an mbarrier

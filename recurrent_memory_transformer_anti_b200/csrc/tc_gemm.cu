@@ -627,9 +627,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else {
         epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
       }
+      // accumulator read: the MMA issuer reads none of the epilogue's stores, so the arrive is
+      // relaxed and does not wait for them
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(tempty_bar(acc));
+      if (lane == 0) sm100::mbar_arrive_relaxed(tempty_bar(acc));
       if (++acc == 2) {
         acc = 0;
         aph ^= 1u;

@@ -449,10 +449,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                             static_cast<uint32_t>(acc * C::ACC_COLS + wg * cnt);
       float* red = red_all + ((acc * 2 + wg) * 4 + quarter) * 128;
       pair_epilogue<EPI, OpT>(args, c, tacc, tok0, cnt, f, lane, rs, red);
-      // accumulator drained: release it to the even CTA's MMA issuer
+      // accumulator drained (every lane's tcgen05.ld waited for): release it to the even CTA's
+      // MMA issuer. The issuer reads none of this warp's global stores, so the arrive is
+      // relaxed and does not wait for them to drain.
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive_cluster(acc ? tempty_lead1 : tempty_lead0);
+      if (lane == 0) sm100::mbar_arrive_cluster_relaxed(acc ? tempty_lead1 : tempty_lead0);
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
         if (ep.ss_out) {
           // the four warps of this warpgroup hold 32-feature sums of the same tokens: combine
