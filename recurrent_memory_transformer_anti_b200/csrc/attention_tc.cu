@@ -290,15 +290,15 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
         sm100::mbar_arrive(bar(kSFree));
         const int k0 = j * 128;
         const bool need_mask = (j == qt) || (k0 + 128 > kvlim);
-        // causal mask (and the cell's ragged end) only on the tiles that need it
+        // causal mask (and the cell's ragged end) only on the tiles that need it: key k0 + e is
+        // visible iff e <= vis, so each element costs one compare with a constant and a select
         if (need_mask) {
+          const int vis = min(qrow, kvlim - 1) - k0;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kv = k0 + 32 * q4 + i;
-              if (kv > qrow || kv >= kvlim) s[q4][i] = __float_as_uint(-INFINITY);
-            }
+            for (int i = 0; i < 32; ++i)
+              if (32 * q4 + i > vis) s[q4][i] = __float_as_uint(-INFINITY);
           }
         }
         // row max over 4 independent partials (short dependency chains)
