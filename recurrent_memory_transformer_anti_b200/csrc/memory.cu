@@ -202,19 +202,34 @@ __global__ void __launch_bounds__(kUpdThreads) mem_update_kernel(const MemUpdate
   float* A = a.A + si * dk * dv;
   float* z = a.z + si * dk;
 
-  for (int e = threadIdx.x; e < n * dkv; e += kUpdThreads) {
-    const int r = e / dkv, j = e % dkv;
-    float val;
-    if (a.part) {
-      const float* p = a.part + ki * a.nsplit * n * dkv + e;
-      const size_t stride = static_cast<size_t>(n) * dkv;
-      val = 0.f;
+  if (a.part) {
+    // each thread sums 4 elements at once over the splits (ascending, as one element at a
+    // time would), so 4 x 8 partial loads are in flight instead of 8
+    constexpr int EPT = 4;
+    const float* p = a.part + ki * a.nsplit * n * dkv;
+    const size_t stride = static_cast<size_t>(n) * dkv;
+    for (int e0 = threadIdx.x; e0 < n * dkv; e0 += EPT * kUpdThreads) {
+      float val[EPT] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-      for (int sp = 0; sp < a.nsplit; ++sp) val += p[sp * stride];
-    } else {
-      val = j < dk ? a.k[(ki * n + r) * dk + j] : a.v[(ki * n + r) * dv + (j - dk)];
+      for (int sp = 0; sp < a.nsplit; ++sp) {
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+          const int e = e0 + u * kUpdThreads;
+          if (e < n * dkv) val[u] += p[sp * stride + e];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < EPT; ++u) {
+        const int e = e0 + u * kUpdThreads;
+        if (e < n * dkv) KV[e] = e % dkv < dk ? phi_f(val[u]) : val[u];
+      }
     }
-    KV[e] = j < dk ? phi_f(val) : val;
+  } else {
+    for (int e = threadIdx.x; e < n * dkv; e += kUpdThreads) {
+      const int r = e / dkv, j = e % dkv;
+      const float val = j < dk ? a.k[(ki * n + r) * dk + j] : a.v[(ki * n + r) * dv + (j - dk)];
+      KV[e] = j < dk ? phi_f(val) : val;
+    }
   }
   for (int e = threadIdx.x; e < dk * dv; e += kUpdThreads) As[e] = A[e];
   for (int e = threadIdx.x; e < dk; e += kUpdThreads) zs[e] = z[e];
