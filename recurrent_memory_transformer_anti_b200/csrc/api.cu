@@ -248,6 +248,12 @@ struct rmt_handle {
   // bf16 mode with d_k = d_v = 64: the memory read runs in the mem-q GEMM's epilogue (the
   // query never goes to memory) and has no launch of its own
   bool fuse_read = false;
+  // with fuse_read and the O projection on CTA pairs: the read-out o sits in d_v extra columns
+  // of the attention output and W_mo in d_v extra columns of W_o, so the O projection adds
+  // W_o att + W_mo o to the layer input in one accumulator; the read-out projection then only
+  // forms the f16 operand copy and RMSNorm statistics of x + W_mo o (no fp32 store)
+  bool fold_mo = false;
+  int ld_att = 0;  // row stride of the attention output (n_heads * head_dim, + d_v with fold_mo)
   std::vector<void*> allocs;
   // activations and memory state, sized for cap_b sequences (rmt_reserve)
   int cap_b = 0;
@@ -425,7 +431,14 @@ rmt_status pack_weights(rmt_handle* h, const rmt_weights* w) {
       RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, hd * d), w->wk[l], kvd * d * es, "wk"));
     }
     RMT_TRY(copy_in(at(h->w_qkv, nqkv * d, l, (hd + kvd) * d), w->wv[l], kvd * d * es, "wv"));
-    RMT_TRY(copy_in(at(h->w_o, d * hd, l), w->wo[l], d * hd * es, "wo"));
+    if (h->fold_mo) {  // row n of layer l: W_o[n][0..hd) then W_mo[n][0..dv)
+      const size_t ldw = hd + dv;
+      if (!w->wo[l] || !w->w_mo[l]) return fail(RMT_EINVAL, "null wo/w_mo");
+      RMT_CUDA(cudaMemcpy2D(at(h->w_o, d * ldw, l), ldw * es, w->wo[l], hd * es, hd * es, d, cudaMemcpyDefault));
+      RMT_CUDA(cudaMemcpy2D(at(h->w_o, d * ldw, l, hd), ldw * es, w->w_mo[l], dv * es, dv * es, d, cudaMemcpyDefault));
+    } else {
+      RMT_TRY(copy_in(at(h->w_o, d * hd, l), w->wo[l], d * hd * es, "wo"));
+    }
     // gate/up interleaved: row by row for the pair GEMM, else in blocks of kSwiGLUBlock rows
     if (!w->w_gate[l] || !w->w_up[l]) return fail(RMT_EINVAL, "null w_gate/w_up");
     const size_t rows = h->pair_gu ? 1 : kSwiGLUBlock, blk = rows * d * es;
@@ -462,16 +475,22 @@ rmt_status build_maps(rmt_handle* h) {
   // weight boxes: 128 rows per CTA on the pair GEMM, else the tile width
   const uint32_t pb = static_cast<uint32_t>(pair_token_tile(static_cast<int>(M)) / 2);
   const bool any_pair = h->pair_mo || h->pair_qkv || h->pair_o || h->pair_gu || h->pair_d;
-  bool ok = map(&h->tm_xb, h->xb, d, M, NS, 128) && map(&h->tm_om, h->om, c.d_v, M, L, 128) &&
-            map(&h->tm_att, h->att, hd, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
+  // the read-out o: its own buffer, or (fold_mo) the last d_v columns of the attention output
+  const uint64_t lda = uint64_t(h->ld_att);
+  auto map_om = [&](CUtensorMap* m, uint32_t box) {
+    return h->fold_mo ? make_tmap_16_3d_strided(m, static_cast<__half*>(h->att) + hd, c.d_v, M, L, lda, box, true)
+                      : map(m, h->om, c.d_v, M, L, box);
+  };
+  bool ok = map(&h->tm_xb, h->xb, d, M, NS, 128) && map_om(&h->tm_om, 128) &&
+            map(&h->tm_att, h->att, lda, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
             map(&h->tm_wmq, h->w_mq, d, c.d_k, LW, h->bn_mq) &&
             map(&h->tm_wmo, h->w_mo, c.d_v, d, LW, h->pair_mo ? 128 : h->bn_mo) &&
             map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, LW, h->pair_qkv ? 128 : h->bn_qkv) &&
-            map(&h->tm_wo, h->w_o, hd, d, LW, h->pair_o ? 128 : h->bn_o) &&
+            map(&h->tm_wo, h->w_o, lda, d, LW, h->pair_o ? 128 : h->bn_o) &&
             map(&h->tm_wgu, h->w_gu, d, 2 * F, LW, h->pair_gu ? 128 : h->bn_gu) &&
             map(&h->tm_wd, h->w_d, F, d, LW, h->pair_d ? 128 : h->bn_d) &&
-            (!any_pair || (map(&h->tp_xb, h->xb, d, M, NS, pb) && map(&h->tp_om, h->om, c.d_v, M, L, pb) &&
-                           map(&h->tp_att, h->att, hd, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
+            (!any_pair || (map(&h->tp_xb, h->xb, d, M, NS, pb) && map_om(&h->tp_om, pb) &&
+                           map(&h->tp_att, h->att, lda, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
             make_tmap_f32_resid(&h->tm_x, h->x, d, M, NS) &&
             (c.head_dim < 64 || map(&h->tm_rope, h->rope_h, c.head_dim, M, 1, 32));
@@ -486,14 +505,14 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
   RMT_CUDA(cudaDeviceSynchronize());
   h->free_acts();
   const rmt_cfg& c = h->cfg;
-  const size_t nb = B, L = c.n_layers, d = c.d_model, M = h->M, es = h->es, hd = size_t(c.n_heads) * c.head_dim,
-               F = c.d_ff, dk = c.d_k, dv = c.d_v, BL = nb * L;
+  const size_t nb = B, L = c.n_layers, d = c.d_model, M = h->M, es = h->es, F = c.d_ff, dk = c.d_k, dv = c.d_v,
+               BL = nb * L;
   struct {
     void** p;
     size_t bytes;
   } plan[] = {
       {reinterpret_cast<void**>(&h->x), nb * n_slots(c.n_layers) * M * d * 4},
-      {&h->qkv, BL * M * h->Nqkv * es},   {&h->att, BL * M * hd * es},
+      {&h->qkv, BL * M * h->Nqkv * es},   {&h->att, BL * M * size_t(h->ld_att) * es},
       {reinterpret_cast<void**>(&h->ss1), BL * M * (d / 16 + 1) * 4},
       {reinterpret_cast<void**>(&h->ss2), BL * M * (d / 16 + 1) * 4},
       {&h->u, BL * M * F * es},           {&h->om, BL * M * dv * es},
@@ -569,13 +588,17 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       a32 = h->x, w = h->w_mq, ta = &h->tm_xb, tb = &h->tm_wmq, bn = h->bn_mq;
       if (h->fuse_read) {  // o = phi(q) A / (phi(q) . z + eps) straight from the accumulator
         epi = kEpiMemRead;
-        ep.out = h->om, ep.ldo = c.d_v;
+        if (h->fold_mo)  // o goes to the last d_v columns of the attention output rows
+          ep.out = static_cast<__half*>(h->att) + hd, ep.ldo = h->ld_att;
+        else
+          ep.out = h->om, ep.ldo = c.d_v;
         ep.mem_A = h->A, ep.mem_z = h->z, ep.mem_dv = c.d_v, ep.mem_eps = c.mem_eps;
       }
       break;
     case kProjMemO:  // x_out = x_in + read-out; emits the row sums of squares of RMSNorm 1
       N = d, K = c.d_v, epi = resid;
       ep.src_mode = kInSlot, ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss1;
+      ep.resid_no_store = h->fold_mo;  // the O projection adds W_mo o itself
       a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
       tp = &h->tp_om, pair = h->pair_mo;
       break;
@@ -588,6 +611,10 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
     case kProjO:  // x_out += attention output; emits the row sums of squares of RMSNorm 2
       N = d, K = hd, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss2;
+      if (h->fold_mo) {  // x_out = x_in + [W_o | W_mo] [att ; o]
+        K = h->ld_att;
+        ep.src_mode = kInSlot;
+      }
       a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
       tp = &h->tp_att, pair = h->pair_o;
       break;
@@ -675,7 +702,11 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                     });
     if (e != cudaSuccess) return e;
   }
-  e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv, g * (m * dv * es + dd * dv * es + 2 * m * dd * 4), st,
+  // with fold_mo the read-out projection stores only the f16 copy, and the O projection
+  // carries the d_v extra columns of K
+  const double fold = h->fold_mo ? 1.0 : 0.0;
+  e = launch_kind(h, RMT_K_MEMO, 2 * g * m * dd * dv,
+                  g * (m * dv * es + dd * dv * es + m * dd * 4 + (fold ? m * dd * 2 : m * dd * 4)), st,
                   [&] { return run_proj(h, kProjMemO, cells, G, st); });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_QKV, 2 * g * m * nq * dd, g * (m * dd * es + nq * dd * es + m * nq * es), st,
@@ -683,13 +714,15 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_ATTENTION, c.n_heads * 4.0 * c.head_dim * pairs,
                   g * (m * nq * es + m * hd * es), st, [&] {
-                    AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err};
+                    AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err,
+                               h->ld_att};
                     if (h->bf16 && attention_tc_supported(c.head_dim))
                       return launch_attention_tc(h->tm_qkv, a, /*f16=*/true, st);
                     return launch_attention(a, h->bf16 ? kElemF16 : kElemF32, st);
                   });
   if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd, g * (m * hd * es + dd * hd * es + 2 * m * dd * 4), st,
+  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * (hd + fold * dv),
+                  g * (m * (hd + fold * dv) * es + dd * (hd + fold * dv) * es + 2 * m * dd * 4), st,
                   [&] { return run_proj(h, kProjO, cells, G, st); });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_GATEUP, 2 * g * m * 2 * F * dd, g * (m * dd * es + 2 * F * dd * es + m * F * es), st,
@@ -929,13 +962,26 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   h->M = c.seg_len + c.n_mem;
   h->Nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
   h->nsplit = (c.d_model + kMemKvSplit - 1) / kMemKvSplit;
-  const size_t L = c.n_layers, d = c.d_model, M = h->M, es = h->es, hd = size_t(c.n_heads) * c.head_dim,
-               F = c.d_ff, dk = c.d_k, dv = c.d_v;
+  const size_t L = c.n_layers, d = c.d_model, M = h->M, es = h->es, F = c.d_ff, dk = c.d_k, dv = c.d_v;
+  if (h->bf16) {
+    const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
+    // the memory read-out projection (K = d_v) is a pure stream over the residual; it stays on
+    // the single-CTA kernel, whose residual epilogue moves whole blocks through TMA
+    h->pair_mo = false;
+    h->fuse_read = c.d_k == 64 && c.d_v == 64 && tc_pick_bn(c.d_k, kEpiStoreF32, 0) == 64;
+    h->pair_qkv = tc_pair_supported(Mi, h->Nqkv, di, kEpiRope, c.head_dim);
+    h->pair_gu = tc_pair_supported(Mi, 2 * Fi, di, kEpiSwiGLU, 0);
+    h->pair_d = tc_pair_supported(Mi, di, Fi, kEpiResidCast, 0);
+    h->pair_o = tc_pair_supported(Mi, di, hdi, kEpiResidCast, 0);
+    h->fold_mo = h->fuse_read && h->pair_o && tc_pair_supported(Mi, di, hdi + c.d_v, kEpiResidCast, 0);
+  }
+  h->ld_att = c.n_heads * c.head_dim + (h->fold_mo ? c.d_v : 0);
+  const size_t ldw_o = size_t(h->ld_att);  // W_o rows: [W_o | W_mo] with fold_mo
   struct {
     void** p;
     size_t bytes;
   } plan[] = {
-      {&h->w_qkv, L * h->Nqkv * d * es}, {&h->w_o, L * d * hd * es},        {&h->w_gu, L * 2 * F * d * es},
+      {&h->w_qkv, L * h->Nqkv * d * es}, {&h->w_o, L * d * ldw_o * es},     {&h->w_gu, L * 2 * F * d * es},
       {&h->w_d, L * d * F * es},         {&h->w_mq, L * dk * d * es},       {&h->w_mo, L * d * dv * es},
       {&h->w_mkv, L * (dk + dv) * d * es}, {&h->g1, L * d * es},            {&h->g2, L * d * es},
       {&h->memtok, size_t(c.n_mem) * d * es},
@@ -947,27 +993,16 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
     *e.p = h->alloc(e.bytes);
     if (!*e.p) return bail(fail(RMT_ENOMEM, "device allocation failed"));
   }
-  if (h->bf16) {
-    const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
-    // the memory read-out projection (K = d_v) is a pure stream over the residual; it stays on
-    // the single-CTA kernel, whose residual epilogue moves whole blocks through TMA
-    h->pair_mo = false;
-    h->fuse_read = c.d_k == 64 && c.d_v == 64 && tc_pick_bn(c.d_k, kEpiStoreF32, 0) == 64;
-    h->pair_qkv = tc_pair_supported(Mi, h->Nqkv, di, kEpiRope, c.head_dim);
-    h->pair_o = tc_pair_supported(Mi, di, hdi, kEpiResidCast, 0);
-    h->pair_gu = tc_pair_supported(Mi, 2 * Fi, di, kEpiSwiGLU, 0);
-    h->pair_d = tc_pair_supported(Mi, di, Fi, kEpiResidCast, 0);
-  }
   rmt_status st = pack_weights(h, weights);
   if (st != RMT_OK) return bail(st);
   // bf16 mode: the tensor-core operands are f16 (3 more mantissa bits than bf16, same MMA
   // rate); the bf16 weight values convert exactly (bar magnitudes below 2^-17).
   if (h->bf16) {
-    const size_t L_ = c.n_layers, d_ = c.d_model, hd_ = size_t(c.n_heads) * c.head_dim, F_ = c.d_ff;
+    const size_t L_ = c.n_layers, d_ = c.d_model, F_ = c.d_ff;
     const struct {
       void* p;
       size_t n;
-    } ops[] = {{h->w_qkv, L_ * h->Nqkv * d_}, {h->w_o, L_ * d_ * hd_},       {h->w_gu, L_ * 2 * F_ * d_},
+    } ops[] = {{h->w_qkv, L_ * h->Nqkv * d_}, {h->w_o, L_ * d_ * size_t(h->ld_att)}, {h->w_gu, L_ * 2 * F_ * d_},
                {h->w_d, L_ * d_ * F_},        {h->w_mq, L_ * c.d_k * d_},    {h->w_mo, L_ * d_ * c.d_v}};
     for (const auto& o : ops)
       if (launch_bf16_to_f16(o.p, o.n, 0) != cudaSuccess) return bail(fail(RMT_ECUDA, "weight conversion failed"));

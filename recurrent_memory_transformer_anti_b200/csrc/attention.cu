@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const Cell c = a.cells[blockIdx.z];
   const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
-  const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.H * HD;
+  const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.ldo ? a.ldo : a.H * HD;
   const size_t slice = cell_index(a.mode, a.L, c);
   const OpT* base = static_cast<const OpT*>(a.qkv) + slice * a.M * ldq;
   const OpT* qsrc = base + h * HD;
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
   const Cell c = a.cells[blockIdx.z];
   const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
-  const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.H * HD;
+  const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.ldo ? a.ldo : a.H * HD;
   const size_t slice = cell_index(a.mode, a.L, c);
   const float* base = static_cast<const float*>(a.qkv) + slice * a.M * ldq;
   const int row = qc * BQ + threadIdx.x;

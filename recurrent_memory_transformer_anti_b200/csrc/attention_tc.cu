@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       if (!ok) break;
       sm100::tc_fence_after();
       const float inv = 1.f / l;
-      const int ldo = a.H * HD;
+      const int ldo = a.ldo ? a.ldo : a.H * HD;
       OpT* dst = static_cast<OpT*>(a.out) + (static_cast<size_t>(slice) * a.M + qrow) * ldo + h * HD;
 #pragma unroll 1
       for (int oc = 0; oc < HD / 32; ++oc) {

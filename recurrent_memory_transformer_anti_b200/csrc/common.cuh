@@ -120,6 +120,10 @@ struct EpiParams {
   const float* mem_z;
   int mem_dv;
   float mem_eps;
+  // kEpiResidCast on the single-CTA kernel: keep the sum x[src] + acc in registers for the
+  // operand copy and the row sums of squares, but do not store it to x[dst] (its consumer
+  // adds the same product itself)
+  int resid_no_store;
 };
 
 // RMSNorm row scale from the per-block sums of squares of one row (fixed summation order).

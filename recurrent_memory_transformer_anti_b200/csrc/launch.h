@@ -48,6 +48,10 @@ struct TcGemmArgs {
 };
 
 // tensor-core path: 16-bit operands (f16 or bf16, one type per launch) in TMA tensor maps
+// As make_tmap_16_3d over a [depth][rows][inner] view whose rows are row_stride elements apart
+// (row_stride >= inner, a multiple of 8; base 16-byte aligned).
+bool make_tmap_16_3d_strided(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                             uint64_t row_stride, uint32_t box_rows, bool f16);
 bool make_tmap_16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
                      uint32_t box_rows, bool f16);
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
@@ -93,6 +97,7 @@ struct AttnArgs {
   IndexMode mode;  // slice index of both buffers
   int L;
   int* err;        // device error word for bounded waits (tensor-core kernel), may be null
+  int ldo;         // row stride of out in elements (0: H * dh, rows packed)
 };
 // mma.sync (bf16) or fp32 FMA kernels, any head_dim in {32, 64, 128}
 cudaError_t launch_attention(const AttnArgs& a, ElemType t, cudaStream_t st);

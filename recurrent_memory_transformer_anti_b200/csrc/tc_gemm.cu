@@ -306,8 +306,10 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
     sm100::fence_async_smem();
     __syncwarp();
     if (lane == 0) {
-      sm100::tma_store_3d(tmX, buf_s + b * BLK, col, rowbase, dst);
-      sm100::bulk_commit();
+      if (!ep.resid_no_store) {
+        sm100::tma_store_3d(tmX, buf_s + b * BLK, col, rowbase, dst);
+        sm100::bulk_commit();
+      }
       if (cc + NBUF < c1) issue(cc + NBUF, b);
     }
   }
@@ -736,6 +738,22 @@ bool make_tmap_16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   if (!encode || !base || inner % 8 != 0 || (reinterpret_cast<uintptr_t>(base) & 15) != 0) return false;
   cuuint64_t dims[3] = {inner, rows, depth};
   cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_16_3d_strided(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t depth,
+                             uint64_t row_stride, uint32_t box_rows, bool f16) {
+  auto encode = get_encode_fn();
+  if (!encode || !base || inner % 8 != 0 || row_stride % 8 != 0 || row_stride < inner ||
+      (reinterpret_cast<uintptr_t>(base) & 15) != 0)
+    return false;
+  cuuint64_t dims[3] = {inner, rows, depth};
+  cuuint64_t strides[2] = {row_stride * 2, row_stride * rows * 2};
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
