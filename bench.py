@@ -44,7 +44,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch of the current kernel (profiles/gateup_gemm_1b.md). Traffic grows with the number of
 # cells (each cell brings its own layer's weights and activations), so a launch's traffic is
 # this figure times its cells. None when no capture of the current kernel exists.
-GATEUP_TRAFFIC_BYTES_PER_CELL = 82.70e6
+GATEUP_TRAFFIC_BYTES_PER_CELL = 82.49e6
 
 
 def parse():

@@ -721,7 +721,8 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                     return launch_attention(a, h->bf16 ? kElemF16 : kElemF32, st);
                   });
   if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * (hd + fold * dv),
+  // (the folded W_mo o is counted once, with the read-out projection, as the model defines it)
+  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd,
                   g * (m * (hd + fold * dv) * es + dd * (hd + fold * dv) * es + 2 * m * dd * 4), st,
                   [&] { return run_proj(h, kProjO, cells, G, st); });
   if (e != cudaSuccess) return e;
