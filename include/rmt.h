@@ -277,7 +277,7 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
  * streams). Same arguments and results as rmt_memory_write; the cell table and the split-K
  * partial sums live in a fixed 8 MiB array in the library's device memory, which every GPU
  * that loads the library holds until the process exits. Sizes whose partial sums need
- * more than 8 MiB - 64 KiB (G*ceil(d/128)*n*(dk+dv)*4 bytes), or G > 8192, return
+ * more than 8 MiB - 256 KiB (G*ceil(d/128)*n*(dk+dv)*4 bytes), or G > 8192, return
  * RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress); make that first call before any
  * stream capture. All calls share the array, which keeps the last call's contents (every

@@ -53,7 +53,7 @@ extern "C" rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv
   if (size_t(G) * sizeof(Cell) > kNoAllocCellBytes || part_bytes > kNoAllocScratchBytes - kNoAllocCellBytes)
     return fail(RMT_EINVAL,
                 "rmt_memory_write_noalloc: G*ceil(d/128)*n*(dk+dv)*4 bytes of partial sums exceed the fixed "
-                "8 MiB - 64 KiB scratch (or G > 8192); use rmt_memory_write");
+                "8 MiB - 256 KiB scratch (or G > 8192); use rmt_memory_write");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(RMT_ECUDA, "cudaGetDevice failed");
   if (!g_noalloc_addr[dev]) {
