@@ -187,6 +187,13 @@ rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap);
  * word of the kernel-level entry points on the current device is checked. */
 rmt_status rmt_sync(rmt_handle* h, void* stream);
 
+/* Check of the failure path: one CTA waits on an mbarrier that nothing signals, with the
+ * bounded wait every kernel of this library uses, limited here to limit_us microseconds
+ * (1 .. 10^7; the kernels use 2 s). The wait gives up, the CTA sets the device error word of
+ * the kernel-level entry points and returns normally; rmt_sync(NULL, stream) then reports
+ * RMT_ETIMEOUT (and clears the word), and the context stays usable. Asynchronous on stream. */
+rmt_status rmt_wait_selftest(uint32_t limit_us, void* stream);
+
 /* Kernel kinds of one schedule step, in launch order (see rmt_forward). */
 typedef enum {
   RMT_K_ASSEMBLE = 0,  /* layer-0 input: segment embeddings + memory tokens */

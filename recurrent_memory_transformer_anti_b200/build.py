@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "librmt.so")
-SOURCES = ["api.cu", "tc_gemm.cu", "tc_gemm_pair.cu", "simt_gemm.cu", "attention.cu", "attention_tc.cu", "memory.cu", "rowops.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "tc_gemm.cu", "tc_gemm_pair.cu", "simt_gemm.cu", "attention.cu", "attention_tc.cu", "memory.cu", "rowops.cu", "noalloc.cu",
+           "selftest.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -1352,6 +1352,15 @@ rmt_status rmt_destroy(rmt_handle* h) {
 
 // ----------------------------------------------------------------- kernel-level entry points
 
+rmt_status rmt_wait_selftest(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 10000000) return fail(RMT_EINVAL, "limit_us must be in 1 .. 10^7");
+  int* err = nullptr;
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(1, &cells, &err));
+  RMT_CUDA(launch_wait_selftest(err, 1000ull * limit_us, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+}
+
 rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t G, int32_t M, int32_t N, int32_t K,
                                  rmt_dtype out_dtype, void* stream) {
   if (!A || !B || !C) return fail(RMT_EINVAL, "null pointer");

@@ -14,6 +14,7 @@ enum : int {
   kErrTimeoutMma = 2,
   kErrTimeoutEpilogue = 4,
   kErrBadArgs = 8,
+  kErrTimeoutSelftest = 16,  // the bounded-wait check (rmt_wait_selftest) gave up, as it should
 };
 
 // Programmatic dependent launch. The forward launches its kernels with programmatic stream

@@ -185,6 +185,9 @@ cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const voi
                             int n_mem, int d, bool bf16, cudaStream_t st);
 // RMSNorm statistics of rows 0..M-1 of an fp32 [M, d] block: ss[row * parts + b] = sum of
 // squares of columns b*w .. b*w+w-1, w = d / parts (a multiple of 4; at most 32 parts).
+// One CTA waits on an mbarrier nothing signals, with the kernels' bounded wait limited to
+// limit_ns, and ORs kErrTimeoutSelftest into *err when the wait gives up (see selftest.cu).
+cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st);
 cudaError_t launch_row_ssq(const float* x, float* ss, int M, int d, int parts, cudaStream_t st);
 // Segment outputs of the G cells: rows 0..m-n_mem-1 of slot c.xout, cast to T, to out rows c.t0...
 cudaError_t launch_emit(const Cell* cells, int G, const float* x, void* out, int M, int n_mem, int d, bool bf16,

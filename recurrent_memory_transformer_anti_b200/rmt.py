@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4
 
 EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "rmt_forward_batch",
             "rmt_full_attention_forward", "rmt_schedule_table",
-            "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync",
+            "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync", "rmt_wait_selftest",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
             "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
             "rmt_probe_read")
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "rmt_get_schedule": [vp, i32, ctypes.c_int, p32, sz],
         "rmt_get_trace": [vp, p32, sz],
         "rmt_sync": [vp, vp],
+        "rmt_wait_selftest": [ctypes.c_uint32, vp],
         "rmt_destroy": [vp],
         "rmt_grouped_gemm_bf16": [vp, vp, vp, i32, i32, i32, i32, ctypes.c_int, vp],
         "rmt_attention": [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp],
@@ -240,6 +241,10 @@ def rmt_get_trace(h: Handle, n_cells: int) -> np.ndarray:
 
 def rmt_sync(h: Handle | None, stream=None) -> None:
     _check(_lib.rmt_sync(h.ptr if h is not None else None, _stream(stream)), "rmt_sync")
+
+
+def rmt_wait_selftest(limit_us: int, stream=None) -> None:
+    _check(_lib.rmt_wait_selftest(int(limit_us), _stream(stream)), "rmt_wait_selftest")
 
 
 def rmt_destroy(h: Handle) -> None:

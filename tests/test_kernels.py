@@ -188,3 +188,30 @@ def test_memory_write_matches_oracle(dtype, G, n, d, dk, dv):
                                     z[g].astype(np.float64), 1e-6)
         assert normwise(to_np(tA[g]), rA) < 2e-5
         assert normwise(to_np(tz[g]), rz) < 2e-6
+
+
+def test_bounded_wait_gives_up_and_reports_without_a_fault(cuda_ok):
+    """The failure path of every kernel: a wait on a barrier that nothing signals gives up after
+    its limit, the error word reaches the host as RMT_ETIMEOUT, and the context stays usable."""
+    import time
+
+    rmt.rmt_sync(None)  # clean error word
+    t0 = time.perf_counter()
+    rmt.rmt_wait_selftest(20000)  # 20 ms
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_sync(None)
+    assert ex.value.status == rmt.RMT_ETIMEOUT
+    assert time.perf_counter() - t0 >= 0.015
+    rmt.rmt_sync(None)  # the word was cleared
+    # the device still runs kernels: a small grouped GEMM after the timeout is correct
+    G, M, N, K = 2, 130, 256, 128
+    a = torch.randn(G, M, K, device="cuda").to(torch.bfloat16)
+    b = (torch.randn(G, N, K, device="cuda") * 0.05).to(torch.bfloat16)
+    c = torch.empty(G, M, N, device="cuda")
+    rmt.rmt_grouped_gemm_bf16(a, b, c, G, M, N, K, "f32")
+    rmt.rmt_sync(None)
+    ref = torch.einsum("gmk,gnk->gmn", a.float(), b.float())
+    assert (c - ref).abs().max().item() / ref.abs().max().item() < 1e-2
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_wait_selftest(0)
+    assert ex.value.status == rmt.RMT_EINVAL
