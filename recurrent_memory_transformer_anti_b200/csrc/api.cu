@@ -14,12 +14,15 @@
 // two schedules give identical bits ("Dependency Preservation" in "Architecture
 // Overview"; arXiv 2506.05229 abstract: a pure run-time reordering with exact recurrence).
 #include <climits>
+#include <cstdio>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <map>
 #include <string>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "launch.h"
 #include "rmt.h"
@@ -646,9 +649,21 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   return launch_simt_gemm(a, st);
 }
 
+// NVTX range names of the kernel kinds (rmt_kernel order). The ranges cost nothing
+// measurable without a tool attached and give a profiler's timeline the step structure.
+const char* const kKindNames[RMT_K_COUNT] = {"assemble", "memq",      "memread",   "memo", "rmsnorm1",
+                                             "qkv",      "attention", "o",         "rmsnorm2", "gateup",
+                                             "down",     "memkv",     "memupdate", "emit"};
+
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 // Launch one kernel of a step: count it and, if its kind is probed, bracket it with events.
 template <typename F>
 cudaError_t launch_kind(rmt_handle* h, int kind, double flops, double bytes, cudaStream_t st, F&& fn) {
+  NvtxRange range(kKindNames[kind]);
   const bool on = (h->probe_mask >> kind) & 1u;
   cudaEvent_t a = nullptr, b = nullptr;
   if (on && (a = h->probe_event()) != nullptr) cudaEventRecord(a, st);
@@ -1144,8 +1159,12 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, const std::vector<int>& 
     RMT_CUDA(cudaMemsetAsync(h->z, 0, BL * c.d_k * sizeof(float), st));
   }
   const bool split_in = in_pinned && emb_dev != emb, split_out = out_host && out_pinned;
+  NvtxRange fwd_range(schedule == RMT_DIAGONAL ? "rmt_forward diagonal" : "rmt_forward sequential");
+  char step_name[48];
   for (int step = 0; step < int(t.off.size()); ++step) {
     const int off = t.off[step], G = t.cnt[step];
+    snprintf(step_name, sizeof(step_name), "step %d (%d cells)", step, G);
+    NvtxRange step_range(step_name);
     if (split_in)
       for (int i = 0; i < t.n_first[step]; ++i)
         RMT_CUDA(cudaStreamWaitEvent(st, h->copy_events[2 + 2 * seg_ord(t.cells[off + i])], 0));

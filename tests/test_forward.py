@@ -458,3 +458,19 @@ def test_full_attention_1b_at_131k(cuda_ok):
     rmt.rmt_destroy(h)
     ref = armt.full_attention_forward(cfg, w, emb[:P], dtype=np.float32)
     assert normwise(part, ref) < BF16_TOL
+
+
+def test_failed_reservation_leaves_the_handle_usable(cuda_ok):
+    """A reservation that cannot fit on the device fails with RMT_ENOMEM (a real cudaMalloc
+    failure, no fault), and the next forward reserves again and gives the same bits."""
+    cfg = CONFIGS["small-bf16"]
+    w, h = build(cfg)
+    emb = embeddings(cfg, 2, seed=50)
+    before = forward(h, cfg, emb, 2, "diagonal")
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_reserve(h, 10_000_000)  # several TB of activations
+    assert ex.value.status == rmt.RMT_ENOMEM
+    after = forward(h, cfg, emb, 2, "diagonal")
+    for a, b in zip(before, after):
+        np.testing.assert_array_equal(a, b)
+    rmt.rmt_destroy(h)
