@@ -429,6 +429,33 @@ def main() -> int:
                             if GATEUP_TRAFFIC_BYTES_PER_CELL and probe["launches"] else None),
                 "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 2-cell launch)"}
 
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    e_host = e.cpu().pin_memory()
+    o_host = torch.empty_like(e_host).pin_memory()
+    A_host = torch.empty(A.shape, dtype=A.dtype).pin_memory()
+    z_host = torch.empty(z.shape, dtype=z.dtype).pin_memory()
+    rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
+    torch.cuda.synchronize()
+    n_e2e = K  # as many steps as the device-resident region, right after it (same clock regime)
+    barrier()
+    torch.cuda.synchronize()
+    sampler_e2e = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    sampler_e2e.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks_e2e = sampler_e2e.stop()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
+    rmt.rmt_sync(h, stream)
+    e2e = {"value": job_throughput(tokens, e2e_ms, world), "unit": UNIT,
+           "h2d_bytes_per_step": e_host.numel() * e_host.element_size(),
+           "d2h_bytes_per_step": o_host.numel() * o_host.element_size() + A_host.numel() * 4 + z_host.numel() * 4,
+           "steps": n_e2e, "sm_mhz": clocks_e2e.get("sm_mhz") if clocks_e2e else None}
+
     # ---- per-kernel breakdown of one forward (outside the timed region)
     rmt.rmt_probe(h, list(rmt.KERNELS))
     run("diagonal", 1)
@@ -472,29 +499,6 @@ def main() -> int:
         full = {"model": "the same 16-layer decoder without the associative memory, causal over all tokens",
                 "ms_per_step": full_ms, "tokens_per_s": job_throughput(tokens, full_ms, world),
                 "armt_diagonal_speedup": full_ms / ms, "pages_speedup": 3.3}
-
-    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
-    e_host = e.cpu().pin_memory()
-    o_host = torch.empty_like(e_host).pin_memory()
-    A_host = torch.empty(A.shape, dtype=A.dtype).pin_memory()
-    z_host = torch.empty(z.shape, dtype=z.dtype).pin_memory()
-    rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
-    torch.cuda.synchronize()
-    n_e2e = max(1, min(K, 3))
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n_e2e):
-        rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
-    rmt.rmt_sync(h, stream)
-    e2e = {"value": job_throughput(tokens, e2e_ms, world), "unit": UNIT,
-           "h2d_bytes_per_step": e_host.numel() * e_host.element_size(),
-           "d2h_bytes_per_step": o_host.numel() * o_host.element_size() + A_host.numel() * 4 + z_host.numel() * 4}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
