@@ -437,6 +437,9 @@ def main() -> int:
     rmt.rmt_forward(h, e_host, S, "diagonal", o_host, A_host, z_host, stream)
     torch.cuda.synchronize()
     n_e2e = K  # as many steps as the device-resident region, right after it (same clock regime)
+    # the same instrumentation as the device-resident region: its gate/up launches are bracketed
+    # by events, which hold back the programmatic overlap around them by about 1-2% of the step
+    rmt.rmt_probe(h, ["gateup"])
     barrier()
     torch.cuda.synchronize()
     sampler_e2e = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
@@ -451,6 +454,7 @@ def main() -> int:
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, dev)
     rmt.rmt_sync(h, stream)
+    rmt.rmt_probe(h, [])
     e2e = {"value": job_throughput(tokens, e2e_ms, world), "unit": UNIT,
            "h2d_bytes_per_step": e_host.numel() * e_host.element_size(),
            "d2h_bytes_per_step": o_host.numel() * o_host.element_size() + A_host.numel() * 4 + z_host.numel() * 4,
