@@ -153,17 +153,19 @@ def test_small_bf16_diagonal_equals_sequential_bitwise(small_bf16):
         np.testing.assert_array_equal(a, b)
 
 
-def test_1b_shape_bench_configuration(cuda_ok):
-    """The 131,072-token LLaMA-1B-shaped workload the bench times (16 layers x 128 segments
-    of 1024 + 16 tokens, bf16). The oracle cannot run 128 segments in seconds, so:
-      - the first four segments of the 128-segment run equal a 4-segment run bit for bit
-        (a segment's output never depends on later segments), and the 4-segment run --
-        hidden states and the memory state after 4 segments -- matches the oracle within
-        the bf16 tolerance;
+@pytest.mark.parametrize("S", [32, 128])
+def test_1b_shape_bench_configuration(cuda_ok, S):
+    """The LLaMA-1B-shaped workloads: 32 segments (32,768 tokens) and the 131,072 tokens the
+    bench times (16 layers x 128 segments of 1024 + 16 tokens, bf16). The oracle cannot run
+    them in seconds, so:
+      - the first four segments of the full run equal a 4-segment run bit for bit (a
+        segment's output never depends on later segments), and the 4-segment run -- hidden
+        states and the memory state after 4 segments -- matches the oracle within the bf16
+        tolerance;
       - DIAGONAL equals SEQUENTIAL bit for bit at the full size."""
     cfg = CONFIGS["1b"]
     w, h = build(cfg)
-    S, P = 128, 4
+    P = 4
     emb = embeddings(cfg, S)
     full_d = forward(h, cfg, emb, S, "diagonal")
     full_s = forward(h, cfg, emb, S, "sequential")
