@@ -194,10 +194,15 @@ rmt_status rmt_sync(rmt_handle* h, void* stream);
  * RMT_ETIMEOUT (and clears the word), and the context stays usable. Asynchronous on stream. */
 rmt_status rmt_wait_selftest(uint32_t limit_us, void* stream);
 
-/* Kernel kinds of one schedule step, in launch order (see rmt_forward). */
+/* Kernel kinds of one schedule step, in launch order (see rmt_forward). Kinds that are fused
+ * into another kind's kernel launch nothing of their own and read zero in rmt_probe_read:
+ * RMSNORM1 and RMSNORM2 always (their statistics come from the residual epilogues and their
+ * gains are folded into the next projection's weights); MEMREAD in bf16 mode with
+ * d_k = d_v = 64, where the read runs in the MEMQ kernel's epilogue (and then MEMO forms only
+ * the operand copy and statistics, the O projection adding the read-out to the residual). */
 typedef enum {
   RMT_K_ASSEMBLE = 0,  /* layer-0 input: segment embeddings + memory tokens */
-  RMT_K_MEMQ = 1,      /* memory-query projection (grouped GEMM) */
+  RMT_K_MEMQ = 1,      /* memory-query projection (grouped GEMM), with the read when fused */
   RMT_K_MEMREAD = 2,   /* associative read */
   RMT_K_MEMO = 3,      /* read-out projection + residual (grouped GEMM) */
   RMT_K_RMSNORM1 = 4,

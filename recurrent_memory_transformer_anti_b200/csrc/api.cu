@@ -10,6 +10,10 @@
 //   -> QKV GEMM (+RoPE) -> attention -> O GEMM (+residual) -> RMSNorm
 //   -> gate/up GEMM (+SwiGLU) -> down GEMM (+residual) -> memory k/v -> memory update
 //   -> [segment output]
+// The RMSNorms launch nothing (statistics from the residual epilogues, gains folded into the
+// next weights). In bf16 mode with d_k = d_v = 64 the read runs in the mem-q GEMM's
+// epilogue, and with the O GEMM on CTA pairs the mem-o residual add moves into the O GEMM
+// (fold_mo), so a step is nine launches.
 // Each kernel does the same arithmetic for a cell whatever else shares its launch, so the
 // two schedules give identical bits ("Dependency Preservation" in "Architecture
 // Overview"; arXiv 2506.05229 abstract: a pure run-time reordering with exact recurrence).
