@@ -53,7 +53,10 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--segments", type=int, default=N_SEGMENTS)
+    p.add_argument("--segments", type=int, default=None,
+                   help="segments of the timed sequence (default: 131,072 tokens' worth of the config)")
+    p.add_argument("--config", choices=["1b", "3b-512", "3b-2048"], default="1b",
+                   help="model shape of the forward (the bench line of record is the 1B-shaped workload)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-sequential", action="store_true")
     p.add_argument("--no-full-attention", action="store_true",
@@ -233,16 +236,16 @@ def run_reference(args, world: int, rank: int) -> int:
 
 # ----------------------------------------------------------------------------- our arm
 
-def cpu_baseline(cfg, w, emb) -> dict:
-    """The oracle as it stands, on one segment (1024 tokens through all 16 layers)."""
+def cpu_baseline(cfg, w, emb, n_segments: int) -> dict:
+    """The oracle as it stands, on one segment of the workload (seg_len tokens through every layer)."""
     from oracle import armt
     seg = cfg.seg_len
     t0 = time.perf_counter()
     armt.forward(cfg, w, emb[:seg], 1, dtype=np.float32)
     dt = time.perf_counter() - t0
     return {"value": seg / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"1 of {N_SEGMENTS} segments (1024 tokens through 16 layers, {dt:.1f} s); per-segment cost "
-                      "is the same for every segment"}
+            "sample": f"1 of {n_segments} segments ({seg} tokens through {cfg.n_layers} layers, {dt:.1f} s); "
+                      "per-segment cost is the same for every segment"}
 
 
 def run_microbench(args, local: int) -> int:
@@ -375,8 +378,8 @@ def main() -> int:
             dist.barrier()
 
     K, W = max(1, args.steps), max(3, args.warmup)
-    S = args.segments
-    cfg = CONFIGS["1b"]
+    cfg = CONFIGS[args.config]
+    S = args.segments if args.segments else 131072 // cfg.seg_len
     w = make_weights(cfg)
     emb = make_embeddings(cfg, S)
     h = rmt.rmt_create(rmt.weights_storage(w, "bf16", dev), cfg)
@@ -426,7 +429,7 @@ def main() -> int:
                 "peak_source": f"bf16_tflops_sustained ({peak_src})",
                 "launches": probe["launches"], "kernel_ms_per_step": probe["ms"] / K,
                 "traffic": (GATEUP_TRAFFIC_BYTES_PER_CELL * cfg.n_layers * S / probe["launches"] * K
-                            if GATEUP_TRAFFIC_BYTES_PER_CELL and probe["launches"] else None),
+                            if GATEUP_TRAFFIC_BYTES_PER_CELL and probe["launches"] and args.config == "1b" else None),
                 "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 2-cell launch)"}
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
@@ -506,17 +509,20 @@ def main() -> int:
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(cfg, w, emb)
+        cpu = cpu_baseline(cfg, w, emb, S)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": DATA,
-            "config": {"workload": WORKLOAD, "layers": cfg.n_layers, "d_model": cfg.d_model, "segments": S,
+            "config": {"workload": WORKLOAD if args.config == "1b" and S == N_SEGMENTS else
+                       f"{args.config}-shaped ARMT prefill of one {tokens:,}-token sequence "
+                       f"({S} x ({cfg.seg_len} + {cfg.n_mem} memory) tokens)",
+                       "layers": cfg.n_layers, "d_model": cfg.d_model, "segments": S,
                        "seg_len": cfg.seg_len, "n_mem": cfg.n_mem, "tokens": tokens, "schedule": "diagonal",
                        "batch": 1, "parallelism": "replicas" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (weights 1.96 GB, embeddings 0.54 GB): no flush"},
+                       "l2": "inputs larger than L2 (weights of 1.96 GB or more, embeddings 0.54 GB or more): no flush"},
             "roofline": roofline,
             "path": {"algorithmic_tflop_per_step": step_flops / 1e12,
                      "achieved_tflops": step_flops / (ms / 1e3) / 1e12,
