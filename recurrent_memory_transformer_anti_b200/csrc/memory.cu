@@ -95,13 +95,15 @@ __global__ void __launch_bounds__(kReadWarps * 32) mem_read_kernel(const MemRead
 }
 
 // ------------------------------------------------------------------ key/value projection
-// CTA = one split of kMemKvSplit columns of d_model for one cell: the n memory rows and the
-// dkv weight rows of that split are staged in shared memory, k-major; each thread then forms
-// a 4-row x 2-column block of the n x dkv partial dot products over the split, k ascending.
+// CTA = one split of kMemKvSplit columns of d_model for one cell and one block of up to
+// kKvCols output columns: the n memory rows and those weight rows of the split are staged in
+// shared memory, k-major; each thread then forms a 4-row x 2-column block of the partial dot
+// products over the split, k ascending.
 // Staging reads 16-byte vectors: one lane takes 8 consecutive columns of one weight row (4 of
 // one memory row) and writes them down a column of the k-major block, so the lanes of a warp
 // write consecutive words.
 constexpr int kKvThreads = 256;
+constexpr int kKvCols = 128;  // output columns per CTA (blockIdx.z selects the block of dkv)
 
 template <typename T>
 __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
@@ -110,15 +112,16 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
   extern __shared__ float sm[];
   constexpr int KS = kMemKvSplit;
   const int n4 = (a.n + 3) & ~3;  // rows padded to a multiple of 4 (padding rows are zero)
+  const int j_base = blockIdx.z * kKvCols, cols = min(kKvCols, a.dkv - j_base);
   float* Ys = sm;                 // [KS][n4]
-  float* Ws = sm + KS * n4;       // [KS][dkv]
+  float* Ws = sm + KS * n4;       // [KS][cols]: weight rows j_base .. j_base + cols - 1
   const Cell c = a.cells[blockIdx.y];
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
   // the cell's memory rows are its last n valid rows
   const int row0 = cell_rows(c, a.M) - a.n;
   const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row0) * a.d + k0;
-  const T* W = static_cast<const T*>(a.w) + static_cast<size_t>(c.l) * a.dkv * a.d + k0;
+  const T* W = static_cast<const T*>(a.w) + (static_cast<size_t>(c.l) * a.dkv + j_base) * a.d + k0;
   // 16-byte vectors only where every row start is 16-byte aligned
   const bool y_vec = (a.d % 4 == 0) && (reinterpret_cast<uintptr_t>(a.x) % 16 == 0);
   const bool w_vec = sizeof(T) == 2 && (a.d % 8 == 0) && (reinterpret_cast<uintptr_t>(a.w) % 16 == 0);
@@ -143,8 +146,8 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
     Ys[(k + 3) * n4 + r] = v.w;
   }
   // weight rows: one lane per (row, 8 columns), rows fastest
-  for (int e = threadIdx.x; e < a.dkv * (KS / 8); e += kKvThreads) {
-    const int j = e % a.dkv, k = 8 * (e / a.dkv);
+  for (int e = threadIdx.x; e < cols * (KS / 8); e += kKvThreads) {
+    const int j = e % cols, k = 8 * (e / cols);
     float w8[8];
     if (w_vec && k + 7 < kw) {
       const uint4 u = *reinterpret_cast<const uint4*>(W + static_cast<size_t>(j) * a.d + k);
@@ -156,20 +159,20 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
       for (int t = 0; t < 8; ++t) w8[t] = k + t < kw ? to_f32<T>(W[static_cast<size_t>(j) * a.d + k + t]) : 0.f;
     }
 #pragma unroll
-    for (int t = 0; t < 8; ++t) Ws[(k + t) * a.dkv + j] = w8[t];
+    for (int t = 0; t < 8; ++t) Ws[(k + t) * cols + j] = w8[t];
   }
   __syncthreads();
   const int nsplit = (a.d + KS - 1) / KS;
   const int nout = a.n * a.dkv;
   float* part = a.part + (static_cast<size_t>(c.k) * nsplit + split) * nout;
-  const int jt = a.dkv / 2, tiles = (n4 / 4) * jt;
+  const int jt = cols / 2, tiles = (n4 / 4) * jt;
   for (int t = threadIdx.x; t < tiles; t += kKvThreads) {
     const int r0 = (t / jt) * 4, j0 = (t % jt) * 2;
     float acc[4][2] = {};
 #pragma unroll 8
     for (int k = 0; k < KS; ++k) {
       const float4 y = *reinterpret_cast<const float4*>(Ys + k * n4 + r0);
-      const float2 w = *reinterpret_cast<const float2*>(Ws + k * a.dkv + j0);
+      const float2 w = *reinterpret_cast<const float2*>(Ws + k * cols + j0);
       const float yv[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -179,7 +182,8 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (r0 + i < a.n) *reinterpret_cast<float2*>(part + (r0 + i) * a.dkv + j0) = make_float2(acc[i][0], acc[i][1]);
+      if (r0 + i < a.n)
+        *reinterpret_cast<float2*>(part + (r0 + i) * a.dkv + j_base + j0) = make_float2(acc[i][0], acc[i][1]);
   }
 }
 
@@ -295,8 +299,9 @@ cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (a.G <= 0) return cudaSuccess;
   if (a.n > 64 || a.dkv % 4) return cudaErrorInvalidValue;
   const size_t n4 = (a.n + 3) & ~3;
-  const size_t smem = (n4 * kMemKvSplit + static_cast<size_t>(kMemKvSplit) * a.dkv) * sizeof(float);
-  dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G);
+  const size_t cols = a.dkv < kKvCols ? a.dkv : kKvCols;
+  const size_t smem = (n4 * kMemKvSplit + static_cast<size_t>(kMemKvSplit) * cols) * sizeof(float);
+  dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G, (a.dkv + kKvCols - 1) / kKvCols);
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(mem_kv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
