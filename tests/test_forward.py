@@ -426,6 +426,12 @@ def test_full_attention_matches_oracle(cuda_ok, T):
     if T > 1:
         _full(h, cfg, embeddings(cfg, 3, seed=41))
         np.testing.assert_array_equal(_full(h, cfg, emb), got)
+    # host buffers (staged through device copies) give the same bits
+    e_host = rmt.storage(emb, cfg.dtype, device="cuda").cpu()
+    o_host = torch.empty_like(e_host)
+    rmt.rmt_full_attention_forward(h, e_host, T, o_host)
+    rmt.rmt_sync(h)
+    np.testing.assert_array_equal(o_host.float().numpy(), got)
     rmt.rmt_destroy(h)
 
 
