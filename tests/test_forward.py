@@ -482,3 +482,46 @@ def test_failed_reservation_leaves_the_handle_usable(cuda_ok):
     for a, b in zip(before, after):
         np.testing.assert_array_equal(a, b)
     rmt.rmt_destroy(h)
+
+
+def _random_bf16_config(seed):
+    """A small valid bf16 shape drawn from a seeded generator: d_model, heads x head_dim, d_v
+    multiples of 64; d_ff a multiple of 64; any segment length; n_mem * (d_k + d_v) <= 4096."""
+    import dataclasses
+    r = np.random.default_rng(seed)
+    dh = int(r.choice([64, 128]))
+    hkv = int(r.integers(1, 3))
+    hq = hkv * int(r.integers(1, 4))
+    d = int(r.choice([128, 192, 256, 320, 512]))  # multiples of 256 put O and down on CTA pairs
+    # d_k = d_v = 64 takes the fused read (and, with O on CTA pairs, the read-out fold)
+    dk, dv = [(32, 64), (64, 64), (64, 64), (64, 128), (128, 128)][int(r.integers(0, 5))]
+    n_mem = int(r.integers(1, 4096 // (dk + dv) + 1)) if r.random() < 0.3 else int(r.integers(1, 17))
+    return dataclasses.replace(CONFIGS["small-bf16"], n_layers=int(r.integers(1, 4)), d_model=d, n_heads=hq,
+                               n_kv_heads=hkv, head_dim=dh, d_ff=64 * int(r.integers(2, 9)),
+                               seg_len=int(r.integers(1, 300)), n_mem=min(n_mem, 64), d_k=dk, d_v=dv)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_random_bf16_shapes_match_oracle(cuda_ok, seed):
+    """Seeded random shapes (head_dim 64 or 128, GQA ratios, widths that put the projections
+    on CTA pairs or single CTAs, d_k / d_v that do or do not take the fused read, ragged
+    token tiles): every one matches the oracle, DIAGONAL equals SEQUENTIAL bit for bit, and a
+    two-sequence batch with a short last segment equals its sequences run alone."""
+    cfg = _random_bf16_config(seed)
+    w, h = build(cfg)
+    S = 3
+    emb = embeddings(cfg, S, seed=60 + seed)
+    got = forward(h, cfg, emb, S, "diagonal")
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32)
+    for g_, r_, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g_, r_) < BF16_TOL, (what, cfg)
+    seq = forward(h, cfg, emb, S, "sequential")
+    for a, b in zip(got, seq):
+        np.testing.assert_array_equal(a, b)
+    lens = [2 * cfg.seg_len + max(1, cfg.seg_len // 3), cfg.seg_len]
+    embs = [emb[:lens[0]], embeddings(cfg, 1, seed=70 + seed)]
+    batch = forward_batch(h, cfg, embs, "diagonal")
+    for b_ in range(2):
+        alone = forward_batch(h, cfg, [embs[b_]], "diagonal")
+        np.testing.assert_array_equal(batch[0][b_], alone[0][0])
+    rmt.rmt_destroy(h)
