@@ -142,7 +142,9 @@ rmt_status rmt_forward_resume(rmt_handle* h, const void* emb, int32_t n_segments
  * puts every cell (b, l, s) with l + s = d of all sequences into step d (layers ascending,
  * then sequences); RMT_SEQUENTIAL runs one cell per step, sequences outermost, then segments,
  * then layers. Both give the same bits. Grows the activations (rmt_reserve) when batch is
- * above the reserved size. RMT_EINVAL on a non-positive batch or length, or more than 2^30
+ * above the reserved size. The handle keeps the cell table of each (n_tokens, schedule) on
+ * the device, at most 64 of them; a new one beyond that frees the oldest (which waits for
+ * the device). RMT_EINVAL on a non-positive batch or length, or more than 2^30
  * tokens. Other behaviour as rmt_forward. */
 rmt_status rmt_forward_batch(rmt_handle* h, const void* emb, int32_t batch, const int32_t* n_tokens,
                              rmt_schedule schedule, const float* in_A, const float* in_z, void* out_hidden,

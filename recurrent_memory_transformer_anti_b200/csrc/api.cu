@@ -22,6 +22,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <deque>
 #include <map>
 #include <string>
 #include <vector>
@@ -245,6 +246,8 @@ struct rmt_handle {
     return true;
   }
   std::map<std::pair<std::vector<int>, int>, Table> tables;  // keyed by (token counts, schedule)
+  std::deque<std::pair<std::vector<int>, int>> table_order;  // insertion order, for eviction
+  static constexpr size_t kMaxTables = 64;
   CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
   // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
   CUtensorMap tp_xb, tp_om, tp_att, tp_u;
@@ -345,6 +348,7 @@ struct rmt_handle {
     for (auto& kv : tables)
       if (kv.second.dev) cudaFree(kv.second.dev);
     tables.clear();
+    table_order.clear();
     if (trace) cudaFree(trace);
     if (emb_stage) cudaFree(emb_stage);
     if (out_stage) cudaFree(out_stage);
@@ -1087,6 +1091,16 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, const std::vector<int>& 
   const auto key = std::make_pair(T, int(schedule));
   auto it = h->tables.find(key);
   if (it == h->tables.end()) {
+    // keep at most kMaxTables cell tables on the device: drop the oldest (cudaFree waits for
+    // the device, so no forward still reads it)
+    while (h->tables.size() >= rmt_handle::kMaxTables && !h->table_order.empty()) {
+      auto old = h->tables.find(h->table_order.front());
+      if (old != h->tables.end()) {
+        if (old->second.dev) cudaFree(old->second.dev);
+        h->tables.erase(old);
+      }
+      h->table_order.pop_front();
+    }
     Table t;
     build_table(c.n_layers, c.seg_len, c.n_mem, T, schedule, t);
     if (cudaMalloc(&t.dev, sizeof(Cell) * t.cells.size()) != cudaSuccess)
@@ -1096,6 +1110,7 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, const std::vector<int>& 
       return fail(RMT_ECUDA, "cell table upload failed");
     }
     it = h->tables.emplace(key, std::move(t)).first;
+    h->table_order.push_back(key);
   }
   const Table& t = it->second;
   const size_t ncell = t.cells.size();

@@ -525,3 +525,20 @@ def test_random_bf16_shapes_match_oracle(cuda_ok, seed):
         alone = forward_batch(h, cfg, [embs[b_]], "diagonal")
         np.testing.assert_array_equal(batch[0][b_], alone[0][0])
     rmt.rmt_destroy(h)
+
+
+def test_many_distinct_lengths_evict_old_tables(tiny):
+    """Each distinct (token counts, schedule) keeps a cell table on the device, at most 64 of
+    them: 70 different lengths evict the oldest, and a length whose table was evicted runs
+    again with the same bits."""
+    cfg, w, h = tiny
+    emb = embeddings(cfg, 2)
+    first = forward_batch(h, cfg, [emb[:1]], "diagonal")
+    for n in range(2, 72):
+        forward_batch(h, cfg, [emb[:n]], "diagonal")
+    again = forward_batch(h, cfg, [emb[:1]], "diagonal")  # its table was evicted and is rebuilt
+    np.testing.assert_array_equal(first[0][0], again[0][0])
+    np.testing.assert_array_equal(first[1], again[1])
+    last = forward_batch(h, cfg, [emb[:71]], "diagonal")
+    ref = armt.forward_tokens(cfg, w, emb[:71], dtype=np.float32)
+    assert normwise(last[0][0], ref[0]) < F32_TOL
