@@ -248,7 +248,8 @@ struct rmt_handle {
   std::map<std::pair<std::vector<int>, int>, Table> tables;  // keyed by (token counts, schedule)
   std::deque<std::pair<std::vector<int>, int>> table_order;  // insertion order, for eviction
   static constexpr size_t kMaxTables = 64;
-  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_x, tm_rope;
+  CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_qkv_tail, tm_x,
+      tm_rope;
   // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
   CUtensorMap tp_xb, tp_om, tp_att, tp_u;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
@@ -279,7 +280,7 @@ struct rmt_handle {
   float2* frope = nullptr;
   __half2* frope_h = nullptr;
   Cell* fcells = nullptr;  // [L]: cell l = layer l of the one segment
-  CUtensorMap fm_xb, fm_att, fm_u, fm_qkv, fm_x, fm_rope, fp_xb, fp_att, fp_u;
+  CUtensorMap fm_xb, fm_att, fm_u, fm_qkv, fm_qkv_tail, fm_x, fm_rope, fp_xb, fp_att, fp_u;
   // launch probe (rmt_probe): CUDA event pairs around the launches of the kinds in mask
   struct ProbeRec {
     int kind;
@@ -503,6 +504,7 @@ rmt_status build_maps(rmt_handle* h) {
             (!any_pair || (map(&h->tp_xb, h->xb, d, M, NS, pb) && map_om(&h->tp_om, pb) &&
                            map(&h->tp_att, h->att, lda, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
+            map(&h->tm_qkv_tail, h->qkv, h->Nqkv, M, L, attn_tail_box(int(M), c.n_heads, c.n_kv_heads)) &&
             make_tmap_f32_resid(&h->tm_x, h->x, d, M, NS) &&
             (c.head_dim < 64 || map(&h->tm_rope, h->rope_h, c.head_dim, M, 1, 32));
   return ok ? RMT_OK : fail(RMT_ECUDA, "cuTensorMapEncodeTiled failed");
@@ -740,7 +742,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                     AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err,
                                h->ld_att};
                     if (h->bf16 && attention_tc_supported(c.head_dim))
-                      return launch_attention_tc(h->tm_qkv, a, /*f16=*/true, st);
+                      return launch_attention_tc(h->tm_qkv, h->tm_qkv_tail, a, /*f16=*/true, st);
                     return launch_attention(a, h->bf16 ? kElemF16 : kElemF32, st);
                   });
   if (e != cudaSuccess) return e;
@@ -834,6 +836,7 @@ rmt_status full_buffers(rmt_handle* h, int T) {
     const uint64_t Tu = uint64_t(T), pb = uint64_t(pair_token_tile(T) / 2);
     const bool ok = map(&h->fm_xb, h->fxb, d, Tu, 2, 128) && map(&h->fm_att, h->fatt, hd, Tu, 1, 128) &&
                     map(&h->fm_u, h->fu, F, Tu, 1, 128) && map(&h->fm_qkv, h->fqkv, h->Nqkv, Tu, 1, 128) &&
+                    map(&h->fm_qkv_tail, h->fqkv, h->Nqkv, Tu, 1, attn_tail_box(T, c.n_heads, c.n_kv_heads)) &&
                     map(&h->fp_xb, h->fxb, d, Tu, 2, uint32_t(pb)) && map(&h->fp_att, h->fatt, hd, Tu, 1, uint32_t(pb)) &&
                     map(&h->fp_u, h->fu, F, Tu, 1, uint32_t(pb)) && make_tmap_f32_resid(&h->fm_x, h->fx, d, Tu, 2) &&
                     (c.head_dim < 64 || map(&h->fm_rope, h->frope_h, c.head_dim, Tu, 1, 32));
@@ -1290,7 +1293,7 @@ rmt_status rmt_full_attention_forward(rmt_handle* h, const void* emb, int32_t n_
     const Cell* cell = h->fcells + l;
     if ((e = run_proj_full(h, kProjQkv, cell, st)) != cudaSuccess) return launch_fail(e);
     AttnArgs a{h->fqkv, h->fatt, T, c.n_heads, c.n_kv_heads, c.head_dim, 1, cell, kByLayer, L, h->err};
-    e = attention_tc_supported(c.head_dim) ? launch_attention_tc(h->fm_qkv, a, /*f16=*/true, st)
+    e = attention_tc_supported(c.head_dim) ? launch_attention_tc(h->fm_qkv, h->fm_qkv_tail, a, /*f16=*/true, st)
                                            : launch_attention(a, kElemF16, st);
     if (e != cudaSuccess) return launch_fail(e);
     if ((e = run_proj_full(h, kProjO, cell, st)) != cudaSuccess) return launch_fail(e);
@@ -1440,10 +1443,12 @@ rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32
   RMT_TRY(device_scratch(G, &cells, &err));
   AttnArgs a{qkv, out, M, H, Hkv, dh, G, cells, kByLayer, G, err};
   if (dtype == RMT_BF16 && attention_tc_supported(dh)) {
-    CUtensorMap tm;
-    if (!make_tmap_bf16_3d(&tm, qkv, uint64_t(H + 2 * Hkv) * dh, M, G, 128))
+    CUtensorMap tm, tt;
+    const uint64_t inner = uint64_t(H + 2 * Hkv) * dh;
+    if (!make_tmap_bf16_3d(&tm, qkv, inner, M, G, 128) ||
+        !make_tmap_bf16_3d(&tt, qkv, inner, M, G, attn_tail_box(M, H, Hkv)))
       return fail(RMT_EINVAL, "tensor map encoding failed (qkv must be 16-byte aligned)");
-    RMT_CUDA(launch_attention_tc(tm, a, /*f16=*/false, static_cast<cudaStream_t>(stream)));
+    RMT_CUDA(launch_attention_tc(tm, tt, a, /*f16=*/false, static_cast<cudaStream_t>(stream)));
     return RMT_OK;
   }
   RMT_CUDA(launch_attention(a, dtype == RMT_BF16 ? kElemBF16 : kElemF32, static_cast<cudaStream_t>(stream)));

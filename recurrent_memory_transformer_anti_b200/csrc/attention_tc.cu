@@ -7,9 +7,13 @@
 // associative memory (arXiv 2506.05229 abstract: recurrent memory transformers process
 // the input segment by segment).
 //
-// A work item is 128 query rows of one head of one cell; key/value tiles have 128 rows. The
-// CTAs are persistent (two per SM for head_dim 64) and take items round-robin, longest
-// first, so the loads of an item overlap the tail of the previous one.
+// A work item is 128 query rows of one head of one cell; key/value tiles have 128 rows. In
+// the last query tile of a cell, which holds rem = M mod 128 rows, the heads of a key/value
+// group share one item when they fit (their rows stacked, see attn_pack_tail): at M = 1040
+// and 4 query heads per group that turns 4 items of 16 useful rows into one of 64, and the
+// softmax warps whose 32 rows hold none of them skip their arithmetic. The CTAs are
+// persistent (two per SM for head_dim 64) and take items round-robin, longest first, so the
+// loads of an item overlap the tail of the previous one.
 //   warp 0      one thread: TMA loads of Q tiles (2 stages, one per item), K and V tiles
 //               (2 stages each, a ring that runs on across items);
 //   warp 1      TMEM allocation; one thread issues S = Q K^T (M=128, N=128) into TMEM and
@@ -69,7 +73,8 @@ __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
 template <int HD, typename OpT>
 __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_tail,
+                   const AttnArgs a) {
   using C = TaCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = sm100::smem_u32(smem_raw);
@@ -79,13 +84,27 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  // the stacking parameters come from the launch (kernel parameters: no registers held)
   const int nqt = (a.M + 127) / 128;
+  const int rem = a.tail_rows, gq = a.group;
+  const bool pack = rem > 0;
   const int per_rank = a.H * a.G;  // items per query-tile rank
-  const int nitems = nqt * per_rank;
-  // item i: query tile nqt-1 - i / (H*G) (longest first), then head (fastest, so the heads
-  // of a key/value group run close together), then cell
+  const int n_tail = a.n_tail;     // items of the last query tile
+  const int nitems = n_tail + (nqt - 1) * per_rank;
+  // item i: the last query tile first (longest first): one item per key/value group when its
+  // heads are stacked (h = the group's first head), else one per head; then query tiles
+  // nqt-2 .. 0. Within a tile the head runs fastest, so the heads of a key/value group run
+  // close together, then the cell.
   auto decode = [&](int i, int& qt, int& h, int& g) {
-    qt = nqt - 1 - i / per_rank;
+    if (i < n_tail) {
+      qt = nqt - 1;
+      const int nh = pack ? a.Hkv : a.H;
+      h = (i % nh) * (pack ? gq : 1);
+      g = i / nh;
+      return;
+    }
+    i -= n_tail;
+    qt = nqt - 2 - i / per_rank;
     const int r = i % per_rank;
     h = r % a.H;
     g = r / a.H;
@@ -111,7 +130,10 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
     sm100::fence_barrier_init();
     sm100::fence_proxy_async_smem();
   }
-  if (warp == 0 && lane == 0) sm100::tma_prefetch_desc(&tm);
+  if (warp == 0 && lane == 0) {
+    sm100::tma_prefetch_desc(&tm);
+    if (pack) sm100::tma_prefetch_desc(&tm_tail);
+  }
   if (warp == 1) sm100::tmem_alloc(sm100::smem_u32(tmem_slot), C::TMEM_COLS);
   sm100::tc_fence_before();
   __syncthreads();
@@ -138,10 +160,20 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
           ok = false;
           break;
         }
-        sm100::mbar_arrive_expect_tx(bar(kQFull + qs), C::TILE);
-        for (int sb = 0; sb < C::NSUB; ++sb)
-          sm100::tma_load_3d(base + C::Q_OFF + qs * C::TILE + sb * C::SUB, &tm, xq + 64 * sb, qt * 128, slice,
-                             bar(kQFull + qs));
+        if (pack && qt == nqt - 1) {
+          // the group's gq heads, rem rows each, stacked at rows hh * rem (1024-byte aligned:
+          // rem is a multiple of 8 rows of 128 bytes); rows gq * rem .. 127 are not loaded
+          sm100::mbar_arrive_expect_tx(bar(kQFull + qs), C::NSUB * gq * rem * 128);
+          for (int hh = 0; hh < gq; ++hh)
+            for (int sb = 0; sb < C::NSUB; ++sb)
+              sm100::tma_load_3d(base + C::Q_OFF + qs * C::TILE + sb * C::SUB + hh * rem * 128, &tm_tail,
+                                 xq + hh * HD + 64 * sb, qt * 128, slice, bar(kQFull + qs));
+        } else {
+          sm100::mbar_arrive_expect_tx(bar(kQFull + qs), C::TILE);
+          for (int sb = 0; sb < C::NSUB; ++sb)
+            sm100::tma_load_3d(base + C::Q_OFF + qs * C::TILE + sb * C::SUB, &tm, xq + 64 * sb, qt * 128, slice,
+                               bar(kQFull + qs));
+        }
         tq = ik;
         for (int j = 0; j <= qt; ++j, ++kv) {  // key/value tiles 0..qt hold every key the rows may see
           const int st = static_cast<int>(kv & 1);
@@ -271,16 +303,34 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
     bool ok = true;
     long t = 0;  // tiles processed so far (barrier phases)
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
-      int qt, h, g;
-      decode(it, qt, h, g);
-      const Cell c = a.cells[g];
-      const int slice = cell_index(a.mode, a.L, c);
-      const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
-      const int qrow = qt * 128 + r;
+      // a stacked tail tile holds head h + r / rem at row r < gq * rem; a warp whose rows are
+      // all past that (warp-uniform) keeps the barrier protocol but skips the arithmetic
+      int qt, vlim, mlim;
+      bool idle;
+      {
+        int h, g;
+        decode(it, qt, h, g);
+        const int kvlim = cell_rows(a.cells[g], a.M);  // keys past the cell's tokens are masked
+        const bool packed = pack && qt == nqt - 1;
+        idle = packed && quarter * 32 >= gq * rem;
+        vlim = min(qt * 128 + (packed ? r % rem : r), kvlim - 1);  // the last key this row sees
+        mlim = min(kvlim, qt * 128 + 1);  // a key tile reaching past this needs the mask
+      }
       float m_use = 0.f, l = 0.f;
       for (int j = 0; j <= qt; ++j, ++t) {
         ok = __all_sync(0xffffffffu, sm100::mbar_wait(bar(kSFull), static_cast<uint32_t>(t & 1), abort_flag));
         if (!ok) break;
+        if (idle) {
+          // the same waits and arrivals as the busy warps, in the same order
+          sm100::mbar_arrive(bar(kSFree));
+          if (j > 0) {
+            ok = __all_sync(0xffffffffu,
+                            sm100::mbar_wait(bar(kOReady), static_cast<uint32_t>((t - 1) & 1), abort_flag));
+            if (!ok) break;
+          }
+          sm100::mbar_arrive(bar(kPReady));
+          continue;
+        }
         sm100::tc_fence_after();
         uint32_t s[4][32];
 #pragma unroll
@@ -289,11 +339,11 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
         sm100::tc_fence_before();
         sm100::mbar_arrive(bar(kSFree));
         const int k0 = j * 128;
-        const bool need_mask = (j == qt) || (k0 + 128 > kvlim);
+        const bool need_mask = k0 + 128 > mlim;  // the diagonal tile, or keys past the cell's end
         // causal mask (and the cell's ragged end) only on the tiles that need it: key k0 + e is
         // visible iff e <= vis, so each element costs one compare with a constant and a select
         if (need_mask) {
-          const int vis = min(qrow, kvlim - 1) - k0;
+          const int vis = vlim - k0;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
 #pragma unroll
@@ -367,14 +417,26 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       if (!ok) break;
       sm100::tc_fence_after();
       const float inv = 1.f / l;
+      // the item's row and head again, from an opaque copy of the item index: recomputing
+      // them here keeps them out of the registers of the tile loop above
+      int it2;
+      asm volatile("mov.b32 %0, %1;" : "=r"(it2) : "r"(it));
+      int qt2, h, g;
+      decode(it2, qt2, h, g);
+      const Cell c = a.cells[g];
+      const bool packed = pack && qt2 == nqt - 1;
+      const int qrow = qt2 * 128 + (packed ? r % rem : r);
+      const bool row_out = packed ? r < gq * rem : qrow < a.M;
       const int ldo = a.ldo ? a.ldo : a.H * HD;
-      OpT* dst = static_cast<OpT*>(a.out) + (static_cast<size_t>(slice) * a.M + qrow) * ldo + h * HD;
+      OpT* const dst = static_cast<OpT*>(a.out) +
+                       (static_cast<size_t>(cell_index(a.mode, a.L, c)) * a.M + qrow) * ldo +
+                       (packed ? h + min(r / rem, gq - 1) : h) * HD;
 #pragma unroll 1
-      for (int oc = 0; oc < HD / 32; ++oc) {
+      for (int oc = 0; oc < (idle ? 0 : HD / 32); ++oc) {
         uint32_t o[32];
         sm100::tmem_ld32(tO + 32 * oc, o);
         sm100::tmem_wait_ld();
-        if (qrow < a.M) {
+        if (row_out) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = u2f(o[i]) * inv;
@@ -397,7 +459,12 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
 }
 
 template <int HD, typename OpT>
-cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st) {
+cudaError_t launch_hd(const CUtensorMap& tm, const CUtensorMap& tm_tail, const AttnArgs& a0, cudaStream_t st) {
+  AttnArgs a = a0;
+  const bool pack = attn_pack_tail(a.M, a.H, a.Hkv);
+  a.tail_rows = pack ? attn_tail_rows(a.M) : 0;
+  a.group = a.H / a.Hkv;
+  a.n_tail = (pack ? a.Hkv : a.H) * a.G;
   using C = TaCfg<HD>;
   static bool attr[64] = {false};
   static int sms[64] = {0};
@@ -410,10 +477,10 @@ cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st)
     cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     attr[dev] = true;
   }
-  const long items = static_cast<long>((a.M + 127) / 128) * a.H * a.G;
+  const long items = a.n_tail + static_cast<long>((a.M + 127) / 128 - 1) * a.H * a.G;
   const long cap = static_cast<long>(sms[dev] > 0 ? sms[dev] : 148) * C::CTAS_PER_SM;
   const int grid = static_cast<int>(items < cap ? items : cap);
-  const cudaError_t e = launch_pdl(attn_tc_kernel<HD, OpT>, dim3(grid), dim3(192), C::SMEM, st, tm, a);
+  const cudaError_t e = launch_pdl(attn_tc_kernel<HD, OpT>, dim3(grid), dim3(192), C::SMEM, st, tm, tm_tail, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -422,11 +489,15 @@ cudaError_t launch_hd(const CUtensorMap& tm, const AttnArgs& a, cudaStream_t st)
 
 bool attention_tc_supported(int dh) { return dh == 64 || dh == 128; }
 
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, bool f16, cudaStream_t st) {
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const CUtensorMap& tm_tail, const AttnArgs& a, bool f16,
+                                cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;
   if (a.Hkv <= 0 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
-  if (a.dh == 64) return f16 ? launch_hd<64, __half>(tm_qkv, a, st) : launch_hd<64, __nv_bfloat16>(tm_qkv, a, st);
-  if (a.dh == 128) return f16 ? launch_hd<128, __half>(tm_qkv, a, st) : launch_hd<128, __nv_bfloat16>(tm_qkv, a, st);
+  const CUtensorMap& tt = tm_tail;
+  if (a.dh == 64)
+    return f16 ? launch_hd<64, __half>(tm_qkv, tt, a, st) : launch_hd<64, __nv_bfloat16>(tm_qkv, tt, a, st);
+  if (a.dh == 128)
+    return f16 ? launch_hd<128, __half>(tm_qkv, tt, a, st) : launch_hd<128, __nv_bfloat16>(tm_qkv, tt, a, st);
   return cudaErrorInvalidValue;
 }
 

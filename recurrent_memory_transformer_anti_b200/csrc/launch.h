@@ -98,12 +98,31 @@ struct AttnArgs {
   int L;
   int* err;        // device error word for bounded waits (tensor-core kernel), may be null
   int ldo;         // row stride of out in elements (0: H * dh, rows packed)
+  // filled in by launch_attention_tc: rows of the stacked last query tile (0: not stacked,
+  // see attn_pack_tail), H / Hkv, and the work items of the last query tile
+  int tail_rows, group, n_tail;
 };
 // mma.sync (bf16) or fp32 FMA kernels, any head_dim in {32, 64, 128}
 cudaError_t launch_attention(const AttnArgs& a, ElemType t, cudaStream_t st);
-// tcgen05 kernel (16-bit, head_dim 64 or 128): tm_qkv maps qkv as [*, M, (H+2Hkv)dh], box 64 x 128
+// The last 128-row query tile of a cell holds rem = M - 128 (ceil(M / 128) - 1) rows. When the
+// H / Hkv query heads of one key/value group fit in a single 128-row tile there, and rem is a
+// multiple of 8 (so that each head's rows start on a 1024-byte swizzle atom), the tcgen05 kernel
+// stacks them: query head kvh * H / Hkv + i at tile rows i * rem .. i * rem + rem - 1, one work
+// item per group instead of one per head.
+__host__ __device__ inline int attn_tail_rows(int M) { return M - ((M + 127) / 128 - 1) * 128; }
+__host__ __device__ inline bool attn_pack_tail(int M, int H, int Hkv) {
+  const int rem = attn_tail_rows(M), gq = Hkv > 0 ? H / Hkv : 0;
+  return gq >= 2 && rem % 8 == 0 && rem * gq <= 128;
+}
+// Box height of the tail map: rem when the tail is stacked, else the 128-row tile
+inline uint32_t attn_tail_box(int M, int H, int Hkv) {
+  return attn_pack_tail(M, H, Hkv) ? static_cast<uint32_t>(attn_tail_rows(M)) : 128u;
+}
+// tcgen05 kernel (16-bit, head_dim 64 or 128): tm_qkv maps qkv as [*, M, (H+2Hkv)dh] with box
+// 64 x 128; tm_tail maps the same tensor with box 64 x attn_tail_box(M, H, Hkv)
 bool attention_tc_supported(int dh);
-cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const AttnArgs& a, bool f16, cudaStream_t st);
+cudaError_t launch_attention_tc(const CUtensorMap& tm_qkv, const CUtensorMap& tm_tail, const AttnArgs& a, bool f16,
+                                cudaStream_t st);
 
 // ------------------------------------------------------------------ associative memory
 struct MemReadArgs {

@@ -231,6 +231,9 @@ MIXED_CONFIGS = {
     # head_dim 128 on CTA pairs; 158 rows per cell end in a ragged token tile
     "pairs-dh128": dict(n_layers=3, d_model=256, n_heads=2, n_kv_heads=1, head_dim=128, d_ff=512, seg_len=150,
                         n_mem=8, d_k=64, d_v=64),
+    # 152 rows per cell: the last query tile (24 rows) stacks the 4 heads of the key/value group
+    "tail-stacked": dict(n_layers=3, d_model=256, n_heads=4, n_kv_heads=1, head_dim=64, d_ff=512, seg_len=144,
+                         n_mem=8, d_k=64, d_v=64),
 }
 
 
@@ -248,6 +251,14 @@ def test_bf16_tile_paths_match_oracle(cuda_ok, name):
     seq = forward(h, cfg, emb, S, "sequential")
     for a, b in zip(got, seq):
         np.testing.assert_array_equal(a, b)
+    if name == "tail-stacked":
+        # short last segments: the stacked tail rows past a cell's tokens are masked keys
+        embs = [emb[:2 * cfg.seg_len + 37], emb[:cfg.seg_len - 5]]
+        outs, A, z = forward_batch(h, cfg, embs, "diagonal")
+        outs_ref, A_ref, z_ref = armt.forward_batch(cfg, w, embs, dtype=np.float32)
+        for b_ in range(2):
+            assert normwise(outs[b_], outs_ref[b_]) < BF16_TOL, b_
+        assert normwise(A, A_ref) < BF16_TOL and normwise(z, z_ref) < BF16_TOL
     rmt.rmt_destroy(h)
 
 
@@ -412,7 +423,7 @@ def _full(h, cfg, emb):
     return out.float().cpu().numpy()
 
 
-@pytest.mark.parametrize("T", [1, 130, 455])
+@pytest.mark.parametrize("T", [1, 130, 176, 455])
 def test_full_attention_matches_oracle(cuda_ok, T):
     """The decoder stack without the memory, causal over T tokens (one or several query tiles
     with a ragged tail), against the oracle's comparison model."""

@@ -66,7 +66,11 @@ def test_grouped_gemm_each_group_uses_its_own_weight(N):
 
 ATTN_CASES = [("bf16", 2, 1040, 32, 8, 64), ("bf16", 3, 208, 4, 2, 64), ("bf16", 2, 300, 4, 1, 128),
               ("bf16", 2, 72, 4, 4, 32), ("bf16", 1, 1, 2, 1, 64), ("bf16", 1, 65, 2, 2, 64),
-              ("f32", 2, 72, 4, 4, 32), ("f32", 2, 208, 4, 2, 64), ("f32", 1, 130, 2, 1, 128)]
+              ("f32", 2, 72, 4, 4, 32), ("f32", 2, 208, 4, 2, 64), ("f32", 1, 130, 2, 1, 128),
+              # last query tile stacked across the heads of a key/value group: 3 x 16 rows
+              # (two warps idle, one half used), 4 x 8, 3 x 40 in the only tile, 4 x 32 (full)
+              ("bf16", 2, 528, 24, 8, 128), ("bf16", 2, 136, 8, 2, 64), ("bf16", 1, 40, 6, 2, 64),
+              ("bf16", 2, 160, 8, 2, 64)]
 
 
 @pytest.mark.parametrize("dtype,G,M,H,Hkv,dh", ATTN_CASES)
