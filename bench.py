@@ -40,11 +40,12 @@ N_SEGMENTS = 128
 WORKLOAD = "LLaMA-1B-shaped ARMT prefill of one 131,072-token sequence (128 x (1024 + 16 memory) tokens)"
 DATA = "synthetic: seeded N(0,1) embeddings, random-init N(0,0.02) weights"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per cell of the gate/up GEMM, from one ncu capture of a 2-cell
-# launch of the current kernel (profiles/gateup_gemm_1b.md). Traffic grows with the number of
-# cells (each cell brings its own layer's weights and activations), so a launch's traffic is
-# this figure times its cells. None when no capture of the current kernel exists.
-GATEUP_TRAFFIC_BYTES_PER_CELL = 82.49e6
+# DRAM bytes (read + write) per cell of the dominant launch -- the chained O / gate-up / down
+# grouped GEMM -- from one ncu capture of a small launch of the current kernel. Traffic grows
+# with the number of cells (each cell brings its own layer's weights and activations), so a
+# launch's traffic is this figure times its cells. None when no capture of the current kernel
+# exists.
+DOMINANT_TRAFFIC_BYTES_PER_CELL = None
 
 
 def parse():
@@ -407,7 +408,8 @@ def main() -> int:
     run("diagonal", W)
     rmt.rmt_sync(h, stream)
 
-    # ---- timed region: K diagonal-batched forwards, gate/up GEMM launches probed
+    # ---- timed region: K diagonal-batched forwards, the chained O / gate-up / down launches
+    # (probe kind "gateup") timed with CUDA events
     rmt.rmt_probe(h, ["gateup"])
     props = torch.cuda.get_device_properties(local)
     sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
@@ -423,13 +425,15 @@ def main() -> int:
     peaks, peak_src = load_peaks()
     achieved = probe["flops"] / (probe["ms"] / 1e3) / 1e12 if probe["ms"] > 0 else None
     peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "kernel": "grouped GEMM gate/up + SwiGLU epilogue (tcgen05)",
+    roofline = {"bound": "tensor",
+                "kernel": "chained grouped GEMM, one launch per diagonal: O projection + residual, gate/up + "
+                          "SwiGLU, down + residual (tcgen05, CTA pairs)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak if achieved else None,
                 "peak_source": f"bf16_tflops_sustained ({peak_src})",
                 "launches": probe["launches"], "kernel_ms_per_step": probe["ms"] / K,
-                "traffic": (GATEUP_TRAFFIC_BYTES_PER_CELL * cfg.n_layers * S / probe["launches"] * K
-                            if GATEUP_TRAFFIC_BYTES_PER_CELL and probe["launches"] and args.config == "1b" else None),
+                "traffic": (DOMINANT_TRAFFIC_BYTES_PER_CELL * cfg.n_layers * S / probe["launches"] * K
+                            if DOMINANT_TRAFFIC_BYTES_PER_CELL and probe["launches"] and args.config == "1b" else None),
                 "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 2-cell launch)"}
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
@@ -522,6 +526,8 @@ def main() -> int:
                        "layers": cfg.n_layers, "d_model": cfg.d_model, "segments": S,
                        "seg_len": cfg.seg_len, "n_mem": cfg.n_mem, "tokens": tokens, "schedule": "diagonal",
                        "batch": 1, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "precision": "bf16 weights, embeddings and outputs; f16 tensor-core operands with fp32 "
+                                    "accumulation; fp32 residual stream, softmax statistics and memory state",
                        "l2": "inputs larger than L2 (weights of 1.96 GB or more, embeddings 0.54 GB or more): no flush"},
             "roofline": roofline,
             "path": {"algorithmic_tflop_per_step": step_flops / 1e12,

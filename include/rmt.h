@@ -36,15 +36,25 @@ typedef enum {
   RMT_ENOMEM = 2,    /* device or pinned allocation failed */
   RMT_ECUDA = 3,     /* a CUDA runtime call or launch failed */
   RMT_ETIMEOUT = 4,  /* a bounded device-side wait gave up (reported by rmt_sync) */
-  RMT_ESTATE = 5     /* call not valid in this state (e.g. trace before any forward) */
+  RMT_ESTATE = 5,    /* call not valid in this state (e.g. trace before any forward) */
+  RMT_ERANGE = 6,    /* bf16 mode: a value overflowed an f16 tensor-core operand (reported by rmt_sync) */
+  RMT_EDEBUG = 7     /* debug build (librmt_debug.so) only: an in-kernel bounds check failed (rmt_sync) */
 } rmt_status;
 
 typedef enum { RMT_DIAGONAL = 0, RMT_SEQUENTIAL = 1 } rmt_schedule;
 
 /* Storage type of weights, embeddings, outputs and inter-kernel activations.
  * RMT_F32: every GEMM is an fp32 FMA kernel (no tensor cores).
- * RMT_BF16: GEMMs and attention run on tensor cores with fp32 accumulation; the residual
- * stream, softmax, RMSNorm statistics and the memory state stay fp32. */
+ * RMT_BF16: weights, embeddings and outputs are bf16. GEMMs and attention run on tensor cores
+ * with f16 operands and fp32 accumulation; the residual stream, softmax, RMSNorm statistics
+ * and the memory state stay fp32. f16 has 3 more mantissa bits than bf16, which the
+ * delta-rule memory update needs, and a smaller range: the values stored as f16 operands --
+ * the residual stream (embeddings included) before each projection, q/k/v, the SwiGLU output
+ * silu(gate)*up and the memory read-out -- must stay below 65504 in magnitude. Weights are
+ * converted to f16 at rmt_create, with the RMSNorm gains folded into the projections that
+ * follow them (exact for bf16 magnitudes from 2^-17 up; smaller ones lose bits).
+ * A forward that stores an operand of magnitude 65520 or more (which rounds to infinity) is
+ * reported by rmt_sync as RMT_ERANGE; its outputs are then not valid. */
 typedef enum { RMT_F32 = 0, RMT_BF16 = 1 } rmt_dtype;
 
 /* Model shape. A cell has M = seg_len + n_mem rows: the segment's tokens followed by the
@@ -185,23 +195,40 @@ rmt_status rmt_schedule_table_batch(int32_t n_layers, int32_t batch, const int32
 rmt_status rmt_get_trace(rmt_handle* h, int32_t* out_dls, size_t cap);
 
 /* Wait for `stream`, then report (and clear) the handle's device error word: RMT_ETIMEOUT
- * if a bounded device wait gave up, RMT_ECUDA on a CUDA error. With h == NULL the error
+ * if a bounded device wait gave up, RMT_ERANGE if the only fault since the last check is an
+ * f16 operand overflow (see rmt_dtype), RMT_EDEBUG if a bounds check of the debug build
+ * failed (see rmt_bounds_selftest), RMT_ECUDA on a CUDA error. With h == NULL the error
  * word of the kernel-level entry points on the current device is checked. */
 rmt_status rmt_sync(rmt_handle* h, void* stream);
 
 /* Check of the failure path: one CTA waits on an mbarrier that nothing signals, with the
- * bounded wait every kernel of this library uses, limited here to limit_us microseconds
- * (1 .. 10^7; the kernels use 2 s). The wait gives up, the CTA sets the device error word of
+ * bounded wait every kernel of this library uses, then on a global counter that nothing
+ * increments, with the bounded wait of the chained projections, each limited here to limit_us
+ * microseconds (1 .. 10^7; the kernels use 2 s). The waits give up, the CTA sets the device error word of
  * the kernel-level entry points and returns normally; rmt_sync(NULL, stream) then reports
  * RMT_ETIMEOUT (and clears the word), and the context stays usable. Asynchronous on stream. */
 rmt_status rmt_wait_selftest(uint32_t limit_us, void* stream);
+
+/* The debug build. librmt_debug.so is this library compiled with -DRMT_DEBUG, a stand-in for
+ * a memory checker: every kernel reads its (layer, segment) cells through a check of each
+ * index against the buffers the host sized for that forward (layer, state slice, residual
+ * slot, rows, token rows); a violation is recorded in the error word, which rmt_sync reports
+ * as RMT_EDEBUG, and the kernel continues with in-range indices, so no access leaves its
+ * buffer. rmt_bounds_selftest checks that mechanism: one thread presents an out-of-range cell
+ * to the check, and rmt_sync(NULL, stream) must then return RMT_EDEBUG with error word 64.
+ * The release library returns RMT_ESTATE here. Asynchronous on stream. */
+rmt_status rmt_bounds_selftest(void* stream);
 
 /* Kernel kinds of one schedule step, in launch order (see rmt_forward). Kinds that are fused
  * into another kind's kernel launch nothing of their own and read zero in rmt_probe_read:
  * RMSNORM1 and RMSNORM2 always (their statistics come from the residual epilogues and their
  * gains are folded into the next projection's weights); MEMREAD in bf16 mode with
  * d_k = d_v = 64, where the read runs in the MEMQ kernel's epilogue (and then MEMO forms only
- * the operand copy and statistics, the O projection adding the read-out to the residual). */
+ * the operand copy and statistics, the O projection adding the read-out to the residual); and
+ * O and DOWN in bf16 mode when O, gate/up and down all run on CTA pairs: the three projections
+ * then run as one chained launch per step (the tiles of each projection start as soon as the
+ * previous projection has stored the rows they read), reported under GATEUP with the flops
+ * and bytes of all three. */
 typedef enum {
   RMT_K_ASSEMBLE = 0,  /* layer-0 input: segment embeddings + memory tokens */
   RMT_K_MEMQ = 1,      /* memory-query projection (grouped GEMM), with the read when fused */
@@ -212,7 +239,7 @@ typedef enum {
   RMT_K_ATTENTION = 6,
   RMT_K_O = 7,         /* output projection + residual (grouped GEMM) */
   RMT_K_RMSNORM2 = 8,
-  RMT_K_GATEUP = 9,    /* gate/up projection + SwiGLU (grouped GEMM) */
+  RMT_K_GATEUP = 9,    /* gate/up projection + SwiGLU (grouped GEMM); or O + gate/up + down chained */
   RMT_K_DOWN = 10,     /* down projection + residual (grouped GEMM) */
   RMT_K_MEMKV = 11,    /* memory key/value projection of the memory-token rows */
   RMT_K_MEMUPDATE = 12,/* delta-rule update */
@@ -263,14 +290,15 @@ rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32
 /* Associative read, per row r of each group g (phi(x) = elu(x) + 1):
  *   o[g,r] = phi(q[g,r]) A[g] / (phi(q[g,r]) . z[g] + eps)
  * q [G, M, dk] fp32 (before phi), A [G, dk, dv] fp32, z [G, dk] fp32, o [G, M, dv] in
- * dtype. dk, dv multiples of 32, <= 128. */
+ * dtype. dk, dv multiples of 32, <= 128; every pointer 16-byte aligned (RMT_EINVAL otherwise). */
 rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void* o, int32_t G,
                            int32_t M, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
 
 /* Delta-rule write of n rows per group, all rows against the pre-update state:
  *   v_bar = phi(k) A / (phi(k) . z + eps);  A += phi(k)^T (v - v_bar);  z += sum_r phi(k_r)
  * k [G, n, dk] fp32 (before phi), v [G, n, dv] fp32, A [G, dk, dv] and z [G, dk] fp32,
- * updated in place. n <= 64; dk, dv multiples of 32, <= 128. */
+ * updated in place. n <= 64; dk, dv multiples of 32, <= 128; every pointer 16-byte aligned
+ * (RMT_EINVAL otherwise). */
 rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G,
                              int32_t n, int32_t dk, int32_t dv, float eps, void* stream);
 
@@ -278,9 +306,10 @@ rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z,
  *   k = y W_mk^T, v = y W_mv^T, then the delta-rule update above (phi applied to k).
  * y [G, n, d] fp32; w_mkv [G, dk + dv, d] in dtype (the dk rows of W_mk, then the dv rows
  * of W_mv); A [G, dk, dv] and z [G, dk] fp32, updated in place. The projection is split
- * along d in blocks of 128 columns whose partial sums go to a library-owned device scratch
- * buffer (grown with cudaMalloc on demand) and are added in a fixed order.
- * n <= 64, n*(dk+dv) <= 4096; dk, dv multiples of 32, <= 128. */
+ * along d in blocks of 128 columns (tensor cores for bf16 weights, the fp32 rows split into
+ * three bf16 terms) whose partial sums go to a library-owned device scratch buffer (grown
+ * with cudaMalloc on demand) and are added in a fixed order.
+ * n <= 64, n*(dk+dv) <= 4096; dk, dv multiples of 32, <= 128; A and z 16-byte aligned. */
 rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n,
                             int32_t d, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
 
@@ -289,12 +318,15 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
  * caching allocator that has already claimed the device memory for its own pool (there a
  * cudaMalloc can fail, and it synchronizes the whole device, stalling the caller's other
  * streams). Same arguments and results as rmt_memory_write; the cell table and the split-K
- * partial sums live in a fixed 8 MiB array in the library's device memory, which every GPU
- * that loads the library holds until the process exits. Sizes whose partial sums need
- * more than 8 MiB - 256 KiB (G*ceil(d/128)*n*(dk+dv)*4 bytes), or G > 8192, return
- * RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each device looks up
- * the array's device address (cudaGetSymbolAddress); make that first call before any
- * stream capture. All calls share the array, which keeps the last call's contents (every
+ * partial sums live in a fixed 8 MiB array in the library's device memory. Sizes whose
+ * partial sums need more than 8 MiB - 256 KiB (G*ceil(d/128)*n*(dk+dv)*4 bytes), or
+ * G > 8192, return RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each
+ * device loads the module that holds the array (CUDA loads modules lazily by default), which
+ * reserves the 8 MiB on that device until the process exits, and looks up the array's
+ * device address (cudaGetSymbolAddress). Make that first call at start-up: before the
+ * caller's allocator claims the device memory, and before any stream capture. The address is
+ * kept per device and does not survive a cudaDeviceReset of that device.
+ * All calls share the array, which keeps the last call's contents (every
  * value a call reads is written earlier in the same call): calls that overlap on the GPU,
  * e.g. on two streams, race and give wrong results. */
 rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv, float* A, float* z, int32_t G,

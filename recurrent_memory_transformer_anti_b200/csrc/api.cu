@@ -49,6 +49,8 @@ rmt_status fail(rmt_status st, const std::string& msg) {
     if (e_ != cudaSuccess) return fail(RMT_ECUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
   } while (0)
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 bool is_host_ptr(const void* p) {
   cudaPointerAttributes attr;
   if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
@@ -265,6 +267,12 @@ struct rmt_handle {
   // forms the f16 operand copy and RMSNorm statistics of x + W_mo o (no fp32 store)
   bool fold_mo = false;
   int ld_att = 0;  // row stride of the attention output (n_heads * head_dim, + d_v with fold_mo)
+  // bf16 mode with O, gate/up and down all on CTA pairs: the three run as one chained launch
+  // per step (launch_tc_pair_chain_o_mlp), ordered per (cell, token tile) by counters in
+  // global memory; the parity alternates from launch to launch
+  bool chain_mlp = false;
+  unsigned* chain_ctr = nullptr;
+  int chain_ctr_len = 0, chain_parity = 0;
   std::vector<void*> allocs;
   // activations and memory state, sized for cap_b sequences (rmt_reserve)
   int cap_b = 0;
@@ -328,6 +336,7 @@ struct rmt_handle {
     xb = nullptr;
     qkv = att = u = om = nullptr;
     qm = part = A = z = ss1 = ss2 = nullptr;
+    chain_ctr = nullptr;
   }
   void free_full() {
     for (void* p : full_allocs) cudaFree(p);
@@ -552,6 +561,17 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
     h->free_acts();
     return fail(RMT_ECUDA, "cudaMemset failed");
   }
+  if (h->chain_mlp) {  // one counter per (cell, token tile) of a step, both parities, both boundaries
+    const int nt = pair_token_tile(M);
+    h->chain_ctr_len = static_cast<int>(BL) * ((M + nt - 1) / nt);
+    const size_t bytes = size_t(2) * (kMaxPhases - 1) * h->chain_ctr_len * sizeof(unsigned);
+    h->chain_ctr = static_cast<unsigned*>(h->act_alloc(bytes));
+    if (!h->chain_ctr || cudaMemset(h->chain_ctr, 0, bytes) != cudaSuccess) {
+      h->free_acts();
+      return fail(RMT_ENOMEM, "activation allocation failed");
+    }
+    h->chain_parity = 0;
+  }
   h->cap_b = B;
   if (h->bf16) {
     rmt_status st = build_maps(h);
@@ -572,7 +592,14 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
 
 enum Proj { kProjMemQ, kProjMemO, kProjQkv, kProjO, kProjGateUp, kProjDown };
 
-cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream_t st) {
+// A CTA-pair projection's launch arguments, collected instead of launched (for the chain).
+struct PairLaunch {
+  TcGemmArgs a;
+  const CUtensorMap* tw;
+  const CUtensorMap* tx;
+};
+
+cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream_t st, PairLaunch* collect = nullptr) {
   const rmt_cfg& c = h->cfg;
   const int d = c.d_model, hd = c.n_heads * c.head_dim;
   EpiParams ep{};
@@ -646,8 +673,13 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   }
   if (h->bf16 && pair) {
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
+    if (collect) {
+      *collect = PairLaunch{a, tb, tp};
+      return cudaSuccess;
+    }
     return launch_tc_pair_gemm(*tb, *tp, a, /*f16=*/true, st);
   }
+  if (collect) return cudaErrorInvalidValue;
   if (h->bf16) {
     const bool rope_tma = p == kProjQkv && c.head_dim >= 64;
     ep.rope_tma = rope_tma;
@@ -657,6 +689,27 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
   SimtGemmArgs a{h->M, N, K, G, cells, c.n_layers, a32, lda, amode, static_cast<const float*>(w), epi, ep};
   return launch_simt_gemm(a, st);
+}
+
+// The O projection, gate/up and down of a step in one chained CTA-pair launch.
+cudaError_t run_chain_o_mlp(rmt_handle* h, const Cell* cells, int G, cudaStream_t st) {
+  PairLaunch o{}, gu{}, dn{};
+  cudaError_t e = run_proj(h, kProjO, cells, G, st, &o);
+  if (e == cudaSuccess) e = run_proj(h, kProjGateUp, cells, G, st, &gu);
+  if (e == cudaSuccess) e = run_proj(h, kProjDown, cells, G, st, &dn);
+  if (e != cudaSuccess) return e;
+  PairChainArgs a{};
+  a.ph[0] = o.a;
+  a.ph[1] = gu.a;
+  a.ph[2] = dn.a;
+  a.nphase = 3;
+  a.ctr = h->chain_ctr;
+  a.ctr_len = h->chain_ctr_len;
+  a.parity = h->chain_parity;
+  const CUtensorMap tw[3] = {*o.tw, *gu.tw, *dn.tw}, tx[3] = {*o.tx, *gu.tx, *dn.tx};
+  e = launch_tc_pair_chain_o_mlp(tw, tx, a, st);
+  if (e == cudaSuccess) h->chain_parity ^= 1;
+  return e;
 }
 
 // NVTX range names of the kernel kinds (rmt_kernel order). The ranges cost nothing
@@ -707,7 +760,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (n_first > 0) {
     e = launch_kind(h, RMT_K_ASSEMBLE, 0, rows_first * dd * (es + 4 + (h->bf16 ? 2 : 0)), st, [&] {
       return launch_assemble(cells, n_first, emb, h->memtok, h->x, h->bf16 ? h->xb : nullptr, M, c.n_mem, d, h->bf16,
-                             st);
+                             h->err, st);
     });
     if (e != cudaSuccess) return e;
   }
@@ -723,7 +776,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
     e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk),
                     g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es), st, [&] {
                       MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
-                      return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st);
+                      return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st, h->err);
                     });
     if (e != cudaSuccess) return e;
   }
@@ -747,17 +800,22 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                   });
   if (e != cudaSuccess) return e;
   // (the folded W_mo o is counted once, with the read-out projection, as the model defines it)
-  e = launch_kind(h, RMT_K_O, 2 * g * m * dd * hd,
-                  g * (m * (hd + fold * dv) * es + dd * (hd + fold * dv) * es + 2 * m * dd * 4), st,
-                  [&] { return run_proj(h, kProjO, cells, G, st); });
-  if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_GATEUP, 2 * g * m * 2 * F * dd, g * (m * dd * es + 2 * F * dd * es + m * F * es), st,
-                  [&] { return run_proj(h, kProjGateUp, cells, G, st); });
-  if (e != cudaSuccess) return e;
-  e = launch_kind(h, RMT_K_DOWN, 2 * g * m * dd * F,
-                  g * (m * F * es + dd * F * es + 2 * m * dd * 4 + (h->bf16 ? m * dd * 2 : 0)), st,
-                  [&] { return run_proj(h, kProjDown, cells, G, st); });
-  if (e != cudaSuccess) return e;
+  const double o_flops = 2 * g * m * dd * hd, gu_flops = 2 * g * m * 2 * F * dd, d_flops = 2 * g * m * dd * F;
+  const double o_bytes = g * (m * (hd + fold * dv) * es + dd * (hd + fold * dv) * es + 2 * m * dd * 4),
+               gu_bytes = g * (m * dd * es + 2 * F * dd * es + m * F * es),
+               d_bytes = g * (m * F * es + dd * F * es + 2 * m * dd * 4 + (h->bf16 ? m * dd * 2 : 0));
+  if (h->chain_mlp) {  // one launch: reported under GATEUP with the work of all three projections
+    e = launch_kind(h, RMT_K_GATEUP, o_flops + gu_flops + d_flops, o_bytes + gu_bytes + d_bytes, st,
+                    [&] { return run_chain_o_mlp(h, cells, G, st); });
+    if (e != cudaSuccess) return e;
+  } else {
+    e = launch_kind(h, RMT_K_O, o_flops, o_bytes, st, [&] { return run_proj(h, kProjO, cells, G, st); });
+    if (e != cudaSuccess) return e;
+    e = launch_kind(h, RMT_K_GATEUP, gu_flops, gu_bytes, st, [&] { return run_proj(h, kProjGateUp, cells, G, st); });
+    if (e != cudaSuccess) return e;
+    e = launch_kind(h, RMT_K_DOWN, d_flops, d_bytes, st, [&] { return run_proj(h, kProjDown, cells, G, st); });
+    if (e != cudaSuccess) return e;
+  }
   e = launch_kind(h, RMT_K_MEMKV, 2 * g * n * (dk + dv) * dd,
                   g * (n * dd * 4 + (dk + dv) * dd * es + h->nsplit * n * (dk + dv) * 4), st, [&] {
                     MemKvArgs a{h->x, M, d, c.n_mem, kOutSlot, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
@@ -828,7 +886,18 @@ rmt_status full_buffers(rmt_handle* h, int T) {
   }
   if (T != h->full_T) {
     std::vector<Cell> cells(c.n_layers);
-    for (int l = 0; l < c.n_layers; ++l) cells[l] = Cell{l, 0, 0, T, 0, l & 1, (l + 1) & 1, 0};
+    for (int l = 0; l < c.n_layers; ++l) {
+      cells[l] = Cell{l, 0, 0, T, 0, l & 1, (l + 1) & 1, 0};
+#ifdef RMT_DEBUG
+      cells[l].lim_L = c.n_layers;
+      cells[l].lim_state = 1;
+      cells[l].lim_slot = 2;
+      cells[l].lim_M = T;
+      cells[l].lim_nmem = 0;
+      cells[l].lim_tokens = T;
+      cells[l].lim_err = h->err;
+#endif
+    }
     RMT_CUDA(cudaMemcpy(h->fcells, cells.data(), cells.size() * sizeof(Cell), cudaMemcpyHostToDevice));
     auto map = [](CUtensorMap* m, const void* q, uint64_t inner, uint64_t rows, uint64_t depth, uint32_t box) {
       return make_tmap_16_3d(m, q, inner, rows, depth, box, true);
@@ -988,7 +1057,7 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   h->es = h->bf16 ? 2 : 4;
   h->M = c.seg_len + c.n_mem;
   h->Nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-  h->nsplit = (c.d_model + kMemKvSplit - 1) / kMemKvSplit;
+  h->nsplit = mem_kv_splits(c.d_model, c.dtype == RMT_BF16);
   const size_t L = c.n_layers, d = c.d_model, M = h->M, es = h->es, F = c.d_ff, dk = c.d_k, dv = c.d_v;
   if (h->bf16) {
     const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
@@ -1001,6 +1070,7 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
     h->pair_d = tc_pair_supported(Mi, di, Fi, kEpiResidCast, 0);
     h->pair_o = tc_pair_supported(Mi, di, hdi, kEpiResidCast, 0);
     h->fold_mo = h->fuse_read && h->pair_o && tc_pair_supported(Mi, di, hdi + c.d_v, kEpiResidCast, 0);
+    h->chain_mlp = h->pair_o && h->pair_gu && h->pair_d;
   }
   h->ld_att = c.n_heads * c.head_dim + (h->fold_mo ? c.d_v : 0);
   const size_t ldw_o = size_t(h->ld_att);  // W_o rows: [W_o | W_mo] with fold_mo
@@ -1106,6 +1176,17 @@ rmt_status forward_impl(rmt_handle* h, const void* emb, const std::vector<int>& 
     }
     Table t;
     build_table(c.n_layers, c.seg_len, c.n_mem, T, schedule, t);
+#ifdef RMT_DEBUG
+    for (Cell& x : t.cells) {  // the buffers this forward's cells address, for the in-kernel checks
+      x.lim_L = c.n_layers;
+      x.lim_state = B * c.n_layers;
+      x.lim_slot = B * n_slots(c.n_layers);
+      x.lim_M = h->M;
+      x.lim_nmem = c.n_mem;
+      x.lim_tokens = static_cast<long long>(total_tokens);
+      x.lim_err = h->err;
+    }
+#endif
     if (cudaMalloc(&t.dev, sizeof(Cell) * t.cells.size()) != cudaSuccess)
       return fail(RMT_ENOMEM, "cell table allocation failed");
     if (cudaMemcpy(t.dev, t.cells.data(), sizeof(Cell) * t.cells.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
@@ -1286,7 +1367,7 @@ rmt_status rmt_full_attention_forward(rmt_handle* h, const void* emb, int32_t n_
     return fail(RMT_ECUDA, std::string("launch failed: ") + cudaGetErrorString(e));
   };
   // the input: the embeddings into slot 0 (fp32 and the f16 copy), and their RMSNorm statistics
-  cudaError_t e = launch_assemble(h->fcells, 1, emb_dev, h->memtok, h->fx, h->fxb, T, 0, d, true, st);
+  cudaError_t e = launch_assemble(h->fcells, 1, emb_dev, h->memtok, h->fx, h->fxb, T, 0, d, true, h->err, st);
   if (e == cudaSuccess) e = launch_row_ssq(h->fx, h->fss1, T, d, h->ss_parts, st);
   if (e != cudaSuccess) return launch_fail(e);
   for (int l = 0; l < L; ++l) {
@@ -1339,6 +1420,13 @@ rmt_status rmt_sync(rmt_handle* h, void* stream) {
   RMT_CUDA(cudaMemcpy(&word, err, sizeof(int), cudaMemcpyDeviceToHost));
   if (word) {
     RMT_CUDA(cudaMemset(err, 0, sizeof(int)));
+    if (word & kErrBounds)
+      return fail(RMT_EDEBUG, "a kernel's bounds check failed: a cell index fell outside its buffers (error word " +
+                                  std::to_string(word) + ")");
+    if (word == kErrF16Range)
+      return fail(RMT_ERANGE,
+                  "a value of magnitude 65520 or more was stored as an f16 tensor-core operand (bf16 mode): the "
+                  "outputs of this forward are not valid");
     return fail(RMT_ETIMEOUT, "a bounded device wait gave up (error word " + std::to_string(word) + ")");
   }
   return RMT_OK;
@@ -1402,6 +1490,19 @@ rmt_status rmt_wait_selftest(uint32_t limit_us, void* stream) {
   return RMT_OK;
 }
 
+rmt_status rmt_bounds_selftest(void* stream) {
+#ifdef RMT_DEBUG
+  int* err = nullptr;
+  const Cell* cells = nullptr;
+  RMT_TRY(device_scratch(1, &cells, &err));
+  RMT_CUDA(launch_bounds_selftest(err, static_cast<cudaStream_t>(stream)));
+  return RMT_OK;
+#else
+  (void)stream;
+  return fail(RMT_ESTATE, "rmt_bounds_selftest needs the debug build (librmt_debug.so)");
+#endif
+}
+
 rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t G, int32_t M, int32_t N, int32_t K,
                                  rmt_dtype out_dtype, void* stream) {
   if (!A || !B || !C) return fail(RMT_EINVAL, "null pointer");
@@ -1458,19 +1559,24 @@ rmt_status rmt_attention(const void* qkv, void* out, int32_t G, int32_t M, int32
 rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void* o, int32_t G, int32_t M, int32_t dk,
                            int32_t dv, float eps, rmt_dtype dtype, void* stream) {
   if (!q || !A || !z || !o) return fail(RMT_EINVAL, "null pointer");
+  if (!aligned16(q) || !aligned16(A) || !aligned16(z) || !aligned16(o))
+    return fail(RMT_EINVAL, "q, A, z and o must be 16-byte aligned");
   if (G <= 0 || M <= 0 || dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128)
     return fail(RMT_EINVAL, "bad sizes");
   if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
   const Cell* cells = nullptr;
-  RMT_TRY(device_scratch(G, &cells, nullptr));
+  int* err = nullptr;
+  RMT_TRY(device_scratch(G, &cells, &err));
   MemReadArgs a{q, A, z, o, M, dk, dv, eps, G, cells, kByLayer, kByLayer, G};
-  RMT_CUDA(launch_mem_read(a, dtype == RMT_BF16 ? kElemBF16 : kElemF32, static_cast<cudaStream_t>(stream)));
+  RMT_CUDA(launch_mem_read(a, dtype == RMT_BF16 ? kElemBF16 : kElemF32, static_cast<cudaStream_t>(stream), err));
   return RMT_OK;
 }
 
 rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n, int32_t dk,
                              int32_t dv, float eps, void* stream) {
   if (!k || !v || !A || !z) return fail(RMT_EINVAL, "null pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(z))
+    return fail(RMT_EINVAL, "k, v, A and z must be 16-byte aligned");
   if (G <= 0 || n <= 0 || n > 64 || dk % 32 || dv % 32 || dk <= 0 || dv <= 0 || dk > 128 || dv > 128)
     return fail(RMT_EINVAL, "bad sizes");
   const Cell* cells = nullptr;
@@ -1495,13 +1601,14 @@ rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int
 rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n, int32_t d,
                             int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream) {
   if (!y || !w_mkv || !A || !z) return fail(RMT_EINVAL, "null pointer");
+  if (!aligned16(A) || !aligned16(z)) return fail(RMT_EINVAL, "A and z must be 16-byte aligned");
   if (G <= 0 || n <= 0 || n > 64 || d <= 0 || dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128 ||
       n * (dk + dv) > 4096)
     return fail(RMT_EINVAL, "bad sizes");
   if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
   const Cell* cells = nullptr;
   RMT_TRY(device_scratch(G, &cells, nullptr));
-  const int nsplit = (d + kMemKvSplit - 1) / kMemKvSplit;
+  const int nsplit = mem_kv_splits(d, dtype == RMT_BF16);
   float* part = nullptr;
   RMT_TRY(partial_scratch(size_t(G) * nsplit * n * (dk + dv), &part));
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnArgs a) {
   const int nqt = (a.M + S::BQ - 1) / S::BQ;
   const int qt = nqt - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y;
-  const Cell c = a.cells[blockIdx.z];
+  const Cell c = load_cell(a.cells, blockIdx.z);
   const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
   const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.ldo ? a.ldo : a.H * HD;
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
   __shared__ float Kc[CK][HD];
   __shared__ float Vc[CK][HD];
   const int qc = blockIdx.x, h = blockIdx.y;
-  const Cell c = a.cells[blockIdx.z];
+  const Cell c = load_cell(a.cells, blockIdx.z);
   const int kvlim = cell_rows(c, a.M);  // keys past the cell's tokens are masked
   const int rep = a.H / a.Hkv, kvh = h / rep;
   const int ldq = (a.H + 2 * a.Hkv) * HD, ldo = a.ldo ? a.ldo : a.H * HD;

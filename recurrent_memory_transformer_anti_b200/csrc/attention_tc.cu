@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++ik) {
         int qt, h, g;
         decode(it, qt, h, g);
-        const Cell c = a.cells[g];
+        const Cell c = load_cell(a.cells, g);
         const int kvh = h / (a.H / a.Hkv);
         const int slice = cell_index(a.mode, a.L, c);
         const int xq = h * HD, xk = (a.H + kvh) * HD, xv = (a.H + a.Hkv + kvh) * HD;
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       {
         int h, g;
         decode(it, qt, h, g);
-        const int kvlim = cell_rows(a.cells[g], a.M);  // keys past the cell's tokens are masked
+        const int kvlim = cell_rows(load_cell(a.cells, g), a.M);  // keys past the cell's tokens are masked
         const bool packed = pack && qt == nqt - 1;
         idle = packed && quarter * 32 >= gq * rem;
         vlim = min(qt * 128 + (packed ? r % rem : r), kvlim - 1);  // the last key this row sees
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(192, TaCfg<HD>::CTAS_PER_SM)
       asm volatile("mov.b32 %0, %1;" : "=r"(it2) : "r"(it));
       int qt2, h, g;
       decode(it2, qt2, h, g);
-      const Cell c = a.cells[g];
+      const Cell c = load_cell(a.cells, g);
       const bool packed = pack && qt2 == nqt - 1;
       const int qrow = qt2 * 128 + (packed ? r % rem : r);
       const bool row_out = packed ? r < gq * rem : qrow < a.M;

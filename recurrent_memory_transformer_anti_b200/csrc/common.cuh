@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace rmt {
 
 // Device error word values (OR-ed together; read and cleared by rmt_sync).
@@ -15,7 +17,35 @@ enum : int {
   kErrTimeoutEpilogue = 4,
   kErrBadArgs = 8,
   kErrTimeoutSelftest = 16,  // the bounded-wait check (rmt_wait_selftest) gave up, as it should
+  kErrF16Range = 32,         // a value stored as an f16 tensor-core operand overflowed (see below)
+  kErrBounds = 64,           // debug build: a cell's index fell outside the buffers it addresses
 };
+
+// f16 operand range. In bf16 mode the tensor-core operands the forward writes (the residual
+// stream's operand copy, q/k/v, the SwiGLU output, the memory read-out) are f16, whose largest
+// finite value is 65504: a magnitude of 65520 or more rounds to infinity. Each kernel that
+// stores such an operand keeps, per thread, the largest magnitude it stored and reports an
+// overflow in the error word (kErrF16Range), which rmt_sync turns into RMT_ERANGE.
+constexpr float kF16Overflow = 65520.f;
+
+template <typename T>
+__device__ __forceinline__ void track_amax(float& m, float v) {
+  if constexpr (std::is_same_v<T, __half>) m = fmaxf(m, fabsf(v));
+}
+template <typename T, int N>
+__device__ __forceinline__ void track_amax(float& m, const float (&v)[N]) {
+  if constexpr (std::is_same_v<T, __half>) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+}
+// Called by all 32 lanes of a warp: one atomic per warp that stored an overflowing value.
+template <typename T>
+__device__ __forceinline__ void report_f16_range(float m, int* err) {
+  if constexpr (std::is_same_v<T, __half>) {
+    if (__any_sync(0xffffffffu, m >= kF16Overflow) && (threadIdx.x & 31) == 0 && err) atomicOr(err, kErrF16Range);
+  }
+}
 
 // Programmatic dependent launch. The forward launches its kernels with programmatic stream
 // serialization, so a kernel may be scheduled while the previous one in the stream is still
@@ -42,7 +72,39 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 //   t0     row of the segment's first token in the packed embeddings / outputs
 struct Cell {
   int l, s, b, m, k, xin, xout, t0;
+#ifdef RMT_DEBUG
+  // Debug build (-DRMT_DEBUG, librmt_debug.so): the sizes of the buffers this cell's indices
+  // address, and the error word a violation is reported to (null: the identity cells of the
+  // kernel-level entry points, whose indices the grid itself bounds). See load_cell.
+  int lim_L, lim_state, lim_slot, lim_M, lim_nmem;
+  long long lim_tokens;
+  int* lim_err;
+#endif
 };
+
+// Every kernel reads its cells through load_cell. In the debug build it checks each index
+// against the limits the host stored in the cell -- layer < L, state and scratch slice <
+// sequences x L, residual slots < sequences x (2L + 2), n_mem <= rows <= M, and the segment's
+// token rows inside the embeddings -- and on a violation records kErrBounds in the error word
+// (rmt_sync then returns RMT_EDEBUG) and hands the kernel a cell whose indices are all in range
+// (slot 0, state 0, no token rows), so that no access leaves its buffer. The release build
+// compiles to the plain load.
+__device__ __forceinline__ Cell load_cell(const Cell* cells, int g) {
+  Cell c = cells[g];
+#ifdef RMT_DEBUG
+  if (c.lim_err) {
+    const bool ok = c.l >= 0 && c.l < c.lim_L && c.k >= 0 && c.k < c.lim_state && c.xin >= 0 &&
+                    c.xin < c.lim_slot && c.xout >= 0 && c.xout < c.lim_slot && c.m >= c.lim_nmem &&
+                    c.m <= c.lim_M && c.t0 >= 0 && static_cast<long long>(c.t0) + (c.m - c.lim_nmem) <= c.lim_tokens;
+    if (!ok) {
+      atomicOr(c.lim_err, kErrBounds);
+      c.l = c.k = c.xin = c.xout = c.t0 = 0;
+      c.m = c.lim_nmem;
+    }
+  }
+#endif
+  return c;
+}
 
 // Activation slots of one sequence, each an [M, d] fp32 residual block; sequence b owns
 // slots b*n_slots(L) .. (b+1)*n_slots(L)-1.
@@ -67,7 +129,12 @@ __host__ __device__ inline int cell_index(IndexMode mode, int /*L*/, Cell c) {
 __host__ __device__ inline int cell_rows(const Cell& c, int M) { return c.m < M ? c.m : M; }
 
 // Cell g of the kernel-level entry points: group g uses slice g of every stacked operand.
-__host__ __device__ inline Cell identity_cell(int g) { return Cell{g, 0, 0, 0x7fffffff, g, g, g, 0}; }
+__host__ __device__ inline Cell identity_cell(int g) {
+  Cell c{};
+  c.l = c.k = c.xin = c.xout = g;
+  c.m = 0x7fffffff;
+  return c;
+}
 
 // GEMM epilogues shared by the tensor-core and the fp32 kernels.
 enum EpiKind : int {

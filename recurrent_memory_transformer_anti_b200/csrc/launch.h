@@ -71,6 +71,26 @@ bool tc_pair_supported(int M, int N, int K, int epi, int head_dim);
 cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, bool f16,
                                 cudaStream_t st);
 
+// Several projections of the same cells in one CTA-pair launch ("phases", run in order; see
+// tc_gemm_pair.cu): phase p >= 1 of (cell g, token tile tt) starts once every tile of phase p-1
+// for those tokens is stored, which a counter per (phase, cell, token tile) in global memory
+// records (one increment per epilogue warp and tile). The counters of one launch sit in block `parity` of ctr, laid out
+// [2 parities][kMaxPhases - 1][ctr_len] with ctr_len >= G * token tiles; the launch zeroes the
+// other parity's block for the next launch, so consecutive launches alternate the parity and
+// the buffer starts zeroed.
+constexpr int kMaxPhases = 3;
+struct PairChainArgs {
+  TcGemmArgs ph[kMaxPhases];  // per phase; M, G, cells, L and err are phase 0's for all
+  int nphase;
+  unsigned* ctr;
+  int ctr_len;
+  int parity;
+};
+// The O projection, gate/up and down of one diagonal in one launch (f16 operands): tw / tx hold
+// each phase's weight and activation maps, as launch_tc_pair_gemm takes them.
+cudaError_t launch_tc_pair_chain_o_mlp(const CUtensorMap* tw, const CUtensorMap* tx, const PairChainArgs& args,
+                                       cudaStream_t st);
+
 // fp32 FMA path (fp32 operands by pointer)
 struct SimtGemmArgs {
   int M, N, K;
@@ -138,12 +158,19 @@ struct MemReadArgs {
   IndexMode state_mode;  // slice of A and z
   int L;
 };
-cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_t st);
+// 16-bit outputs take the tcgen05 read when it supports d_k (err: its bounded waits' error word,
+// may be null), else the mma.sync read; fp32 outputs the fp32 FMA read
+cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_t st, int* err = nullptr);
+// tcgen05 read for 16-bit outputs with d_k of 64 or 128 (memory_tc.cu); err: error word of the
+// bounded waits (may be null)
+bool mem_read_tc_supported(int dk, int dv);
+cudaError_t launch_mem_read_tc(const MemReadArgs& a, bool f16, int* err, cudaStream_t st);
 
 // Partial products of the memory-token rows with [W_mk; W_mv], split along d_model so the
 // reduction order is fixed: part[l][split][r][j] = sum_{k in split} Y[r][k] W_mkv[l][j][k],
-// Y = rows row0 .. row0+n-1 of the cell's output slot.
+// Y = rows row0 .. row0+n-1 of the cell's output slot; the update adds the splits in order.
 constexpr int kMemKvSplit = 128;  // d_model columns per split
+inline int mem_kv_splits(int d, bool /*bf16*/) { return (d + kMemKvSplit - 1) / kMemKvSplit; }
 struct MemKvArgs {
   const float* x;  // [*, M, d] fp32: the residual stream slots (forward) or caller rows
   int M, d, n;     // the n rows read are the cell's last n valid rows (cell_rows(c, M) - n ..)
@@ -199,14 +226,19 @@ cudaError_t launch_scale_cols(void* w, const void* g, int L, int N, int K, bool 
 cudaError_t launch_bf16_to_f16(void* p, size_t n, cudaStream_t st);
 // Layer-0 inputs of the G cells (all of layer 0): in slot c.xin of x (and of xb, if given),
 // rows 0..m-n_mem-1 from emb rows c.t0.., rows m-n_mem..m-1 from the memory tokens, rows
-// m..M-1 zero (m = cell_rows(c, M)).
+// m..M-1 zero (m = cell_rows(c, M)). An f16 copy that overflows sets kErrF16Range in *err.
 cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
-                            int n_mem, int d, bool bf16, cudaStream_t st);
+                            int n_mem, int d, bool bf16, int* err, cudaStream_t st);
 // RMSNorm statistics of rows 0..M-1 of an fp32 [M, d] block: ss[row * parts + b] = sum of
 // squares of columns b*w .. b*w+w-1, w = d / parts (a multiple of 4; at most 32 parts).
 // One CTA waits on an mbarrier nothing signals, with the kernels' bounded wait limited to
 // limit_ns, and ORs kErrTimeoutSelftest into *err when the wait gives up (see selftest.cu).
 cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st);
+#ifdef RMT_DEBUG
+// Debug build: one thread passes load_cell a cell with an out-of-range slot; kErrBounds must
+// reach *err (and kErrBadArgs too if the returned cell is not the in-range substitute).
+cudaError_t launch_bounds_selftest(int* err, cudaStream_t st);
+#endif
 cudaError_t launch_row_ssq(const float* x, float* ss, int M, int d, int parts, cudaStream_t st);
 // Segment outputs of the G cells: rows 0..m-n_mem-1 of slot c.xout, cast to T, to out rows c.t0...
 cudaError_t launch_emit(const Cell* cells, int G, const float* x, void* out, int M, int n_mem, int d, bool bf16,

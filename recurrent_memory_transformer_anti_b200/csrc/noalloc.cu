@@ -5,6 +5,7 @@
 // fail, and it synchronizes the whole device, stalling the caller's other streams). This
 // entry point keeps its scratch -- the cell table and the split-K partial sums of the
 // key/value projection -- in a fixed array in the library's own device memory instead.
+#include <atomic>
 #include <string>
 
 #include "common.cuh"
@@ -15,15 +16,19 @@ namespace {
 
 using rmt::Cell;
 
-// Scratch for rmt_memory_write_noalloc: the cell table, then the partial sums. Every GPU
-// that loads the library holds these 8 MiB until the process exits.
+// Scratch for rmt_memory_write_noalloc: the cell table, then the partial sums. With CUDA's
+// lazy module loading (the default), a device gets these 8 MiB when this file's module is
+// first loaded there -- at the first rmt_memory_write_noalloc call on that device -- and
+// holds them until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 constexpr size_t kNoAllocCellBytes = 256 << 10;  // room for 8192 cells
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch, looked up once per device (host code cannot use the
-// symbol itself: on the host it names a stand-in, not device memory).
-void* g_noalloc_addr[64] = {};
+// symbol itself: on the host it names a stand-in, not device memory). Host threads may race
+// on the first lookup; each stores the same address. The cached address belongs to the
+// device's context of the time: it does not survive a cudaDeviceReset of that device.
+std::atomic<void*> g_noalloc_addr[64] = {};
 
 __global__ void fill_cells_kernel(Cell* cells, int G) {
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
@@ -44,11 +49,13 @@ extern "C" rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv
     return st;
   };
   if (!y || !w_mkv || !A || !z) return fail(RMT_EINVAL, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(z)) & 15u)
+    return fail(RMT_EINVAL, "A and z must be 16-byte aligned");
   if (G <= 0 || n <= 0 || n > 64 || d <= 0 || dk <= 0 || dv <= 0 || dk % 32 || dv % 32 || dk > 128 || dv > 128 ||
       n * (dk + dv) > 4096)
     return fail(RMT_EINVAL, "bad sizes");
   if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
-  const size_t nsplit = (size_t(d) + rmt::kMemKvSplit - 1) / rmt::kMemKvSplit;
+  const size_t nsplit = static_cast<size_t>(rmt::mem_kv_splits(d, dtype == RMT_BF16));
   const size_t part_bytes = size_t(G) * nsplit * n * (dk + dv) * sizeof(float);
   if (size_t(G) * sizeof(Cell) > kNoAllocCellBytes || part_bytes > kNoAllocScratchBytes - kNoAllocCellBytes)
     return fail(RMT_EINVAL,
@@ -56,14 +63,14 @@ extern "C" rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv
                 "8 MiB - 256 KiB scratch (or G > 8192); use rmt_memory_write");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(RMT_ECUDA, "cudaGetDevice failed");
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
+  void* addr = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (!addr) {
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess || !addr)
       return fail(RMT_ECUDA, "rmt_memory_write_noalloc: cudaGetSymbolAddress of the scratch array failed");
-    g_noalloc_addr[dev] = p;
+    g_noalloc_addr[dev].store(addr, std::memory_order_release);
   }
-  unsigned char* base = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+  unsigned char* base = static_cast<unsigned char*>(addr);
   Cell* cells = reinterpret_cast<Cell*>(base);
   float* part = reinterpret_cast<float*>(base + kNoAllocCellBytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -46,7 +46,7 @@ constexpr int kRmsWarps = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a) {
-  const Cell c = a.cells[blockIdx.y];
+  const Cell c = load_cell(a.cells, blockIdx.y);
   const int row = blockIdx.x * kRmsWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= a.M) return;
   const float* x = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row) * a.d;
@@ -67,22 +67,28 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a
 }
 
 // Layer-0 input of cell blockIdx.y (row blockIdx.x of M): the segment's tokens from the packed
-// embeddings, then the memory tokens, then zero padding up to M.
+// embeddings, then the memory tokens, then zero padding up to M. An f16 operand copy that
+// overflows is reported in the error word.
 template <typename T>
 __global__ void assemble_kernel(const Cell* cells, const T* emb, const T* mem, float* x, __half* xb, int M, int n_mem,
-                                int d) {
+                                int d, int* err) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
-  const Cell c = cells[blockIdx.y];
+  const Cell c = load_cell(cells, blockIdx.y);
   const int r = blockIdx.x, m = cell_rows(c, M), seg = m - n_mem;
   const T* src = r < seg ? emb + (static_cast<size_t>(c.t0) + r) * d
                          : (r < m ? mem + static_cast<size_t>(r - seg) * d : nullptr);
   const size_t row = (static_cast<size_t>(c.xin) * M + r) * d;
+  float amax = 0.f;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
     const float4 v = src ? Vec4<T>::load(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
     Vec4<float>::store(x + row + k, v);
-    if (xb) Vec4<__half>::store(xb + row + k, v);
+    if (xb) {
+      Vec4<__half>::store(xb + row + k, v);
+      amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
+    }
   }
+  report_f16_range<__half>(amax, err);
 }
 
 // Output rows of cell blockIdx.y: its segment's tokens (row blockIdx.x), cast to T, to the
@@ -91,7 +97,7 @@ template <typename T>
 __global__ void emit_kernel(const Cell* cells, const float* x, T* out, int M, int n_mem, int d) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
-  const Cell c = cells[blockIdx.y];
+  const Cell c = load_cell(cells, blockIdx.y);
   const int r = blockIdx.x;
   if (r >= cell_rows(c, M) - n_mem) return;
   const float* src = x + (static_cast<size_t>(c.xout) * M + r) * d;
@@ -172,15 +178,15 @@ cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
 }
 
 cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
-                            int n_mem, int d, bool bf16, cudaStream_t st) {
+                            int n_mem, int d, bool bf16, int* err, cudaStream_t st) {
   if (d % 4) return cudaErrorInvalidValue;
   if (G <= 0) return cudaSuccess;
   const int threads = d >= 1024 ? 256 : 128;
   if (bf16)
     return launch_pdl(assemble_kernel<__nv_bfloat16>, dim3(M, G), dim3(threads), 0, st, cells,
-                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d);
+                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d, err);
   return launch_pdl(assemble_kernel<float>, dim3(M, G), dim3(threads), 0, st, cells, static_cast<const float*>(emb),
-                    static_cast<const float*>(mem), x, xb, M, n_mem, d);
+                    static_cast<const float*>(mem), x, xb, M, n_mem, d, err);
 }
 
 cudaError_t launch_row_ssq(const float* x, float* ss, int M, int d, int parts, cudaStream_t st) {

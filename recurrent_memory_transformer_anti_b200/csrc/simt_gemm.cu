@@ -17,7 +17,7 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(const SimtGemmArgs a) {
   __shared__ float As[BK][BM];
   __shared__ float Bs[BK][BN];
   __shared__ float Cs[BM][BN + 1];
-  const Cell c = a.cells[blockIdx.z];
+  const Cell c = load_cell(a.cells, blockIdx.z);
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const float* A = a.a + static_cast<size_t>(cell_index(a.a_mode, a.L, c)) * a.M * a.lda;
   const float* W = a.w + static_cast<size_t>(c.l) * a.N * a.K;

@@ -68,7 +68,7 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 // values of the chunk for the residual kinds (loaded by the caller before the TMEM wait).
 template <int EPI, typename OpT>
 __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row, int col, const uint32_t (&r)[32],
-                                           const float4 (&src)[8]) {
+                                           const float4 (&src)[8], float& amax) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = u2f(r[j]);
@@ -79,6 +79,7 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
   } else if constexpr (EPI == kEpiStoreAct) {
     const size_t idx = cell_index(ep.out_mode, a.L, c);
     store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
+    track_amax<OpT>(amax, v);
   } else if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
     const size_t di = cell_index(ep.dst_mode, a.L, c);
     float* dst = ep.x + (di * a.M + row) * ep.ldx + col;
@@ -90,7 +91,10 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
       v[4 * q + 3] += src[q].w;
     }
     store32_f32(dst, v);
-    if constexpr (EPI == kEpiResidCast) store32_16(static_cast<OpT*>(ep.xb) + (di * a.M + row) * ep.ldx + col, v);
+    if constexpr (EPI == kEpiResidCast) {
+      store32_16(static_cast<OpT*>(ep.xb) + (di * a.M + row) * ep.ldx + col, v);
+      track_amax<OpT>(amax, v);
+    }
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
@@ -101,7 +105,8 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
 
 // Epilogue of one tile row for column half `part` (0 or 1) of the tile.
 template <int BN, int EPI, typename OpT>
-__device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0, int part) {
+__device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int n0, int part,
+                                              float& amax) {
   const bool valid = row < a.M;
   const EpiParams& ep = a.ep;
   float rs = 1.f;  // folded RMSNorm scale of this row (RoPE and SwiGLU epilogues)
@@ -148,6 +153,8 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
           }
           store32_16(orow + n0 + h0 + p, x1);
           store32_16(orow + n0 + h0 + half + p, x2);
+          track_amax<OpT>(amax, x1);
+          track_amax<OpT>(amax, x2);
         }
       } else {  // head_dim 32: both halves of the head in one 32-column chunk
         uint32_t r[32];
@@ -168,6 +175,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
             }
           }
           store32_16(orow + n0 + h0, x);
+          track_amax<OpT>(amax, x);
         }
       }
     }
@@ -189,6 +197,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
 #pragma unroll
         for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j]) * rs) * (u2f(up[j]) * rs);
         store32_16(orow + (n0 + b0) / 2 + p, y);
+        track_amax<OpT>(amax, y);
       }
     }
   } else {
@@ -211,7 +220,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         }
       }
       sm100::tmem_wait_ld();
-      if (valid) ss += epi_chunk<EPI, OpT>(a, c, row, n0 + cc * 32, r, src);
+      if (valid) ss += epi_chunk<EPI, OpT>(a, c, row, n0 + cc * 32, r, src, amax);
     }
     if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
       if (ep.ss_out && valid)
@@ -231,7 +240,7 @@ template <int BN, int EPI, typename OpT, int NBUF>
 __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CUtensorMap* tmX, uint32_t tacc, Cell c,
                                                    int rowbase, int n0, int part, int lane, uint8_t* buf,
                                                    uint32_t buf_s, uint32_t rbar, uint32_t& rph,
-                                                   volatile int* abort_flag, uint8_t* xstage) {
+                                                   volatile int* abort_flag, uint8_t* xstage, float& amax) {
   const EpiParams& ep = a.ep;
   if (rowbase >= a.M) return true;  // the whole block lies past the cell
   const int row = rowbase + lane;
@@ -285,6 +294,7 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
       for (int j = 0; j < 32; ++j) ss = fmaf(y[j], y[j], ss);
     }
     if constexpr (EPI == kEpiResidCast) {
+      if (valid) track_amax<OpT>(amax, y);
       // the 16-bit copy: stage the warp's 32 x 32 block, then store it row by row, each
       // instruction covering 8 rows x 64 contiguous bytes
       uint4* mine = reinterpret_cast<uint4*>(xstage + lane * 80);
@@ -326,7 +336,7 @@ template <int BN, typename OpT>
 __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUtensorMap* tmR, uint32_t tacc, Cell c,
                                                   int rowbase, int n0, int part, int lane, const uint8_t* buf,
                                                   uint32_t buf_s, uint32_t rbar, uint32_t& rph,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag, float& amax) {
   const EpiParams& ep = a.ep;
   if (rowbase >= a.M) return true;
   const int row = rowbase + lane;
@@ -384,6 +394,8 @@ __device__ __forceinline__ bool epilogue_rope_tma(const TcGemmArgs& a, const CUt
       }
       store32_16(orow + n0 + h0 + p, x1);
       store32_16(orow + n0 + h0 + half + p, x2);
+      track_amax<OpT>(amax, x1);
+      track_amax<OpT>(amax, x2);
     }
   }
   return true;
@@ -412,7 +424,7 @@ __device__ __forceinline__ void stage_mem_state(const TcGemmArgs& a, Cell c, int
 // both sums over i ascending in fp32.
 template <int BN, typename OpT>
 __device__ __forceinline__ void epilogue_mem_read(const TcGemmArgs& a, uint32_t tacc, Cell c, int row, int part,
-                                                  const float* As, const float* zs) {
+                                                  const float* As, const float* zs, float& amax) {
   const EpiParams& ep = a.ep;
   constexpr int HV = 32;  // output columns per thread (d_v = 64)
   float fq[BN];
@@ -449,6 +461,7 @@ __device__ __forceinline__ void epilogue_mem_read(const TcGemmArgs& a, uint32_t 
   for (int j = 0; j < HV; ++j) acc[j] *= inv;
   const size_t idx = cell_index(ep.out_mode, a.L, c);
   store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + part * HV, acc);
+  track_amax<OpT>(amax, acc);
 }
 
 template <int BN, int EPI, typename OpT, int NBUF>
@@ -512,7 +525,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int g = t / (mt * nt), r = t % (mt * nt);
         const int n_tile = r / mt, m_tile = r % mt;
-        const Cell c = args.cells[g];
+        const Cell c = load_cell(args.cells, g);
         const int a3 = cell_index(args.a_mode, args.L, c);
         for (int kb = 0; kb < kbn; ++kb) {
           if (!sm100::mbar_wait(empty_bar(stage), ph ^ 1u, abort_flag)) {
@@ -593,10 +606,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t rph = 0;
     int acc = 0;
     uint32_t aph = 0;
+    float amax = 0.f;  // largest magnitude stored as an f16 operand
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int g = t / (mt * nt), r = t % (mt * nt);
       const int n_tile = r / mt, m_tile = r % mt;
-      const Cell c = args.cells[g];
+      const Cell c = load_cell(args.cells, g);
       if constexpr (EPI == kEpiMemRead)
         stage_mem_state<BN>(args, c, part, lane, reinterpret_cast<float*>(rbuf),
                             reinterpret_cast<float*>(smem + C::XS_OFF + ew * C::XS_BUF));
@@ -610,14 +624,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
         ok = epilogue_resid_tma<BN, EPI, OpT, NBUF>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part,
                                                     lane, rbuf, rbuf_s, resid_bar(ew), rph, abort_flag,
-                                                    smem + C::XS_OFF + ew * C::XS_BUF);
+                                                    smem + C::XS_OFF + ew * C::XS_BUF, amax);
         if (!ok) {
           if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
           break;
         }
       } else if (EPI == kEpiRope && args.ep.rope_tma) {
         ok = epilogue_rope_tma<BN, OpT>(args, &tmX, tacc, c, m_tile * C::BM + quarter * 32, n_tile * BN, part, lane,
-                                        rbuf, rbuf_s, resid_bar(ew), rph, abort_flag);
+                                        rbuf, rbuf_s, resid_bar(ew), rph, abort_flag, amax);
         if (!ok) {
           if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
           break;
@@ -625,9 +639,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else if constexpr (EPI == kEpiMemRead) {
         epilogue_mem_read<BN, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, part,
                                    reinterpret_cast<const float*>(rbuf),
-                                   reinterpret_cast<const float*>(smem + C::XS_OFF + ew * C::XS_BUF));
+                                   reinterpret_cast<const float*>(smem + C::XS_OFF + ew * C::XS_BUF), amax);
       } else {
-        epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part);
+        epilogue_tile<BN, EPI, OpT>(args, tacc, c, m_tile * C::BM + quarter * 32 + lane, n_tile * BN, part, amax);
       }
       // accumulator read: the MMA issuer reads none of the epilogue's stores, so the arrive is
       // relaxed and does not wait for them
@@ -639,6 +653,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         aph ^= 1u;
       }
     }
+    report_f16_range<OpT>(amax, args.err);
     if (lane == 0) sm100::bulk_wait_all();  // residual stores complete before the CTA leaves
   }
 

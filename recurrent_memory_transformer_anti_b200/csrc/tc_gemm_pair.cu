@@ -111,7 +111,7 @@ __device__ __forceinline__ float row_scale(const float* ss_row, int parts, float
 // from tacc. A step covers 32 columns; columns past cnt (at most 24) are read, not stored.
 template <int EPI, typename OpT>
 __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint32_t tacc, int tok0, int cnt, int f,
-                                              int lane, const float* rs, float* red) {
+                                              int lane, const float* rs, float* red, float& amax) {
   const EpiParams& ep = a.ep;
   const int M = a.M;
   const int lim = min(cnt, M - tok0);  // valid tokens of this warp's range
@@ -140,7 +140,10 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const float y = xs[j] + u2f(r[j]);
         if (j0 + j < lim) {
           dst[static_cast<size_t>(j0 + j) * ep.ldx] = y;
-          if constexpr (EPI == kEpiResidCast) xb[static_cast<size_t>(j0 + j) * ep.ldx] = from_f32<OpT>(y);
+          if constexpr (EPI == kEpiResidCast) {
+            xb[static_cast<size_t>(j0 + j) * ep.ldx] = from_f32<OpT>(y);
+            track_amax<OpT>(amax, y);
+          }
         }
         sq[j] = j0 + j < lim ? y * y : 0.f;
         xs[j] = xn[j];
@@ -163,8 +166,10 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
           const size_t o = o0 + static_cast<size_t>(j0 + j) * ep.ldo;
           if constexpr (EPI == kEpiStoreF32)
             static_cast<float*>(ep.out)[o] = u2f(r[j]);
-          else
+          else {
             static_cast<OpT*>(ep.out)[o] = from_f32<OpT>(u2f(r[j]));
+            track_amax<OpT>(amax, u2f(r[j]));
+          }
         }
       }
     }
@@ -189,7 +194,10 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const float x = u2f(r[j]) * rs[j0 + j];
         const float other = __shfl_xor_sync(0xffffffffu, x, 1);
         const float y = odd ? fmaf(x, cs.x, other * cs.y) : fmaf(x, cs.x, -other * cs.y);
-        if (j0 + j < lim) out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
+        if (j0 + j < lim) {
+          out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
+          track_amax<OpT>(amax, y);
+        }
         cs = make_float2(fmaf(cs.x, step.x, -cs.y * step.y), fmaf(cs.y, step.x, cs.x * step.y));
       }
     }
@@ -212,17 +220,40 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const float got = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[16 + j], 1);
         const float g = odd ? got : v[j], u = odd ? v[16 + j] : got;
         const int t = j0 + (odd ? 16 : 0) + j;
-        if (t < lim) out[static_cast<size_t>(t) * ep.ldo] = from_f32<OpT>(silu_fast(g) * u);
+        if (t < lim) {
+          const float y = silu_fast(g) * u;
+          out[static_cast<size_t>(t) * ep.ldo] = from_f32<OpT>(y);
+          track_amax<OpT>(amax, y);
+        }
       }
     }
   }
 }
 
-template <int EPI, typename OpT>
+// Chained projections. One launch runs one to three projections ("phases") of the same cells
+// in order -- in the forward: the O projection, gate/up, then down. Tiles are numbered phase by
+// phase (cell, feature pair, token tile within a phase) and each CTA pair takes its tiles in
+// increasing order, so a pair reaches its tiles of phase p only after all of its tiles of
+// phase p-1. A tile of phase p >= 1 for (cell g, token tile tt) reads what phase p-1 wrote for
+// the same tokens over all of its feature pairs (residual rows and RMSNorm statistics, or the
+// SwiGLU output): its loads and its epilogue wait (bounded) until a counter in global memory
+// shows that every one of those tiles has been stored. Each epilogue warp adds 1 to the
+// counter of (phase, g, tt) with a release once it has stored its share of a tile and made the
+// stores visible to the tensor-memory-access proxy; waiters read it with acquire loads. No wait closes a cycle: a tile waits only on tiles of the previous phase, which every
+// pair reaches before any of its own tiles of a later phase, and the grid never holds more
+// pairs than can be resident together. The launch ends as soon as the last tile is stored, so
+// the drain and refill between the projections of a diagonal disappear with their launches.
+constexpr int kNoEpi = -1;  // an unused phase slot
+constexpr unsigned kSignalsPerTile = 2 * PairCfg::EPI_WARPS;  // one per epilogue warp of each CTA of the pair
+
+template <int E0, int E1, int E2, typename OpT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
-    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                        const TcGemmArgs args) {
+    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
+                        const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX1,
+                        const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmX2,
+                        const PairChainArgs args) {
   using C = PairCfg;
+  constexpr int NP = E1 == kNoEpi ? 1 : (E2 == kNoEpi ? 2 : 3);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = sm100::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -236,7 +267,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * C::MAX_STAGES + 6);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int M = args.M;
+  const TcGemmArgs& a0 = args.ph[0];
+  const int M = a0.M, G = a0.G;
   const int NT = pair_token_tile(M);
   const int STAGES = C::stages(NT);
   const uint32_t BLK = static_cast<uint32_t>(C::block_bytes(NT));
@@ -260,8 +292,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     sm100::fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) {
-    sm100::tma_prefetch_desc(&tmW);
-    sm100::tma_prefetch_desc(&tmX);
+    sm100::tma_prefetch_desc(&tmW0);
+    sm100::tma_prefetch_desc(&tmX0);
+    if (NP > 1) {
+      sm100::tma_prefetch_desc(&tmW1);
+      sm100::tma_prefetch_desc(&tmX1);
+    }
+    if (NP > 2) {
+      sm100::tma_prefetch_desc(&tmW2);
+      sm100::tma_prefetch_desc(&tmX2);
+    }
   }
   if (warp == 1) sm100::tmem_alloc_pair(sm100::smem_u32(tmem_slot), C::TMEM_COLS);
   sm100::tc_fence_before();
@@ -270,12 +310,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_trigger();  // this CTA holds its TMEM: the next kernel may be scheduled
   pdl_wait();     // operands and residuals come from the previous kernels of the stream
+  if (NP > 1 && blockIdx.x == 0) {
+    // the next chained launch uses the other parity's counters: this launch started after the
+    // one that used them ended, and the next one starts after this one ends
+    unsigned* next = args.ctr + static_cast<size_t>(args.parity ^ 1) * (kMaxPhases - 1) * args.ctr_len;
+    for (int i = threadIdx.x; i < (kMaxPhases - 1) * args.ctr_len; i += blockDim.x) next[i] = 0u;
+  }
 
   const int ntt = (M + NT - 1) / NT;
-  const int npair = args.N / 256;
-  const int kblk = args.K / C::BK;  // 64-column blocks
-  const int kst = (kblk + 1) / 2;   // ring stages per tile (the last may hold one block)
-  const int tiles = args.G * npair * ntt;
+  // tiles of the phases: [0, t1) phase 0, [t1, t2) phase 1, [t2, tiles) phase 2
+  const int np0 = a0.N / 256, np1 = NP > 1 ? args.ph[1].N / 256 : 0, np2 = NP > 2 ? args.ph[2].N / 256 : 0;
+  const int t1 = G * np0 * ntt, t2 = t1 + G * np1 * ntt, tiles = t2 + G * np2 * ntt;
+  auto npair_of = [&](int p) { return p == 0 ? np0 : (p == 1 ? np1 : np2); };
+  auto k_of = [&](int p) { return p == 0 ? a0.K : (p == 1 ? args.ph[1].K : args.ph[2].K); };
+  auto decode = [&](int t, int& p, int& g, int& fp, int& tt) {
+    p = (NP > 1 && t >= t1) ? ((NP > 2 && t >= t2) ? 2 : 1) : 0;
+    const int r0 = t - (p == 0 ? 0 : (p == 1 ? t1 : t2)), per = npair_of(p) * ntt;
+    g = r0 / per;
+    const int r = r0 % per;
+    fp = r / ntt;
+    tt = r % ntt;
+  };
+  // completed CTA halves of phase p's tiles of (cell g, token tile tt)
+  auto counter = [&](int p, int g, int tt) {
+    return args.ctr + (static_cast<size_t>(args.parity) * (kMaxPhases - 1) + p) * args.ctr_len + g * ntt + tt;
+  };
   const int cl = static_cast<int>(sm100::cluster_id_x()), ncl = static_cast<int>(sm100::cluster_count_x());
   // tokens of token tile tt (the last one rounded up to 16; rows past M read as zeros)
   auto tile_tokens = [&](int tt) {
@@ -291,10 +350,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       bool ok = true;
       auto acquire = [&]() { return sm100::mbar_wait(empty_bar(stage), ph ^ 1u, abort_flag); };
       for (int t = cl; t < tiles && ok; t += ncl) {
-        const int g = t / (npair * ntt), r = t % (npair * ntt);
-        const int fp = r / ntt, tt = r % ntt;
-        const Cell c = args.cells[g];
-        const int a3 = cell_index(args.a_mode, args.L, c);
+        int p, g, fp, tt;
+        decode(t, p, g, fp, tt);
+        const CUtensorMap* tw = p == 0 ? &tmW0 : (p == 1 ? &tmW1 : &tmW2);
+        const CUtensorMap* tx = p == 0 ? &tmX0 : (p == 1 ? &tmX1 : &tmX2);
+        const IndexMode amode = p == 0 ? a0.a_mode : (p == 1 ? args.ph[1].a_mode : args.ph[2].a_mode);
+        const int kblk = k_of(p) / C::BK;  // 64-column blocks
+        const int kst = (kblk + 1) / 2;    // ring stages per tile (the last may hold one block)
+        const Cell c = load_cell(a0.cells, g);
+        const int a3 = cell_index(amode, a0.L, c);
+        if (NP > 1 && p > 0) {
+          // every tile of the previous phase for these tokens is stored
+          if (!sm100::counter_wait(counter(p - 1, g, tt), kSignalsPerTile * static_cast<unsigned>(npair_of(p - 1)),
+                                   abort_flag)) {
+            ok = false;
+            break;
+          }
+          sm100::fence_proxy_async_global();
+        }
         const int wrow = fp * 256 + static_cast<int>(rank) * C::FM;
         const int xrow = tt * NT + static_cast<int>(rank) * (tile_tokens(tt) / 2);
         for (int ks = 0; ks < kst; ++ks) {
@@ -307,8 +380,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           const uint32_t sa = ring + static_cast<uint32_t>(stage) * 2u * BLK;
           const uint32_t fb = sm100::mapa_shared(full_bar(stage), 0);
           for (int b = 0; b < nb; ++b) {
-            sm100::tma_load_3d_pair(sa + b * BLK, &tmW, (2 * ks + b) * C::BK, wrow, c.l, fb);
-            sm100::tma_load_3d_pair(sa + b * BLK + C::W_BYTES, &tmX, (2 * ks + b) * C::BK, xrow, a3, fb);
+            sm100::tma_load_3d_pair(sa + b * BLK, tw, (2 * ks + b) * C::BK, wrow, c.l, fb);
+            sm100::tma_load_3d_pair(sa + b * BLK + C::W_BYTES, tx, (2 * ks + b) * C::BK, xrow, a3, fb);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -326,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
       }
       if (!ok) {
-        if (args.err) atomicOr(args.err, kErrTimeoutProducer);
+        if (a0.err) atomicOr(a0.err, kErrTimeoutProducer);
         // copies already issued complete on the even CTA's barriers, which this CTA cannot
         // wait on: give them a millisecond to land before shared memory can be released
         const uint64_t t0 = sm100::global_timer_ns();
@@ -341,7 +414,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       uint32_t ph = 0, aph = 0;
       bool ok = true;
       for (int t = cl; t < tiles && ok; t += ncl) {
-        const int tt = (t % (npair * ntt)) % ntt;
+        int p, g, fp, tt;
+        decode(t, p, g, fp, tt);
+        const int kblk = k_of(p) / C::BK, kst = (kblk + 1) / 2;
         const uint32_t idesc = idesc0 | (static_cast<uint32_t>(tile_tokens(tt) >> 3) << 17);
         if (!sm100::mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) {
           ok = false;
@@ -378,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
       }
       if (!ok) {
-        if (args.err) atomicOr(args.err, kErrTimeoutMma);
+        if (a0.err) atomicOr(a0.err, kErrTimeoutMma);
         sm100::mma_commit_pair(sm100::mapa_shared(drain_bar, 0));
         sm100::mbar_wait_drain(drain_bar, 0);
       }
@@ -393,22 +468,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     float* rs_all = reinterpret_cast<float*>(smem + C::RS_OFF);
     const uint32_t tempty_lead0 = sm100::mapa_shared(tempty_bar(0), 0);
     const uint32_t tempty_lead1 = sm100::mapa_shared(tempty_bar(1), 0);
-    const EpiParams& ep = args.ep;
     int acc = 0;
     uint32_t aph = 0, wph = 0;
+    float amax = 0.f;  // largest magnitude stored as an f16 operand
+    bool ok = true;
     // the four warps of this warpgroup meet (bounded); false on a timeout
     auto wg_sync = [&]() {
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(wg_bar(wg));
-      const bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(wg_bar(wg), wph, abort_flag));
+      const bool r = __all_sync(0xffffffffu, sm100::mbar_wait(wg_bar(wg), wph, abort_flag));
       wph ^= 1u;
-      if (!ok && lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
-      return ok;
+      if (!r && lane == 0 && a0.err) atomicOr(a0.err, kErrTimeoutEpilogue);
+      return r;
     };
-    for (int t = cl; t < tiles; t += ncl) {
-      const int g = t / (npair * ntt), r = t % (npair * ntt);
-      const int fp = r / ntt, tt = r % ntt;
-      const Cell c = args.cells[g];
+    // one tile of phase epilogue kind EPI with that phase's arguments; the next tile's cell and
+    // position (gn < 0: none in this phase) for the residual epilogue's L2 warm-up
+    auto epi_tile = [&](auto epi_kind, const TcGemmArgs& a, const Cell& c, int fp, int tt, int gn, int fpn,
+                        int ttn) -> bool {
+      constexpr int EPI = decltype(epi_kind)::value;
+      const EpiParams& ep = a.ep;
       const int nt = tile_tokens(tt), cnt = nt / 2;
       const int tok0 = tt * NT + wg * cnt;
       const int fcta = fp * 256 + static_cast<int>(rank) * C::FM;  // first feature of this CTA
@@ -423,32 +501,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                       ? row_scale(ep.ss_in + (static_cast<size_t>(c.k) * M + tok) * ep.ss_parts, ep.ss_parts, ep.inv_d,
                                   ep.rms_eps)
                       : 1.f;
-        if (!wg_sync()) break;
+        if (!wg_sync()) return false;
       }
       if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
         // warm L2 with the residual rows of this CTA's next tile (its rows of 128 features)
-        const int tn = t + ncl;
-        if (tn < tiles) {
-          const int gn = tn / (npair * ntt), rn = tn % (npair * ntt);
-          const int fpn = rn / ntt, ttn = rn % ntt;
-          const Cell cn = args.cells[gn];
+        if (gn >= 0) {
+          const Cell cn = load_cell(a.cells, gn);
           const int k = ew * 32 + lane, ntn = tile_tokens(ttn);
           if (k < ntn && ttn * NT + k < M) {
-            const size_t si = cell_index(ep.src_mode, args.L, cn);
+            const size_t si = cell_index(ep.src_mode, a.L, cn);
             sm100::prefetch_l2_bulk(ep.x + (si * M + ttn * NT + k) * ep.ldx + fpn * 256 + rank * C::FM, C::FM * 4);
           }
         }
       }
-      bool ok = __all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag));
-      if (!ok) {
-        if (lane == 0 && args.err) atomicOr(args.err, kErrTimeoutEpilogue);
-        break;
+      if (!__all_sync(0xffffffffu, sm100::mbar_wait(tfull_bar(acc), aph, abort_flag))) {
+        if (lane == 0 && a0.err) atomicOr(a0.err, kErrTimeoutEpilogue);
+        return false;
       }
       sm100::tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(acc * C::ACC_COLS + wg * cnt);
       float* red = red_all + ((acc * 2 + wg) * 4 + quarter) * 128;
-      pair_epilogue<EPI, OpT>(args, c, tacc, tok0, cnt, f, lane, rs, red);
+      pair_epilogue<EPI, OpT>(a, c, tacc, tok0, cnt, f, lane, rs, red, amax);
       // accumulator drained (every lane's tcgen05.ld waited for): release it to the even CTA's
       // MMA issuer. The issuer reads none of this warp's global stores, so the arrive is
       // relaxed and does not wait for them to drain.
@@ -459,7 +533,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (ep.ss_out) {
           // the four warps of this warpgroup hold 32-feature sums of the same tokens: combine
           // them in quarter order into one partial per (token, 128-feature block)
-          if (!wg_sync()) break;
+          if (!wg_sync()) return false;
           const float* rb = red_all + (acc * 2 + wg) * 4 * 128;
           const int k = wq * 32 + lane;
           const int tok = tok0 + k;
@@ -472,7 +546,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         acc = 0;
         aph ^= 1u;
       }
+      return true;
+    };
+    for (int t = cl; t < tiles && ok; t += ncl) {
+      int p, g, fp, tt;
+      decode(t, p, g, fp, tt);
+      const Cell c = load_cell(a0.cells, g);
+      int gn = -1, fpn = 0, ttn = 0;
+      if (t + ncl < tiles) {
+        int pn;
+        decode(t + ncl, pn, gn, fpn, ttn);
+        if (pn != p) gn = -1;
+      }
+      if (NP > 1 && p > 0) {
+        // the stores of the previous phase this tile's epilogue reads (residual rows, RMSNorm
+        // statistics) are complete: the producer saw the same counter, and this acquire makes
+        // them visible to this warp as well
+        bool r = true;
+        if (lane == 0)
+          r = sm100::counter_wait(counter(p - 1, g, tt), kSignalsPerTile * static_cast<unsigned>(npair_of(p - 1)),
+                                  abort_flag);
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, r ? 1 : 0, 0)) {
+          if (lane == 0 && a0.err) atomicOr(a0.err, kErrTimeoutEpilogue);
+          ok = false;
+          break;
+        }
+      }
+      if (p == 0) {
+        ok = epi_tile(std::integral_constant<int, E0>{}, args.ph[0], c, fp, tt, gn, fpn, ttn);
+      } else if (p == 1) {
+        if constexpr (NP > 1) ok = epi_tile(std::integral_constant<int, E1>{}, args.ph[1], c, fp, tt, gn, fpn, ttn);
+      } else {
+        if constexpr (NP > 2) ok = epi_tile(std::integral_constant<int, E2>{}, args.ph[2], c, fp, tt, gn, fpn, ttn);
+      }
+      if (!ok) break;
+      if (NP > 1 && p < NP - 1) {
+        // this warp's share of the tile is stored: publish it to the next phase's tiles of the
+        // same tokens (one release add per warp, after the warp's stores are ordered before it
+        // and made visible to the tensor-memory-access proxy)
+        sm100::fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) sm100::counter_release_add(counter(p, g, tt), 1u);
+      }
     }
+    report_f16_range<OpT>(amax, a0.err);
   }
 
   sm100::tc_fence_before();
@@ -503,37 +621,45 @@ int max_pair_clusters(const void* fn) {
   return cached[dev];
 }
 
-template <int EPI, typename OpT>
-cudaError_t launch_pair_epi(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, cudaStream_t st) {
+template <int E0, int E1, int E2, typename OpT>
+cudaError_t launch_pair_chain_t(const CUtensorMap* tw, const CUtensorMap* tx, const PairChainArgs& args,
+                                cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  const void* fn = reinterpret_cast<const void*>(tc_pair_gemm_kernel<EPI, OpT>);
+  const void* fn = reinterpret_cast<const void*>(tc_pair_gemm_kernel<E0, E1, E2, OpT>);
   if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int NT = pair_token_tile(args.M);
-  const long tiles = static_cast<long>(args.G) * (args.N / 256) * ((args.M + NT - 1) / NT);
+  const TcGemmArgs& a0 = args.ph[0];
+  const int NT = pair_token_tile(a0.M), ntt = (a0.M + NT - 1) / NT;
+  long tiles = 0;
+  for (int p = 0; p < args.nphase; ++p) tiles += static_cast<long>(a0.G) * (args.ph[p].N / 256) * ntt;
   if (tiles <= 0) return cudaSuccess;
-  const int maxc = max_pair_clusters(fn);
+  const int maxc = max_pair_clusters(fn);  // every pair resident at once (the chained waits rely on it)
   const int clusters = static_cast<int>(tiles < maxc ? tiles : maxc);
-  const cudaError_t e = launch_pdl(tc_pair_gemm_kernel<EPI, OpT>, dim3(2 * clusters), dim3(PairCfg::THREADS),
-                                   PairCfg::SMEM_BYTES, st, tw, tx, args);
+  const int np = args.nphase;
+  const cudaError_t e = launch_pdl(tc_pair_gemm_kernel<E0, E1, E2, OpT>, dim3(2 * clusters), dim3(PairCfg::THREADS),
+                                   PairCfg::SMEM_BYTES, st, tw[0], tx[0], tw[np > 1 ? 1 : 0], tx[np > 1 ? 1 : 0],
+                                   tw[np > 2 ? 2 : 0], tx[np > 2 ? 2 : 0], args);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <typename OpT>
 cudaError_t launch_pair_op(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, cudaStream_t st) {
+  PairChainArgs c{};
+  c.ph[0] = args;
+  c.nphase = 1;
   switch (args.epi) {
-    case kEpiStoreF32: return launch_pair_epi<kEpiStoreF32, OpT>(tw, tx, args, st);
-    case kEpiStoreAct: return launch_pair_epi<kEpiStoreAct, OpT>(tw, tx, args, st);
-    case kEpiResidCast: return launch_pair_epi<kEpiResidCast, OpT>(tw, tx, args, st);
-    case kEpiRope: return launch_pair_epi<kEpiRope, OpT>(tw, tx, args, st);
-    case kEpiSwiGLU: return launch_pair_epi<kEpiSwiGLU, OpT>(tw, tx, args, st);
+    case kEpiStoreF32: return launch_pair_chain_t<kEpiStoreF32, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
+    case kEpiStoreAct: return launch_pair_chain_t<kEpiStoreAct, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
+    case kEpiResidCast: return launch_pair_chain_t<kEpiResidCast, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
+    case kEpiRope: return launch_pair_chain_t<kEpiRope, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
+    case kEpiSwiGLU: return launch_pair_chain_t<kEpiSwiGLU, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -551,6 +677,22 @@ cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, co
                                 cudaStream_t st) {
   if (!tc_pair_supported(args.M, args.N, args.K, args.epi, args.ep.head_dim)) return cudaErrorInvalidValue;
   return f16 ? launch_pair_op<__half>(tw, tx, args, st) : launch_pair_op<__nv_bfloat16>(tw, tx, args, st);
+}
+
+cudaError_t launch_tc_pair_chain_o_mlp(const CUtensorMap* tw, const CUtensorMap* tx, const PairChainArgs& args,
+                                       cudaStream_t st) {
+  const TcGemmArgs* a = args.ph;
+  if (args.nphase != 3 || !args.ctr || args.ctr_len <= 0 || a[0].epi != kEpiResidCast || a[1].epi != kEpiSwiGLU ||
+      a[2].epi != kEpiResidCast)
+    return cudaErrorInvalidValue;
+  for (int p = 0; p < 3; ++p) {
+    if (!tc_pair_supported(a[p].M, a[p].N, a[p].K, a[p].epi, a[p].ep.head_dim) || a[p].M != a[0].M ||
+        a[p].G != a[0].G || a[p].cells != a[0].cells)
+      return cudaErrorInvalidValue;
+  }
+  const int NT = pair_token_tile(a[0].M);
+  if (static_cast<long>(a[0].G) * ((a[0].M + NT - 1) / NT) > args.ctr_len) return cudaErrorInvalidValue;
+  return launch_pair_chain_t<kEpiResidCast, kEpiSwiGLU, kEpiResidCast, __half>(tw, tx, args, st);
 }
 
 }  // namespace rmt

@@ -2,7 +2,9 @@
 
 Every step of the ARMT prefill runs in the library's CUDA kernels. Arrays may be torch
 tensors (device or host) or numpy arrays (host); pointers are passed through unchanged.
-If librmt.so is missing this module raises at import: there is no fallback path.
+If librmt.so is missing this module raises at import: there is no fallback path. The
+environment variable RMT_LIBRARY selects another build of the same ABI (librmt_debug.so,
+the in-kernel bounds-checking build).
 """
 from __future__ import annotations
 
@@ -12,18 +14,21 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librmt.so")
+LIB_PATH = os.environ.get("RMT_LIBRARY") or os.path.join(_HERE, "librmt.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "librmt_debug.so")
 
-RMT_OK, RMT_EINVAL, RMT_ENOMEM, RMT_ECUDA, RMT_ETIMEOUT, RMT_ESTATE = range(6)
+RMT_OK, RMT_EINVAL, RMT_ENOMEM, RMT_ECUDA, RMT_ETIMEOUT, RMT_ESTATE, RMT_ERANGE, RMT_EDEBUG = range(8)
 RMT_DIAGONAL, RMT_SEQUENTIAL = 0, 1
 RMT_F32, RMT_BF16 = 0, 1
 SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
 DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16}
-STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE"}
+STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE",
+                6: "RMT_ERANGE", 7: "RMT_EDEBUG"}
 
 EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "rmt_forward_batch",
             "rmt_full_attention_forward", "rmt_schedule_table",
             "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync", "rmt_wait_selftest",
+            "rmt_bounds_selftest",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
             "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
             "rmt_probe_read")
@@ -72,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "rmt_get_trace": [vp, p32, sz],
         "rmt_sync": [vp, vp],
         "rmt_wait_selftest": [ctypes.c_uint32, vp],
+        "rmt_bounds_selftest": [vp],
         "rmt_destroy": [vp],
         "rmt_grouped_gemm_bf16": [vp, vp, vp, i32, i32, i32, i32, ctypes.c_int, vp],
         "rmt_attention": [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp],
@@ -245,6 +251,10 @@ def rmt_sync(h: Handle | None, stream=None) -> None:
 
 def rmt_wait_selftest(limit_us: int, stream=None) -> None:
     _check(_lib.rmt_wait_selftest(int(limit_us), _stream(stream)), "rmt_wait_selftest")
+
+
+def rmt_bounds_selftest(stream=None) -> None:
+    _check(_lib.rmt_bounds_selftest(_stream(stream)), "rmt_bounds_selftest")
 
 
 def rmt_destroy(h: Handle) -> None:

@@ -19,13 +19,22 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(rmt_[a-z0-9_]+)\s*\(", text)))
 
 
-def test_every_declared_symbol_is_exported():
+@pytest.mark.parametrize("which", ["release", "debug"])
+def test_every_declared_symbol_is_exported(which):
     names = declared_functions()
     assert len(names) >= 13
-    lib = ctypes.CDLL(rmt.LIB_PATH)
+    path = rmt.LIB_PATH if which == "release" else rmt.DEBUG_LIB_PATH
+    assert os.path.exists(path), path
+    lib = ctypes.CDLL(path)
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(rmt.EXPORTED)
+
+
+def test_release_library_has_no_bounds_selftest():
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_bounds_selftest()
+    assert ex.value.status == rmt.RMT_ESTATE
 
 
 @pytest.mark.parametrize("schedule", ["diagonal", "sequential"])

@@ -8,6 +8,8 @@
 * The device trace of executed cells equals the schedule, which equals the oracle's
   enumeration.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -21,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 F32_TOL = 1e-4
 BF16_TOL = 2e-2
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 @pytest.fixture(scope="module")
@@ -153,56 +156,74 @@ def test_small_bf16_diagonal_equals_sequential_bitwise(small_bf16):
         np.testing.assert_array_equal(a, b)
 
 
-@pytest.mark.parametrize("S", [32, 128])
-def test_1b_shape_bench_configuration(cuda_ok, S):
-    """The LLaMA-1B-shaped workloads: 32 segments (32,768 tokens) and the 131,072 tokens the
-    bench times (16 layers x 128 segments of 1024 + 16 tokens, bf16). The oracle cannot run
-    them in seconds, so:
-      - the first four segments of the full run equal a 4-segment run bit for bit (a
-        segment's output never depends on later segments), and the 4-segment run -- hidden
-        states and the memory state after 4 segments -- matches the oracle within the bf16
-        tolerance;
-      - DIAGONAL equals SEQUENTIAL bit for bit at the full size."""
+# ------------------------------------------- the full-length workloads against oracle goldens
+#
+# tests/golden/long_*.npz hold the fp32 oracle's results for the bench's workloads, written by
+# tests/golden/make_long_goldens.py (which calls only the oracle and the input generators):
+# every layer's A and z after the last segment, and the last layer's hidden states at 40
+# sampled rows of the first, middle and last segments.
+
+
+def _golden(name):
+    return np.load(os.path.join(GOLDEN, f"long_{name}.npz"))
+
+
+def _check_golden(got, g, cfg):
+    out, A, z = got
+    n = int(g["n_segments"])
+    assert str(g["config"]) in CONFIGS and CONFIGS[str(g["config"])] == cfg
+    assert out.shape == (n * cfg.seg_len, cfg.d_model)
+    errs = {"hidden": normwise(out[g["rows"]], g["hidden"]), "A": normwise(A, g["A"]), "z": normwise(z, g["z"])}
+    per_layer_A = [normwise(A[l], g["A"][l]) for l in range(cfg.n_layers)]
+    assert max(errs.values()) < BF16_TOL, (errs, per_layer_A)
+    assert np.isfinite(out).all()
+    return errs
+
+
+@pytest.fixture(scope="module")
+def model_1b(cuda_ok):
     cfg = CONFIGS["1b"]
     w, h = build(cfg)
-    P = 4
+    yield cfg, w, h
+    rmt.rmt_destroy(h)
+
+
+def test_1b_131k_matches_oracle_golden(model_1b):
+    """The bench's workload: the LLaMA-1B-shaped ARMT over 128 segments of 1024 + 16 tokens
+    (131,072 tokens, bf16). The hidden states at the sampled rows of segments 0, 64 and 127
+    and every layer's final A and z match the oracle within the bf16 tolerance; SEQUENTIAL
+    gives the bits of DIAGONAL; and the first 32 segments, run alone, give the same bits and
+    match the oracle's 32-segment results (the 32,768-token workload)."""
+    cfg, w, h = model_1b
+    S, P = 128, 32
     emb = embeddings(cfg, S)
     full_d = forward(h, cfg, emb, S, "diagonal")
+    _check_golden(full_d, _golden("1b_s128"), cfg)
     full_s = forward(h, cfg, emb, S, "sequential")
     for a, b in zip(full_d, full_s):
         np.testing.assert_array_equal(a, b)
+    del full_s
     part = forward(h, cfg, emb[:P * cfg.seg_len], P, "diagonal")
     np.testing.assert_array_equal(full_d[0][:P * cfg.seg_len], part[0])
-    ref = armt.forward(cfg, w, emb[:P * cfg.seg_len], P, dtype=np.float32)
-    for g, r, name in zip(part, ref, ("out", "A", "z")):
-        assert normwise(g, r) < BF16_TOL, name
-    assert np.isfinite(full_d[0]).all() and np.isfinite(full_d[1]).all()
-    rmt.rmt_destroy(h)
+    _check_golden(part, _golden("1b_s32"), cfg)
 
 
-@pytest.mark.parametrize("name", ["3b-512", "3b-2048"])
-def test_3b_shape_full_size(cuda_ok, name):
+@pytest.mark.parametrize("name,S", [("3b-512", 256), ("3b-2048", 64)])
+def test_3b_131k_matches_oracle_golden(cuda_ok, name, S):
     """The LLaMA-3B-shaped workloads at 131,072 tokens (28 layers, d 3072, 24/8 heads of 128,
     d_k = d_v = 128, segments of 512 or 2048 + 16 tokens; the 2064-row cells end in a ragged
-    token tile). DIAGONAL equals SEQUENTIAL bit for bit at the full size; the first segment
-    of the full run equals a one-segment run bit for bit, and that run (hidden states and the
-    28 layers' memory states) matches the oracle within the bf16 tolerance."""
+    token tile): the sampled hidden rows and all 28 layers' final A and z match the oracle
+    within the bf16 tolerance, and SEQUENTIAL gives the bits of DIAGONAL."""
     cfg = CONFIGS[name]
     w, h = build(cfg)
-    S = 131072 // cfg.seg_len
+    del w
     emb = embeddings(cfg, S)
     full_d = forward(h, cfg, emb, S, "diagonal")
+    _check_golden(full_d, _golden(f"{name}_s{S}"), cfg)
     full_s = forward(h, cfg, emb, S, "sequential")
+    rmt.rmt_destroy(h)
     for a, b in zip(full_d, full_s):
         np.testing.assert_array_equal(a, b)
-    assert np.isfinite(full_d[0]).all() and np.isfinite(full_d[1]).all()
-    del full_s
-    part = forward(h, cfg, emb[:cfg.seg_len], 1, "diagonal")
-    np.testing.assert_array_equal(full_d[0][:cfg.seg_len], part[0])
-    rmt.rmt_destroy(h)
-    ref = armt.forward(cfg, w, emb[:cfg.seg_len], 1, dtype=np.float32)
-    for g, r, what in zip(part, ref, ("out", "A", "z")):
-        assert normwise(g, r) < BF16_TOL, what
 
 
 @pytest.mark.parametrize("name,S,tol", [("tiny", 3, F32_TOL), ("small-bf16", 3, BF16_TOL)])
@@ -222,6 +243,53 @@ def test_random_rmsnorm_gains_match_oracle(cuda_ok, name, S, tol):
     for g_, r, what in zip(got, ref, ("out", "A", "z")):
         assert normwise(g_, r) < tol, what
     rmt.rmt_destroy(h)
+
+
+@pytest.mark.parametrize("name", ["small-bf16", "mixed-tiles"])
+def test_large_magnitudes_within_f16_range_match_oracle(cuda_ok, name):
+    """bf16 mode keeps its tensor-core operands in f16 (largest finite value 65504): the
+    residual stream's operand copy, q/k/v, the SwiGLU output and the memory read-out.
+    Embeddings scaled to magnitudes of about 10^4 and RMSNorm gains between 0 and 8 keep
+    every such operand in range; the result still matches the oracle and no overflow is
+    reported. Both the CTA-pair and the single-CTA GEMM epilogues store operands here."""
+    import dataclasses
+
+    from armt_synthetic import make_weights, round_to_bf16
+    cfg = CONFIGS["small-bf16"]
+    if name != "small-bf16":
+        cfg = dataclasses.replace(cfg, **MIXED_CONFIGS[name])
+    w = make_weights(cfg, seed=21)
+    rng = np.random.default_rng(22)
+    for key in ("g_attn", "g_mlp"):
+        w[key] = [round_to_bf16(np.abs(1 + 2 * rng.standard_normal(cfg.d_model)).astype(np.float32))
+                  for _ in range(cfg.n_layers)]
+    w, h = build(cfg, weights=w)
+    S = 3
+    emb = round_to_bf16(embeddings(cfg, S, seed=23) * np.float32(3000))
+    assert 9e3 < np.abs(emb).max() < 3e4
+    got = forward(h, cfg, emb, S, "diagonal")
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32)
+    for g_, r, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g_, r) < BF16_TOL, what
+    rmt.rmt_destroy(h)
+
+
+def test_f16_operand_overflow_is_reported(small_bf16):
+    """Embeddings of magnitude 10^5 overflow the f16 operand copy of the residual stream:
+    rmt_sync reports RMT_ERANGE (no fault; the infinities only spoil the outputs), and the
+    handle's next forward gives the bits it gave before."""
+    cfg, w, h = small_bf16
+    S = 2
+    emb = embeddings(cfg, S, seed=24)
+    before = forward(h, cfg, emb, S, "diagonal")
+    big = rmt.storage(emb * np.float32(1e5), cfg.dtype, device="cuda")
+    rmt.rmt_forward(h, big, S, "diagonal", torch.empty_like(big))
+    with pytest.raises(rmt.RmtError) as ex:
+        rmt.rmt_sync(h)
+    assert ex.value.status == rmt.RMT_ERANGE
+    after = forward(h, cfg, emb, S, "diagonal")
+    for a, b in zip(before, after):
+        np.testing.assert_array_equal(a, b)
 
 
 MIXED_CONFIGS = {
@@ -461,20 +529,18 @@ def test_full_attention_argument_errors(tiny, cuda_ok):
     rmt.rmt_destroy(h2)
 
 
-def test_full_attention_1b_at_131k(cuda_ok):
+def test_full_attention_1b_at_131k(model_1b):
     """The comparison model at the bench's size: LLaMA-1B shape, 131,072 tokens, one causal
     segment. The oracle cannot run it in seconds, so: the first 1024 rows equal a 1024-token
     run bit for bit (a row never depends on later tokens, and both runs tile tokens by 256),
     and that run matches the oracle within the bf16 tolerance."""
-    cfg = CONFIGS["1b"]
-    w, h = build(cfg)
+    cfg, w, h = model_1b
     T, P = 131072, 1024
     emb = embeddings(cfg, T // cfg.seg_len)
     full = _full(h, cfg, emb)
     assert np.isfinite(full).all()
     part = _full(h, cfg, emb[:P])
     np.testing.assert_array_equal(full[:P], part)
-    rmt.rmt_destroy(h)
     ref = armt.full_attention_forward(cfg, w, emb[:P], dtype=np.float32)
     assert normwise(part, ref) < BF16_TOL
 

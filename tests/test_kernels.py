@@ -96,9 +96,14 @@ def test_attention_matches_oracle(dtype, G, M, H, Hkv, dh):
 
 # ------------------------------------------------------------------------------ memory
 
+# 16-bit outputs with d_k of 64 or 128 take the tcgen05 read (persistent CTAs over 128-row
+# tiles, crossing cells: G = 300 puts several cells and a ragged tile in every CTA's range),
+# other d_k the mma.sync read; fp32 outputs the fp32 read
 @pytest.mark.parametrize("dtype,G,M,dk,dv", [("f32", 3, 1040, 64, 64), ("bf16", 3, 1040, 64, 64),
                                              ("f32", 2, 72, 32, 32), ("f32", 2, 77, 128, 128),
-                                             ("f32", 2, 50, 32, 96), ("bf16", 4, 130, 128, 64)])
+                                             ("f32", 2, 50, 32, 96), ("bf16", 4, 130, 128, 64),
+                                             ("bf16", 2, 2064, 128, 128), ("bf16", 300, 130, 64, 32),
+                                             ("bf16", 1, 1, 64, 64), ("bf16", 2, 300, 32, 64), ("bf16", 3, 77, 96, 96)])
 def test_memory_read_matches_oracle(dtype, G, M, dk, dv):
     r = rng(300 + M + dk)
     q = r.standard_normal((G, M, dk), dtype=np.float32)
@@ -114,8 +119,12 @@ def test_memory_read_matches_oracle(dtype, G, M, dk, dv):
         assert normwise(got[g], ref) < (8e-3 if dtype == "bf16" else 1e-5)
 
 
+# a launch picks its kernel from G: column slices of 16 (a cluster of d_v / 16 CTAs per cell)
+# for few cells, 32 or 64 for more, and the streaming kernel (persistent CTAs, one cell ahead
+# in shared memory) for at least four cells per SM; the sums run in the same order in all
 @pytest.mark.parametrize("G,n,dk,dv", [(5, 16, 64, 64), (3, 8, 32, 32), (2, 16, 128, 128), (2, 64, 64, 32),
-                                       (1, 1, 32, 64)])
+                                       (1, 1, 32, 64), (200, 16, 64, 64), (300, 16, 64, 64), (150, 13, 128, 128),
+                                       (700, 16, 64, 64), (650, 7, 32, 96)])
 def test_memory_update_matches_oracle(G, n, dk, dv):
     r = rng(400 + n + dk)
     k = r.standard_normal((G, n, dk), dtype=np.float32)
@@ -130,6 +139,24 @@ def test_memory_update_matches_oracle(G, n, dk, dv):
                                     z[g].astype(np.float64), 1e-6)
         assert normwise(to_np(tA[g]), rA) < 1e-5
         assert normwise(to_np(tz[g]), rz) < 1e-6
+
+
+def test_memory_update_bits_do_not_depend_on_the_column_slicing():
+    """The same cells updated in a launch of 4 cells (16-column slices), of 400 cells (64-column
+    slices) and of 700 cells (the streaming kernel) give the same bits."""
+    r = rng(450)
+    G, n, dk, dv = 700, 16, 64, 64
+    k = torch.from_numpy(r.standard_normal((G, n, dk), dtype=np.float32)).cuda()
+    v = torch.from_numpy(r.standard_normal((G, n, dv), dtype=np.float32)).cuda()
+    A0 = torch.from_numpy(r.standard_normal((G, dk, dv), dtype=np.float32)).cuda()
+    z0 = torch.from_numpy(r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)).cuda()
+    A_all, z_all = A0.clone(), z0.clone()
+    rmt.rmt_memory_update(k, v, A_all, z_all, G, n, dk, dv, 1e-6)
+    for m in (4, 400):
+        A_few, z_few = A0[:m].clone(), z0[:m].clone()
+        rmt.rmt_memory_update(k[:m].contiguous(), v[:m].contiguous(), A_few, z_few, m, n, dk, dv, 1e-6)
+        rmt.rmt_sync(None)
+        assert torch.equal(A_all[:m], A_few) and torch.equal(z_all[:m], z_few), m
 
 
 def test_memory_write_then_read_orthonormal_keys_on_gpu():
@@ -195,8 +222,10 @@ def test_memory_write_matches_oracle(dtype, G, n, d, dk, dv):
 
 
 def test_bounded_wait_gives_up_and_reports_without_a_fault(cuda_ok):
-    """The failure path of every kernel: a wait on a barrier that nothing signals gives up after
-    its limit, the error word reaches the host as RMT_ETIMEOUT, and the context stays usable."""
+    """The failure path of every kernel: a wait on a barrier that nothing signals, and a wait on a
+    global counter that nothing increments (the chained projections' dependency wait), each
+    give up after their limit, the error word reaches the host as RMT_ETIMEOUT, and the context
+    stays usable."""
     import time
 
     rmt.rmt_sync(None)  # clean error word
@@ -205,7 +234,7 @@ def test_bounded_wait_gives_up_and_reports_without_a_fault(cuda_ok):
     with pytest.raises(rmt.RmtError) as ex:
         rmt.rmt_sync(None)
     assert ex.value.status == rmt.RMT_ETIMEOUT
-    assert time.perf_counter() - t0 >= 0.015
+    assert time.perf_counter() - t0 >= 0.035
     rmt.rmt_sync(None)  # the word was cleared
     # the device still runs kernels: a small grouped GEMM after the timeout is correct
     G, M, N, K = 2, 130, 256, 128

@@ -41,6 +41,26 @@ def test_noalloc_memory_write_matches_allocating_entry_point(cuda_ok, dtype, G, 
         assert normwise(A_new, A0) > 1e-6  # the state really moved
 
 
+def test_noalloc_allocates_no_device_memory(cuda_ok):
+    """After one call on the device (which loads the module that holds the fixed array), a
+    call larger than any before it leaves the device's free memory exactly as it was: no
+    allocation, no growth of a scratch buffer."""
+    G0, G, n, d, dk, dv = 2, 48, 16, 2048, 64, 64  # 48*16*16*128*4 B = 6 MiB of partial sums
+    r = np.random.Generator(np.random.PCG64(710))
+    y = torch.from_numpy(r.standard_normal((G, n, d), dtype=np.float32)).cuda()
+    w = rmt.storage(round_to_bf16(r.standard_normal((G, dk + dv, d), dtype=np.float32) * np.float32(0.02)), "bf16",
+                    "cuda")
+    A = torch.zeros((G, dk, dv), device="cuda")
+    z = torch.zeros((G, dk), device="cuda")
+    rmt.rmt_memory_write_noalloc(y, w, A, z, G0, n, d, dk, dv, 1e-6, "bf16")
+    rmt.rmt_sync(None)
+    free_before = torch.cuda.mem_get_info()[0]
+    rmt.rmt_memory_write_noalloc(y, w, A, z, G, n, d, dk, dv, 1e-6, "bf16")
+    rmt.rmt_sync(None)
+    assert torch.cuda.mem_get_info()[0] == free_before
+    assert torch.isfinite(A).all() and A.abs().max() > 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
     G, n, d, dk, dv = 64, 16, 2048, 128, 128  # 64*16*16*256*4 B = 16 MiB of partial sums > 8 MiB
     y = torch.zeros((G, n, d), device="cuda")
