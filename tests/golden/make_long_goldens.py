@@ -16,15 +16,18 @@ and the last segment. Workloads (the LLaMA-1B- and LLaMA-3B-shaped ARMTs of the 
 
   long_1b_s32.npz        1b, 32 segments of 1024 + 16 tokens (32,768 tokens)
   long_1b_s128.npz       1b, 128 segments (131,072 tokens); continues the 32-segment run
-  long_3b-512_s256.npz   3b-512, 256 segments of 512 + 16 tokens (131,072 tokens)
+  long_3b-512_s64.npz    3b-512, 64 segments of 512 + 16 tokens (32,768 tokens)
+  long_3b-512_s256.npz   3b-512, 256 segments of 512 + 16 tokens (131,072 tokens); continues
+                         the 64-segment run
   long_3b-2048_s64.npz   3b-2048, 64 segments of 2048 + 16 tokens (131,072 tokens)
 
-The 128-segment run resumes the oracle from the 32-segment run's state (the state after a
-segment depends only on the segments before it, which the oracle tests pin). On an 8-core
+The longer run of a workload resumes the oracle from the shorter run's state (the state after
+a segment depends only on the segments before it, which the oracle tests pin). On an 8-core
 host the oracle takes about 16 min for the 1B runs, 35 min for 3b-512 and 45 min for
 3b-2048.
 
-Usage: python tests/golden/make_long_goldens.py [1b] [3b-512] [3b-2048]
+Usage: python tests/golden/make_long_goldens.py [1b] [3b-512] [3b-2048] [NAME:STOP,...]
+(NAME:STOP,... runs that workload to the given stops only, e.g. 3b-512:64.)
 """
 from __future__ import annotations
 
@@ -86,8 +89,9 @@ def run(cfg_name: str, stops: list) -> None:
         save(f"{cfg_name}_s{stop}", cfg_name, stop, out[:stop * seg], A, z)
 
 
-JOBS = {"1b": [32, 128], "3b-512": [256], "3b-2048": [64]}
+JOBS = {"1b": [32, 128], "3b-512": [64, 256], "3b-2048": [64]}
 
 if __name__ == "__main__":
-    for name in sys.argv[1:] or list(JOBS):
-        run(name, JOBS[name])
+    for job in sys.argv[1:] or list(JOBS):
+        name, _, stops = job.partition(":")
+        run(name, [int(x) for x in stops.split(",")] if stops else JOBS[name])
