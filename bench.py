@@ -18,6 +18,7 @@ workload instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -45,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # with the number of cells (each cell brings its own layer's weights and activations), so a
 # launch's traffic is this figure times its cells. None when no capture of the current kernel
 # exists.
-DOMINANT_TRAFFIC_BYTES_PER_CELL = None
+DOMINANT_TRAFFIC_BYTES_PER_CELL = 206.7e6  # 674.3 MB read + 152.6 MB written by a 4-cell launch (1B shape)
 
 
 def parse():
@@ -58,6 +59,9 @@ def parse():
                    help="segments of the timed sequence (default: 131,072 tokens' worth of the config)")
     p.add_argument("--config", choices=["1b", "3b-512", "3b-2048"], default="1b",
                    help="model shape of the forward (the bench line of record is the 1B-shaped workload)")
+    p.add_argument("--operands", choices=["f16", "split"], default="f16",
+                   help="tensor-core operands of the bf16 forward: f16 (RMT_BF16, the line of record) or "
+                        "split high + low f16 terms (RMT_BF16_SPLIT: twice the GEMM work, fp32 attention)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-sequential", action="store_true")
     p.add_argument("--no-full-attention", action="store_true",
@@ -383,7 +387,8 @@ def main() -> int:
     S = args.segments if args.segments else 131072 // cfg.seg_len
     w = make_weights(cfg)
     emb = make_embeddings(cfg, S)
-    h = rmt.rmt_create(rmt.weights_storage(w, "bf16", dev), cfg)
+    hcfg = dataclasses.replace(cfg, dtype="bf16-split" if args.operands == "split" else "bf16")
+    h = rmt.rmt_create(rmt.weights_storage(w, "bf16", dev), hcfg)
     e = rmt.storage(emb, "bf16", dev)
     out = torch.empty_like(e)
     A = torch.empty(cfg.n_layers, cfg.d_k, cfg.d_v, device=dev)
@@ -434,7 +439,7 @@ def main() -> int:
                 "launches": probe["launches"], "kernel_ms_per_step": probe["ms"] / K,
                 "traffic": (DOMINANT_TRAFFIC_BYTES_PER_CELL * cfg.n_layers * S / probe["launches"] * K
                             if DOMINANT_TRAFFIC_BYTES_PER_CELL and probe["launches"] and args.config == "1b" else None),
-                "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 2-cell launch)"}
+                "traffic_note": "ncu DRAM bytes per cell x average cells per launch (capture of a 4-cell launch)"}
 
     # ---- end to end through the C ABI with host buffers (copies inside the timed region)
     e_host = e.cpu().pin_memory()
@@ -526,8 +531,12 @@ def main() -> int:
                        "layers": cfg.n_layers, "d_model": cfg.d_model, "segments": S,
                        "seg_len": cfg.seg_len, "n_mem": cfg.n_mem, "tokens": tokens, "schedule": "diagonal",
                        "batch": 1, "parallelism": "replicas" if world > 1 else "single GPU",
-                       "precision": "bf16 weights, embeddings and outputs; f16 tensor-core operands with fp32 "
-                                    "accumulation; fp32 residual stream, softmax statistics and memory state",
+                       "precision": ("bf16 weights, embeddings and outputs; f16 tensor-core operands with fp32 "
+                                     "accumulation; fp32 residual stream, softmax statistics and memory state")
+                       if args.operands == "f16" else
+                       ("bf16 weights, embeddings and outputs; split high + low f16 tensor-core activation "
+                        "operands (2x the GEMM MMAs) with fp32 accumulation; fp32 q/k/v and attention; fp32 "
+                        "residual stream and memory state"),
                        "l2": "inputs larger than L2 (weights of 1.96 GB or more, embeddings 0.54 GB or more): no flush"},
             "roofline": roofline,
             "path": {"algorithmic_tflop_per_step": step_flops / 1e12,

@@ -55,7 +55,15 @@ typedef enum { RMT_DIAGONAL = 0, RMT_SEQUENTIAL = 1 } rmt_schedule;
  * follow them (exact for bf16 magnitudes from 2^-17 up; smaller ones lose bits).
  * A forward that stores an operand of magnitude 65520 or more (which rounds to infinity) is
  * reported by rmt_sync as RMT_ERANGE; its outputs are then not valid. */
-typedef enum { RMT_F32 = 0, RMT_BF16 = 1 } rmt_dtype;
+/* RMT_BF16_SPLIT: bf16 storage and f16 range as RMT_BF16, with every activation operand of a
+ * tensor-core GEMM carried as two f16 terms (hi = f16(v), lo = f16(v - hi): about 22
+ * significant bits), so each projection runs twice the MMAs of RMT_BF16 against the same
+ * weights; q, k and v stay fp32 and attention runs on the fp32 FMA kernel. The memory
+ * recurrence carries rounding differences from segment to segment and amplifies them, so
+ * over hundreds of segments RMT_BF16's f16 rounding can drift past the bf16 tolerance of the
+ * outputs and memory state where this mode does not; it costs about twice the GEMM time.
+ * Needs d_k of 64 or 128. rmt_full_attention_forward does not take it. */
+typedef enum { RMT_F32 = 0, RMT_BF16 = 1, RMT_BF16_SPLIT = 2 } rmt_dtype;
 
 /* Model shape. A cell has M = seg_len + n_mem rows: the segment's tokens followed by the
  * n_mem memory tokens. Limits (else RMT_EINVAL): all sizes > 0; n_heads % n_kv_heads == 0;

@@ -213,6 +213,10 @@ struct rmt_handle {
   rmt_cfg cfg{};
   int dev = 0;
   bool bf16 = false;
+  // RMT_BF16_SPLIT: every f16 activation operand is stored as high and low terms side by side
+  // in one row ([hi | lo], twice the width), each tensor-core GEMM reads 2K columns against
+  // its K weight columns, q/k/v stay fp32 and attention runs on the fp32 kernel
+  bool split = false;
   int M = 0, es = 4, Nqkv = 0, nsplit = 0;
   // packed weights (cfg dtype)
   void *w_qkv = nullptr, *w_o = nullptr, *w_gu = nullptr, *w_d = nullptr, *w_mq = nullptr, *w_mo = nullptr,
@@ -384,7 +388,8 @@ bool validate_cfg(const rmt_cfg* c, std::string& why) {
     why = "all sizes must be positive";
     return false;
   }
-  if (c->dtype != RMT_F32 && c->dtype != RMT_BF16) return why = "dtype must be RMT_F32 or RMT_BF16", false;
+  if (c->dtype != RMT_F32 && c->dtype != RMT_BF16 && c->dtype != RMT_BF16_SPLIT)
+    return why = "dtype must be RMT_F32, RMT_BF16 or RMT_BF16_SPLIT", false;
   if (c->n_heads % c->n_kv_heads) return why = "n_heads must be a multiple of n_kv_heads", false;
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return why = "head_dim must be 32, 64 or 128", false;
   if (c->d_k % 32 || c->d_v % 32 || c->d_k > 128 || c->d_v > 128)
@@ -394,7 +399,9 @@ bool validate_cfg(const rmt_cfg* c, std::string& why) {
   if (c->d_model % 4) return why = "d_model must be a multiple of 4", false;
   if (!(c->rope_theta > 0.f) || !(c->rms_eps >= 0.f) || !(c->mem_eps >= 0.f))
     return why = "rope_theta > 0, rms_eps >= 0, mem_eps >= 0", false;
-  if (c->dtype == RMT_BF16) {
+  if (c->dtype == RMT_BF16_SPLIT && c->d_k != 64 && c->d_k != 128)
+    return why = "bf16 split operands: d_k must be 64 or 128", false;
+  if (c->dtype != RMT_F32) {
     const int hd = c->n_heads * c->head_dim, nqkv = (c->n_heads + 2 * c->n_kv_heads) * c->head_dim;
     if (c->d_model % 64 || hd % 64 || c->d_v % 64)
       return why = "bf16: d_model, n_heads*head_dim and d_v must be multiples of 64", false;
@@ -498,20 +505,24 @@ rmt_status build_maps(rmt_handle* h) {
   const bool any_pair = h->pair_mo || h->pair_qkv || h->pair_o || h->pair_gu || h->pair_d;
   // the read-out o: its own buffer, or (fold_mo) the last d_v columns of the attention output
   const uint64_t lda = uint64_t(h->ld_att);
+  // split-operand mode: the activation rows hold [high terms | low terms], twice as wide
+  const uint64_t sw = h->split ? 2 : 1, xw = sw * d, aw = sw * lda, uw = sw * F, ow = sw * c.d_v;
   auto map_om = [&](CUtensorMap* m, uint32_t box) {
-    return h->fold_mo ? make_tmap_16_3d_strided(m, static_cast<__half*>(h->att) + hd, c.d_v, M, L, lda, box, true)
-                      : map(m, h->om, c.d_v, M, L, box);
+    // folded: from column hd of the attention rows, the high terms of o, then (split) the rest
+    // of the row up to its low terms ld_att columns further
+    return h->fold_mo ? make_tmap_16_3d_strided(m, static_cast<__half*>(h->att) + hd, aw - hd, M, L, aw, box, true)
+                      : map(m, h->om, ow, M, L, box);
   };
-  bool ok = map(&h->tm_xb, h->xb, d, M, NS, 128) && map_om(&h->tm_om, 128) &&
-            map(&h->tm_att, h->att, lda, M, L, 128) && map(&h->tm_u, h->u, F, M, L, 128) &&
+  bool ok = map(&h->tm_xb, h->xb, xw, M, NS, 128) && map_om(&h->tm_om, 128) &&
+            map(&h->tm_att, h->att, aw, M, L, 128) && map(&h->tm_u, h->u, uw, M, L, 128) &&
             map(&h->tm_wmq, h->w_mq, d, c.d_k, LW, h->bn_mq) &&
             map(&h->tm_wmo, h->w_mo, c.d_v, d, LW, h->pair_mo ? 128 : h->bn_mo) &&
             map(&h->tm_wqkv, h->w_qkv, d, h->Nqkv, LW, h->pair_qkv ? 128 : h->bn_qkv) &&
             map(&h->tm_wo, h->w_o, lda, d, LW, h->pair_o ? 128 : h->bn_o) &&
             map(&h->tm_wgu, h->w_gu, d, 2 * F, LW, h->pair_gu ? 128 : h->bn_gu) &&
             map(&h->tm_wd, h->w_d, F, d, LW, h->pair_d ? 128 : h->bn_d) &&
-            (!any_pair || (map(&h->tp_xb, h->xb, d, M, NS, pb) && map_om(&h->tp_om, pb) &&
-                           map(&h->tp_att, h->att, lda, M, L, pb) && map(&h->tp_u, h->u, F, M, L, pb))) &&
+            (!any_pair || (map(&h->tp_xb, h->xb, xw, M, NS, pb) && map_om(&h->tp_om, pb) &&
+                           map(&h->tp_att, h->att, aw, M, L, pb) && map(&h->tp_u, h->u, uw, M, L, pb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
             map(&h->tm_qkv_tail, h->qkv, h->Nqkv, M, L, attn_tail_box(int(M), c.n_heads, c.n_kv_heads)) &&
             make_tmap_f32_resid(&h->tm_x, h->x, d, M, NS) &&
@@ -528,16 +539,16 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
   h->free_acts();
   const rmt_cfg& c = h->cfg;
   const size_t nb = B, L = c.n_layers, d = c.d_model, M = h->M, es = h->es, F = c.d_ff, dk = c.d_k, dv = c.d_v,
-               BL = nb * L;
+               BL = nb * L, sw = h->split ? 2 : 1;  // sw: operand row width factor (split: hi | lo)
   struct {
     void** p;
     size_t bytes;
   } plan[] = {
       {reinterpret_cast<void**>(&h->x), nb * n_slots(c.n_layers) * M * d * 4},
-      {&h->qkv, BL * M * h->Nqkv * es},   {&h->att, BL * M * size_t(h->ld_att) * es},
+      {&h->qkv, BL * M * h->Nqkv * (h->split ? 4 : es)}, {&h->att, BL * M * size_t(h->ld_att) * es * sw},
       {reinterpret_cast<void**>(&h->ss1), BL * M * (d / 16 + 1) * 4},
       {reinterpret_cast<void**>(&h->ss2), BL * M * (d / 16 + 1) * 4},
-      {&h->u, BL * M * F * es},           {&h->om, BL * M * dv * es},
+      {&h->u, BL * M * F * es * sw},      {&h->om, BL * M * dv * es * sw},
       {reinterpret_cast<void**>(&h->qm), BL * M * dk * 4},
       {reinterpret_cast<void**>(&h->part), BL * h->nsplit * size_t(c.n_mem) * (dk + dv) * 4},
       {reinterpret_cast<void**>(&h->A), BL * dk * dv * 4},
@@ -551,7 +562,7 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
     }
   }
   if (h->bf16) {
-    h->xb = static_cast<__half*>(h->act_alloc(nb * n_slots(c.n_layers) * M * d * 2));
+    h->xb = static_cast<__half*>(h->act_alloc(nb * n_slots(c.n_layers) * M * d * 2 * sw));
     if (!h->xb) {
       h->free_acts();
       return fail(RMT_ENOMEM, "activation allocation failed");
@@ -613,6 +624,10 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   ep.inv_d = 1.f / float(d);
   ep.rms_eps = c.rms_eps;
   const EpiKind resid = h->bf16 ? kEpiResidCast : kEpiResid;  // bf16: also refresh the bf16 copy
+  // split-operand mode: X rows are [high terms | low terms]; kx_lo = column of the low terms
+  const int sw = h->split ? 2 : 1;
+  int kx_lo = 0;
+  if (h->split) ep.ldxb = 2 * d;
   int N = 0, K = 0;
   EpiKind epi = kEpiStoreF32;
   IndexMode amode = kByLayer;
@@ -629,11 +644,12 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       if (h->fuse_read) {  // o = phi(q) A / (phi(q) . z + eps) straight from the accumulator
         epi = kEpiMemRead;
         if (h->fold_mo)  // o goes to the last d_v columns of the attention output rows
-          ep.out = static_cast<__half*>(h->att) + hd, ep.ldo = h->ld_att;
+          ep.out = static_cast<__half*>(h->att) + hd, ep.ldo = sw * h->ld_att, ep.lo_off = h->split ? h->ld_att : 0;
         else
-          ep.out = h->om, ep.ldo = c.d_v;
+          ep.out = h->om, ep.ldo = sw * c.d_v, ep.lo_off = h->split ? c.d_v : 0;
         ep.mem_A = h->A, ep.mem_z = h->z, ep.mem_dv = c.d_v, ep.mem_eps = c.mem_eps;
       }
+      kx_lo = h->split ? d : 0;
       break;
     case kProjMemO:  // x_out = x_in + read-out; emits the row sums of squares of RMSNorm 1
       N = d, K = c.d_v, epi = resid;
@@ -641,12 +657,16 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       ep.resid_no_store = h->fold_mo;  // the O projection adds W_mo o itself
       a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
       tp = &h->tp_om, pair = h->pair_mo;
+      ep.lo_off = h->split ? d : 0;
+      kx_lo = h->split ? (h->fold_mo ? h->ld_att : c.d_v) : 0;
       break;
     case kProjQkv:  // rows of x_out scaled by RMSNorm 1 (gain folded into the weight), then RoPE
       N = h->Nqkv, K = d, epi = kEpiRope, amode = kOutSlot;
       ep.out = h->qkv, ep.ldo = h->Nqkv, ep.ss_in = h->ss1;
       a32 = h->x, w = h->w_qkv, ta = &h->tm_xb, tb = &h->tm_wqkv, bn = h->bn_qkv;
       tp = &h->tp_xb, pair = h->pair_qkv;
+      ep.out_f32 = h->split;  // split-operand mode: attention reads fp32 q, k, v
+      kx_lo = h->split ? d : 0;
       break;
     case kProjO:  // x_out += attention output; emits the row sums of squares of RMSNorm 2
       N = d, K = hd, epi = resid;
@@ -657,22 +677,28 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       }
       a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
       tp = &h->tp_att, pair = h->pair_o;
+      ep.lo_off = h->split ? d : 0;
+      kx_lo = h->split ? h->ld_att : 0;
       break;
     case kProjGateUp:  // rows of x_out scaled by RMSNorm 2 (gain folded into the weight), SwiGLU
       N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU, amode = kOutSlot;
-      ep.out = h->u, ep.ldo = c.d_ff, ep.ss_in = h->ss2;
+      ep.out = h->u, ep.ldo = sw * c.d_ff, ep.ss_in = h->ss2;
       a32 = h->x, w = h->w_gu, ta = &h->tm_xb, tb = &h->tm_wgu, bn = h->bn_gu;
       tp = &h->tp_xb, pair = h->pair_gu;
+      ep.lo_off = h->split ? c.d_ff : 0;
+      kx_lo = h->split ? d : 0;
       break;
     case kProjDown:  // x_out += MLP output; the bf16 copy feeds the next layer's memory query
       N = d, K = c.d_ff, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb;
       a32 = static_cast<const float*>(h->u), w = h->w_d, ta = &h->tm_u, tb = &h->tm_wd, bn = h->bn_d;
       tp = &h->tp_u, pair = h->pair_d;
+      ep.lo_off = h->split ? d : 0;
+      kx_lo = h->split ? c.d_ff : 0;
       break;
   }
   if (h->bf16 && pair) {
-    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
+    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err, kx_lo};
     if (collect) {
       *collect = PairLaunch{a, tb, tp};
       return cudaSuccess;
@@ -681,9 +707,9 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   }
   if (collect) return cudaErrorInvalidValue;
   if (h->bf16) {
-    const bool rope_tma = p == kProjQkv && c.head_dim >= 64;
+    const bool rope_tma = p == kProjQkv && c.head_dim >= 64 && !h->split;
     ep.rope_tma = rope_tma;
-    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err};
+    TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err, kx_lo};
     return launch_tc_gemm(*ta, *tb, rope_tma ? h->tm_rope : h->tm_x, a, bn, /*f16=*/true, st);
   }
   const int lda = (p == kProjMemQ || p == kProjQkv || p == kProjGateUp) ? d : K;
@@ -760,7 +786,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   if (n_first > 0) {
     e = launch_kind(h, RMT_K_ASSEMBLE, 0, rows_first * dd * (es + 4 + (h->bf16 ? 2 : 0)), st, [&] {
       return launch_assemble(cells, n_first, emb, h->memtok, h->x, h->bf16 ? h->xb : nullptr, M, c.n_mem, d, h->bf16,
-                             h->err, st);
+                             h->err, st, h->split);
     });
     if (e != cudaSuccess) return e;
   }
@@ -776,6 +802,7 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
     e = launch_kind(h, RMT_K_MEMREAD, g * m * (2 * dk * dv + 2 * dk),
                     g * (m * dk * 4 + dk * dv * 4 + dk * 4 + m * dv * es), st, [&] {
                       MemReadArgs a{h->qm, h->A, h->z, h->om, M, c.d_k, c.d_v, c.mem_eps, G, cells, kByLayer, kByLayer, L};
+                      if (h->split) a.ldo = 2 * c.d_v, a.lo_off = c.d_v;  // [high terms | low terms] rows
                       return launch_mem_read(a, h->bf16 ? kElemF16 : kElemF32, st, h->err);
                     });
     if (e != cudaSuccess) return e;
@@ -794,6 +821,10 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
                   g * (m * nq * es + m * hd * es), st, [&] {
                     AttnArgs a{h->qkv, h->att, M, c.n_heads, c.n_kv_heads, c.head_dim, G, cells, kByLayer, L, h->err,
                                h->ld_att};
+                    if (h->split) {  // fp32 q, k, v in; f16 high and low terms out
+                      a.ldo = 2 * h->ld_att, a.out_lo = h->ld_att;
+                      return launch_attention(a, kElemF32, st);
+                    }
                     if (h->bf16 && attention_tc_supported(c.head_dim))
                       return launch_attention_tc(h->tm_qkv, h->tm_qkv_tail, a, /*f16=*/true, st);
                     return launch_attention(a, h->bf16 ? kElemF16 : kElemF32, st);
@@ -1053,11 +1084,12 @@ rmt_status rmt_create(const rmt_weights* weights, const rmt_cfg* cfg, rmt_handle
   };
   if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(RMT_ECUDA, "no CUDA device"));
   const rmt_cfg& c = h->cfg;
-  h->bf16 = c.dtype == RMT_BF16;
+  h->bf16 = c.dtype != RMT_F32;
+  h->split = c.dtype == RMT_BF16_SPLIT;
   h->es = h->bf16 ? 2 : 4;
   h->M = c.seg_len + c.n_mem;
   h->Nqkv = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-  h->nsplit = mem_kv_splits(c.d_model, c.dtype == RMT_BF16);
+  h->nsplit = mem_kv_splits(c.d_model, h->bf16);
   const size_t L = c.n_layers, d = c.d_model, M = h->M, es = h->es, F = c.d_ff, dk = c.d_k, dv = c.d_v;
   if (h->bf16) {
     const int Mi = h->M, di = c.d_model, hdi = c.n_heads * c.head_dim, Fi = c.d_ff;
@@ -1329,7 +1361,7 @@ rmt_status rmt_full_attention_forward(rmt_handle* h, const void* emb, int32_t n_
                                       void* stream) {
   if (!h) return fail(RMT_EINVAL, "null handle");
   if (!emb || !out_hidden) return fail(RMT_EINVAL, "emb and out_hidden must not be null");
-  if (!h->bf16) return fail(RMT_EINVAL, "the full-attention forward needs a bf16 handle");
+  if (!h->bf16 || h->split) return fail(RMT_EINVAL, "the full-attention forward needs an RMT_BF16 handle");
   if (n_tokens <= 0) return fail(RMT_EINVAL, "n_tokens must be positive");
   const rmt_cfg& c = h->cfg;
   if (h->ss_parts > 32 || c.d_model % h->ss_parts || (c.d_model / h->ss_parts) % 4)

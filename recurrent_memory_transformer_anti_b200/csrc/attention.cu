@@ -286,8 +286,19 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(const AttnArgs a) {
     }
   }
   if (!valid) return;
-  float* dst = static_cast<float*>(a.out) + slice * a.M * ldo + static_cast<size_t>(row) * ldo + h * HD;
+  const size_t off = slice * a.M * ldo + static_cast<size_t>(row) * ldo + h * HD;
   const float inv = 1.f / l;
+  if (a.out_lo) {  // split-operand mode: f16 high and low terms for the O projection
+    __half* dst = static_cast<__half*>(a.out) + off;
+#pragma unroll
+    for (int i = 0; i < HD; ++i) {
+      const float v = o[i] * inv;
+      dst[i] = __float2half_rn(v);
+      dst[i + a.out_lo] = __float2half_rn(lo_term<__half>(v));
+    }
+    return;
+  }
+  float* dst = static_cast<float*>(a.out) + off;
 #pragma unroll
   for (int i = 0; i < HD; ++i) dst[i] = o[i] * inv;
 }
@@ -332,7 +343,7 @@ cudaError_t launch_typed(const AttnArgs& a, ElemType t, cudaStream_t st) {
 
 cudaError_t launch_attention(const AttnArgs& a, ElemType t, cudaStream_t st) {
   if (a.G <= 0 || a.M <= 0) return cudaSuccess;
-  if (a.Hkv <= 0 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+  if (a.Hkv <= 0 || a.H % a.Hkv != 0 || (a.out_lo && t != kElemF32)) return cudaErrorInvalidValue;
   switch (a.dh) {
     case 32: return launch_typed<32>(a, t, st);
     case 64: return launch_typed<64>(a, t, st);

@@ -192,6 +192,13 @@ struct EpiParams {
   // operand copy and the row sums of squares, but do not store it to x[dst] (its consumer
   // adds the same product itself)
   int resid_no_store;
+  // Split-operand mode (RMT_BF16_SPLIT): every 16-bit operand this epilogue writes (the
+  // residual copy xb, the SwiGLU output, the memory read-out o) also gets its low term, lo_off
+  // elements after the high term in the same row (0: high terms only). xb rows are ldxb
+  // elements apart (0: ldx). kEpiRope with out_f32 writes q, k and v as fp32 instead.
+  int lo_off;
+  int ldxb;
+  int out_f32;
 };
 
 // RMSNorm row scale from the per-block sums of squares of one row (fixed summation order).
@@ -226,6 +233,11 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) 
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) { return pack2<__nv_bfloat16>(a, b); }
 
+// Split-operand mode: v reaches the tensor cores as hi = T(v) and lo = T(v - hi); the pair
+// carries about twice the significand bits of T (22 for f16), and one MMA per term with the
+// same weight operand accumulates W.hi + W.lo in fp32.
+template <typename T> __device__ __forceinline__ float lo_term(float v) { return v - to_f32<T>(from_f32<T>(v)); }
+
 // Store 32 consecutive fp32 values as a 16-bit type (64 bytes, four 16-byte stores).
 template <typename T>
 __device__ __forceinline__ void store32_16(T* dst, const float* v) {
@@ -237,6 +249,18 @@ __device__ __forceinline__ void store32_16(T* dst, const float* v) {
   }
 }
 __device__ __forceinline__ void store32_bf16(__nv_bfloat16* dst, const float* v) { store32_16(dst, v); }
+
+// store32_16, plus (lo_off != 0) the 32 low terms at dst + lo_off.
+template <typename T>
+__device__ __forceinline__ void store32_16_split(T* dst, const float* v, int lo_off) {
+  store32_16(dst, v);
+  if (lo_off) {
+    float l[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) l[j] = lo_term<T>(v[j]);
+    store32_16(dst + lo_off, l);
+  }
+}
 
 // Tensor-core operand format code of the instruction descriptor (kind::f16): f16 0, bf16 1.
 template <typename T> struct OpFormat;

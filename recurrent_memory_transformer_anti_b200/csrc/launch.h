@@ -45,6 +45,10 @@ struct TcGemmArgs {
   EpiKind epi;
   EpiParams ep;
   int* err;  // device error word (may be null)
+  // split-operand mode: the X operand holds each row's high terms in columns 0..K-1 and its
+  // low terms from column kx_lo on; the GEMM runs 2K/64 blocks, block b reading X at column
+  // (b mod K/64) * 64 + (b div K/64) * kx_lo and W at (b mod K/64) * 64 (0: K blocks)
+  int kx_lo;
 };
 
 // tensor-core path: 16-bit operands (f16 or bf16, one type per launch) in TMA tensor maps
@@ -118,6 +122,9 @@ struct AttnArgs {
   int L;
   int* err;        // device error word for bounded waits (tensor-core kernel), may be null
   int ldo;         // row stride of out in elements (0: H * dh, rows packed)
+  // fp32 kernel only: write out as f16 high terms and, out_lo elements further, low terms
+  // (split-operand mode; 0: fp32 out)
+  int out_lo;
   // filled in by launch_attention_tc: rows of the stacked last query tile (0: not stacked,
   // see attn_pack_tail), H / Hkv, and the work items of the last query tile
   int tail_rows, group, n_tail;
@@ -157,6 +164,8 @@ struct MemReadArgs {
   IndexMode mode;        // slice of q and o
   IndexMode state_mode;  // slice of A and z
   int L;
+  int ldo;     // row stride of o in elements (0: dv)
+  int lo_off;  // tcgen05 read, split-operand mode: low terms of o lo_off elements after the high terms (0: none)
 };
 // 16-bit outputs take the tcgen05 read when it supports d_k (err: its bounded waits' error word,
 // may be null), else the mma.sync read; fp32 outputs the fp32 FMA read
@@ -227,8 +236,9 @@ cudaError_t launch_bf16_to_f16(void* p, size_t n, cudaStream_t st);
 // Layer-0 inputs of the G cells (all of layer 0): in slot c.xin of x (and of xb, if given),
 // rows 0..m-n_mem-1 from emb rows c.t0.., rows m-n_mem..m-1 from the memory tokens, rows
 // m..M-1 zero (m = cell_rows(c, M)). An f16 copy that overflows sets kErrF16Range in *err.
+// split: xb rows are 2d wide, the high terms then the low terms (split-operand mode).
 cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
-                            int n_mem, int d, bool bf16, int* err, cudaStream_t st);
+                            int n_mem, int d, bool bf16, int* err, cudaStream_t st, bool split = false);
 // RMSNorm statistics of rows 0..M-1 of an fp32 [M, d] block: ss[row * parts + b] = sum of
 // squares of columns b*w .. b*w+w-1, w = d / parts (a multiple of 4; at most 32 parts).
 // One CTA waits on an mbarrier nothing signals, with the kernels' bounded wait limited to

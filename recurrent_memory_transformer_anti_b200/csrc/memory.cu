@@ -509,8 +509,8 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
 //      order, then phi) and its own value columns into shared memory; the cluster meets, and
 //      each CTA copies the other key rows from its peers' shared memory;
 //   2. den[r] = phi(k_r) . z + eps, one warp per row (lanes over i, then a butterfly);
-//   3. v_bar and D = V - v_bar for the slice's columns over i ascending (4 x 4 register blocks
-//      of rows x columns for whole-cell CTAs, 1 x 4 for slices, which have fewer columns);
+//   3. v_bar and D = V - v_bar for the slice's columns over i ascending (one row x 4 columns
+//      per thread);
 //   4. A' = A + phi(K)^T D for the slice's columns, 4 x 4 blocks over rows ascending; the CTA of
 //      slice 0 also writes z' = z + sum of the phi(k) rows.
 // Every sum runs in a fixed order whatever S is, so the bits do not depend on the slicing or on
@@ -519,12 +519,11 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
 constexpr int kUpdThreads = 256;
 
 struct UpdLayout {  // shared-memory layout in floats (every region starts 16-byte aligned)
-  int n4, fk, fkT, As, Vs, D, zs, den, total;
+  int n4, fk, As, Vs, D, zs, den, total;
   __host__ __device__ UpdLayout(int n, int dk, int cs) {
     n4 = (n + 3) & ~3;
     fk = 0;                 // [n][dk]    phi(keys)
-    fkT = fk + n * dk;      // [dk][n4]   the same, transposed (whole cells only); rows past n are zero
-    As = fkT + dk * n4;     // [dk][cs]   this slice's columns of A
+    As = fk + n * dk;       // [dk][cs]   this slice's columns of A
     Vs = As + dk * cs;      // [n][cs]    this slice's columns of V
     D = Vs + n * cs;        // [n4][cs]   V - v_bar
     zs = D + n4 * cs;       // [dk]
@@ -574,9 +573,7 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
   const int slice = static_cast<int>(blockIdx.x) % S, g = static_cast<int>(blockIdx.x) / S;
   const int j0 = slice * cs;
   const UpdLayout lay(n, dk, cs);
-  const int n4 = lay.n4;
   float* fk = sm + lay.fk;
-  float* fkT = sm + lay.fkT;
   float* As = sm + lay.As;
   float* Vs = sm + lay.Vs;
   float* D = sm + lay.D;
@@ -640,14 +637,7 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
   }
   __syncthreads();
 
-  // 2. row denominators (and, for whole-cell CTAs, the transposed keys)
-  const bool wide = cs >= 64;  // many cells per launch: 4-row blocks, for fewer shared-memory reads
-  if (wide) {
-    for (int e = tid; e < dk * n4; e += kUpdThreads) {
-      const int i = e / n4, r = e % n4;
-      fkT[e] = r < n ? fk[r * dk + i] : 0.f;
-    }
-  }
+  // 2. row denominators
   const int warp = tid >> 5, lane = tid & 31;
   for (int r = warp; r < n; r += kUpdThreads / 32) {
     float d = 0.f;
@@ -657,48 +647,26 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
   }
   __syncthreads();
 
-  // 3. D = V - phi(K) A / den for this slice's columns, i ascending per element
-  if (wide) {  // 4 rows x 4 columns per thread
-    for (int b = tid; b < (n4 / 4) * (cs / 4); b += kUpdThreads) {
-      const int r0 = 4 * (b / (cs / 4)), c0 = 4 * (b % (cs / 4));
-      float acc[4][4] = {};
-      for (int i = 0; i < dk; ++i) {
-        const float4 f = *reinterpret_cast<const float4*>(fkT + i * n4 + r0);
-        const float4 av = *reinterpret_cast<const float4*>(As + i * cs + c0);
-        const float fr[4] = {f.x, f.y, f.z, f.w}, ar[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(fr[x], ar[y], acc[x][y]);
-      }
+  // 3. D = V - phi(K) A / den for this slice's columns, i ascending per element: one row x 4
+  //    columns per thread, so every thread has work; a warp's reads of a key row and of an A
+  //    row are broadcasts
+  for (int b = tid; b < n * (cs / 4); b += kUpdThreads) {
+    const int r = b / (cs / 4), c0 = 4 * (b % (cs / 4));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i0 = 0; i0 < dk; i0 += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
+      const float fr[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
-        const int r = r0 + x;
-        if (r < n) {
-#pragma unroll
-          for (int y = 0; y < 4; ++y) D[r * cs + c0 + y] = Vs[r * cs + c0 + y] - acc[x][y] / den[r];
-        }
+        const float4 av = *reinterpret_cast<const float4*>(As + (i0 + x) * cs + c0);
+        acc[0] = fmaf(fr[x], av.x, acc[0]);
+        acc[1] = fmaf(fr[x], av.y, acc[1]);
+        acc[2] = fmaf(fr[x], av.z, acc[2]);
+        acc[3] = fmaf(fr[x], av.w, acc[3]);
       }
     }
-  } else {  // one row x 4 columns per thread: more threads on a short chain
-    for (int b = tid; b < n * (cs / 4); b += kUpdThreads) {
-      const int r = b / (cs / 4), c0 = 4 * (b % (cs / 4));
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i0 = 0; i0 < dk; i0 += 4) {
-        const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
-        const float fr[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float4 av = *reinterpret_cast<const float4*>(As + (i0 + x) * cs + c0);
-          acc[0] = fmaf(fr[x], av.x, acc[0]);
-          acc[1] = fmaf(fr[x], av.y, acc[1]);
-          acc[2] = fmaf(fr[x], av.z, acc[2]);
-          acc[3] = fmaf(fr[x], av.w, acc[3]);
-        }
-      }
-#pragma unroll
-      for (int y = 0; y < 4; ++y) D[r * cs + c0 + y] = Vs[r * cs + c0 + y] - acc[y] / den[r];
-    }
+    for (int y = 0; y < 4; ++y) D[r * cs + c0 + y] = Vs[r * cs + c0 + y] - acc[y] / den[r];
   }
   __syncthreads();
 
@@ -743,38 +711,39 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
 // cell ahead (two stages), so that the loads of the next cell overlap the arithmetic of this
 // one. The arithmetic is mem_update_kernel's, element for element in the same order (the
 // same bits): den by one warp per row, then v_bar and D over i ascending, then A' over rows
-// ascending, here in 8 x 4 register blocks for fewer shared-memory reads per FMA. Keys and
-// values come as plain arrays or as whole sums (one split, [n][d_k + d_v] per cell).
+// ascending. Every thread works in every phase (1 x 4 and 4 x 4 register blocks), laid out so
+// that a warp's shared-memory reads of a key row or an A row are broadcasts. Keys and values
+// come as plain arrays or as whole sums (one split, [n][d_k + d_v] per cell).
 constexpr int kUpdStreamThreads = 256;
 
 struct UpdStreamLayout {  // in floats; every region starts 16-byte aligned
-  int n8, stage, fk, fkT, D, den, total;
-  __host__ __device__ UpdStreamLayout(int n, int dk, int dv) {
+  int n8, stage, fk, D, den, total;
+  __host__ __device__ UpdStreamLayout(int n, int dk, int dv, int nst) {
     n8 = (n + 7) & ~7;
     stage = n * dk + n * dv + dk * dv + dk;  // K [n][dk], V [n][dv], A [dk][dv], z [dk]
-    fk = 2 * stage;                          // phi(K) [n][dk]
-    fkT = fk + n * dk;                       // [dk][n8]
-    D = fkT + dk * n8;                       // [n8][dv]
+    fk = nst * stage;                        // phi(K) [n][dk]
+    D = fk + n * dk;                         // [n8][dv]
     den = D + n8 * dv;                       // [n8]
     total = den + n8;
   }
 };
 
+// A ring of NST cell stages: the loads of cells g+1 .. g+NST-1 are in flight while cell g is
+// computed (the stage of cell g+NST-1 is the one cell g-1 just released).
+template <int NST>
 __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel(const MemUpdateArgs a) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ __align__(16) float us[];
   const int n = a.n, dk = a.dk, dv = a.dv, dkv = dk + dv;
-  const UpdStreamLayout lay(n, dk, dv);
-  const int n8 = lay.n8;
+  const UpdStreamLayout lay(n, dk, dv, NST);
   float* fk = us + lay.fk;
-  float* fkT = us + lay.fkT;
   float* D = us + lay.D;
   float* den = us + lay.den;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int per = (a.G + gridDim.x - 1) / gridDim.x;
   const int c_beg = blockIdx.x * per, c_end = min(a.G, c_beg + per);
-  auto stage = [&](int i) { return us + (i & 1) * lay.stage; };
+  auto stage = [&](int i) { return us + (i % NST) * lay.stage; };
   auto issue = [&](int g, float* dst) {
     const Cell c = load_cell(a.cells, g);
     const size_t ki = cell_index(a.kv_mode, a.L, c), si = cell_index(a.state_mode, a.L, c);
@@ -795,24 +764,26 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel
       cp_async16(sm100::smem_u32(dst + n * dk + n * dv + 4 * e), src, 16u);
     }
   };
-  if (c_beg < c_end) issue(c_beg, stage(0));
-  cp_async_commit();
-  if (c_beg + 1 < c_end) issue(c_beg + 1, stage(1));
-  cp_async_commit();
+#pragma unroll
+  for (int j = 0; j < NST - 1; ++j) {
+    if (c_beg + j < c_end) issue(c_beg + j, stage(j));
+    cp_async_commit();
+  }
   for (int g = c_beg; g < c_end; ++g) {
-    float* st = stage(g - c_beg);
+    const int i = g - c_beg;
+    float* st = stage(i);
     const float* Kr = st;
     const float* Vr = st + n * dk;
     const float* Ar = Vr + n * dv;
     const float* zr = Ar + dk * dv;
-    cp_async_wait<1>();  // this cell's stage has landed (the next cell's may still be in flight)
+    // the stage of cell g-1 is free (the barrier that closed its iteration): refill it with
+    // cell g+NST-1
+    if (g + NST - 1 < c_end) issue(g + NST - 1, stage(i + NST - 1));
+    cp_async_commit();
+    cp_async_wait<NST - 1>();  // this cell's stage has landed (the later ones may still be in flight)
     __syncthreads();
     for (int e = tid; e < n * dk; e += kUpdStreamThreads) fk[e] = phi_f(Kr[e]);
     __syncthreads();
-    for (int e = tid; e < dk * n8; e += kUpdStreamThreads) {
-      const int i = e / n8, r = e % n8;
-      fkT[e] = r < n ? fk[r * dk + i] : 0.f;
-    }
     for (int r = warp; r < n; r += kUpdStreamThreads / 32) {
       float d = 0.f;
       for (int i = lane; i < dk; i += 32) d = fmaf(fk[r * dk + i], zr[i], d);
@@ -820,52 +791,48 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel
       if (lane == 0) den[r] = d + a.eps;
     }
     __syncthreads();
-    // D = V - phi(K) A / den: 8 rows x 4 columns per thread, i ascending
-    for (int b = tid; b < (n8 / 8) * (dv / 4); b += kUpdStreamThreads) {
-      const int r0 = 8 * (b / (dv / 4)), c0 = 4 * (b % (dv / 4));
-      float acc[8][4] = {};
-      for (int i = 0; i < dk; ++i) {
-        const float4 f0 = *reinterpret_cast<const float4*>(fkT + i * n8 + r0);
-        const float4 f1 = *reinterpret_cast<const float4*>(fkT + i * n8 + r0 + 4);
-        const float4 av = *reinterpret_cast<const float4*>(Ar + i * dv + c0);
-        const float fr[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w}, ar[4] = {av.x, av.y, av.z, av.w};
+    // D = V - phi(K) A / den: one row x 4 columns per thread, i ascending; a warp holds two rows
+    // x 16 column blocks, so its reads of a row of phi(K) and of a row of A are broadcasts
+    for (int b = tid; b < n * (dv / 4); b += kUpdStreamThreads) {
+      const int r = b / (dv / 4), c0 = 4 * (b % (dv / 4));
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i0 = 0; i0 < dk; i0 += 4) {
+        const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
+        const float fr[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(fr[x], ar[y], acc[x][y]);
-      }
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int r = r0 + x;
-        if (r < n) {
-#pragma unroll
-          for (int y = 0; y < 4; ++y) D[r * dv + c0 + y] = Vr[r * dv + c0 + y] - acc[x][y] / den[r];
+        for (int x = 0; x < 4; ++x) {
+          const float4 av = *reinterpret_cast<const float4*>(Ar + (i0 + x) * dv + c0);
+          acc[0] = fmaf(fr[x], av.x, acc[0]);
+          acc[1] = fmaf(fr[x], av.y, acc[1]);
+          acc[2] = fmaf(fr[x], av.z, acc[2]);
+          acc[3] = fmaf(fr[x], av.w, acc[3]);
         }
       }
+#pragma unroll
+      for (int y = 0; y < 4; ++y) D[r * dv + c0 + y] = Vr[r * dv + c0 + y] - acc[y] / den[r];
     }
     __syncthreads();
-    // A' = A + phi(K)^T D: 8 rows of A x 4 columns per thread, rows of K ascending
+    // A' = A + phi(K)^T D: 4 rows of A x 4 columns per thread, rows of K ascending
     const Cell c = load_cell(a.cells, g);
     const size_t si = cell_index(a.state_mode, a.L, c);
     float* A = a.A + si * dk * dv;
-    for (int b = tid; b < (dk / 8) * (dv / 4); b += kUpdStreamThreads) {
-      const int i0 = 8 * (b / (dv / 4)), c0 = 4 * (b % (dv / 4));
-      float s8[8][4] = {};
+    for (int b = tid; b < (dk / 4) * (dv / 4); b += kUpdStreamThreads) {
+      const int i0 = 4 * (b / (dv / 4)), c0 = 4 * (b % (dv / 4));
+      float s4[4][4] = {};
       for (int r = 0; r < n; ++r) {
-        const float4 f0 = *reinterpret_cast<const float4*>(fk + r * dk + i0);
-        const float4 f1 = *reinterpret_cast<const float4*>(fk + r * dk + i0 + 4);
+        const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
         const float4 dd = *reinterpret_cast<const float4*>(D + r * dv + c0);
-        const float fr[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w}, dr[4] = {dd.x, dd.y, dd.z, dd.w};
+        const float fr[4] = {f.x, f.y, f.z, f.w}, dr[4] = {dd.x, dd.y, dd.z, dd.w};
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
+        for (int x = 0; x < 4; ++x)
 #pragma unroll
-          for (int y = 0; y < 4; ++y) s8[x][y] = fmaf(fr[x], dr[y], s8[x][y]);
+          for (int y = 0; y < 4; ++y) s4[x][y] = fmaf(fr[x], dr[y], s4[x][y]);
       }
 #pragma unroll
-      for (int x = 0; x < 8; ++x) {
+      for (int x = 0; x < 4; ++x) {
         const float4 old = *reinterpret_cast<const float4*>(Ar + (i0 + x) * dv + c0);
         *reinterpret_cast<float4*>(A + static_cast<size_t>(i0 + x) * dv + c0) =
-            make_float4(old.x + s8[x][0], old.y + s8[x][1], old.z + s8[x][2], old.w + s8[x][3]);
+            make_float4(old.x + s4[x][0], old.y + s4[x][1], old.z + s4[x][2], old.w + s4[x][3]);
       }
     }
     for (int i = tid; i < dk; i += kUpdStreamThreads) {
@@ -880,8 +847,6 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel
       t[2] = c.s;
     }
     __syncthreads();  // the stage, phi(K) and D are free again
-    if (g + 2 < c_end) issue(g + 2, st);
-    cp_async_commit();
   }
   cp_async_wait<0>();
 }
@@ -935,6 +900,11 @@ cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_
   if (a.dk % 32 || a.dv % 32 || a.dk > 128 || a.dv > 128) return cudaErrorInvalidValue;
   const size_t smem = (static_cast<size_t>(a.dk) * a.dv + a.dk) * sizeof(float);
   const bool tc = mem_read_tc_supported(a.dk, a.dv);
+  // an output row stride and low terms only on the tensor-core read
+  if ((a.ldo && a.ldo != a.dv) || a.lo_off) {
+    if (!tc || out_type == kElemF32 || a.ldo < a.dv + a.lo_off || a.ldo % 8 || a.lo_off % 8)
+      return cudaErrorInvalidValue;
+  }
   switch (out_type) {
     case kElemF32: return launch_mem_read_t<float>(a, smem, st);
     case kElemBF16: return tc ? launch_mem_read_tc(a, false, err, st) : launch_mem_read_mma_t<__nv_bfloat16>(a, st);
@@ -976,21 +946,25 @@ cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st) {
   int sms = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // many cells, whole keys and values: the streaming kernel (the same bits as the one below)
-  const size_t smem_stream = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv).total) * sizeof(float);
-  if (static_cast<long>(a.G) >= 4L * sms && (!a.part || a.nsplit == 1) && smem_stream <= 200 * 1024) {
+  // many cells, whole keys and values: the streaming kernel (the same bits as the one below),
+  // with a 4-stage ring when two CTAs of it fit on an SM (d_k = d_v = 64), else 2 stages
+  const size_t smem4 = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv, 4).total) * sizeof(float);
+  const size_t smem2 = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv, 2).total) * sizeof(float);
+  if (static_cast<long>(a.G) >= 4L * sms && (!a.part || a.nsplit == 1) && smem2 <= 200 * 1024) {
+    const bool four = smem4 <= 110 * 1024;
+    const size_t smem_stream = four ? smem4 : smem2;
+    void (*kern)(MemUpdateArgs) = four ? mem_update_stream_kernel<4> : mem_update_stream_kernel<2>;
     if (smem_stream > 48 * 1024)
-      cudaFuncSetAttribute(mem_update_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_stream);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_stream);
     int fit = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, mem_update_stream_kernel, kUpdStreamThreads, smem_stream) !=
-            cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kern, kUpdStreamThreads, smem_stream) != cudaSuccess ||
         fit <= 0) {
       cudaGetLastError();
       fit = 1;
     }
     const long cap = static_cast<long>(sms) * fit;
     const int grid = static_cast<int>(a.G < cap ? a.G : cap);
-    const cudaError_t e = launch_pdl(mem_update_stream_kernel, dim3(grid), dim3(kUpdStreamThreads), smem_stream, st, a);
+    const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kUpdStreamThreads), smem_stream, st, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

@@ -18,6 +18,8 @@
 // and the warps finish the previous tile: read its accumulator rows (one row per TMEM lane),
 // divide, round and store. Loads of tile i+1, the MMAs of tile i and the epilogue of tile i-1
 // overlap. Every wait is bounded; on a timeout the CTA records it in the error word and stops.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -48,6 +50,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 __device__ __forceinline__ uint32_t swz128(int r, int c) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
+
+// phi(x) = elu(x) + 1 without a branch, the exponential from the fast intrinsic (relative error
+// about 2^-21, far below the 16-bit output's rounding): x + 1 for x > 0, exp(x) otherwise.
+__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(fminf(x, 0.f)); }
 
 // Bounded CTA-wide barrier on an mbarrier that counts every thread's arrival.
 __device__ __forceinline__ bool cta_sync_bounded(uint32_t bar, uint32_t& phase, volatile int* abort) {
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(kRtThreads, DK == 64 ? 2 : 1) mem_read_tc_kern
       uint32_t h1[4], h2[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float p0 = phi_f(v[2 * k]), p1 = phi_f(v[2 * k + 1]);
+        const float p0 = phi_fast(v[2 * k]), p1 = phi_fast(v[2 * k + 1]);
         const float b0 = __bfloat162float(__float2bfloat16_rn(p0)), b1 = __bfloat162float(__float2bfloat16_rn(p1));
         h1[k] = pack_bf16x2(b0, b1);
         h2[k] = pack_bf16x2(p0 - b0, p1 - b1);
@@ -199,19 +205,30 @@ __global__ void __launch_bounds__(kRtThreads, DK == 64 ? 2 : 1) mem_read_tc_kern
     sm100::tmem_ld16(acc + dv, dn);
     sm100::tmem_wait_ld();
     const float inv = 1.f / (__uint_as_float(dn[0]) + a.eps);
-    T* o = static_cast<T*>(a.o) + (static_cast<size_t>(cell_index(a.mode, a.L, c)) * M + row) * dv;
+    const int ldo = a.ldo ? a.ldo : dv;
+    T* o = static_cast<T*>(a.o) + (static_cast<size_t>(cell_index(a.mode, a.L, c)) * M + row) * ldo;
     const int half = dv / 2, c0 = (warp >> 2) * half;
     for (int cc = c0; cc < c0 + half; cc += 16) {
       uint32_t v[16];
       sm100::tmem_ld16(acc + cc, v);
       sm100::tmem_wait_ld();
       if (row < M) {
-        uint32_t p[8];
+        float y[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) p[k] = pack2<T>(__uint_as_float(v[2 * k]) * inv, __uint_as_float(v[2 * k + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(o + cc);
-        dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
-        dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+        for (int k = 0; k < 16; ++k) y[k] = __uint_as_float(v[k]) * inv;
+#pragma unroll 1
+        for (int pass = 0; pass < (a.lo_off ? 2 : 1); ++pass) {  // split-operand mode: then the low terms
+          if (pass == 1) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) y[k] = lo_term<T>(y[k]);
+          }
+          uint32_t p[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) p[k] = pack2<T>(y[2 * k], y[2 * k + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(o + cc + pass * a.lo_off);
+          dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+          dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+        }
       }
     }
   };
@@ -294,21 +311,25 @@ cudaError_t launch_dk(const MemReadArgs& a, int* err, cudaStream_t st) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!attr[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(mem_read_tc_kernel<T, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem_max));
+    const void* fn = reinterpret_cast<const void*>(mem_read_tc_kernel<T, DK>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
+    // as many CTAs per SM as the registers and shared memory allow (two at d_k = 64: two tiles'
+    // loads in flight per SM)
+    cudaFuncAttributes fa{};
+    int smem_sm = 0, regs_sm = 0;
+    cudaFuncGetAttributes(&fa, fn);
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    const int by_smem = static_cast<int>(smem_sm / (smem_max + 1024));
+    const int by_regs = fa.numRegs > 0 ? regs_sm / (fa.numRegs * kRtThreads) : 1;
+    per_sm[dev] = std::max(1, std::min(by_smem, by_regs));
     attr[dev] = true;
   }
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // as many CTAs as fit at once (two per SM at d_k = 64: two tiles' loads in flight per SM)
-  int fit = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, mem_read_tc_kernel<T, DK>, kRtThreads, smem) != cudaSuccess ||
-      fit <= 0) {
-    cudaGetLastError();
-    fit = 1;
-  }
-  per_sm[dev] = fit;
   const long tiles = static_cast<long>(a.G) * ((a.M + kRtRows - 1) / kRtRows);
   const long cap = static_cast<long>(sms) * per_sm[dev];
   const int grid = static_cast<int>(tiles < cap ? tiles : cap);

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kRmsWarps * 32) rmsnorm_kernel(const RmsArgs a
 // overflows is reported in the error word.
 template <typename T>
 __global__ void assemble_kernel(const Cell* cells, const T* emb, const T* mem, float* x, __half* xb, int M, int n_mem,
-                                int d, int* err) {
+                                int d, int split, int* err) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   const Cell c = load_cell(cells, blockIdx.y);
@@ -79,12 +79,16 @@ __global__ void assemble_kernel(const Cell* cells, const T* emb, const T* mem, f
   const T* src = r < seg ? emb + (static_cast<size_t>(c.t0) + r) * d
                          : (r < m ? mem + static_cast<size_t>(r - seg) * d : nullptr);
   const size_t row = (static_cast<size_t>(c.xin) * M + r) * d;
+  const size_t rowb = split ? 2 * row : row;  // split-operand mode: [high terms | low terms] rows of 2d
   float amax = 0.f;
   for (int k = threadIdx.x * 4; k < d; k += blockDim.x * 4) {
     const float4 v = src ? Vec4<T>::load(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
     Vec4<float>::store(x + row + k, v);
     if (xb) {
-      Vec4<__half>::store(xb + row + k, v);
+      Vec4<__half>::store(xb + rowb + k, v);
+      if (split)
+        Vec4<__half>::store(xb + rowb + d + k, make_float4(lo_term<__half>(v.x), lo_term<__half>(v.y),
+                                                           lo_term<__half>(v.z), lo_term<__half>(v.w)));
       amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
     }
   }
@@ -178,15 +182,17 @@ cudaError_t launch_rmsnorm(const RmsArgs& a, bool bf16, cudaStream_t st) {
 }
 
 cudaError_t launch_assemble(const Cell* cells, int G, const void* emb, const void* mem, float* x, __half* xb, int M,
-                            int n_mem, int d, bool bf16, int* err, cudaStream_t st) {
+                            int n_mem, int d, bool bf16, int* err, cudaStream_t st, bool split) {
   if (d % 4) return cudaErrorInvalidValue;
   if (G <= 0) return cudaSuccess;
   const int threads = d >= 1024 ? 256 : 128;
+  const int sp = split ? 1 : 0;
   if (bf16)
     return launch_pdl(assemble_kernel<__nv_bfloat16>, dim3(M, G), dim3(threads), 0, st, cells,
-                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d, err);
+                      static_cast<const __nv_bfloat16*>(emb), static_cast<const __nv_bfloat16*>(mem), x, xb, M, n_mem, d,
+                      sp, err);
   return launch_pdl(assemble_kernel<float>, dim3(M, G), dim3(threads), 0, st, cells, static_cast<const float*>(emb),
-                    static_cast<const float*>(mem), x, xb, M, n_mem, d, err);
+                    static_cast<const float*>(mem), x, xb, M, n_mem, d, sp, err);
 }
 
 cudaError_t launch_row_ssq(const float* x, float* ss, int M, int d, int parts, cudaStream_t st) {

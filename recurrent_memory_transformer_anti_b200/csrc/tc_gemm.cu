@@ -78,7 +78,7 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
     store32_f32(static_cast<float*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
   } else if constexpr (EPI == kEpiStoreAct) {
     const size_t idx = cell_index(ep.out_mode, a.L, c);
-    store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v);
+    store32_16_split(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + col, v, ep.lo_off);
     track_amax<OpT>(amax, v);
   } else if constexpr (EPI == kEpiResid || EPI == kEpiResidCast) {
     const size_t di = cell_index(ep.dst_mode, a.L, c);
@@ -92,7 +92,8 @@ __device__ __forceinline__ float epi_chunk(const TcGemmArgs& a, Cell c, int row,
     }
     store32_f32(dst, v);
     if constexpr (EPI == kEpiResidCast) {
-      store32_16(static_cast<OpT*>(ep.xb) + (di * a.M + row) * ep.ldx + col, v);
+      const int ldxb = ep.ldxb ? ep.ldxb : ep.ldx;
+      store32_16_split(static_cast<OpT*>(ep.xb) + (di * a.M + row) * ldxb + col, v, ep.lo_off);
       track_amax<OpT>(amax, v);
     }
     float ss = 0.f;
@@ -119,6 +120,13 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
     const int dh = ep.head_dim, half = dh >> 1;
     const size_t idx = cell_index(ep.out_mode, a.L, c);
     OpT* orow = static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo;
+    float* orow32 = static_cast<float*>(ep.out) + (idx * a.M + row) * ep.ldo;  // out_f32
+    auto put = [&](int col, const float* v) {
+      if (ep.out_f32)
+        store32_f32(orow32 + col, v);
+      else
+        store32_16(orow + col, v);
+    };
     const int heads = BN / dh;
     // rotation pairs (i, i + dh/2) of each head, in 32-wide units: heads * max(1, half/32)
     const int per_head = half >= 32 ? half / 32 : 1;
@@ -151,8 +159,8 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
               x2[j] = a2;
             }
           }
-          store32_16(orow + n0 + h0 + p, x1);
-          store32_16(orow + n0 + h0 + half + p, x2);
+          put(n0 + h0 + p, x1);
+          put(n0 + h0 + half + p, x2);
           track_amax<OpT>(amax, x1);
           track_amax<OpT>(amax, x2);
         }
@@ -174,7 +182,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
               x[j + 16] = a2;
             }
           }
-          store32_16(orow + n0 + h0, x);
+          put(n0 + h0, x);
           track_amax<OpT>(amax, x);
         }
       }
@@ -196,7 +204,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& a, uint32_t tacc
         float y[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) y[j] = silu_f(u2f(g[j]) * rs) * (u2f(up[j]) * rs);
-        store32_16(orow + (n0 + b0) / 2 + p, y);
+        store32_16_split(orow + (n0 + b0) / 2 + p, y, ep.lo_off);
         track_amax<OpT>(amax, y);
       }
     }
@@ -297,21 +305,31 @@ __device__ __forceinline__ bool epilogue_resid_tma(const TcGemmArgs& a, const CU
       if (valid) track_amax<OpT>(amax, y);
       // the 16-bit copy: stage the warp's 32 x 32 block, then store it row by row, each
       // instruction covering 8 rows x 64 contiguous bytes
+      // (split-operand mode: a second pass stores the low terms lo_off columns further)
+      const int ldxb = ep.ldxb ? ep.ldxb : ep.ldx;
       uint4* mine = reinterpret_cast<uint4*>(xstage + lane * 80);
+      OpT* xb = static_cast<OpT*>(ep.xb) + ((size_t)dst * a.M + rowbase) * ldxb + col + (lane & 3) * 8;
+#pragma unroll 1
+      for (int pass = 0; pass < (ep.lo_off ? 2 : 1); ++pass) {
+        if (pass == 1) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        mine[q] = make_uint4(pack2<OpT>(y[8 * q], y[8 * q + 1]), pack2<OpT>(y[8 * q + 2], y[8 * q + 3]),
-                             pack2<OpT>(y[8 * q + 4], y[8 * q + 5]), pack2<OpT>(y[8 * q + 6], y[8 * q + 7]));
-      __syncwarp();
-      OpT* xb = static_cast<OpT*>(ep.xb) + ((size_t)dst * a.M + rowbase) * ep.ldx + col + (lane & 3) * 8;
+          for (int j = 0; j < 32; ++j) y[j] = lo_term<OpT>(y[j]);
+        }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int r2 = (lane >> 2) + 8 * k;
-        if (rowbase + r2 < a.M)
-          *reinterpret_cast<uint4*>(xb + static_cast<size_t>(r2) * ep.ldx) =
-              *reinterpret_cast<const uint4*>(xstage + r2 * 80 + (lane & 3) * 16);
+        for (int q = 0; q < 4; ++q)
+          mine[q] = make_uint4(pack2<OpT>(y[8 * q], y[8 * q + 1]), pack2<OpT>(y[8 * q + 2], y[8 * q + 3]),
+                               pack2<OpT>(y[8 * q + 4], y[8 * q + 5]), pack2<OpT>(y[8 * q + 6], y[8 * q + 7]));
+        __syncwarp();
+        OpT* xp = xb + pass * ep.lo_off;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r2 = (lane >> 2) + 8 * k;
+          if (rowbase + r2 < a.M)
+            *reinterpret_cast<uint4*>(xp + static_cast<size_t>(r2) * ldxb) =
+                *reinterpret_cast<const uint4*>(xstage + r2 * 80 + (lane & 3) * 16);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     sm100::fence_async_smem();
     __syncwarp();
@@ -460,7 +478,7 @@ __device__ __forceinline__ void epilogue_mem_read(const TcGemmArgs& a, uint32_t 
 #pragma unroll
   for (int j = 0; j < HV; ++j) acc[j] *= inv;
   const size_t idx = cell_index(ep.out_mode, a.L, c);
-  store32_16(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + part * HV, acc);
+  store32_16_split(static_cast<OpT*>(ep.out) + (idx * a.M + row) * ep.ldo + part * HV, acc, ep.lo_off);
   track_amax<OpT>(amax, acc);
 }
 
@@ -513,7 +531,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int mt = (args.M + C::BM - 1) / C::BM;
   const int nt = args.N / BN;
-  const int kbn = args.K / C::BK;
+  const int kbw = args.K / C::BK;                    // 64-column blocks of the weight
+  const int kbn = args.kx_lo ? 2 * kbw : kbw;        // of the product (split-operand mode: twice)
   const int tiles = args.G * mt * nt;
 
   if (warp == 0) {
@@ -534,8 +553,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t sa = base + stage * C::STAGE_BYTES;
           sm100::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-          sm100::tma_load_3d(sa, &tmA, kb * C::BK, m_tile * C::BM, a3, full_bar(stage));
-          sm100::tma_load_3d(sa + C::A_BYTES, &tmB, kb * C::BK, n_tile * BN, c.l, full_bar(stage));
+          const int kw = (kb % kbw) * C::BK, kx = kw + (kb / kbw) * args.kx_lo;
+          sm100::tma_load_3d(sa, &tmA, kx, m_tile * C::BM, a3, full_bar(stage));
+          sm100::tma_load_3d(sa + C::A_BYTES, &tmB, kw, n_tile * BN, c.l, full_bar(stage));
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -809,6 +829,8 @@ bool make_tmap_f32_resid(CUtensorMap* map, const float* base, uint64_t inner, ui
 cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tx, const TcGemmArgs& args,
                            int bn, bool f16, cudaStream_t st) {
   if (args.K % 64 != 0 || args.M <= 0) return cudaErrorInvalidValue;
+  if (args.kx_lo && (args.kx_lo < args.K || args.kx_lo % 8 != 0)) return cudaErrorInvalidValue;
+  if (args.ep.out_f32 && (args.epi != kEpiRope || args.ep.rope_tma)) return cudaErrorInvalidValue;
   return f16 ? launch_op<__half>(ta, tb, tx, args, bn, st) : launch_op<__nv_bfloat16>(ta, tb, tx, args, bn, st);
 }
 

@@ -121,7 +121,8 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
     const float* src = ep.x + (si * M + tok0) * ep.ldx + f;
     float* dst = ep.x + (di * M + tok0) * ep.ldx + f;
     OpT* xb = nullptr;
-    if constexpr (EPI == kEpiResidCast) xb = static_cast<OpT*>(ep.xb) + (di * M + tok0) * ep.ldx + f;
+    const int ldxb = ep.ldxb ? ep.ldxb : ep.ldx;
+    if constexpr (EPI == kEpiResidCast) xb = static_cast<OpT*>(ep.xb) + (di * M + tok0) * ldxb + f;
     const bool want_ss = ep.ss_out != nullptr;
     float xs[16];
 #pragma unroll
@@ -141,7 +142,9 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         if (j0 + j < lim) {
           dst[static_cast<size_t>(j0 + j) * ep.ldx] = y;
           if constexpr (EPI == kEpiResidCast) {
-            xb[static_cast<size_t>(j0 + j) * ep.ldx] = from_f32<OpT>(y);
+            OpT* xr = xb + static_cast<size_t>(j0 + j) * ldxb;
+            *xr = from_f32<OpT>(y);
+            if (ep.lo_off) xr[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
             track_amax<OpT>(amax, y);
           }
         }
@@ -181,7 +184,9 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
     const int dh = ep.head_dim, hh = dh >> 1;
     const int i = f % dh, p = i >> 1;
     const bool odd = i & 1, rot = f < ep.rope_cols;
-    OpT* out = static_cast<OpT*>(ep.out) + (static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * M + tok0) * ep.ldo + f;
+    const size_t o0 = (static_cast<size_t>(cell_index(ep.out_mode, a.L, c)) * M + tok0) * ep.ldo + f;
+    OpT* out = static_cast<OpT*>(ep.out) + o0;
+    float* out32 = static_cast<float*>(ep.out) + o0;  // out_f32
     const float2 step = (rot && M > 1) ? ep.rope[hh + p] : make_float2(1.f, 0.f);
 #pragma unroll 1
     for (int j0 = 0; j0 < cnt; j0 += 32) {
@@ -195,8 +200,12 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const float other = __shfl_xor_sync(0xffffffffu, x, 1);
         const float y = odd ? fmaf(x, cs.x, other * cs.y) : fmaf(x, cs.x, -other * cs.y);
         if (j0 + j < lim) {
-          out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
-          track_amax<OpT>(amax, y);
+          if (ep.out_f32) {
+            out32[static_cast<size_t>(j0 + j) * ep.ldo] = y;
+          } else {
+            out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
+            track_amax<OpT>(amax, y);
+          }
         }
         cs = make_float2(fmaf(cs.x, step.x, -cs.y * step.y), fmaf(cs.y, step.x, cs.x * step.y));
       }
@@ -222,7 +231,9 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const int t = j0 + (odd ? 16 : 0) + j;
         if (t < lim) {
           const float y = silu_fast(g) * u;
-          out[static_cast<size_t>(t) * ep.ldo] = from_f32<OpT>(y);
+          OpT* o = out + static_cast<size_t>(t) * ep.ldo;
+          *o = from_f32<OpT>(y);
+          if (ep.lo_off) o[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
           track_amax<OpT>(amax, y);
         }
       }
@@ -323,6 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   const int t1 = G * np0 * ntt, t2 = t1 + G * np1 * ntt, tiles = t2 + G * np2 * ntt;
   auto npair_of = [&](int p) { return p == 0 ? np0 : (p == 1 ? np1 : np2); };
   auto k_of = [&](int p) { return p == 0 ? a0.K : (p == 1 ? args.ph[1].K : args.ph[2].K); };
+  auto kx_lo_of = [&](int p) { return p == 0 ? a0.kx_lo : (p == 1 ? args.ph[1].kx_lo : args.ph[2].kx_lo); };
   auto decode = [&](int t, int& p, int& g, int& fp, int& tt) {
     p = (NP > 1 && t >= t1) ? ((NP > 2 && t >= t2) ? 2 : 1) : 0;
     const int r0 = t - (p == 0 ? 0 : (p == 1 ? t1 : t2)), per = npair_of(p) * ntt;
@@ -355,7 +367,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         const CUtensorMap* tw = p == 0 ? &tmW0 : (p == 1 ? &tmW1 : &tmW2);
         const CUtensorMap* tx = p == 0 ? &tmX0 : (p == 1 ? &tmX1 : &tmX2);
         const IndexMode amode = p == 0 ? a0.a_mode : (p == 1 ? args.ph[1].a_mode : args.ph[2].a_mode);
-        const int kblk = k_of(p) / C::BK;  // 64-column blocks
+        const int kbw = k_of(p) / C::BK;            // 64-column blocks of the weight
+        const int kxl = kx_lo_of(p);                 // split-operand mode: column of the low terms
+        const int kblk = kxl ? 2 * kbw : kbw;        // 64-column blocks of the product
         const int kst = (kblk + 1) / 2;    // ring stages per tile (the last may hold one block)
         const Cell c = load_cell(a0.cells, g);
         const int a3 = cell_index(amode, a0.L, c);
@@ -380,8 +394,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           const uint32_t sa = ring + static_cast<uint32_t>(stage) * 2u * BLK;
           const uint32_t fb = sm100::mapa_shared(full_bar(stage), 0);
           for (int b = 0; b < nb; ++b) {
-            sm100::tma_load_3d_pair(sa + b * BLK, tw, (2 * ks + b) * C::BK, wrow, c.l, fb);
-            sm100::tma_load_3d_pair(sa + b * BLK + C::W_BYTES, tx, (2 * ks + b) * C::BK, xrow, a3, fb);
+            const int blk = 2 * ks + b, kw = (blk % kbw) * C::BK, kx = kw + (blk / kbw) * kxl;
+            sm100::tma_load_3d_pair(sa + b * BLK, tw, kw, wrow, c.l, fb);
+            sm100::tma_load_3d_pair(sa + b * BLK + C::W_BYTES, tx, kx, xrow, a3, fb);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -416,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       for (int t = cl; t < tiles && ok; t += ncl) {
         int p, g, fp, tt;
         decode(t, p, g, fp, tt);
-        const int kblk = k_of(p) / C::BK, kst = (kblk + 1) / 2;
+        const int kblk = (k_of(p) / C::BK) * (kx_lo_of(p) ? 2 : 1), kst = (kblk + 1) / 2;
         const uint32_t idesc = idesc0 | (static_cast<uint32_t>(tile_tokens(tt) >> 3) << 17);
         if (!sm100::mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag)) {
           ok = false;
@@ -673,9 +688,13 @@ bool tc_pair_supported(int M, int N, int K, int epi, int head_dim) {
   return pair_token_tile(M) <= 256;
 }
 
+// A split-operand X keeps its low terms at a 16-byte aligned column at or past its high terms.
+static bool kx_lo_ok(const TcGemmArgs& a) { return a.kx_lo == 0 || (a.kx_lo >= a.K && a.kx_lo % 8 == 0); }
+
 cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, bool f16,
                                 cudaStream_t st) {
-  if (!tc_pair_supported(args.M, args.N, args.K, args.epi, args.ep.head_dim)) return cudaErrorInvalidValue;
+  if (!tc_pair_supported(args.M, args.N, args.K, args.epi, args.ep.head_dim) || !kx_lo_ok(args))
+    return cudaErrorInvalidValue;
   return f16 ? launch_pair_op<__half>(tw, tx, args, st) : launch_pair_op<__nv_bfloat16>(tw, tx, args, st);
 }
 
@@ -686,7 +705,7 @@ cudaError_t launch_tc_pair_chain_o_mlp(const CUtensorMap* tw, const CUtensorMap*
       a[2].epi != kEpiResidCast)
     return cudaErrorInvalidValue;
   for (int p = 0; p < 3; ++p) {
-    if (!tc_pair_supported(a[p].M, a[p].N, a[p].K, a[p].epi, a[p].ep.head_dim) || a[p].M != a[0].M ||
+    if (!tc_pair_supported(a[p].M, a[p].N, a[p].K, a[p].epi, a[p].ep.head_dim) || !kx_lo_ok(a[p]) || a[p].M != a[0].M ||
         a[p].G != a[0].G || a[p].cells != a[0].cells)
       return cudaErrorInvalidValue;
   }

@@ -19,9 +19,11 @@ DEBUG_LIB_PATH = os.path.join(_HERE, "librmt_debug.so")
 
 RMT_OK, RMT_EINVAL, RMT_ENOMEM, RMT_ECUDA, RMT_ETIMEOUT, RMT_ESTATE, RMT_ERANGE, RMT_EDEBUG = range(8)
 RMT_DIAGONAL, RMT_SEQUENTIAL = 0, 1
-RMT_F32, RMT_BF16 = 0, 1
+RMT_F32, RMT_BF16, RMT_BF16_SPLIT = 0, 1, 2
 SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
-DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16}
+# "bf16-split": bf16 storage, split (high + low f16 term) tensor-core operands (include/rmt.h)
+DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16, "bf16-split": RMT_BF16_SPLIT}
+STORAGE_BF16 = ("bf16", "bf16-split")
 STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE",
                 6: "RMT_ERANGE", 7: "RMT_EDEBUG"}
 
@@ -317,7 +319,7 @@ def storage(a, dtype: str, device=None):
     """A float32 array as a torch tensor in the model's storage dtype (marshalling helper)."""
     import torch
     t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
-    t = t.to(torch.bfloat16) if dtype == "bf16" else t
+    t = t.to(torch.bfloat16) if dtype in STORAGE_BF16 else t
     return t.to(device) if device is not None else t
 
 
