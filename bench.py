@@ -512,7 +512,7 @@ def main() -> int:
         barrier()
         full_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         rmt.rmt_sync(h, stream)
-        full = {"model": "the same 16-layer decoder without the associative memory, causal over all tokens",
+        full = {"model": f"the same {cfg.n_layers}-layer decoder without the associative memory, causal over all tokens",
                 "ms_per_step": full_ms, "tokens_per_s": job_throughput(tokens, full_ms, world),
                 "armt_diagonal_speedup": full_ms / ms, "pages_speedup": 3.3}
 

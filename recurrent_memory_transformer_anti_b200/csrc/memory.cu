@@ -392,12 +392,21 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
 // y3 = bf16(y - y1 - y2)), which carry all of its 24 significand bits; the weights are exact in
 // bf16, so the three products per 16-column step go into one fp32 accumulator, terms in that
 // order, steps ascending. The rows and the weight rows of the split are staged with cp.async
-// (all of a CTA's 16-byte chunks in flight at once); the rows are split while the A fragments
-// are formed and the weights read as B fragments with ldmatrix. Warp w computes the 8-column
-// output tiles w and w + 8 of every 16-row tile.
+// (all of a CTA's 16-byte chunks in flight at once); the CTA then splits the rows once into
+// three bf16 planes, and every warp reads its A fragments from them and its B fragments from
+// the weights with ldmatrix (the warps share the rows: splitting while forming the fragments
+// would repeat the conversion in every warp). Warp w computes the 8-column output tiles w and
+// w + 8 of every 16-row tile.
 constexpr int kKvMmaThreads = 256;
-constexpr int kKvYStride = kMemKvSplit + 8;  // fp32 row stride of the staged rows (fragment loads spread over all banks)
+constexpr int kKvYStride = kMemKvSplit + 8;  // fp32 row stride of the staged rows
 constexpr int kKvWStride = kMemKvSplit + 8;  // bf16 row stride of the staged weights (272 B: ldmatrix rows on distinct banks)
+constexpr int kKvPStride = kMemKvSplit + 8;  // bf16 row stride of the split planes (same reason)
+
+// Shared memory of the tensor-core k/v kernel: fp32 rows, weight rows, three split planes.
+inline size_t kv_mma_smem(int n, int cols) {
+  const size_t n16 = (n + 15) & ~15, wrows = (cols + 7) / 8 * 8;
+  return sizeof(float) * n16 * kKvYStride + 2 * wrows * kKvWStride + 3 * 2 * n16 * kKvPStride;
+}
 
 __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvArgs a) {
   pdl_trigger();
@@ -409,6 +418,7 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
   const int ntiles = (cols + 7) / 8;
   float* Ys = reinterpret_cast<float*>(kv_sm);                                                      // [n16][kKvYStride]
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(kv_sm + sizeof(float) * n16 * kKvYStride);  // [8*ntiles][kKvWStride]
+  __nv_bfloat16* Ps = Ws + 8 * ntiles * kKvWStride;  // [3][n16][kKvPStride]: y1, y2, y3
   const Cell c = load_cell(a.cells, blockIdx.y);
   const int split = blockIdx.x, k0 = split * KS;
   const int kw = min(KS, a.d - k0);
@@ -456,6 +466,17 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
+  // the rows' three bf16 terms, two columns per step
+  for (int e = tid; e < n16 * (KS / 2); e += kKvMmaThreads) {
+    const int r = e / (KS / 2), k = 2 * (e % (KS / 2));
+    uint32_t t1, t2, t3;
+    split3(*reinterpret_cast<const float2*>(Ys + r * kKvYStride + k), t1, t2, t3);
+    uint32_t* p = reinterpret_cast<uint32_t*>(Ps + r * kKvPStride + k);
+    p[0] = t1;
+    p[n16 * kKvPStride / 2] = t2;
+    p[n16 * kKvPStride] = t3;
+  }
+  __syncthreads();
   const int warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
   const int nsplit = (a.d + KS - 1) / KS;
   float* part = a.part + (static_cast<size_t>(c.k) * nsplit + split) * a.n * a.dkv;
@@ -466,17 +487,19 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
   const int lr = lane & 7, lk = ((lane >> 3) & 1) * 8;
   const uint32_t wb0 = sm100::smem_u32(Ws + (nt0 * 8 + lr) * kKvWStride + lk);
   const uint32_t wb1 = has1 ? sm100::smem_u32(Ws + (nt1 * 8 + lr) * kKvWStride + lk) : wb0;
+  // ldmatrix x4 row addresses of a 16 x 16 A tile: lanes 0-15 rows 0-15 at k 0, lanes 16-31 at k 8
+  const uint32_t plane = 2u * n16 * kKvPStride;  // bytes
+  const uint32_t pa0 =
+      sm100::smem_u32(Ps + ((lane & 7) + ((lane >> 3) & 1) * 8) * kKvPStride + (lane >> 4) * 8);
   for (int mt = 0; mt < n16 / 16; ++mt) {
     float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* y0 = Ys + (mt * 16 + gq) * kKvYStride + 2 * tq;
-    const float* y8 = y0 + 8 * kKvYStride;
+    const uint32_t pa = pa0 + 2u * 16 * kKvPStride * mt;
 #pragma unroll 2
     for (int ks = 0; ks < KS / 16; ++ks) {
       uint32_t t1[4], t2[4], t3[4];
-      split3(*reinterpret_cast<const float2*>(y0 + 16 * ks), t1[0], t2[0], t3[0]);
-      split3(*reinterpret_cast<const float2*>(y8 + 16 * ks), t1[1], t2[1], t3[1]);
-      split3(*reinterpret_cast<const float2*>(y0 + 16 * ks + 8), t1[2], t2[2], t3[2]);
-      split3(*reinterpret_cast<const float2*>(y8 + 16 * ks + 8), t1[3], t2[3], t3[3]);
+      ldmatrix_x4(pa + 32u * ks, t1);
+      ldmatrix_x4(pa + plane + 32u * ks, t2);
+      ldmatrix_x4(pa + 2 * plane + 32u * ks, t3);
       uint32_t b0, b1;
       ldmatrix_x2(wb0 + 32u * ks, b0, b1);
       mma_bf16_16816(acc0, t1, b0, b1);
@@ -731,7 +754,7 @@ struct UpdStreamLayout {  // in floats; every region starts 16-byte aligned
 // A ring of NST cell stages: the loads of cells g+1 .. g+NST-1 are in flight while cell g is
 // computed (the stage of cell g+NST-1 is the one cell g-1 just released).
 template <int NST>
-__global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel(const MemUpdateArgs a) {
+__global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel(const MemUpdateArgs a) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ __align__(16) float us[];
@@ -796,6 +819,7 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel
     for (int b = tid; b < n * (dv / 4); b += kUpdStreamThreads) {
       const int r = b / (dv / 4), c0 = 4 * (b % (dv / 4));
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
       for (int i0 = 0; i0 < dk; i0 += 4) {
         const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
         const float fr[4] = {f.x, f.y, f.z, f.w};
@@ -819,6 +843,7 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 2) mem_update_stream_kernel
     for (int b = tid; b < (dk / 4) * (dv / 4); b += kUpdStreamThreads) {
       const int i0 = 4 * (b / (dv / 4)), c0 = 4 * (b % (dv / 4));
       float s4[4][4] = {};
+#pragma unroll 4
       for (int r = 0; r < n; ++r) {
         const float4 f = *reinterpret_cast<const float4*>(fk + r * dk + i0);
         const float4 dd = *reinterpret_cast<const float4*>(D + r * dv + c0);
@@ -919,8 +944,8 @@ cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (a.n > 64 || a.dkv % 4) return cudaErrorInvalidValue;
   dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G, (a.dkv + kKvCols - 1) / kKvCols);
   if (bf16) {  // tensor cores: three-term split of the fp32 rows against the bf16 weights
-    const int n16 = (a.n + 15) & ~15, cols = a.dkv < kKvCols ? a.dkv : kKvCols;
-    const size_t smem = sizeof(float) * n16 * kKvYStride + 2 * static_cast<size_t>((cols + 7) / 8 * 8) * kKvWStride;
+    const int cols = a.dkv < kKvCols ? a.dkv : kKvCols;
+    const size_t smem = kv_mma_smem(a.n, cols);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(mem_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     const cudaError_t e = launch_pdl(mem_kv_mma_kernel, grid, dim3(kKvMmaThreads), smem, st, a);
@@ -947,13 +972,11 @@ cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // many cells, whole keys and values: the streaming kernel (the same bits as the one below),
-  // with a 4-stage ring when two CTAs of it fit on an SM (d_k = d_v = 64), else 2 stages
-  const size_t smem4 = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv, 4).total) * sizeof(float);
-  const size_t smem2 = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv, 2).total) * sizeof(float);
-  if (static_cast<long>(a.G) >= 4L * sms && (!a.part || a.nsplit == 1) && smem2 <= 200 * 1024) {
-    const bool four = smem4 <= 110 * 1024;
-    const size_t smem_stream = four ? smem4 : smem2;
-    void (*kern)(MemUpdateArgs) = four ? mem_update_stream_kernel<4> : mem_update_stream_kernel<2>;
+  // two cell stages per CTA (a 4-stage ring measured no faster: the arithmetic, not the loads,
+  // sets its pace)
+  const size_t smem_stream = static_cast<size_t>(UpdStreamLayout(a.n, a.dk, a.dv, 2).total) * sizeof(float);
+  if (static_cast<long>(a.G) >= 4L * sms && (!a.part || a.nsplit == 1) && smem_stream <= 200 * 1024) {
+    void (*kern)(MemUpdateArgs) = mem_update_stream_kernel<2>;
     if (smem_stream > 48 * 1024)
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_stream);
     int fit = 0;

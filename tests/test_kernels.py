@@ -103,6 +103,7 @@ def test_attention_matches_oracle(dtype, G, M, H, Hkv, dh):
                                              ("f32", 2, 72, 32, 32), ("f32", 2, 77, 128, 128),
                                              ("f32", 2, 50, 32, 96), ("bf16", 4, 130, 128, 64),
                                              ("bf16", 2, 2064, 128, 128), ("bf16", 300, 130, 64, 32),
+                                             ("bf16", 300, 130, 64, 64), ("bf16", 40, 1040, 64, 128),
                                              ("bf16", 1, 1, 64, 64), ("bf16", 2, 300, 32, 64), ("bf16", 3, 77, 96, 96)])
 def test_memory_read_matches_oracle(dtype, G, M, dk, dv):
     r = rng(300 + M + dk)
