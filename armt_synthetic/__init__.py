@@ -52,6 +52,7 @@ class ArmtConfig:
     rms_eps: float = 1e-5
     mem_eps: float = 1e-6
     dtype: str = "f32"          # "f32" or "bf16": storage type of weights and activations
+    mem_update: str = "batched"  # "batched" or "sequential": how a cell writes its memory rows
 
     @property
     def m_tokens(self) -> int:

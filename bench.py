@@ -337,6 +337,10 @@ def run_microbench(args, local: int) -> int:
         ms = median_ms(lambda: rmt.rmt_memory_update(k, v, A, z, G, n, dk, dv, eps))
         emit("memory_update", {"G": G, "n": n, "dk": dk, "dv": dv}, ms,
              G * (n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), "GB/s", hbm, "hbm_gbs")
+        # the per-token rule: the same bytes, plus the rows' Gram matrix and a forward substitution
+        ms = median_ms(lambda: rmt.rmt_memory_update_sequential(k, v, A, z, G, n, dk, dv, eps))
+        emit("memory_update_sequential", {"G": G, "n": n, "dk": dk, "dv": dv}, ms,
+             G * (n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), "GB/s", hbm, "hbm_gbs")
         del k, v, A, z
     for G in (16, 2048):
         y = torch.randn(G, n, d, device=dev, generator=gen)

@@ -65,6 +65,12 @@ typedef enum { RMT_DIAGONAL = 0, RMT_SEQUENTIAL = 1 } rmt_schedule;
  * Needs d_k of 64 or 128. rmt_full_attention_forward does not take it. */
 typedef enum { RMT_F32 = 0, RMT_BF16 = 1, RMT_BF16_SPLIT = 2 } rmt_dtype;
 
+/* How a cell writes its n_mem memory rows (the delta rule of rmt_memory_update):
+ * RMT_MEM_BATCHED: every row against the pre-update A, z (the rows' writes are summed).
+ * RMT_MEM_SEQUENTIAL: the rows one after another, each against the state the earlier rows of
+ * the cell left -- the per-token delta rule (rmt_memory_update_sequential). */
+typedef enum { RMT_MEM_BATCHED = 0, RMT_MEM_SEQUENTIAL = 1 } rmt_mem_update;
+
 /* Model shape. A cell has M = seg_len + n_mem rows: the segment's tokens followed by the
  * n_mem memory tokens. Limits (else RMT_EINVAL): all sizes > 0; n_heads % n_kv_heads == 0;
  * head_dim in {32, 64, 128}; d_k, d_v multiples of 32, at most 128; n_mem <= 64 and
@@ -78,6 +84,7 @@ typedef struct {
   float rms_eps;    /* RMSNorm epsilon (1e-5) */
   float mem_eps;    /* associative-memory epsilon in both denominators (1e-6) */
   rmt_dtype dtype;
+  rmt_mem_update mem_update; /* RMT_MEM_BATCHED or RMT_MEM_SEQUENTIAL */
 } rmt_cfg;
 
 /* Model weights, in cfg.dtype. Each `const void* const*` member is a host array of
@@ -309,6 +316,16 @@ rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void*
  * (RMT_EINVAL otherwise). */
 rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G,
                              int32_t n, int32_t dk, int32_t dv, float eps, void* stream);
+
+/* The per-token delta rule: rows r = 0 .. n-1 of each group written one after another, row r
+ * against the state rows 0 .. r-1 left:
+ *   v_bar_r = phi(k_r) A_r / (phi(k_r) . z_r + eps);  A_{r+1} = A_r + phi(k_r)^T (v_r - v_bar_r);
+ *   z_{r+1} = z_r + phi(k_r).
+ * Same arguments, layouts and errors as rmt_memory_update. The kernels form it from the
+ * batched quantities and the rows' Gram matrix G_rj = phi(k_r) . phi(k_j) (forward
+ * substitution over the rows), so it agrees with the row-by-row loop up to rounding. */
+rmt_status rmt_memory_update_sequential(const float* k, const float* v, float* A, float* z, int32_t G,
+                                        int32_t n, int32_t dk, int32_t dv, float eps, void* stream);
 
 /* Memory write from n rows per group (a layer's memory-token outputs):
  *   k = y W_mk^T, v = y W_mv^T, then the delta-rule update above (phi applied to k).

@@ -23,7 +23,9 @@ Readings where the pages are silent (the pages cite ARMT by name only and print 
 layer equations):
 * memory: phi(x) = elu(x) + 1; read o = phi(q) A / (phi(q) . z + eps); delta-rule update
   A += phi(K)^T (V - phi(K) A / (phi(K) . z + eps)), z += sum of phi(K) rows, batched over
-  the memory-token rows of the cell with the pre-update A, z; eps = 1e-6.
+  the memory-token rows of the cell with the pre-update A, z; eps = 1e-6. The rule is
+  written for one key; cfg.mem_update = "sequential" applies it to the cell's rows one
+  after another instead (each row against the state the earlier rows left).
 * the read sits at the layer input (all rows of the cell) and is added back through W_mo;
   the update keys/values are projected from the layer's memory-token output rows.
 * the layer is a LLaMA decoder layer: RMSNorm (eps 1e-5), RoPE rotate-half with
@@ -46,8 +48,8 @@ import math
 import numpy as np
 
 __all__ = ["phi", "silu", "rms_norm", "rope", "causal_gqa_attention", "memory_read",
-           "memory_update", "decoder_layer", "armt_cell", "forward", "forward_tokens", "forward_batch",
-           "full_attention_forward", "diagonals",
+           "memory_update", "memory_update_sequential", "decoder_layer", "armt_cell", "forward",
+           "forward_tokens", "forward_batch", "full_attention_forward", "diagonals",
            "sequential_steps", "schedule_triples", "schedule_quads"]
 
 
@@ -193,6 +195,22 @@ def memory_update(k_raw: np.ndarray, v: np.ndarray, A: np.ndarray, z: np.ndarray
     return A + fk.T @ (v - v_bar), z + fk.sum(axis=0)
 
 
+def memory_update_sequential(k_raw: np.ndarray, v: np.ndarray, A: np.ndarray, z: np.ndarray, eps: float):
+    """Delta-rule write of n key/value rows, one after another: row r is written into the
+    state that rows 0 .. r-1 left (for each row, the single-key rule of memory_update).
+    k_raw: [n, dk] (before phi); v: [n, dv]. Returns (A', z')."""
+    fk = phi(k_raw)
+    e = k_raw.dtype.type(eps)
+    A = A.copy()
+    z = z.copy()
+    for r in range(fk.shape[0]):
+        k = fk[r]
+        v_bar = (k @ A) / (k @ z + e)
+        A = A + np.outer(k, v[r] - v_bar)
+        z = z + k
+    return A, z
+
+
 # ------------------------------------------------------------------------------- model
 
 def decoder_layer(x: np.ndarray, lw: dict, cfg) -> np.ndarray:
@@ -225,7 +243,8 @@ def armt_cell(x: np.ndarray, lw: dict, A: np.ndarray, z: np.ndarray, cfg) -> tup
     x = decoder_layer(x, lw, cfg)
     # memory write from this layer's memory-token output rows (the cell's last n_mem rows)
     y = x[m - cfg.n_mem:]
-    A, z = memory_update(y @ lw["w_mk"].T, y @ lw["w_mv"].T, A, z, cfg.mem_eps)
+    write = memory_update_sequential if getattr(cfg, "mem_update", "batched") == "sequential" else memory_update
+    A, z = write(y @ lw["w_mk"].T, y @ lw["w_mv"].T, A, z, cfg.mem_eps)
     return x, A, z
 
 

@@ -17,6 +17,7 @@
 // Each kernel does the same arithmetic for a cell whatever else shares its launch, so the
 // two schedules give identical bits ("Dependency Preservation" in "Architecture
 // Overview"; arXiv 2506.05229 abstract: a pure run-time reordering with exact recurrence).
+#include <algorithm>
 #include <climits>
 #include <cstdio>
 #include <cmath>
@@ -256,8 +257,9 @@ struct rmt_handle {
   static constexpr size_t kMaxTables = 64;
   CUtensorMap tm_xb, tm_om, tm_att, tm_u, tm_wqkv, tm_wo, tm_wgu, tm_wd, tm_wmq, tm_wmo, tm_qkv, tm_qkv_tail, tm_x,
       tm_rope;
-  // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes)
-  CUtensorMap tp_xb, tp_om, tp_att, tp_u;
+  // activation maps of the CTA-pair GEMM (pair_token_tile(M)/2-row boxes), and the same with
+  // kPairFineTile/2-row boxes for launches of few cells (pair_pick_nt)
+  CUtensorMap tp_xb, tp_om, tp_att, tp_u, tq_xb, tq_om, tq_att, tq_u;
   int bn_mq = 0, bn_mo = 0, bn_qkv = 0, bn_o = 0, bn_gu = 0, bn_d = 0;
   // bf16 mode: projections that run on the CTA-pair GEMM (decided before packing, which
   // depends on it for the RoPE and SwiGLU row orders)
@@ -390,6 +392,8 @@ bool validate_cfg(const rmt_cfg* c, std::string& why) {
   }
   if (c->dtype != RMT_F32 && c->dtype != RMT_BF16 && c->dtype != RMT_BF16_SPLIT)
     return why = "dtype must be RMT_F32, RMT_BF16 or RMT_BF16_SPLIT", false;
+  if (c->mem_update != RMT_MEM_BATCHED && c->mem_update != RMT_MEM_SEQUENTIAL)
+    return why = "mem_update must be RMT_MEM_BATCHED or RMT_MEM_SEQUENTIAL", false;
   if (c->n_heads % c->n_kv_heads) return why = "n_heads must be a multiple of n_kv_heads", false;
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return why = "head_dim must be 32, 64 or 128", false;
   if (c->d_k % 32 || c->d_v % 32 || c->d_k > 128 || c->d_v > 128)
@@ -501,7 +505,8 @@ rmt_status build_maps(rmt_handle* h) {
     return make_tmap_16_3d(m, p, inner, rows, depth, box, true);
   };
   // weight boxes: 128 rows per CTA on the pair GEMM, else the tile width
-  const uint32_t pb = static_cast<uint32_t>(pair_token_tile(static_cast<int>(M)) / 2);
+  const uint32_t pb = static_cast<uint32_t>(pair_token_tile(static_cast<int>(M)) / 2),
+                 qb = static_cast<uint32_t>(std::min(pair_token_tile(static_cast<int>(M)), kPairFineTile) / 2);
   const bool any_pair = h->pair_mo || h->pair_qkv || h->pair_o || h->pair_gu || h->pair_d;
   // the read-out o: its own buffer, or (fold_mo) the last d_v columns of the attention output
   const uint64_t lda = uint64_t(h->ld_att);
@@ -522,7 +527,9 @@ rmt_status build_maps(rmt_handle* h) {
             map(&h->tm_wgu, h->w_gu, d, 2 * F, LW, h->pair_gu ? 128 : h->bn_gu) &&
             map(&h->tm_wd, h->w_d, F, d, LW, h->pair_d ? 128 : h->bn_d) &&
             (!any_pair || (map(&h->tp_xb, h->xb, xw, M, NS, pb) && map_om(&h->tp_om, pb) &&
-                           map(&h->tp_att, h->att, aw, M, L, pb) && map(&h->tp_u, h->u, uw, M, L, pb))) &&
+                           map(&h->tp_att, h->att, aw, M, L, pb) && map(&h->tp_u, h->u, uw, M, L, pb) &&
+                           map(&h->tq_xb, h->xb, xw, M, NS, qb) && map_om(&h->tq_om, qb) &&
+                           map(&h->tq_att, h->att, aw, M, L, qb) && map(&h->tq_u, h->u, uw, M, L, qb))) &&
             map(&h->tm_qkv, h->qkv, h->Nqkv, M, L, 128) &&
             map(&h->tm_qkv_tail, h->qkv, h->Nqkv, M, L, attn_tail_box(int(M), c.n_heads, c.n_kv_heads)) &&
             make_tmap_f32_resid(&h->tm_x, h->x, d, M, NS) &&
@@ -573,7 +580,7 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
     return fail(RMT_ECUDA, "cudaMemset failed");
   }
   if (h->chain_mlp) {  // one counter per (cell, token tile) of a step, both parities, both boundaries
-    const int nt = pair_token_tile(M);
+    const int nt = std::min(pair_token_tile(M), kPairFineTile);  // the finer of the two token tiles
     h->chain_ctr_len = static_cast<int>(BL) * ((M + nt - 1) / nt);
     const size_t bytes = size_t(2) * (kMaxPhases - 1) * h->chain_ctr_len * sizeof(unsigned);
     h->chain_ctr = static_cast<unsigned*>(h->act_alloc(bytes));
@@ -603,11 +610,13 @@ rmt_status reserve_acts(rmt_handle* h, int B) {
 
 enum Proj { kProjMemQ, kProjMemO, kProjQkv, kProjO, kProjGateUp, kProjDown };
 
-// A CTA-pair projection's launch arguments, collected instead of launched (for the chain).
+// A CTA-pair projection's launch arguments, collected instead of launched (for the chain):
+// tx maps the activations in pair_token_tile(M) token tiles, tq in kPairFineTile ones.
 struct PairLaunch {
   TcGemmArgs a;
   const CUtensorMap* tw;
   const CUtensorMap* tx;
+  const CUtensorMap* tq;
 };
 
 cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream_t st, PairLaunch* collect = nullptr) {
@@ -633,7 +642,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   IndexMode amode = kByLayer;
   const float* a32 = nullptr;
   const void* w = nullptr;
-  const CUtensorMap *ta = nullptr, *tb = nullptr, *tp = nullptr;
+  const CUtensorMap *ta = nullptr, *tb = nullptr, *tp = nullptr, *tq = nullptr;
   int bn = 0;
   bool pair = false;
   switch (p) {
@@ -656,7 +665,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       ep.src_mode = kInSlot, ep.dst_mode = kOutSlot, ep.xb = h->xb, ep.ss_out = h->ss1;
       ep.resid_no_store = h->fold_mo;  // the O projection adds W_mo o itself
       a32 = static_cast<const float*>(h->om), w = h->w_mo, ta = &h->tm_om, tb = &h->tm_wmo, bn = h->bn_mo;
-      tp = &h->tp_om, pair = h->pair_mo;
+      tp = &h->tp_om, tq = &h->tq_om, pair = h->pair_mo;
       ep.lo_off = h->split ? d : 0;
       kx_lo = h->split ? (h->fold_mo ? h->ld_att : c.d_v) : 0;
       break;
@@ -664,7 +673,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       N = h->Nqkv, K = d, epi = kEpiRope, amode = kOutSlot;
       ep.out = h->qkv, ep.ldo = h->Nqkv, ep.ss_in = h->ss1;
       a32 = h->x, w = h->w_qkv, ta = &h->tm_xb, tb = &h->tm_wqkv, bn = h->bn_qkv;
-      tp = &h->tp_xb, pair = h->pair_qkv;
+      tp = &h->tp_xb, tq = &h->tq_xb, pair = h->pair_qkv;
       ep.out_f32 = h->split;  // split-operand mode: attention reads fp32 q, k, v
       kx_lo = h->split ? d : 0;
       break;
@@ -676,7 +685,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
         ep.src_mode = kInSlot;
       }
       a32 = static_cast<const float*>(h->att), w = h->w_o, ta = &h->tm_att, tb = &h->tm_wo, bn = h->bn_o;
-      tp = &h->tp_att, pair = h->pair_o;
+      tp = &h->tp_att, tq = &h->tq_att, pair = h->pair_o;
       ep.lo_off = h->split ? d : 0;
       kx_lo = h->split ? h->ld_att : 0;
       break;
@@ -684,7 +693,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       N = 2 * c.d_ff, K = d, epi = kEpiSwiGLU, amode = kOutSlot;
       ep.out = h->u, ep.ldo = sw * c.d_ff, ep.ss_in = h->ss2;
       a32 = h->x, w = h->w_gu, ta = &h->tm_xb, tb = &h->tm_wgu, bn = h->bn_gu;
-      tp = &h->tp_xb, pair = h->pair_gu;
+      tp = &h->tp_xb, tq = &h->tq_xb, pair = h->pair_gu;
       ep.lo_off = h->split ? c.d_ff : 0;
       kx_lo = h->split ? d : 0;
       break;
@@ -692,7 +701,7 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
       N = d, K = c.d_ff, epi = resid;
       ep.src_mode = ep.dst_mode = kOutSlot, ep.xb = h->xb;
       a32 = static_cast<const float*>(h->u), w = h->w_d, ta = &h->tm_u, tb = &h->tm_wd, bn = h->bn_d;
-      tp = &h->tp_u, pair = h->pair_d;
+      tp = &h->tp_u, tq = &h->tq_u, pair = h->pair_d;
       ep.lo_off = h->split ? d : 0;
       kx_lo = h->split ? c.d_ff : 0;
       break;
@@ -700,10 +709,11 @@ cudaError_t run_proj(rmt_handle* h, Proj p, const Cell* cells, int G, cudaStream
   if (h->bf16 && pair) {
     TcGemmArgs a{h->M, N, K, G, cells, c.n_layers, amode, epi, ep, h->err, kx_lo};
     if (collect) {
-      *collect = PairLaunch{a, tb, tp};
+      *collect = PairLaunch{a, tb, tp, tq};
       return cudaSuccess;
     }
-    return launch_tc_pair_gemm(*tb, *tp, a, /*f16=*/true, st);
+    a.nt = pair_pick_nt(h->M, G, N / 256);
+    return launch_tc_pair_gemm(*tb, a.nt == pair_token_tile(h->M) ? *tp : *tq, a, /*f16=*/true, st);
   }
   if (collect) return cudaErrorInvalidValue;
   if (h->bf16) {
@@ -732,7 +742,11 @@ cudaError_t run_chain_o_mlp(rmt_handle* h, const Cell* cells, int G, cudaStream_
   a.ctr = h->chain_ctr;
   a.ctr_len = h->chain_ctr_len;
   a.parity = h->chain_parity;
-  const CUtensorMap tw[3] = {*o.tw, *gu.tw, *dn.tw}, tx[3] = {*o.tx, *gu.tx, *dn.tx};
+  const int nt = pair_pick_nt(h->M, G, (o.a.N + gu.a.N + dn.a.N) / 256);
+  const bool fine = nt != pair_token_tile(h->M);
+  for (int p = 0; p < 3; ++p) a.ph[p].nt = nt;
+  const CUtensorMap tw[3] = {*o.tw, *gu.tw, *dn.tw};
+  const CUtensorMap tx[3] = {fine ? *o.tq : *o.tx, fine ? *gu.tq : *gu.tx, fine ? *dn.tq : *dn.tx};
   e = launch_tc_pair_chain_o_mlp(tw, tx, a, st);
   if (e == cudaSuccess) h->chain_parity ^= 1;
   return e;
@@ -856,7 +870,8 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
   e = launch_kind(h, RMT_K_MEMUPDATE, g * 4 * n * dk * dv,
                   g * (h->nsplit * n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), st, [&] {
                     MemUpdateArgs a{h->part, h->nsplit, nullptr, nullptr, h->A, h->z, c.n_mem, c.d_k, c.d_v, c.mem_eps,
-                                    G, cells, kByLayer, kByLayer, L, h->trace, off, step};
+                                    G, cells, kByLayer, kByLayer, L, h->trace, off, step,
+                                    c.mem_update == RMT_MEM_SEQUENTIAL ? 1 : 0};
                     return launch_mem_update(a, st);
                   });
   if (e != cudaSuccess) return e;
@@ -1552,7 +1567,8 @@ rmt_status rmt_grouped_gemm_bf16(const void* A, const void* B, void* C, int32_t 
   ep.out_mode = kByLayer;
   TcGemmArgs a{M, N, K, G, cells, G, kByLayer, static_cast<EpiKind>(epi), ep, err};
   if (tc_pair_supported(M, N, K, epi, 0)) {  // widths in multiples of 256: CTA-pair kernel
-    if (!make_tmap_bf16_3d(&ta, A, K, M, G, static_cast<uint32_t>(pair_token_tile(M) / 2)) ||
+    a.nt = pair_pick_nt(M, G, N / 256);
+    if (!make_tmap_bf16_3d(&ta, A, K, M, G, static_cast<uint32_t>(a.nt / 2)) ||
         !make_tmap_bf16_3d(&tb, B, K, N, G, 128))
       return fail(RMT_EINVAL, "tensor map encoding failed (pointers must be 16-byte aligned)");
     RMT_CUDA(launch_tc_pair_gemm(tb, ta, a, /*f16=*/false, static_cast<cudaStream_t>(stream)));
@@ -1604,8 +1620,9 @@ rmt_status rmt_memory_read(const float* q, const float* A, const float* z, void*
   return RMT_OK;
 }
 
-rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n, int32_t dk,
-                             int32_t dv, float eps, void* stream) {
+namespace {
+rmt_status memory_update_impl(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n, int32_t dk,
+                              int32_t dv, float eps, int seq, void* stream) {
   if (!k || !v || !A || !z) return fail(RMT_EINVAL, "null pointer");
   if (!aligned16(k) || !aligned16(v) || !aligned16(A) || !aligned16(z))
     return fail(RMT_EINVAL, "k, v, A and z must be 16-byte aligned");
@@ -1613,9 +1630,20 @@ rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z,
     return fail(RMT_EINVAL, "bad sizes");
   const Cell* cells = nullptr;
   RMT_TRY(device_scratch(G, &cells, nullptr));
-  MemUpdateArgs a{nullptr, 0, k, v, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0};
+  MemUpdateArgs a{nullptr, 0, k, v, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0, seq};
   RMT_CUDA(launch_mem_update(a, static_cast<cudaStream_t>(stream)));
   return RMT_OK;
+}
+}  // namespace
+
+rmt_status rmt_memory_update(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n, int32_t dk,
+                             int32_t dv, float eps, void* stream) {
+  return memory_update_impl(k, v, A, z, G, n, dk, dv, eps, 0, stream);
+}
+
+rmt_status rmt_memory_update_sequential(const float* k, const float* v, float* A, float* z, int32_t G, int32_t n,
+                                        int32_t dk, int32_t dv, float eps, void* stream) {
+  return memory_update_impl(k, v, A, z, G, n, dk, dv, eps, 1, stream);
 }
 
 rmt_status rmt_rmsnorm(const float* x, const void* g, void* y, int32_t rows, int32_t d, float eps, rmt_dtype dtype,

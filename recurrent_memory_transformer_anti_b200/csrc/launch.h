@@ -49,6 +49,9 @@ struct TcGemmArgs {
   // low terms from column kx_lo on; the GEMM runs 2K/64 blocks, block b reading X at column
   // (b mod K/64) * 64 + (b div K/64) * kx_lo and W at (b mod K/64) * 64 (0: K blocks)
   int kx_lo;
+  // CTA-pair kernel: tokens per tile (a multiple of 16, at most 256; the activation maps' box
+  // is nt / 2 rows); 0: pair_token_tile(M). In a chained launch phase 0's value holds for all.
+  int nt;
 };
 
 // tensor-core path: 16-bit operands (f16 or bf16, one type per launch) in TMA tensor maps
@@ -72,6 +75,12 @@ cudaError_t launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const C
 // 128-row boxes, tx the [*, M, K] activations with pair_token_tile(M)/2-row boxes. RoPE and
 // SwiGLU expect the pair packing described with pair_token_tile.
 bool tc_pair_supported(int M, int N, int K, int epi, int head_dim);
+// Token tile of a CTA-pair launch over G cells of M rows whose phases have `pairs` 256-row
+// feature pairs in all: pair_token_tile(M), or kPairFineTile when a launch of few tiles
+// finishes sooner in more, smaller ones (fewer rounds of the resident CTA pairs; each tile
+// also costs a fixed pipeline fill and drain).
+constexpr int kPairFineTile = 128;
+int pair_pick_nt(int M, long G, long pairs);
 cudaError_t launch_tc_pair_gemm(const CUtensorMap& tw, const CUtensorMap& tx, const TcGemmArgs& args, bool f16,
                                 cudaStream_t st);
 
@@ -211,6 +220,9 @@ struct MemUpdateArgs {
   int L;
   int* trace;         // optional: trace[3*(trace_base+g) + {0,1,2}] = (step, l, s)
   int trace_base, step;
+  // 0: every row is written against the pre-update A, z (batched). 1: the rows are written one
+  // after another, each against the state the earlier rows left (per-token delta rule).
+  int seq;
 };
 cudaError_t launch_mem_update(const MemUpdateArgs& a, cudaStream_t st);
 

@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
 constexpr int kUpdThreads = 256;
 
 struct UpdLayout {  // shared-memory layout in floats (every region starts 16-byte aligned)
-  int n4, fk, As, Vs, D, zs, den, total;
+  int n4, fk, As, Vs, D, zs, den, gram, total;
   __host__ __device__ UpdLayout(int n, int dk, int cs) {
     n4 = (n + 3) & ~3;
     fk = 0;                 // [n][dk]    phi(keys)
@@ -551,9 +551,48 @@ struct UpdLayout {  // shared-memory layout in floats (every region starts 16-by
     D = Vs + n * cs;        // [n4][cs]   V - v_bar
     zs = D + n4 * cs;       // [dk]
     den = zs + dk;          // [n4]
-    total = den + n4;
+    gram = den + n4;        // [n][n4]    per-token rule: phi(k_r) . phi(k_j), j < r
+    total = gram + n * n4;
   }
 };
+
+// Per-token delta rule (rows written one after another) from the batched quantities. Row r
+// meets the state A_r = A + sum_{j<r} phi(k_j)^T d_j, z_r = z + sum_{j<r} phi(k_j), so with
+// G_rj = phi(k_r) . phi(k_j):
+//   den_r = phi(k_r) . z + eps + sum_{j<r} G_rj
+//   d_r   = V_r - phi(k_r) A / den_r - sum_{j<r} G_rj d_j / den_r
+// and after the last row A' = A + phi(K)^T D, z' = z + sum_r phi(k_r), as in the batched rule.
+// seq_gram_den: G (lower triangle, i ascending) and the denominators (den holds phi(k_r) . z
+// + eps on entry; j ascending). seq_substitute: D holds V_r - phi(k_r) A / den_r on entry and
+// d_r on exit, rows ascending, one thread per column. Both run the same order in every kernel.
+__device__ __forceinline__ void seq_gram_den(const float* fk, int n, int dk, int ldg, float* gram, float* den,
+                                             int tid, int nthreads) {
+  for (int p = tid; p < n * n; p += nthreads) {
+    const int r = p / n, j = p % n;
+    if (j >= r) continue;
+    float s = 0.f;
+    for (int i = 0; i < dk; ++i) s = fmaf(fk[r * dk + i], fk[j * dk + i], s);
+    gram[r * ldg + j] = s;
+  }
+  __syncthreads();
+  for (int r = tid; r < n; r += nthreads) {
+    float d = den[r];
+    for (int j = 0; j < r; ++j) d += gram[r * ldg + j];
+    den[r] = d;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void seq_substitute(float* D, int ldd, int cols, int n, const float* gram, int ldg,
+                                               const float* den, int tid, int nthreads) {
+  for (int c = tid; c < cols; c += nthreads) {
+    for (int r = 1; r < n; ++r) {
+      float acc = 0.f;
+      for (int j = 0; j < r; ++j) acc = fmaf(gram[r * ldg + j], D[j * ldd + c], acc);
+      D[r * ldd + c] -= acc / den[r];
+    }
+  }
+}
 
 // Raw key|value elements (r, col) of the cell, as the sum of the split partials in split order,
 // starting from the first (or the plain inputs without partials). EPT elements per call; their partial loads go out
@@ -602,6 +641,7 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
   float* D = sm + lay.D;
   float* zs = sm + lay.zs;
   float* den = sm + lay.den;
+  float* gram = sm + lay.gram;
   const Cell c = load_cell(a.cells, g);
   const size_t ki = cell_index(a.kv_mode, a.L, c), si = cell_index(a.state_mode, a.L, c);
   float* A = a.A + si * dk * dv;
@@ -669,6 +709,7 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
     if (lane == 0) den[r] = d + a.eps;
   }
   __syncthreads();
+  if (a.seq) seq_gram_den(fk, n, dk, lay.n4, gram, den, tid, kUpdThreads);
 
   // 3. D = V - phi(K) A / den for this slice's columns, i ascending per element: one row x 4
   //    columns per thread, so every thread has work; a warp's reads of a key row and of an A
@@ -692,6 +733,10 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
     for (int y = 0; y < 4; ++y) D[r * cs + c0 + y] = Vs[r * cs + c0 + y] - acc[y] / den[r];
   }
   __syncthreads();
+  if (a.seq) {  // per-token rule: the innovations row after row
+    seq_substitute(D, cs, cs, n, gram, lay.n4, den, tid, kUpdThreads);
+    __syncthreads();
+  }
 
   // 4. A' = A + phi(K)^T D for this slice's columns: 4 rows of A x 4 columns per thread
   for (int b = tid; b < (dk / 4) * (cs / 4); b += kUpdThreads) {
@@ -740,14 +785,15 @@ __global__ void __launch_bounds__(kUpdThreads, 2) mem_update_kernel(const MemUpd
 constexpr int kUpdStreamThreads = 256;
 
 struct UpdStreamLayout {  // in floats; every region starts 16-byte aligned
-  int n8, stage, fk, D, den, total;
+  int n8, stage, fk, D, den, gram, total;
   __host__ __device__ UpdStreamLayout(int n, int dk, int dv, int nst) {
     n8 = (n + 7) & ~7;
     stage = n * dk + n * dv + dk * dv + dk;  // K [n][dk], V [n][dv], A [dk][dv], z [dk]
     fk = nst * stage;                        // phi(K) [n][dk]
     D = fk + n * dk;                         // [n8][dv]
     den = D + n8 * dv;                       // [n8]
-    total = den + n8;
+    gram = den + n8;                         // [n][n8] (per-token rule)
+    total = gram + n * n8;
   }
 };
 
@@ -763,6 +809,7 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel
   float* fk = us + lay.fk;
   float* D = us + lay.D;
   float* den = us + lay.den;
+  float* gram = us + lay.gram;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int per = (a.G + gridDim.x - 1) / gridDim.x;
   const int c_beg = blockIdx.x * per, c_end = min(a.G, c_beg + per);
@@ -814,6 +861,7 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel
       if (lane == 0) den[r] = d + a.eps;
     }
     __syncthreads();
+    if (a.seq) seq_gram_den(fk, n, dk, lay.n8, gram, den, tid, kUpdStreamThreads);
     // D = V - phi(K) A / den: one row x 4 columns per thread, i ascending; a warp holds two rows
     // x 16 column blocks, so its reads of a row of phi(K) and of a row of A are broadcasts
     for (int b = tid; b < n * (dv / 4); b += kUpdStreamThreads) {
@@ -836,6 +884,10 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel
       for (int y = 0; y < 4; ++y) D[r * dv + c0 + y] = Vr[r * dv + c0 + y] - acc[y] / den[r];
     }
     __syncthreads();
+    if (a.seq) {  // per-token rule: the innovations row after row
+      seq_substitute(D, dv, dv, n, gram, lay.n8, den, tid, kUpdStreamThreads);
+      __syncthreads();
+    }
     // A' = A + phi(K)^T D: 4 rows of A x 4 columns per thread, rows of K ascending
     const Cell c = load_cell(a.cells, g);
     const size_t si = cell_index(a.state_mode, a.L, c);

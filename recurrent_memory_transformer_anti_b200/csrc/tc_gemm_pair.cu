@@ -109,7 +109,9 @@ __device__ __forceinline__ float row_scale(const float* ss_row, int parts, float
 // Epilogue of one warp: its 32 features (f = this lane's output column) over tokens
 // tok0 .. tok0 + cnt - 1 of the cell (cnt a multiple of 8, at most 128), accumulator columns
 // from tacc. A step covers 32 columns; columns past cnt (at most 24) are read, not stored.
-template <int EPI, typename OpT>
+// SPLIT: the split-operand mode's stores (low terms, fp32 q/k/v) are compiled in; without it
+// the epilogue carries no trace of them.
+template <int EPI, typename OpT, bool SPLIT>
 __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint32_t tacc, int tok0, int cnt, int f,
                                               int lane, const float* rs, float* red, float& amax) {
   const EpiParams& ep = a.ep;
@@ -144,7 +146,7 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
           if constexpr (EPI == kEpiResidCast) {
             OpT* xr = xb + static_cast<size_t>(j0 + j) * ldxb;
             *xr = from_f32<OpT>(y);
-            if (ep.lo_off) xr[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
+            if constexpr (SPLIT) xr[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
             track_amax<OpT>(amax, y);
           }
         }
@@ -200,7 +202,7 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
         const float other = __shfl_xor_sync(0xffffffffu, x, 1);
         const float y = odd ? fmaf(x, cs.x, other * cs.y) : fmaf(x, cs.x, -other * cs.y);
         if (j0 + j < lim) {
-          if (ep.out_f32) {
+          if constexpr (SPLIT) {
             out32[static_cast<size_t>(j0 + j) * ep.ldo] = y;
           } else {
             out[static_cast<size_t>(j0 + j) * ep.ldo] = from_f32<OpT>(y);
@@ -233,7 +235,7 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
           const float y = silu_fast(g) * u;
           OpT* o = out + static_cast<size_t>(t) * ep.ldo;
           *o = from_f32<OpT>(y);
-          if (ep.lo_off) o[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
+          if constexpr (SPLIT) o[ep.lo_off] = from_f32<OpT>(lo_term<OpT>(y));
           track_amax<OpT>(amax, y);
         }
       }
@@ -257,7 +259,7 @@ __device__ __forceinline__ void pair_epilogue(const TcGemmArgs& a, Cell c, uint3
 constexpr int kNoEpi = -1;  // an unused phase slot
 constexpr unsigned kSignalsPerTile = 2 * PairCfg::EPI_WARPS;  // one per epilogue warp of each CTA of the pair
 
-template <int E0, int E1, int E2, typename OpT>
+template <int E0, int E1, int E2, typename OpT, bool SPLIT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
                         const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX1,
@@ -280,7 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const TcGemmArgs& a0 = args.ph[0];
   const int M = a0.M, G = a0.G;
-  const int NT = pair_token_tile(M);
+  const int NT = a0.nt > 0 ? a0.nt : pair_token_tile(M);
   const int STAGES = C::stages(NT);
   const uint32_t BLK = static_cast<uint32_t>(C::block_bytes(NT));
   const uint32_t ring = base + C::RING_OFF;
@@ -537,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                             static_cast<uint32_t>(acc * C::ACC_COLS + wg * cnt);
       float* red = red_all + ((acc * 2 + wg) * 4 + quarter) * 128;
-      pair_epilogue<EPI, OpT>(a, c, tacc, tok0, cnt, f, lane, rs, red, amax);
+      pair_epilogue<EPI, OpT, SPLIT>(a, c, tacc, tok0, cnt, f, lane, rs, red, amax);
       // accumulator drained (every lane's tcgen05.ld waited for): release it to the even CTA's
       // MMA issuer. The issuer reads none of this warp's global stores, so the arrive is
       // relaxed and does not wait for them to drain.
@@ -636,28 +638,36 @@ int max_pair_clusters(const void* fn) {
   return cached[dev];
 }
 
-template <int E0, int E1, int E2, typename OpT>
+// Split-operand launches (any phase with low terms, or fp32 q/k/v) take the SPLIT kernel.
+inline bool pair_split(const PairChainArgs& args) {
+  for (int p = 0; p < args.nphase; ++p)
+    if (args.ph[p].kx_lo || args.ph[p].ep.lo_off || args.ph[p].ep.out_f32) return true;
+  return false;
+}
+
+template <int E0, int E1, int E2, typename OpT, bool SPLIT>
 cudaError_t launch_pair_chain_t(const CUtensorMap* tw, const CUtensorMap* tx, const PairChainArgs& args,
                                 cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  const void* fn = reinterpret_cast<const void*>(tc_pair_gemm_kernel<E0, E1, E2, OpT>);
+  const void* fn = reinterpret_cast<const void*>(tc_pair_gemm_kernel<E0, E1, E2, OpT, SPLIT>);
   if (!attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const TcGemmArgs& a0 = args.ph[0];
-  const int NT = pair_token_tile(a0.M), ntt = (a0.M + NT - 1) / NT;
+  const int NT = a0.nt > 0 ? a0.nt : pair_token_tile(a0.M), ntt = (a0.M + NT - 1) / NT;
+  if (NT % 16 != 0 || NT > 256) return cudaErrorInvalidValue;
   long tiles = 0;
   for (int p = 0; p < args.nphase; ++p) tiles += static_cast<long>(a0.G) * (args.ph[p].N / 256) * ntt;
   if (tiles <= 0) return cudaSuccess;
   const int maxc = max_pair_clusters(fn);  // every pair resident at once (the chained waits rely on it)
   const int clusters = static_cast<int>(tiles < maxc ? tiles : maxc);
   const int np = args.nphase;
-  const cudaError_t e = launch_pdl(tc_pair_gemm_kernel<E0, E1, E2, OpT>, dim3(2 * clusters), dim3(PairCfg::THREADS),
+  const cudaError_t e = launch_pdl(tc_pair_gemm_kernel<E0, E1, E2, OpT, SPLIT>, dim3(2 * clusters), dim3(PairCfg::THREADS),
                                    PairCfg::SMEM_BYTES, st, tw[0], tx[0], tw[np > 1 ? 1 : 0], tx[np > 1 ? 1 : 0],
                                    tw[np > 2 ? 2 : 0], tx[np > 2 ? 2 : 0], args);
   if (e != cudaSuccess) return e;
@@ -669,12 +679,22 @@ cudaError_t launch_pair_op(const CUtensorMap& tw, const CUtensorMap& tx, const T
   PairChainArgs c{};
   c.ph[0] = args;
   c.nphase = 1;
+  if (pair_split(c)) {  // split-operand mode: the f16 operands only
+    if constexpr (std::is_same<OpT, __half>::value) {
+      switch (args.epi) {
+        case kEpiResidCast: return launch_pair_chain_t<kEpiResidCast, kNoEpi, kNoEpi, OpT, true>(&tw, &tx, c, st);
+        case kEpiRope: return launch_pair_chain_t<kEpiRope, kNoEpi, kNoEpi, OpT, true>(&tw, &tx, c, st);
+        case kEpiSwiGLU: return launch_pair_chain_t<kEpiSwiGLU, kNoEpi, kNoEpi, OpT, true>(&tw, &tx, c, st);
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (args.epi) {
-    case kEpiStoreF32: return launch_pair_chain_t<kEpiStoreF32, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
-    case kEpiStoreAct: return launch_pair_chain_t<kEpiStoreAct, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
-    case kEpiResidCast: return launch_pair_chain_t<kEpiResidCast, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
-    case kEpiRope: return launch_pair_chain_t<kEpiRope, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
-    case kEpiSwiGLU: return launch_pair_chain_t<kEpiSwiGLU, kNoEpi, kNoEpi, OpT>(&tw, &tx, c, st);
+    case kEpiStoreF32: return launch_pair_chain_t<kEpiStoreF32, kNoEpi, kNoEpi, OpT, false>(&tw, &tx, c, st);
+    case kEpiStoreAct: return launch_pair_chain_t<kEpiStoreAct, kNoEpi, kNoEpi, OpT, false>(&tw, &tx, c, st);
+    case kEpiResidCast: return launch_pair_chain_t<kEpiResidCast, kNoEpi, kNoEpi, OpT, false>(&tw, &tx, c, st);
+    case kEpiRope: return launch_pair_chain_t<kEpiRope, kNoEpi, kNoEpi, OpT, false>(&tw, &tx, c, st);
+    case kEpiSwiGLU: return launch_pair_chain_t<kEpiSwiGLU, kNoEpi, kNoEpi, OpT, false>(&tw, &tx, c, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -686,6 +706,27 @@ bool tc_pair_supported(int M, int N, int K, int epi, int head_dim) {
   if (epi == kEpiResid) return false;  // 16-bit operands always refresh the operand copy (kEpiResidCast)
   if (epi == kEpiRope && (head_dim <= 0 || head_dim % 2 != 0)) return false;
   return pair_token_tile(M) <= 256;
+}
+
+int pair_pick_nt(int M, long G, long pairs) {
+  const int coarse = pair_token_tile(M);
+  if (coarse <= kPairFineTile) return coarse;
+  static int clusters[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!clusters[dev]) {
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    clusters[dev] = sms > 1 ? sms / 2 : 1;
+  }
+  // makespan in token-equivalents: rounds of the resident pairs x (tile tokens + a fixed
+  // pipeline fill and drain of about 48 tokens' worth of MMA)
+  auto cost = [&](int nt) {
+    const long tiles = G * pairs * ((M + nt - 1) / nt);
+    return ((tiles + clusters[dev] - 1) / clusters[dev]) * (nt + 48);
+  };
+  return cost(kPairFineTile) < cost(coarse) ? kPairFineTile : coarse;
 }
 
 // A split-operand X keeps its low terms at a 16-byte aligned column at or past its high terms.
@@ -709,9 +750,10 @@ cudaError_t launch_tc_pair_chain_o_mlp(const CUtensorMap* tw, const CUtensorMap*
         a[p].G != a[0].G || a[p].cells != a[0].cells)
       return cudaErrorInvalidValue;
   }
-  const int NT = pair_token_tile(a[0].M);
+  const int NT = a[0].nt > 0 ? a[0].nt : pair_token_tile(a[0].M);
   if (static_cast<long>(a[0].G) * ((a[0].M + NT - 1) / NT) > args.ctr_len) return cudaErrorInvalidValue;
-  return launch_pair_chain_t<kEpiResidCast, kEpiSwiGLU, kEpiResidCast, __half>(tw, tx, args, st);
+  if (pair_split(args)) return launch_pair_chain_t<kEpiResidCast, kEpiSwiGLU, kEpiResidCast, __half, true>(tw, tx, args, st);
+  return launch_pair_chain_t<kEpiResidCast, kEpiSwiGLU, kEpiResidCast, __half, false>(tw, tx, args, st);
 }
 
 }  // namespace rmt

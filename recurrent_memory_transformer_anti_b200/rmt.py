@@ -23,6 +23,8 @@ RMT_F32, RMT_BF16, RMT_BF16_SPLIT = 0, 1, 2
 SCHEDULES = {"diagonal": RMT_DIAGONAL, "sequential": RMT_SEQUENTIAL}
 # "bf16-split": bf16 storage, split (high + low f16 term) tensor-core operands (include/rmt.h)
 DTYPES = {"f32": RMT_F32, "bf16": RMT_BF16, "bf16-split": RMT_BF16_SPLIT}
+# how a cell writes its memory rows (include/rmt.h rmt_mem_update)
+MEM_UPDATES = {"batched": 0, "sequential": 1}
 STORAGE_BF16 = ("bf16", "bf16-split")
 STATUS_NAMES = {0: "RMT_OK", 1: "RMT_EINVAL", 2: "RMT_ENOMEM", 3: "RMT_ECUDA", 4: "RMT_ETIMEOUT", 5: "RMT_ESTATE",
                 6: "RMT_ERANGE", 7: "RMT_EDEBUG"}
@@ -32,7 +34,7 @@ EXPORTED = ("rmt_create", "rmt_reserve", "rmt_forward", "rmt_forward_resume", "r
             "rmt_schedule_table_batch", "rmt_get_schedule", "rmt_get_trace", "rmt_sync", "rmt_wait_selftest",
             "rmt_bounds_selftest",
             "rmt_destroy", "rmt_last_error", "rmt_grouped_gemm_bf16", "rmt_attention", "rmt_memory_read",
-            "rmt_memory_update", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
+            "rmt_memory_update", "rmt_memory_update_sequential", "rmt_memory_write", "rmt_memory_write_noalloc", "rmt_rmsnorm", "rmt_probe",
             "rmt_probe_read")
 
 KERNELS = ("assemble", "memq", "memread", "memo", "rmsnorm1", "qkv", "attention", "o", "rmsnorm2", "gateup", "down",
@@ -49,7 +51,7 @@ class rmt_cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("n_layers", "d_model", "n_heads", "n_kv_heads", "head_dim", "d_ff",
                                                "seg_len", "n_mem", "d_k", "d_v")] + \
                [("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("mem_eps", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("mem_update", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -85,6 +87,7 @@ def _load() -> ctypes.CDLL:
         "rmt_attention": [vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp],
         "rmt_memory_read": [vp, vp, vp, vp, i32, i32, i32, i32, f32, ctypes.c_int, vp],
         "rmt_memory_update": [vp, vp, vp, vp, i32, i32, i32, i32, f32, vp],
+        "rmt_memory_update_sequential": [vp, vp, vp, vp, i32, i32, i32, i32, f32, vp],
         "rmt_memory_write": [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, ctypes.c_int, vp],
         "rmt_memory_write_noalloc": [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, ctypes.c_int, vp],
         "rmt_rmsnorm": [vp, vp, vp, i32, i32, f32, ctypes.c_int, vp],
@@ -149,6 +152,8 @@ def make_cfg(cfg) -> rmt_cfg:
         setattr(c, n, int(getattr(cfg, n)))
     c.rope_theta, c.rms_eps, c.mem_eps = float(cfg.rope_theta), float(cfg.rms_eps), float(cfg.mem_eps)
     c.dtype = DTYPES[cfg.dtype] if isinstance(cfg.dtype, str) else int(cfg.dtype)
+    mu = getattr(cfg, "mem_update", "batched")
+    c.mem_update = MEM_UPDATES[mu] if isinstance(mu, str) else int(mu)
     return c
 
 
@@ -298,6 +303,11 @@ def rmt_memory_read(q, A, z, o, G, M, dk, dv, eps, dtype="f32", stream=None) -> 
 def rmt_memory_update(k, v, A, z, G, n, dk, dv, eps, stream=None) -> None:
     _check(_lib.rmt_memory_update(_ptr(k), _ptr(v), _ptr(A), _ptr(z), G, n, dk, dv, eps, _stream(stream)),
            "rmt_memory_update")
+
+
+def rmt_memory_update_sequential(k, v, A, z, G, n, dk, dv, eps, stream=None) -> None:
+    _check(_lib.rmt_memory_update_sequential(_ptr(k), _ptr(v), _ptr(A), _ptr(z), G, n, dk, dv, eps,
+                                             _stream(stream)), "rmt_memory_update_sequential")
 
 
 def rmt_memory_write(y, w_mkv, A, z, G, n, d, dk, dv, eps, dtype="f32", stream=None) -> None:

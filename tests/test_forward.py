@@ -260,6 +260,27 @@ def test_split_operands_match_oracle(small_split, S):
     assert normwise(A, ref[1]) < F32_TOL and normwise(z, ref[2]) < F32_TOL, (normwise(A, ref[1]), normwise(z, ref[2]))
 
 
+@pytest.mark.parametrize("name,S,tol", [("tiny", 4, F32_TOL), ("small-bf16", 3, BF16_TOL)])
+def test_per_token_memory_update_matches_oracle(cuda_ok, name, S, tol):
+    """cfg.mem_update = "sequential": each cell writes its memory rows one after another (the
+    oracle's row loop; the kernels' Gram forward substitution). DIAGONAL gives the bits of
+    SEQUENTIAL, and the result differs from the batched write."""
+    base = CONFIGS[name]
+    cfg = dataclasses.replace(base, mem_update="sequential")
+    w = make_weights(base)
+    _, h = build(cfg, weights=w)
+    emb = embeddings(base, S)
+    got = forward(h, cfg, emb, S, "diagonal")
+    ref = armt.forward(cfg, w, emb, S, dtype=np.float32)
+    for g, r, what in zip(got, ref, ("out", "A", "z")):
+        assert normwise(g, r) < tol, what
+    for a, b in zip(got, forward(h, cfg, emb, S, "sequential")):
+        np.testing.assert_array_equal(a, b)
+    rmt.rmt_destroy(h)
+    batched = armt.forward(base, w, emb, S, dtype=np.float32)
+    assert normwise(ref[1], batched[1]) > 5 * tol  # A differs by 12-18% between the two rules
+
+
 def test_split_operands_diagonal_equals_sequential_bitwise(small_split):
     base, cfg, w, h = small_split
     S = 5

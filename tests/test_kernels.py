@@ -160,6 +160,60 @@ def test_memory_update_bits_do_not_depend_on_the_column_slicing():
         assert torch.equal(A_all[:m], A_few) and torch.equal(z_all[:m], z_few), m
 
 
+@pytest.mark.parametrize("G,n,dk,dv", [(5, 16, 64, 64), (3, 8, 32, 32), (2, 16, 128, 128), (2, 64, 64, 32),
+                                       (1, 1, 32, 64), (300, 16, 64, 64), (150, 13, 128, 128), (700, 16, 64, 64)])
+def test_memory_update_sequential_matches_oracle(G, n, dk, dv):
+    """The per-token delta rule (rows written one after another) against the oracle's row loop;
+    G = 700 runs the streaming kernel, the others the cluster kernel."""
+    r = rng(600 + n + dk)
+    k = r.standard_normal((G, n, dk), dtype=np.float32)
+    v = r.standard_normal((G, n, dv), dtype=np.float32)
+    A = r.standard_normal((G, dk, dv), dtype=np.float32)
+    z = r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)
+    tk, tv, tA, tz = (torch.from_numpy(x).cuda() for x in (k, v, A, z))
+    rmt.rmt_memory_update_sequential(tk, tv, tA, tz, G, n, dk, dv, 1e-6)
+    rmt.rmt_sync(None)
+    for g in range(G):
+        rA, rz = armt.memory_update_sequential(k[g].astype(np.float64), v[g].astype(np.float64),
+                                               A[g].astype(np.float64), z[g].astype(np.float64), 1e-6)
+        assert normwise(to_np(tA[g]), rA) < 1e-5
+        assert normwise(to_np(tz[g]), rz) < 1e-6
+
+
+def test_memory_update_sequential_bits_do_not_depend_on_the_launch():
+    r = rng(650)
+    G, n, dk, dv = 700, 16, 64, 64
+    k = torch.from_numpy(r.standard_normal((G, n, dk), dtype=np.float32)).cuda()
+    v = torch.from_numpy(r.standard_normal((G, n, dv), dtype=np.float32)).cuda()
+    A0 = torch.from_numpy(r.standard_normal((G, dk, dv), dtype=np.float32)).cuda()
+    z0 = torch.from_numpy(r.uniform(1.0, 100.0, (G, dk)).astype(np.float32)).cuda()
+    A_all, z_all = A0.clone(), z0.clone()
+    rmt.rmt_memory_update_sequential(k, v, A_all, z_all, G, n, dk, dv, 1e-6)
+    for m in (4, 400):
+        A_few, z_few = A0[:m].clone(), z0[:m].clone()
+        rmt.rmt_memory_update_sequential(k[:m].contiguous(), v[:m].contiguous(), A_few, z_few, m, n, dk, dv, 1e-6)
+        rmt.rmt_sync(None)
+        assert torch.equal(A_all[:m], A_few) and torch.equal(z_all[:m], z_few), m
+
+
+def test_memory_update_sequential_overwrites_a_key_written_twice():
+    """phi(k) = e_0 for both rows of one cell, values v then v': the per-token rule leaves
+    e_0 reading (v' + v eps/(1+eps)) / (2+eps) (the batched rule would give the average)."""
+    dk, dv, eps = 32, 32, 1e-6
+    k = np.full((1, 2, dk), -1000.0, np.float32)
+    k[0, :, 0] = 0.0
+    v = rng(8).standard_normal((1, 2, dv), dtype=np.float32)
+    A = torch.zeros((1, dk, dv), device="cuda")
+    z = torch.zeros((1, dk), device="cuda")
+    tk = torch.from_numpy(k).cuda()
+    rmt.rmt_memory_update_sequential(tk, torch.from_numpy(v).cuda(), A, z, 1, 2, dk, dv, eps)
+    o = torch.empty((1, 1, dv), device="cuda")
+    rmt.rmt_memory_read(tk[:, :1].contiguous(), A, z, o, 1, 1, dk, dv, eps, "f32")
+    rmt.rmt_sync(None)
+    expect = (v[0, 1].astype(np.float64) + v[0, 0] * eps / (1 + eps)) / (2 + eps)
+    np.testing.assert_allclose(to_np(o)[0, 0], expect, rtol=1e-6, atol=1e-7)
+
+
 def test_memory_write_then_read_orthonormal_keys_on_gpu():
     """phi(k_i) = e_i (k = 0 on the diagonal, -1000 elsewhere): after one write from an empty
     memory, the read of k_j returns v_j / (1 + eps)."""

@@ -161,6 +161,66 @@ def test_memory_rewrite_of_stored_pair_is_nearly_noop():
     np.testing.assert_array_equal((A2 - A)[1:], 0.0)
 
 
+# per-token delta rule (cfg.mem_update = "sequential")
+
+def test_sequential_update_of_one_row_is_the_batched_update():
+    rng = np.random.default_rng(21)
+    k, v = rng.standard_normal((1, 24)), rng.standard_normal((1, 40))
+    A, z = rng.standard_normal((24, 40)), rng.uniform(1, 10, 24)
+    for got, want in zip(armt.memory_update_sequential(k, v, A, z, 1e-6), armt.memory_update(k, v, A, z, 1e-6)):
+        np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-14)
+
+
+def test_sequential_update_writes_the_same_key_twice_as_two_writes():
+    """Keys with phi(k) = e_0 twice in one cell, values v then v': the per-token rule stores v,
+    reads it back as v/(1+eps) and corrects toward v', so a read of e_0 returns
+    (v' + v eps/(1+eps)) / (2+eps); the batched rule sees the empty memory for both rows and
+    returns the average (v + v')/(2+eps)."""
+    eps = 1e-6
+    rng = np.random.default_rng(23)
+    k = np.full((2, 5), -1000.0)
+    k[:, 0] = 0.0
+    v = rng.standard_normal((2, 3))
+    A0, z0 = np.zeros((5, 3)), np.zeros(5)
+    q = k[:1]
+    A, z = armt.memory_update_sequential(k, v, A0, z0, eps)
+    np.testing.assert_array_equal(z, [2.0, 0, 0, 0, 0])
+    np.testing.assert_allclose(armt.memory_read(q, A, z, eps)[0], (v[1] + v[0] * eps / (1 + eps)) / (2 + eps),
+                               rtol=1e-13, atol=1e-15)
+    Ab, zb = armt.memory_update(k, v, A0, z0, eps)
+    np.testing.assert_allclose(armt.memory_read(q, Ab, zb, eps)[0], (v[0] + v[1]) / (2 + eps), rtol=1e-13, atol=1e-15)
+
+
+def test_sequential_update_equals_one_row_writes_in_order():
+    rng = np.random.default_rng(25)
+    k, v = rng.standard_normal((9, 16)), rng.standard_normal((9, 12))
+    A, z = rng.standard_normal((16, 12)), rng.uniform(1, 10, 16)
+    As, zs = armt.memory_update_sequential(k, v, A, z, 1e-6)
+    for r in range(9):
+        A, z = armt.memory_update(k[r:r + 1], v[r:r + 1], A, z, 1e-6)
+    np.testing.assert_allclose(As, A, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(zs, z, rtol=1e-13, atol=1e-13)
+
+
+def test_sequential_update_matches_the_gram_forward_substitution():
+    """The same write from the batched quantities: with G = phi(K) phi(K)^T,
+    den_r = phi(k_r) . z + eps + sum_{j<r} G_rj and d_r = V_r - (phi(k_r) A + sum_{j<r} G_rj d_j) / den_r,
+    A' = A + phi(K)^T D, z' = z + sum_r phi(k_r) (the form the kernels use)."""
+    rng = np.random.default_rng(27)
+    n, dk, dv, eps = 16, 32, 24, 1e-6
+    k, v = rng.standard_normal((n, dk)), rng.standard_normal((n, dv))
+    A, z = 0.1 * rng.standard_normal((dk, dv)), rng.uniform(1, 10, dk)
+    fk = np.where(k > 0, k + 1.0, np.exp(np.minimum(k, 0.0)))
+    G = fk @ fk.T
+    den = fk @ z + eps + np.array([G[r, :r].sum() for r in range(n)])
+    D = np.zeros((n, dv))
+    for r in range(n):
+        D[r] = v[r] - (fk[r] @ A + G[r, :r] @ D[:r]) / den[r]
+    As, zs = armt.memory_update_sequential(k, v, A, z, eps)
+    np.testing.assert_allclose(As, A + fk.T @ D, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(zs, z + fk.sum(axis=0), rtol=1e-13, atol=1e-13)
+
+
 # ------------------------------------------------------ independent torch reference model
 
 def _torch_cell(x, lw, A, z, cfg):
