@@ -375,6 +375,10 @@ MIXED_CONFIGS = {
     # 152 rows per cell: the last query tile (24 rows) stacks the 4 heads of the key/value group
     "tail-stacked": dict(n_layers=3, d_model=256, n_heads=4, n_kv_heads=1, head_dim=64, d_ff=512, seg_len=144,
                          n_mem=8, d_k=64, d_v=64),
+    # d_k = d_v = 128: the mem-q GEMM stores q, the tcgen05 read runs as a launch of its own and
+    # the read-out projection keeps its residual store (no fold)
+    "memory-128": dict(n_layers=3, d_model=256, n_heads=4, n_kv_heads=2, head_dim=64, d_ff=512, seg_len=200,
+                       n_mem=8, d_k=128, d_v=128),
 }
 
 
