@@ -46,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # with the number of cells (each cell brings its own layer's weights and activations), so a
 # launch's traffic is this figure times its cells. None when no capture of the current kernel
 # exists.
-DOMINANT_TRAFFIC_BYTES_PER_CELL = 206.7e6  # 674.3 MB read + 152.6 MB written by a 4-cell launch (1B shape)
+DOMINANT_TRAFFIC_BYTES_PER_CELL = 206.8e6  # 677.8 MB read + 149.4 MB written by a 4-cell launch (1B shape)
 
 
 def parse():
