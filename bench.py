@@ -301,6 +301,16 @@ def run_microbench(args, local: int) -> int:
                                            "kernel": "CTA pairs" if N % 256 == 0 else "single CTAs"},
                      ms, 2.0 * G * M * N * K, "TFLOP/s", peaks["bf16_tflops"], "bf16_tflops")
                 del a, b, c
+        # tokens per cell: how a cell's token count splits into token tiles of at most 256
+        G, N = 16, 8192
+        for Mc in (1024, 1040, 1088, 1152, 1280, 768, 784, 528, 512):
+            a = torch.randn(G, Mc, K, device=dev, generator=gen).to(torch.bfloat16)
+            b = (torch.randn(G, N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+            c = torch.empty(G, Mc, N, device=dev, dtype=torch.bfloat16)
+            ms = median_ms(lambda: rmt.rmt_grouped_gemm_bf16(a, b, c, G, Mc, N, K, "bf16"))
+            emit("grouped_gemm_bf16_tokens", {"G": G, "M": Mc, "N": N, "K": K, "kernel": "CTA pairs"},
+                 ms, 2.0 * G * Mc * N * K, "TFLOP/s", peaks["bf16_tflops"], "bf16_tflops")
+            del a, b, c
         return 0
 
     if args.microbench == "attention":
