@@ -562,17 +562,21 @@ struct UpdLayout {  // shared-memory layout in floats (every region starts 16-by
 //   den_r = phi(k_r) . z + eps + sum_{j<r} G_rj
 //   d_r   = V_r - phi(k_r) A / den_r - sum_{j<r} G_rj d_j / den_r
 // and after the last row A' = A + phi(K)^T D, z' = z + sum_r phi(k_r), as in the batched rule.
-// seq_gram_den: G (lower triangle, i ascending) and the denominators (den holds phi(k_r) . z
-// + eps on entry; j ascending). seq_substitute: D holds V_r - phi(k_r) A / den_r on entry and
-// d_r on exit, rows ascending, one thread per column. Both run the same order in every kernel.
+// seq_gram_den: G (lower triangle; one warp per row, lanes over i, then a butterfly) and the
+// denominators (den holds phi(k_r) . z + eps on entry; j ascending). seq_substitute: D holds
+// V_r - phi(k_r) A / den_r on entry and d_r on exit, rows ascending, one thread per column.
+// Both run the same order in every kernel.
 __device__ __forceinline__ void seq_gram_den(const float* fk, int n, int dk, int ldg, float* gram, float* den,
                                              int tid, int nthreads) {
-  for (int p = tid; p < n * n; p += nthreads) {
-    const int r = p / n, j = p % n;
-    if (j >= r) continue;
-    float s = 0.f;
-    for (int i = 0; i < dk; ++i) s = fmaf(fk[r * dk + i], fk[j * dk + i], s);
-    gram[r * ldg + j] = s;
+  // one warp per row r: lanes over i (ascending within a lane), then the butterfly, per j < r
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = 1 + warp; r < n; r += nthreads >> 5) {
+    for (int j = 0; j < r; ++j) {
+      float s = 0.f;
+      for (int i = lane; i < dk; i += 32) s = fmaf(fk[r * dk + i], fk[j * dk + i], s);
+      s = warp_sum(s);
+      if (lane == 0) gram[r * ldg + j] = s;
+    }
   }
   __syncthreads();
   for (int r = tid; r < n; r += nthreads) {
