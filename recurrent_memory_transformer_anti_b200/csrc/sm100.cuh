@@ -147,6 +147,14 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
                "r"(c0), "r"(c1), "r"(c2), "r"(src)
                : "memory");
 }
+// Untiled bulk copy global -> this CTA's shared memory, completion counted in bytes on `bar`.
+// Both addresses 16-byte aligned, `bytes` a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -187,6 +195,17 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
 
 // Instruction descriptor, kind::f16 with an fp32 accumulator: A and B both of format `fmt`
 // (0 = f16, 1 = bf16; the two operands of one MMA always share a type), both K-major.
+// The same layout with 8-row groups `sbo` bytes apart (a multiple of 1024): another operand, or
+// other data, can sit in the gaps.
+__device__ __forceinline__ uint64_t smem_desc_k128_sbo(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address (16-byte units)
+  d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset: 16 B (unused here)
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;  // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (tcgen05)
+  d |= static_cast<uint64_t>(2) << 61;                  // swizzle: 128 B
+  return d;
+}
 __host__ __device__ constexpr uint32_t idesc_f32acc(int m, int n, uint32_t fmt) {
   return (1u << 4)                                   // D format: f32
          | (fmt << 7)                                // A format
