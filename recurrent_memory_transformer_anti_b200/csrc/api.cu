@@ -861,15 +861,17 @@ cudaError_t enqueue_step(rmt_handle* h, const Table& t, int step, const void* em
     e = launch_kind(h, RMT_K_DOWN, d_flops, d_bytes, st, [&] { return run_proj(h, kProjDown, cells, G, st); });
     if (e != cudaSuccess) return e;
   }
+  // many cells: whole sums in one "split" (the same bits as the partials' sum)
+  const int kv_splits = mem_kv_written_splits(G, c.n_mem, d, h->bf16);
   e = launch_kind(h, RMT_K_MEMKV, 2 * g * n * (dk + dv) * dd,
-                  g * (n * dd * 4 + (dk + dv) * dd * es + h->nsplit * n * (dk + dv) * 4), st, [&] {
+                  g * (n * dd * 4 + (dk + dv) * dd * es + kv_splits * n * (dk + dv) * 4), st, [&] {
                     MemKvArgs a{h->x, M, d, c.n_mem, kOutSlot, h->w_mkv, h->part, c.d_k + c.d_v, G, cells, L};
                     return launch_mem_kv(a, h->bf16, st);
                   });
   if (e != cudaSuccess) return e;
   e = launch_kind(h, RMT_K_MEMUPDATE, g * 4 * n * dk * dv,
-                  g * (h->nsplit * n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), st, [&] {
-                    MemUpdateArgs a{h->part, h->nsplit, nullptr, nullptr, h->A, h->z, c.n_mem, c.d_k, c.d_v, c.mem_eps,
+                  g * (kv_splits * n * (dk + dv) * 4 + 2 * (dk * dv + dk) * 4), st, [&] {
+                    MemUpdateArgs a{h->part, kv_splits, nullptr, nullptr, h->A, h->z, c.n_mem, c.d_k, c.d_v, c.mem_eps,
                                     G, cells, kByLayer, kByLayer, L, h->trace, off, step,
                                     c.mem_update == RMT_MEM_SEQUENTIAL ? 1 : 0};
                     return launch_mem_update(a, st);
@@ -1674,7 +1676,8 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MemKvArgs ka{y, n, d, n, kByLayer, w_mkv, part, dk + dv, G, cells, G};
   RMT_CUDA(launch_mem_kv(ka, dtype == RMT_BF16, st));
-  MemUpdateArgs ua{part, nsplit, nullptr, nullptr, A, z, n, dk, dv, eps, G, cells, kByLayer, kByLayer, G, nullptr, 0, 0};
+  MemUpdateArgs ua{part, mem_kv_written_splits(G, n, d, dtype == RMT_BF16), nullptr, nullptr, A, z, n, dk, dv, eps, G,
+                   cells, kByLayer, kByLayer, G, nullptr, 0, 0};
   RMT_CUDA(launch_mem_update(ua, st));
   return RMT_OK;
 }

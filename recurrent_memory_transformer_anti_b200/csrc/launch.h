@@ -200,6 +200,13 @@ struct MemKvArgs {
   const Cell* cells;
   int L;
 };
+// Launches of many cells (at least four per SM, bf16 weights) write whole sums instead: one
+// split, [L, 1, n, dkv], each element the sum of the partials above in split order (the same
+// bits the update forms from them). The update then takes nsplit = 1.
+bool mem_kv_whole(int G, int n, bool bf16);
+inline int mem_kv_written_splits(int G, int n, int d, bool bf16) {
+  return mem_kv_whole(G, n, bf16) ? 1 : mem_kv_splits(d, bf16);
+}
 cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st);
 
 // Delta-rule update of A, z from raw keys/values of n rows. Keys/values come either from

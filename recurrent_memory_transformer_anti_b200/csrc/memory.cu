@@ -397,102 +397,118 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
 // the weights with ldmatrix (the warps share the rows: splitting while forming the fragments
 // would repeat the conversion in every warp). Warp w computes the 8-column output tiles w and
 // w + 8 of every 16-row tile.
+// WHOLE: one CTA per (cell, block of output columns) runs the splits one after another (the
+// next split's rows and weights in flight while this one is multiplied, two stages), forms each
+// split's partial exactly as above and adds it to a running sum in split order -- the sum the
+// update forms from the partials, bit for bit -- and writes that sum alone (one "split"). For
+// launches of many cells, where the partials' round trip through memory would cost more than
+// the splits' parallelism gains.
 constexpr int kKvMmaThreads = 256;
 constexpr int kKvYStride = kMemKvSplit + 8;  // fp32 row stride of the staged rows
 constexpr int kKvWStride = kMemKvSplit + 8;  // bf16 row stride of the staged weights (272 B: ldmatrix rows on distinct banks)
 constexpr int kKvPStride = kMemKvSplit + 8;  // bf16 row stride of the split planes (same reason)
 
-// Shared memory of the tensor-core k/v kernel: fp32 rows, weight rows, three split planes.
-inline size_t kv_mma_smem(int n, int cols) {
+// Shared memory of the tensor-core k/v kernel: `stages` x (fp32 rows, weight rows), then three
+// split planes.
+inline size_t kv_mma_smem(int n, int cols, int stages = 1) {
   const size_t n16 = (n + 15) & ~15, wrows = (cols + 7) / 8 * 8;
-  return sizeof(float) * n16 * kKvYStride + 2 * wrows * kKvWStride + 3 * 2 * n16 * kKvPStride;
+  return stages * (sizeof(float) * n16 * kKvYStride + 2 * wrows * kKvWStride) + 3 * 2 * n16 * kKvPStride;
 }
 
+template <bool WHOLE>
 __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvArgs a) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ __align__(16) unsigned char kv_sm[];
   constexpr int KS = kMemKvSplit;
+  constexpr int NB = WHOLE ? 2 : 1;  // stages of rows and weights
   const int n16 = (a.n + 15) & ~15;
   const int j_base = blockIdx.z * kKvCols, cols = min(kKvCols, a.dkv - j_base);
   const int ntiles = (cols + 7) / 8;
-  float* Ys = reinterpret_cast<float*>(kv_sm);                                                      // [n16][kKvYStride]
-  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(kv_sm + sizeof(float) * n16 * kKvYStride);  // [8*ntiles][kKvWStride]
-  __nv_bfloat16* Ps = Ws + 8 * ntiles * kKvWStride;  // [3][n16][kKvPStride]: y1, y2, y3
+  const size_t ybytes = sizeof(float) * n16 * kKvYStride, wbytes = 2 * 8 * ntiles * kKvWStride;
+  auto Ys_of = [&](int b) { return reinterpret_cast<float*>(kv_sm + b * (ybytes + wbytes)); };  // [n16][kKvYStride]
+  auto Ws_of = [&](int b) {  // [8*ntiles][kKvWStride]
+    return reinterpret_cast<__nv_bfloat16*>(kv_sm + b * (ybytes + wbytes) + ybytes);
+  };
+  __nv_bfloat16* Ps = reinterpret_cast<__nv_bfloat16*>(kv_sm + NB * (ybytes + wbytes));  // [3][n16][kKvPStride]
   const Cell c = load_cell(a.cells, blockIdx.y);
-  const int split = blockIdx.x, k0 = split * KS;
-  const int kw = min(KS, a.d - k0);
+  const int nsplit = (a.d + KS - 1) / KS;
   const int row0 = cell_rows(c, a.M) - a.n;  // the cell's memory rows are its last n valid rows
-  const float* Y = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row0) * a.d + k0;
-  const __nv_bfloat16* W =
-      static_cast<const __nv_bfloat16*>(a.w) + (static_cast<size_t>(c.l) * a.dkv + j_base) * a.d + k0;
+  const float* Yc = a.x + (static_cast<size_t>(cell_index(a.x_mode, a.L, c)) * a.M + row0) * a.d;
+  const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(a.w) + (static_cast<size_t>(c.l) * a.dkv + j_base) * a.d;
   const bool y_vec = (a.d % 4 == 0) && (reinterpret_cast<uintptr_t>(a.x) % 16 == 0);
   const bool w_vec = (a.d % 8 == 0) && (reinterpret_cast<uintptr_t>(a.w) % 16 == 0);
   const int tid = threadIdx.x;
   // rows (zero past n and past the split's columns) and the weight rows of this column block
-  // (zero past cols and past the split's columns): whole 16-byte chunks by cp.async; chunks at a
-  // ragged edge, or of unaligned rows, element by element
-  for (int e = tid; e < n16 * (KS / 4); e += kKvMmaThreads) {
-    const int r = e / (KS / 4), k = 4 * (e % (KS / 4));
-    float* dst = Ys + r * kKvYStride + k;
-    const float* yr = Y + static_cast<size_t>(r < a.n ? r : 0) * a.d + k;
-    if (y_vec && (r >= a.n || k + 3 < kw)) {
-      cp_async16(sm100::smem_u32(dst), r < a.n ? yr : Y, r < a.n ? 16u : 0u);
-    } else {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < a.n) {
-        if (k < kw) v.x = yr[0];
-        if (k + 1 < kw) v.y = yr[1];
-        if (k + 2 < kw) v.z = yr[2];
-        if (k + 3 < kw) v.w = yr[3];
+  // (zero past cols and past the split's columns) of one split into stage b: whole 16-byte chunks
+  // by cp.async; chunks at a ragged edge, or of unaligned rows, element by element
+  auto issue = [&](int split, int b) {
+    const int k0 = split * KS, kw = min(KS, a.d - k0);
+    const float* Y = Yc + k0;
+    const __nv_bfloat16* W = Wc + k0;
+    float* Ys = Ys_of(b);
+    __nv_bfloat16* Ws = Ws_of(b);
+    for (int e = tid; e < n16 * (KS / 4); e += kKvMmaThreads) {
+      const int r = e / (KS / 4), k = 4 * (e % (KS / 4));
+      float* dst = Ys + r * kKvYStride + k;
+      const float* yr = Y + static_cast<size_t>(r < a.n ? r : 0) * a.d + k;
+      if (y_vec && (r >= a.n || k + 3 < kw)) {
+        cp_async16(sm100::smem_u32(dst), r < a.n ? yr : Y, r < a.n ? 16u : 0u);
+      } else {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < a.n) {
+          if (k < kw) v.x = yr[0];
+          if (k + 1 < kw) v.y = yr[1];
+          if (k + 2 < kw) v.z = yr[2];
+          if (k + 3 < kw) v.w = yr[3];
+        }
+        *reinterpret_cast<float4*>(dst) = v;
       }
-      *reinterpret_cast<float4*>(dst) = v;
     }
-  }
-  for (int e = tid; e < 8 * ntiles * (KS / 8); e += kKvMmaThreads) {
-    const int j = e / (KS / 8), k = 8 * (e % (KS / 8));
-    __nv_bfloat16* dst = Ws + j * kKvWStride + k;
-    const __nv_bfloat16* wr = W + static_cast<size_t>(j < cols ? j : 0) * a.d + k;
-    if (w_vec && (j >= cols || k + 7 < kw)) {
-      cp_async16(sm100::smem_u32(dst), j < cols ? wr : W, j < cols ? 16u : 0u);
-    } else {
-      uint32_t h[8];
+    for (int e = tid; e < 8 * ntiles * (KS / 8); e += kKvMmaThreads) {
+      const int j = e / (KS / 8), k = 8 * (e % (KS / 8));
+      __nv_bfloat16* dst = Ws + j * kKvWStride + k;
+      const __nv_bfloat16* wr = W + static_cast<size_t>(j < cols ? j : 0) * a.d + k;
+      if (w_vec && (j >= cols || k + 7 < kw)) {
+        cp_async16(sm100::smem_u32(dst), j < cols ? wr : W, j < cols ? 16u : 0u);
+      } else {
+        uint32_t h[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) h[t] = (j < cols && k + t < kw) ? __bfloat16_as_ushort(wr[t]) : 0u;
-      *reinterpret_cast<uint4*>(dst) =
-          make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+        for (int t = 0; t < 8; ++t) h[t] = (j < cols && k + t < kw) ? __bfloat16_as_ushort(wr[t]) : 0u;
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+      }
     }
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  // the rows' three bf16 terms, two columns per step
-  for (int e = tid; e < n16 * (KS / 2); e += kKvMmaThreads) {
-    const int r = e / (KS / 2), k = 2 * (e % (KS / 2));
-    uint32_t t1, t2, t3;
-    split3(*reinterpret_cast<const float2*>(Ys + r * kKvYStride + k), t1, t2, t3);
-    uint32_t* p = reinterpret_cast<uint32_t*>(Ps + r * kKvPStride + k);
-    p[0] = t1;
-    p[n16 * kKvPStride / 2] = t2;
-    p[n16 * kKvPStride] = t3;
-  }
-  __syncthreads();
+  };
+  // the rows of stage b -> their three bf16 terms, two columns per step
+  auto split_rows = [&](int b) {
+    const float* Ys = Ys_of(b);
+    for (int e = tid; e < n16 * (KS / 2); e += kKvMmaThreads) {
+      const int r = e / (KS / 2), k = 2 * (e % (KS / 2));
+      uint32_t t1, t2, t3;
+      split3(*reinterpret_cast<const float2*>(Ys + r * kKvYStride + k), t1, t2, t3);
+      uint32_t* p = reinterpret_cast<uint32_t*>(Ps + r * kKvPStride + k);
+      p[0] = t1;
+      p[n16 * kKvPStride / 2] = t2;
+      p[n16 * kKvPStride] = t3;
+    }
+  };
   const int warp = tid >> 5, lane = tid & 31, gq = lane >> 2, tq = lane & 3;
-  const int nsplit = (a.d + KS - 1) / KS;
-  float* part = a.part + (static_cast<size_t>(c.k) * nsplit + split) * a.n * a.dkv;
   const int nt0 = warp, nt1 = warp + 8;  // this warp's output tiles (kKvCols = 128: at most 16)
-  const bool has1 = nt1 < ntiles;
-  if (nt0 >= ntiles) return;
+  const bool has0 = nt0 < ntiles, has1 = nt1 < ntiles;
   // ldmatrix row addresses: lanes 0-7 give the rows of the k 0..7 matrix, lanes 8-15 of k 8..15
   const int lr = lane & 7, lk = ((lane >> 3) & 1) * 8;
-  const uint32_t wb0 = sm100::smem_u32(Ws + (nt0 * 8 + lr) * kKvWStride + lk);
-  const uint32_t wb1 = has1 ? sm100::smem_u32(Ws + (nt1 * 8 + lr) * kKvWStride + lk) : wb0;
   // ldmatrix x4 row addresses of a 16 x 16 A tile: lanes 0-15 rows 0-15 at k 0, lanes 16-31 at k 8
   const uint32_t plane = 2u * n16 * kKvPStride;  // bytes
   const uint32_t pa0 =
       sm100::smem_u32(Ps + ((lane & 7) + ((lane >> 3) & 1) * 8) * kKvPStride + (lane >> 4) * 8);
-  for (int mt = 0; mt < n16 / 16; ++mt) {
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+  // the partial of 16-row tile mt over the split in stage b: acc0 (tile nt0), acc1 (tile nt1)
+  auto partial = [&](int b, int mt, float (&acc0)[4], float (&acc1)[4]) {
+    const __nv_bfloat16* Ws = Ws_of(b);
+    const uint32_t wb0 = sm100::smem_u32(Ws + (nt0 * 8 + lr) * kKvWStride + lk);
+    const uint32_t wb1 = has1 ? sm100::smem_u32(Ws + (nt1 * 8 + lr) * kKvWStride + lk) : wb0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc0[q] = acc1[q] = 0.f;
     const uint32_t pa = pa0 + 2u * 16 * kKvPStride * mt;
 #pragma unroll 2
     for (int ks = 0; ks < KS / 16; ++ks) {
@@ -512,15 +528,69 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
         mma_bf16_16816(acc1, t3, b0, b1);
       }
     }
-    const int r = mt * 16 + gq;
-    auto store = [&](const float (&acc)[4], int nt) {
-      const int col = nt * 8 + 2 * tq;
-      if (col >= cols) return;
-      if (r < a.n) *reinterpret_cast<float2*>(part + r * a.dkv + j_base + col) = make_float2(acc[0], acc[1]);
-      if (r + 8 < a.n) *reinterpret_cast<float2*>(part + (r + 8) * a.dkv + j_base + col) = make_float2(acc[2], acc[3]);
-    };
-    store(acc0, nt0);
-    if (has1) store(acc1, nt1);
+  };
+  auto store = [&](float* part, const float (&acc)[4], int mt, int nt) {
+    const int r = mt * 16 + gq, col = nt * 8 + 2 * tq;
+    if (col >= cols) return;
+    if (r < a.n) *reinterpret_cast<float2*>(part + r * a.dkv + j_base + col) = make_float2(acc[0], acc[1]);
+    if (r + 8 < a.n) *reinterpret_cast<float2*>(part + (r + 8) * a.dkv + j_base + col) = make_float2(acc[2], acc[3]);
+  };
+
+  if constexpr (!WHOLE) {
+    const int split = blockIdx.x;
+    issue(split, 0);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    split_rows(0);
+    __syncthreads();
+    float* part = a.part + (static_cast<size_t>(c.k) * nsplit + split) * a.n * a.dkv;
+    if (!has0) return;
+    for (int mt = 0; mt < n16 / 16; ++mt) {
+      float acc0[4], acc1[4];
+      partial(0, mt, acc0, acc1);
+      store(part, acc0, mt, nt0);
+      if (has1) store(part, acc1, mt, nt1);
+    }
+  } else {
+    float s0[4][4], s1[4][4];  // running sums of row tiles mt < 4 (n <= 64)
+    issue(0, 0);
+    cp_async_commit();
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const int b = sp & 1;
+      if (sp + 1 < nsplit) issue(sp + 1, b ^ 1);  // stage b ^ 1 was freed by the barrier that closed split sp - 1
+      cp_async_commit();
+      cp_async_wait<1>();  // this split's stage has landed
+      __syncthreads();
+      split_rows(b);
+      __syncthreads();
+      if (has0) {
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          if (mt < n16 / 16) {
+            float acc0[4], acc1[4];
+            partial(b, mt, acc0, acc1);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              s0[mt][q] = sp == 0 ? acc0[q] : s0[mt][q] + acc0[q];
+              s1[mt][q] = sp == 0 ? acc1[q] : s1[mt][q] + acc1[q];
+            }
+          }
+        }
+      }
+      __syncthreads();  // the planes and stage b are free
+    }
+    cp_async_wait<0>();
+    float* part = a.part + static_cast<size_t>(c.k) * a.n * a.dkv;
+    if (has0) {
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        if (mt < n16 / 16) {
+          store(part, s0[mt], mt, nt0);
+          if (has1) store(part, s1[mt], mt, nt1);
+        }
+      }
+    }
   }
 }
 
@@ -995,16 +1065,26 @@ cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_
 }
 
 
+bool mem_kv_whole(int G, int n, bool bf16) {
+  if (!bf16 || n > 64) return false;
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return static_cast<long>(G) >= 4L * (sms > 0 ? sms : 148);
+}
+
 cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (a.G <= 0) return cudaSuccess;
   if (a.n > 64 || a.dkv % 4) return cudaErrorInvalidValue;
   dim3 grid((a.d + kMemKvSplit - 1) / kMemKvSplit, a.G, (a.dkv + kKvCols - 1) / kKvCols);
   if (bf16) {  // tensor cores: three-term split of the fp32 rows against the bf16 weights
     const int cols = a.dkv < kKvCols ? a.dkv : kKvCols;
-    const size_t smem = kv_mma_smem(a.n, cols);
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(mem_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    const cudaError_t e = launch_pdl(mem_kv_mma_kernel, grid, dim3(kKvMmaThreads), smem, st, a);
+    const bool whole = mem_kv_whole(a.G, a.n, true);
+    const size_t smem = kv_mma_smem(a.n, cols, whole ? 2 : 1);
+    void (*kern)(MemKvArgs) = whole ? mem_kv_mma_kernel<true> : mem_kv_mma_kernel<false>;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (whole) grid.x = 1;
+    const cudaError_t e = launch_pdl(kern, grid, dim3(kKvMmaThreads), smem, st, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

@@ -55,11 +55,13 @@ extern "C" rmt_status rmt_memory_write_noalloc(const float* y, const void* w_mkv
       n * (dk + dv) > 4096)
     return fail(RMT_EINVAL, "bad sizes");
   if (dtype != RMT_F32 && dtype != RMT_BF16) return fail(RMT_EINVAL, "bad dtype");
-  const size_t nsplit = static_cast<size_t>(rmt::mem_kv_splits(d, dtype == RMT_BF16));
+  // the projection writes ceil(d/128) partial sums per cell, or their whole sum when the launch is
+  // large (mem_kv_written_splits)
+  const size_t nsplit = static_cast<size_t>(rmt::mem_kv_written_splits(G, n, d, dtype == RMT_BF16));
   const size_t part_bytes = size_t(G) * nsplit * n * (dk + dv) * sizeof(float);
   if (size_t(G) * sizeof(Cell) > kNoAllocCellBytes || part_bytes > kNoAllocScratchBytes - kNoAllocCellBytes)
     return fail(RMT_EINVAL,
-                "rmt_memory_write_noalloc: G*ceil(d/128)*n*(dk+dv)*4 bytes of partial sums exceed the fixed "
+                "rmt_memory_write_noalloc: G*splits*n*(dk+dv)*4 bytes of partial sums exceed the fixed "
                 "8 MiB - 256 KiB scratch (or G > 8192); use rmt_memory_write");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(RMT_ECUDA, "cudaGetDevice failed");

@@ -276,6 +276,41 @@ def test_memory_write_matches_oracle(dtype, G, n, d, dk, dv):
         assert normwise(to_np(tz[g]), rz) < 2e-6
 
 
+def test_memory_write_whole_sums_equal_split_partials_bitwise():
+    """A write of many groups (at least four per SM, bf16 weights) adds each group's split-K
+    partials inside one CTA and hands the update whole sums (the streaming update kernel); a
+    write of few groups goes through the partials and the cluster update. The same groups give
+    the same bits either way, so one launch of 600 groups equals six launches of 100."""
+    G, chunk, n, d, dk, dv = 600, 100, 16, 2048, 64, 64
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert G >= 4 * sms > chunk  # the two routes
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    y = torch.randn(G, n, d, device="cuda", generator=gen)
+    w = (torch.randn(G, dk + dv, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+    A0 = torch.randn(G, dk, dv, device="cuda", generator=gen)
+    z0 = torch.rand(G, dk, device="cuda", generator=gen) * 99 + 1
+    A1, z1 = A0.clone(), z0.clone()
+    rmt.rmt_memory_write(y, w, A1, z1, G, n, d, dk, dv, 1e-6, "bf16")
+    A2, z2 = A0.clone(), z0.clone()
+    for g0 in range(0, G, chunk):
+        sl = slice(g0, g0 + chunk)
+        a_, z_ = A2[sl].contiguous(), z2[sl].contiguous()
+        rmt.rmt_memory_write(y[sl].contiguous(), w[sl].contiguous(), a_, z_, chunk, n, d, dk, dv, 1e-6, "bf16")
+        A2[sl], z2[sl] = a_, z_
+    rmt.rmt_sync(None)
+    assert torch.equal(A1, A2) and torch.equal(z1, z2)
+    assert not torch.equal(A1, A0)
+    # and the whole route against the oracle on a few groups
+    for g in (0, 299, 599):
+        y64 = y[g].double().cpu().numpy()
+        w64 = w[g].float().double().cpu().numpy()
+        rA, rz = armt.memory_update(y64 @ w64[:dk].T, y64 @ w64[dk:].T, A0[g].double().cpu().numpy(),
+                                    z0[g].double().cpu().numpy(), 1e-6)
+        assert normwise(to_np(A1[g]), rA) < 2e-5
+        assert normwise(to_np(z1[g]), rz) < 2e-6
+
+
 def test_bounded_wait_gives_up_and_reports_without_a_fault(cuda_ok):
     """The failure path of every kernel: a wait on a barrier that nothing signals, and a wait on a
     global counter that nothing increments (the chained projections' dependency wait), each
