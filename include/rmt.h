@@ -333,9 +333,9 @@ rmt_status rmt_memory_update_sequential(const float* k, const float* v, float* A
  * of W_mv); A [G, dk, dv] and z [G, dk] fp32, updated in place. The projection is split
  * along d in blocks of 128 columns (tensor cores for bf16 weights, the fp32 rows split into
  * three bf16 terms) whose partial sums go to a library-owned device scratch buffer (grown
- * with cudaMalloc on demand) and are added in a fixed order. With bf16 weights and at least
- * four groups per SM, one CTA adds a group's partials in that same order itself and only the
- * sums go through the buffer (the same bits).
+ * with cudaMalloc on demand) and are added in a fixed order. With bf16 weights, n <= 16 and at
+ * least four groups per SM, one CTA adds a group's partials in that same order itself and only
+ * the sums go through the buffer (the same bits).
  * n <= 64, n*(dk+dv) <= 4096; dk, dv multiples of 32, <= 128; A and z 16-byte aligned. */
 rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* z, int32_t G, int32_t n,
                             int32_t d, int32_t dk, int32_t dv, float eps, rmt_dtype dtype, void* stream);
@@ -347,7 +347,7 @@ rmt_status rmt_memory_write(const float* y, const void* w_mkv, float* A, float* 
  * streams). Same arguments and results as rmt_memory_write; the cell table and the split-K
  * partial sums live in a fixed 8 MiB array in the library's device memory. Sizes whose
  * partial sums need more than 8 MiB - 256 KiB (G*s*n*(dk+dv)*4 bytes, s = ceil(d/128), or s = 1
- * with bf16 weights and at least four groups per SM), or
+ * with bf16 weights, n <= 16 and at least four groups per SM), or
  * G > 8192, return RMT_EINVAL. It calls no cudaMalloc or cudaFree. The first call on each
  * device loads the module that holds the array (CUDA loads modules lazily by default), which
  * reserves the 8 MiB on that device until the process exits, and looks up the array's

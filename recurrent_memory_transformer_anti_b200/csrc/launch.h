@@ -200,7 +200,7 @@ struct MemKvArgs {
   const Cell* cells;
   int L;
 };
-// Launches of many cells (at least four per SM, bf16 weights) write whole sums instead: one
+// Launches of many cells (at least four per SM, bf16 weights, n <= 16) write whole sums instead: one
 // split, [L, 1, n, dkv], each element the sum of the partials above in split order (the same
 // bits the update forms from them). The update then takes nsplit = 1.
 bool mem_kv_whole(int G, int n, bool bf16);

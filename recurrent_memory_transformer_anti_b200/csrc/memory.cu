@@ -397,13 +397,15 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
 // the weights with ldmatrix (the warps share the rows: splitting while forming the fragments
 // would repeat the conversion in every warp). Warp w computes the 8-column output tiles w and
 // w + 8 of every 16-row tile.
-// WHOLE: one CTA per (cell, block of output columns) runs the splits one after another (the
-// next split's rows and weights in flight while this one is multiplied, two stages), forms each
+// WHOLE: one CTA per (cell, block of output columns) runs the splits one after another (three
+// such CTAs per SM, whose loads and products interleave; a ring of four stages in one CTA per
+// SM measured slower), forms each
 // split's partial exactly as above and adds it to a running sum in split order -- the sum the
 // update forms from the partials, bit for bit -- and writes that sum alone (one "split"). For
 // launches of many cells, where the partials' round trip through memory would cost more than
 // the splits' parallelism gains.
 constexpr int kKvMmaThreads = 256;
+constexpr int kKvWholeStages = 1;  // 57 KB at n <= 16: three CTAs per SM
 constexpr int kKvYStride = kMemKvSplit + 8;  // fp32 row stride of the staged rows
 constexpr int kKvWStride = kMemKvSplit + 8;  // bf16 row stride of the staged weights (272 B: ldmatrix rows on distinct banks)
 constexpr int kKvPStride = kMemKvSplit + 8;  // bf16 row stride of the split planes (same reason)
@@ -416,12 +418,12 @@ inline size_t kv_mma_smem(int n, int cols, int stages = 1) {
 }
 
 template <bool WHOLE>
-__global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvArgs a) {
+__global__ void __launch_bounds__(kKvMmaThreads, WHOLE ? 3 : 1) mem_kv_mma_kernel(const MemKvArgs a) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ __align__(16) unsigned char kv_sm[];
   constexpr int KS = kMemKvSplit;
-  constexpr int NB = WHOLE ? 2 : 1;  // stages of rows and weights
+  constexpr int NB = WHOLE ? kKvWholeStages : 1;  // stages of rows and weights
   const int n16 = (a.n + 15) & ~15;
   const int j_base = blockIdx.z * kKvCols, cols = min(kKvCols, a.dkv - j_base);
   const int ntiles = (cols + 7) / 8;
@@ -553,14 +555,18 @@ __global__ void __launch_bounds__(kKvMmaThreads) mem_kv_mma_kernel(const MemKvAr
       if (has1) store(part, acc1, mt, nt1);
     }
   } else {
-    float s0[4][4], s1[4][4];  // running sums of row tiles mt < 4 (n <= 64)
-    issue(0, 0);
-    cp_async_commit();
-    for (int sp = 0; sp < nsplit; ++sp) {
-      const int b = sp & 1;
-      if (sp + 1 < nsplit) issue(sp + 1, b ^ 1);  // stage b ^ 1 was freed by the barrier that closed split sp - 1
+    float s0[4][4], s1[4][4];  // running sums of row tiles mt < 4 (n <= 64; this route takes n <= 16)
+#pragma unroll
+    for (int j = 0; j < NB - 1; ++j) {
+      if (j < nsplit) issue(j, j);
       cp_async_commit();
-      cp_async_wait<1>();  // this split's stage has landed
+    }
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const int b = sp % NB;
+      // the stage of split sp - 1, freed by the barrier that closed it, takes split sp + NB - 1
+      if (sp + NB - 1 < nsplit) issue(sp + NB - 1, (sp + NB - 1) % NB);
+      cp_async_commit();
+      cp_async_wait<NB - 1>();  // this split's stage has landed
       __syncthreads();
       split_rows(b);
       __syncthreads();
@@ -1066,7 +1072,7 @@ cudaError_t launch_mem_read(const MemReadArgs& a, ElemType out_type, cudaStream_
 
 
 bool mem_kv_whole(int G, int n, bool bf16) {
-  if (!bf16 || n > 64) return false;
+  if (!bf16 || n > 16) return false;  // the running sums of one 16-row tile in registers
   int sms = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1080,7 +1086,8 @@ cudaError_t launch_mem_kv(const MemKvArgs& a, bool bf16, cudaStream_t st) {
   if (bf16) {  // tensor cores: three-term split of the fp32 rows against the bf16 weights
     const int cols = a.dkv < kKvCols ? a.dkv : kKvCols;
     const bool whole = mem_kv_whole(a.G, a.n, true);
-    const size_t smem = kv_mma_smem(a.n, cols, whole ? 2 : 1);
+    size_t smem = kv_mma_smem(a.n, cols, whole ? kKvWholeStages : 1);
+    if (whole && smem > 227 * 1024) return cudaErrorInvalidValue;  // n > 16 is kept off this route
     void (*kern)(MemKvArgs) = whole ? mem_kv_mma_kernel<true> : mem_kv_mma_kernel<false>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (whole) grid.x = 1;
