@@ -71,3 +71,25 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_ok):
         rmt.rmt_memory_write_noalloc(y, w, A, z, G, n, d, dk, dv, 1e-6, "f32")
     assert ex.value.status == rmt.RMT_EINVAL
     assert "scratch" in str(ex.value)
+
+
+def test_noalloc_many_groups_take_whole_sums_and_match_bitwise(cuda_ok):
+    """A launch of at least four groups per SM (bf16 weights, n <= 16) adds each group's split-K
+    partials inside one CTA, so only the sums (G*n*(dk+dv)*4 bytes, 4.9 MB at 600 groups) use the
+    fixed scratch: a size whose partials (78 MB) it could not hold. The results are the
+    allocating entry point's, bit for bit."""
+    G, n, d, dk, dv = 600, 16, 2048, 64, 64
+    assert G >= 4 * torch.cuda.get_device_properties(0).multi_processor_count
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(12)
+    y = torch.randn(G, n, d, device="cuda", generator=gen)
+    w = (torch.randn(G, dk + dv, d, device="cuda", generator=gen) * 0.02).to(torch.bfloat16)
+    A0 = torch.randn(G, dk, dv, device="cuda", generator=gen)
+    z0 = torch.rand(G, dk, device="cuda", generator=gen) * 99 + 1
+    A_ref, z_ref = A0.clone(), z0.clone()
+    A_new, z_new = A0.clone(), z0.clone()
+    rmt.rmt_memory_write(y, w, A_ref, z_ref, G, n, d, dk, dv, 1e-6, "bf16")
+    rmt.rmt_memory_write_noalloc(y, w, A_new, z_new, G, n, d, dk, dv, 1e-6, "bf16")
+    rmt.rmt_sync(None)
+    assert torch.equal(A_new, A_ref) and torch.equal(z_new, z_ref)
+    assert not torch.equal(A_new, A0)
