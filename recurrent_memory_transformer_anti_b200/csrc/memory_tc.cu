@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kRtThreads, DK == 64 ? 2 : 1) mem_read_tc_kern
 //     d_v + 16 > 128) and hands the stage back to the stream when they finish;
 //   - 4 epilogue warps (one per TMEM lane quarter) read a finished accumulator, release it,
 //     and divide, round and store their rows.
-// A stage is thus held from its load to its MMAs, and the ring (4-5 stages) keeps that many
+// A stage is thus held from its load to its MMAs, and the ring (4-6 stages) keeps that many
 // tiles in flight. The arithmetic is the same as in mem_read_tc_kernel, term for term.
 constexpr int kWsConvWarps = 8;
 constexpr int kWsEpiWarps = 4;  // 8 (two per lane quarter, half the columns each) measured the same
