@@ -866,12 +866,14 @@ constexpr int kUpdStreamThreads = 256;
 
 struct UpdStreamLayout {  // in floats; every region starts 16-byte aligned
   int n8, stage, fk, D, den, gram, total;
+  bool d_in_stage;  // D [n8][dv] over the cell's raw keys in its stage, dead once phi(K) is formed
   __host__ __device__ UpdStreamLayout(int n, int dk, int dv, int nst) {
     n8 = (n + 7) & ~7;
     stage = n * dk + n * dv + dk * dv + dk;  // K [n][dk], V [n][dv], A [dk][dv], z [dk]
     fk = nst * stage;                        // phi(K) [n][dk]
-    D = fk + n * dk;                         // [n8][dv]
-    den = D + n8 * dv;                       // [n8]
+    d_in_stage = n8 * dv <= n * dk;
+    D = d_in_stage ? -1 : fk + n * dk;       // [n8][dv] when it has a region of its own
+    den = d_in_stage ? fk + n * dk : D + n8 * dv;  // [n8]
     gram = den + n8;                         // [n][n8] (per-token rule)
     total = gram + n * n8;
   }
@@ -880,14 +882,13 @@ struct UpdStreamLayout {  // in floats; every region starts 16-byte aligned
 // A ring of NST cell stages: the loads of cells g+1 .. g+NST-1 are in flight while cell g is
 // computed (the stage of cell g+NST-1 is the one cell g-1 just released).
 template <int NST>
-__global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel(const MemUpdateArgs a) {
+__global__ void __launch_bounds__(kUpdStreamThreads, 4) mem_update_stream_kernel(const MemUpdateArgs a) {
   pdl_trigger();
   pdl_wait();  // inputs come from the previous kernels of the stream
   extern __shared__ __align__(16) float us[];
   const int n = a.n, dk = a.dk, dv = a.dv, dkv = dk + dv;
   const UpdStreamLayout lay(n, dk, dv, NST);
   float* fk = us + lay.fk;
-  float* D = us + lay.D;
   float* den = us + lay.den;
   float* gram = us + lay.gram;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -923,6 +924,7 @@ __global__ void __launch_bounds__(kUpdStreamThreads, 3) mem_update_stream_kernel
     const int i = g - c_beg;
     float* st = stage(i);
     const float* Kr = st;
+    float* D = lay.d_in_stage ? st : us + lay.D;  // over Kr: written only after phi(K) is formed
     const float* Vr = st + n * dk;
     const float* Ar = Vr + n * dv;
     const float* zr = Ar + dk * dv;
