@@ -397,13 +397,12 @@ __global__ void __launch_bounds__(kKvThreads) mem_kv_kernel(const MemKvArgs a) {
 // the weights with ldmatrix (the warps share the rows: splitting while forming the fragments
 // would repeat the conversion in every warp). Warp w computes the 8-column output tiles w and
 // w + 8 of every 16-row tile.
-// WHOLE: one CTA per (cell, block of output columns) runs the splits one after another (three
-// such CTAs per SM, whose loads and products interleave; a ring of four stages in one CTA per
-// SM measured slower), forms each
-// split's partial exactly as above and adds it to a running sum in split order -- the sum the
-// update forms from the partials, bit for bit -- and writes that sum alone (one "split"). For
-// launches of many cells, where the partials' round trip through memory would cost more than
-// the splits' parallelism gains.
+// WHOLE: one CTA per (cell, block of output columns) runs the splits one after another, forms
+// each split's partial exactly as above and adds it to a running sum in split order -- the sum
+// the update forms from the partials, bit for bit -- and writes that sum alone (one "split").
+// Three such CTAs per SM interleave their loads and products (a ring of four stages in one CTA
+// per SM measured slower). For launches of many cells, where the partials' round trip through
+// memory would cost more than the splits' parallelism gains.
 constexpr int kKvMmaThreads = 256;
 constexpr int kKvWholeStages = 1;  // 57 KB at n <= 16: three CTAs per SM
 constexpr int kKvYStride = kMemKvSplit + 8;  // fp32 row stride of the staged rows
